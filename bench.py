@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the fused exact-attention forward on B200.
+
+One step = one call of the hot path on one batch of seeded synthetic input,
+inputs already resident in HBM.  Default workload: GQA prefill with per-head
+sinks (B=1, H=64 over Hkv=8, T=1400 causal, D=512, bf16) -- the configuration
+the headline metric is quoted on.  Other workloads: --config c1 c3 c4 c5q8 c5q4.
+
+Timing: W untimed warm-up steps, then K steps; before each timed step a
+256 MiB buffer is written to flush L2 (outside the timed interval), and the
+step is bracketed by CUDA events on the launching stream.  Multi-GPU (torchrun):
+every rank runs the same per-GPU work (weak scaling, no data-path collective);
+the time is the max over ranks.  --impl reference times the CPU oracle on the
+host cores on a bounded sample of the same workload.
+
+Prints ONE JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+CONFIGS = {
+    "c1": dict(cfg=1, name="tiny dense causal fp32, B=1 H=4 Hkv=1 T=64 D=64", metric="attention fwd TFLOP/s",
+               dtype="f32"),
+    "c2": dict(cfg=2, name="GQA prefill with sinks, B=1 H=64 Hkv=8 T=1400 D=512 causal", metric="attention fwd TFLOP/s",
+               dtype="bf16"),
+    "c3": dict(cfg=3, name="MLA prefill, B=2 H=16 T=4096 d_qk=192 (128+64) d_v=128 causal",
+               metric="attention fwd TFLOP/s", dtype="bf16"),
+    "c4": dict(cfg=4, name="sparse MLA fwd, 13312 q x 64 h x 2176 top-k, d_qk=d_v=512, pool 65536",
+               metric="attention fwd TFLOP/s", dtype="bf16"),
+    "c5q8": dict(cfg=5, kv_type=W.KV_Q8_0, name="multi-seq decode, 4 seq x 4 tok, H=32 Hkv=8 D=128, 8192 cells/seq, q8_0",
+                 metric="decode GB/s", dtype="q8_0"),
+    "c5q4": dict(cfg=5, kv_type=W.KV_Q4_0, name="multi-seq decode, 4 seq x 4 tok, H=32 Hkv=8 D=128, 8192 cells/seq, q4_0",
+                 metric="decode GB/s", dtype="q4_0"),
+}
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def dense_pairs(Tq, Tk, causal):
+    if not causal:
+        return Tq * Tk
+    return sum(max(0, min(Tk, t + (Tk - Tq) + 1)) for t in range(Tq))
+
+
+def work(case):
+    """(algorithmic units, unit name) of one call: FLOPs over visible pairs, or bytes for decode."""
+    if isinstance(case, W.DenseCase):
+        pairs = case.B * case.H * dense_pairs(case.Tq, case.Tk, case.causal)
+        return pairs * (2 * case.D + 2 * case.Dv), "flop"
+    if isinstance(case, W.MlaCase):
+        pairs = case.B * case.H * dense_pairs(case.Tq, case.Tk, case.causal)
+        return pairs * (2 * (case.Dn + case.Dr) + 2 * case.Dv), "flop"
+    if isinstance(case, W.SparseCase):
+        valid = int(((case.idx >= 0) & (case.idx < case.Skv)).sum())
+        return valid * case.H * (2 * case.Dqk + 2 * case.Dv), "flop"
+    if isinstance(case, W.DecodeCase):
+        kv = case.k_cache.nbytes + case.v_cache.nbytes
+        qo = case.q.nbytes * 2 + case.n_tok * case.H * 4
+        return kv + qo, "byte"
+    raise TypeError(type(case))
+
+
+# ------------------------------------------------------------------ GPU arm
+
+class Uploaded:
+    """Device copies of a case plus the call that runs one step."""
+
+    def __init__(self, case, torch, arc):
+        self.case, self.torch, self.arc = case, torch, arc
+        self.h2d = 0
+
+    def to_dev(self, x):
+        torch = self.torch
+        x = np.ascontiguousarray(x)
+        t = torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x)
+        t = t.cuda()
+        return t.view(torch.bfloat16) if x.dtype == np.uint16 else t
+
+
+def build_call(case, torch, arc, status):
+    """Returns (call(), inputs dict of device tensors, outputs list, n_launches, kernel name)."""
+    U = Uploaded(case, torch, arc)
+    if isinstance(case, W.DenseCase):
+        q, k, v = U.to_dev(case.q), U.to_dev(case.k), U.to_dev(case.v)
+        s = U.to_dev(case.sinks) if case.sinks is not None else None
+        o = torch.empty(case.B, case.H, case.Tq, case.Dv, dtype=q.dtype, device="cuda")
+        lse = torch.empty(case.B, case.H, case.Tq, dtype=torch.float32, device="cuda")
+        info = arc.plan_attn(q, k, v, o, lse, causal=case.causal, sinks=s)
+
+        def call():
+            arc.attn_fwd(q, k, v, scale=case.scale, causal=case.causal, sinks=s, out=o, lse=lse, status=status)
+        ins = {"q": q, "k": k, "v": v}
+        if s is not None:
+            ins["sinks"] = s
+        return call, ins, [o, lse], info
+    if isinstance(case, W.MlaCase):
+        t = [U.to_dev(x) for x in (case.q_nope, case.q_rope, case.k_nope, case.k_rope, case.v)]
+        o = torch.empty(case.B, case.H, case.Tq, case.Dv, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(case.B, case.H, case.Tq, dtype=torch.float32, device="cuda")
+        info = arc.plan_mla(*t, o, lse, causal=case.causal)
+
+        def call():
+            arc.mla_fwd(*t, scale=case.scale, causal=case.causal, out=o, lse=lse, status=status)
+        return call, dict(zip(["q_nope", "q_rope", "k_nope", "k_rope", "v"], t)), [o, lse], info
+    if isinstance(case, W.SparseCase):
+        q, kv, idx = U.to_dev(case.q), U.to_dev(case.kv), U.to_dev(case.idx)
+        o = torch.empty(case.Sq, case.H, case.Dv, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(case.Sq, case.H, dtype=torch.float32, device="cuda")
+        info = arc.plan_sparse(q, kv, idx, o, lse, Dv=case.Dv)
+
+        def call():
+            arc.sparse_mla_fwd(q, kv, idx, Dv=case.Dv, scale=case.scale, out=o, lse=lse, status=status)
+        return call, {"q": q, "kv": kv, "idx": idx}, [o, lse], info
+    if isinstance(case, W.DecodeCase):
+        q, kc, vc = U.to_dev(case.q), U.to_dev(case.k_cache), U.to_dev(case.v_cache)
+        o = torch.empty(case.n_tok, case.H, case.D, dtype=torch.float32, device="cuda")
+        lse = torch.empty(case.n_tok, case.H, dtype=torch.float32, device="cuda")
+        kw = dict(kv_type=case.kv_type, Hkv=case.Hkv, q_begin=case.q_begin, n_q=case.n_q,
+                  kv_begin=case.kv_begin, n_kv=case.n_kv)
+        ws_n = arc.decode_workspace_size(case.kv_type, q, case.Hkv, case.n_cells, case.q_begin, case.n_q,
+                                         case.kv_begin, case.n_kv)
+        ws = torch.empty(max(ws_n, 256), dtype=torch.uint8, device="cuda")
+        info = arc.plan_decode(case.kv_type, q, kc, vc, **kw)
+
+        def call():
+            arc.attn_decode_q8(q, kc, vc, scale=case.scale, workspace=ws, out=o, lse=lse, status=status, **kw)
+        return call, {"q": q, "k_cache": kc, "v_cache": vc}, [o, lse], info
+    raise TypeError(type(case))
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report no clocks rather than guess
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def result(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvml unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash(kernel):
+    files = {"tc_attn_kernel": "attn_tc.cu", "tc_attn_kernel<mla>": "attn_tc.cu",
+             "sparse_tc_kernel": "sparse_tc.cu", "simple_attn_kernel<sparse>": "simple_kernels.cu",
+             "simple_attn_kernel": "simple_kernels.cu"}
+    f = files.get(kernel)
+    if kernel.startswith("decode_split_kernel"):
+        f = "decode.cu"
+    if not f:
+        return None
+    path = os.path.join(ROOT, "exact_attention_131_b200", "csrc", f)
+    h = hashlib.sha256(open(path, "rb").read())
+    h.update(open(os.path.join(ROOT, "exact_attention_131_b200", "csrc", "ptx.cuh"), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config_key, kernel):
+    """DRAM bytes per launch from a committed ncu summary, if its kernel source still matches."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(config_key)
+    if not rec or rec.get("kernel") != kernel or rec.get("source_hash") != kernel_source_hash(kernel):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
+    """The oracle as it stands, on the host cores, on a bounded sample of the workload."""
+    import oracle
+    oracle.build()
+    cores = oracle.num_threads()
+    rng = np.random.default_rng(0)
+    done_units, spent, n_rows = 0, 0.0, 0
+    if isinstance(case, (W.DenseCase, W.MlaCase)):
+        T = case.Tq
+        batch = 8
+        while spent < budget_s[0]:
+            rows = np.sort(rng.choice(T, size=batch, replace=False)).astype(np.int32)
+            t0 = time.perf_counter()
+            oracle.run_case(case, rows=rows)
+            spent += time.perf_counter() - t0
+            Dqk = case.D if isinstance(case, W.DenseCase) else case.Dn + case.Dr
+            heads = case.B * case.H
+            vis = sum(min(case.Tk, r + case.Tk - case.Tq + 1) if case.causal else case.Tk for r in rows)
+            done_units += heads * vis * (2 * Dqk + 2 * case.Dv)
+            n_rows += batch
+            if spent > budget_s[1]:
+                break
+        sample = f"{n_rows} random query positions x all {case.B * case.H} (batch, head) rows"
+        return {"value": done_units / spent / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": sample, "seconds": round(spent, 2)}
+    if isinstance(case, W.SparseCase):
+        batch = 4
+        while spent < budget_s[0]:
+            rows = np.sort(rng.choice(case.Sq, size=batch, replace=False))
+            t0 = time.perf_counter()
+            oracle.run_case(case, rows=rows)
+            spent += time.perf_counter() - t0
+            valid = int(((case.idx[rows] >= 0) & (case.idx[rows] < case.Skv)).sum())
+            done_units += valid * case.H * (2 * case.Dqk + 2 * case.Dv)
+            n_rows += batch
+            if spent > budget_s[1]:
+                break
+        return {"value": done_units / spent / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"{n_rows} random query tokens x 64 heads x all top-k slots", "seconds": round(spent, 2)}
+    if isinstance(case, W.DecodeCase):
+        reps = 0
+        units, _ = work(case)
+        while spent < budget_s[0] and reps < 50:
+            t0 = time.perf_counter()
+            oracle.run_case(case)
+            spent += time.perf_counter() - t0
+            reps += 1
+        return {"value": units * reps / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                "sample": f"the whole decode step, {reps} repetitions", "seconds": round(spent, 2)}
+    raise TypeError(type(case))
+
+
+def run_ours(args, spec, case):
+    import torch
+    import torch.distributed as dist
+    import exact_attention_131_b200 as arc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    call, ins, outs, info = build_call(case, torch, arc, status)
+    units, unit_kind = work(case)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            call()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    barrier()
+    times_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_ms = sum(times_ms) / len(times_ms)
+    total_ms = sum(times_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    assert arc.check_device_error(status) == arc.ARC_OK, "a device-side wait timed out"
+
+    # ---- end to end through the public API with host buffers
+    host_ins = {k: v.cpu().pin_memory() for k, v in ins.items()}
+    host_outs = [o.cpu().pin_memory() for o in outs]
+    h2d = sum(v.numel() * v.element_size() for v in host_ins.values())
+    d2h = sum(o.numel() * o.element_size() for o in host_outs)
+    e2e_steps = max(3, min(args.steps, 20))
+    e2e_ms = []
+    for i in range(e2e_steps + 2):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for kname, hv in host_ins.items():
+            ins[kname].copy_(hv, non_blocking=True)
+        call()
+        for o, ho in zip(outs, host_outs):
+            ho.copy_(o, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i >= 2:
+            e2e_ms.append(a.elapsed_time(b))
+    e2e_mean = sum(e2e_ms) / len(e2e_ms)
+
+    peaks = load_peaks()
+    if unit_kind == "flop":
+        value = units * world * args.steps / (total_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        achieved = units / (mean_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst bf16",
+                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None}
+        e2e_val = units / (e2e_mean * 1e-3) / 1e12
+    else:
+        value = units * world * args.steps / (total_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        achieved = units / (mean_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
+                "note": "whole call (split kernel + combine) timed"}
+        e2e_val = units / (e2e_mean * 1e-3) / 1e9
+    roof["traffic"] = recorded_traffic(args.config, info["kernel"])
+    roof["kernel"] = info["kernel"]
+
+    line = {
+        "metric": spec["metric"], "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": spec["dtype"], "data": "synthetic",
+        "config": {"workload": spec["name"], "config": args.config, "seed": spec["cfg"],
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world}, no collective" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_mean},
+        "gpu_launches": int(info["launches"]) * args.steps,
+        "clocks": sampler.result(),
+        "wall_s_timed_region": wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, args.config)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_reference(args, spec, case):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    cores = oracle.num_threads()
+    rng = np.random.default_rng(1)
+    per_step_units, times = [], []
+    for i in range(args.warmup + args.steps):
+        if isinstance(case, (W.DenseCase, W.MlaCase)):
+            rows = np.sort(rng.choice(case.Tq, size=2, replace=False)).astype(np.int32)
+            Dqk = case.D if isinstance(case, W.DenseCase) else case.Dn + case.Dr
+            vis = sum(min(case.Tk, r + case.Tk - case.Tq + 1) if case.causal else case.Tk for r in rows)
+            u = case.B * case.H * vis * (2 * Dqk + 2 * case.Dv)
+            t0 = time.perf_counter()
+            oracle.run_case(case, rows=rows)
+        elif isinstance(case, W.SparseCase):
+            rows = np.array([rng.integers(case.Sq)])
+            valid = int(((case.idx[rows] >= 0) & (case.idx[rows] < case.Skv)).sum())
+            u = valid * case.H * (2 * case.Dqk + 2 * case.Dv)
+            t0 = time.perf_counter()
+            oracle.run_case(case, rows=rows)
+        else:
+            u, _ = work(case)
+            t0 = time.perf_counter()
+            oracle.run_case(case)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+            per_step_units.append(u)
+    total = sum(times)
+    scale = 1e12 if spec["metric"].startswith("attention") else 1e9
+    unit = "TFLOP/s" if scale == 1e12 else "GB/s"
+    value = sum(per_step_units) / total / scale
+    sample = ("2 random query positions x all heads per step" if isinstance(case, (W.DenseCase, W.MlaCase))
+              else "1 random query token x all heads x all slots per step" if isinstance(case, W.SparseCase)
+              else "the whole decode step per step")
+    line = {"impl": "reference", "metric": spec["metric"], "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": spec["name"], "config": args.config, "seed": spec["cfg"]},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="c2")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    spec = CONFIGS[args.config]
+    kw = {"kv_type": spec["kv_type"]} if "kv_type" in spec else {}
+    case = W.config(spec["cfg"], **kw)
+    if args.impl == "reference":
+        run_reference(args, spec, case)
+    else:
+        run_ours(args, spec, case)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,602 @@
+// api.cu -- the C ABI declared in include/arc_attn.h: host-side validation,
+// planning (which kernel, which tiling), TMA descriptor encoding and launch.
+// Nothing here allocates device memory; nothing is launched when validation
+// fails.
+#include <cudaTypedefs.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+using namespace arc;
+
+namespace arc {
+int decode_smem_bytes(int kv_type, int D);
+}
+
+namespace {
+
+constexpr int kTcBM = 128, kTcBN = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool in_set(int x, std::initializer_list<int> s) { return std::find(s.begin(), s.end(), x) != s.end(); }
+
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+void set_name(arc_plan_info *pi, const char *name)
+{
+    memset(pi, 0, sizeof(*pi));
+    snprintf(pi->kernel, sizeof(pi->kernel), "%s", name);
+}
+
+bool log_enabled()
+{
+    const char *e = getenv("ARC_LOG");
+    return e && e[0] == '1';
+}
+
+// First dispatch per kernel name is logged when ARC_LOG=1 (host-side logging
+// only; it never influences what a call computes).
+void note_dispatch(const char *kernel)
+{
+    if (!log_enabled()) return;
+    static std::mutex mu;
+    static std::vector<std::string> seen;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto &s : seen)
+        if (s == kernel) return;
+    seen.emplace_back(kernel);
+    fprintf(stderr, "arc_attn: first dispatch on %s\n", kernel);
+}
+
+// ------------------------------------------------------------------ TMA maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void *f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, box {64, rows, 1...}; dims/strides innermost first,
+// strides in elements for dims 1..rank-1.
+bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const int64_t *strides_el,
+              uint32_t box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[5], gstr[4];
+    cuuint32_t box[5], estr[5];
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        estr[i] = 1;
+        box[i] = i == 0 ? 64 : (i == 1 ? box_rows : 1);
+    }
+    for (int i = 0; i < rank - 1; ++i) gstr[i] = (cuuint64_t)strides_el[i] * 2;
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gdim, gstr, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool tma_strides_ok(std::initializer_list<int64_t> strides_el)
+{
+    for (int64_t s : strides_el)
+        if (s <= 0 || (s * 2) % 16 != 0 || s * 2 >= (int64_t(1) << 40)) return false;
+    return true;
+}
+
+// Tile order: heavier tiles (more KV tiles under the causal mask) first.
+void order_tiles(TcParams &p, int n_tiles)
+{
+    if (n_tiles > 1024) {
+        for (int i = 0; i < 1024; ++i) p.tile_order[i] = (uint16_t)i;
+        return;
+    }
+    std::vector<std::pair<int, int>> w(n_tiles);
+    const int rows = p.G * p.Tq;
+    for (int t = 0; t < n_tiles; ++t) {
+        const int r0 = t * kTcBM, r_last = std::min(r0 + kTcBM, rows) - 1;
+        const int t_max = (r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
+        const int last = p.causal ? std::min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
+        w[t] = {last < 0 ? 0 : last / kTcBN + 1, t};
+    }
+    std::stable_sort(w.begin(), w.end(), [](auto &a, auto &b) { return a.first > b.first; });
+    for (int i = 0; i < n_tiles; ++i) p.tile_order[i] = (uint16_t)w[i].second;
+    for (int i = n_tiles; i < 1024; ++i) p.tile_order[i] = (uint16_t)i;
+}
+
+// ------------------------------------------------------------------ dense
+
+bool tc_pair_supported(int dqk, int dvs, bool mla)
+{
+    static const int dense[][2] = {{64, 64}, {128, 64}, {128, 128}, {192, 128}, {256, 128},
+                                   {256, 256}, {512, 256}, {512, 128}};
+    static const int mlas[][2] = {{128, 128}, {192, 128}, {192, 64}, {256, 128}, {256, 256}};
+    if (mla) {
+        for (auto &x : mlas)
+            if (x[0] == dqk && x[1] == dvs) return true;
+    } else {
+        for (auto &x : dense)
+            if (x[0] == dqk && x[1] == dvs) return true;
+    }
+    return false;
+}
+
+arc_status check_attn(const arc_attn_args *a)
+{
+    if (!a) return ARC_ERR_INVALID_ARG;
+    if (a->dtype != ARC_DTYPE_BF16 && a->dtype != ARC_DTYPE_F32) return ARC_ERR_INVALID_ARG;
+    if (a->B < 0 || a->H <= 0 || a->Hkv <= 0 || a->H % a->Hkv || a->Tq < 0 || a->Tk < 0) return ARC_ERR_INVALID_ARG;
+    if (a->D <= 0 || a->Dv <= 0 || a->D > 512 || a->Dv > 512) return ARC_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    if (!a->q || !a->o || !a->lse || (a->Tk > 0 && (!a->k || !a->v))) return ARC_ERR_INVALID_ARG;
+    if (!(a->scale == a->scale)) return ARC_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (a->q_strides[i] < 0 || a->k_strides[i] < 0 || a->v_strides[i] < 0 || a->o_strides[i] < 0)
+            return ARC_ERR_INVALID_ARG;
+    return ARC_OK;
+}
+
+enum class Path { None, Simple, Tc };
+
+struct AttnPlan {
+    Path path = Path::None;
+    int dvs = 0, n_slices = 0, n_tiles = 0, grid = 0, stages = 0;
+};
+
+AttnPlan plan_attn(const arc_attn_args *a)
+{
+    AttnPlan pl;
+    if (a->B == 0 || a->Tq == 0) return pl;
+    const bool force_simple = (a->flags & ARC_FLAG_FORCE_SIMPLE) != 0;
+    if (a->dtype == ARC_DTYPE_F32 || force_simple || a->Tk == 0) {
+        if (a->D <= 512 && a->Dv <= 512) pl.path = Path::Simple;
+        return pl;
+    }
+    pl.dvs = a->Dv > 256 ? 256 : a->Dv;
+    pl.n_slices = (a->Dv + pl.dvs - 1) / pl.dvs;
+    if (a->Dv % pl.dvs || !tc_pair_supported(a->D, pl.dvs, false)) return pl;
+    // the fold view needs the g*Tq rows of a kv group evenly spaced
+    if (a->q_strides[1] != (int64_t)a->Tq * a->q_strides[2] && a->H > 1) return pl;
+    if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o)) return pl;
+    if (!tma_strides_ok({a->q_strides[2], a->q_strides[0] ? a->q_strides[0] : 8, a->k_strides[2],
+                         a->k_strides[1] ? a->k_strides[1] : 8, a->k_strides[0] ? a->k_strides[0] : 8,
+                         a->v_strides[2], a->v_strides[1] ? a->v_strides[1] : 8,
+                         a->v_strides[0] ? a->v_strides[0] : 8}))
+        return pl;
+    for (int i = 0; i < 3; ++i)
+        if ((a->o_strides[i] * 2) % 16) return pl;
+    pl.path = Path::Tc;
+    pl.n_tiles = (a->H / a->Hkv * a->Tq + kTcBM - 1) / kTcBM;
+    pl.grid = pl.n_tiles * a->B * a->Hkv * pl.n_slices;
+    pl.stages = tc_max_stages(a->D);
+    return pl;
+}
+
+SimpleParams simple_from_attn(const arc_attn_args *a)
+{
+    SimpleParams p{};
+    p.mode = 0;
+    p.dtype = a->dtype;
+    p.B = a->B, p.H = a->H, p.Hkv = a->Hkv, p.Tq = a->Tq, p.Tk = a->Tk, p.Dqk = a->D, p.Dv = a->Dv, p.Dn = a->D;
+    p.q = a->q, p.k = a->k, p.v = a->v, p.o = a->o;
+    for (int i = 0; i < 3; ++i) p.qs[i] = a->q_strides[i], p.ks[i] = a->k_strides[i], p.vs[i] = a->v_strides[i],
+                                p.os[i] = a->o_strides[i];
+    p.lse = a->lse, p.sinks = a->sinks, p.scale = a->scale, p.causal = a->causal, p.status = a->status;
+    return p;
+}
+
+// ------------------------------------------------------------------ MLA
+
+arc_status check_mla(const arc_mla_args *a)
+{
+    if (!a) return ARC_ERR_INVALID_ARG;
+    if (a->B < 0 || a->H <= 0 || a->Tq < 0 || a->Tk < 0 || a->Dn <= 0 || a->Dr < 0 || a->Dv <= 0)
+        return ARC_ERR_INVALID_ARG;
+    if (a->Dn + a->Dr > 512 || a->Dv > 512) return ARC_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    if (!a->q_nope || (a->Dr > 0 && !a->q_rope) || !a->o || !a->lse) return ARC_ERR_INVALID_ARG;
+    if (a->Tk > 0 && (!a->k_nope || (a->Dr > 0 && !a->k_rope) || !a->v)) return ARC_ERR_INVALID_ARG;
+    return ARC_OK;
+}
+
+AttnPlan plan_mla(const arc_mla_args *a)
+{
+    AttnPlan pl;
+    if (a->B == 0 || a->Tq == 0) return pl;
+    if ((a->flags & ARC_FLAG_FORCE_SIMPLE) || a->Tk == 0) {
+        pl.path = Path::Simple;
+        return pl;
+    }
+    const int dqk = a->Dn + a->Dr;
+    if (a->Dn % 64 || a->Dr % 64 || a->Dr == 0 || a->Dv > 256 || !tc_pair_supported(dqk, a->Dv, true)) return pl;
+    if (a->q_nope_strides[1] != (int64_t)a->Tq * a->q_nope_strides[2] && a->H > 1) return pl;
+    if (a->q_rope_strides[1] != (int64_t)a->Tq * a->q_rope_strides[2] && a->H > 1) return pl;
+    if (!aligned16(a->q_nope) || !aligned16(a->q_rope) || !aligned16(a->k_nope) || !aligned16(a->k_rope) ||
+        !aligned16(a->v) || !aligned16(a->o))
+        return pl;
+    auto nz = [](int64_t s) { return s ? s : (int64_t)8; };
+    if (!tma_strides_ok({a->q_nope_strides[2], nz(a->q_nope_strides[0]), a->q_rope_strides[2],
+                         nz(a->q_rope_strides[0]), a->k_nope_strides[2], nz(a->k_nope_strides[1]),
+                         nz(a->k_nope_strides[0]), a->k_rope_strides[1], nz(a->k_rope_strides[0]),
+                         a->v_strides[2], nz(a->v_strides[1]), nz(a->v_strides[0])}))
+        return pl;
+    for (int i = 0; i < 3; ++i)
+        if ((a->o_strides[i] * 2) % 16) return pl;
+    pl.path = Path::Tc;
+    pl.dvs = a->Dv;
+    pl.n_slices = 1;
+    pl.n_tiles = (a->Tq + kTcBM - 1) / kTcBM;
+    pl.grid = pl.n_tiles * a->B * a->H;
+    pl.stages = tc_max_stages(dqk);
+    return pl;
+}
+
+// ------------------------------------------------------------------ sparse
+
+arc_status check_sparse(const arc_sparse_args *a)
+{
+    if (!a) return ARC_ERR_INVALID_ARG;
+    if (a->Sq < 0 || a->H <= 0 || a->Skv < 0 || a->topk < 0 || a->Dqk <= 0 || a->Dv <= 0) return ARC_ERR_INVALID_ARG;
+    if (a->Dqk > 512 || a->Dv > 512) return ARC_ERR_UNSUPPORTED;
+    if (!a->v && a->Dv > a->Dqk) return ARC_ERR_INVALID_ARG;
+    if (a->Sq == 0) return ARC_OK;
+    if (!a->q || !a->o || !a->lse || (a->topk > 0 && (!a->idx || !a->kv))) return ARC_ERR_INVALID_ARG;
+    return ARC_OK;
+}
+
+// ------------------------------------------------------------------ decode
+
+struct DecodePlan {
+    bool simple = false;
+    int splits = 0, chunk = 0, max_kv = 0;
+    size_t ws = 0;
+};
+
+arc_status check_decode(const arc_decode_args *a, bool need_ptrs = true)
+{
+    if (!a) return ARC_ERR_INVALID_ARG;
+    if (a->kv_type != ARC_KV_Q8_0 && a->kv_type != ARC_KV_Q4_0) return ARC_ERR_INVALID_ARG;
+    if (a->n_tok < 0 || a->H <= 0 || a->Hkv <= 0 || a->H % a->Hkv || a->n_cells < 0 || a->n_seq < 0)
+        return ARC_ERR_INVALID_ARG;
+    if (a->n_seq > ARC_DECODE_MAX_SEQ) return ARC_ERR_UNSUPPORTED;
+    if (!in_set(a->D, {64, 128})) return ARC_ERR_UNSUPPORTED;
+    if (a->n_seq > 0 && !a->seqs) return ARC_ERR_INVALID_ARG;
+    const int G = a->H / a->Hkv;
+    for (int s = 0; s < a->n_seq; ++s) {
+        const arc_seq &q = a->seqs[s];
+        if (q.n_q < 0 || q.n_kv < q.n_q || q.q_begin < 0 || q.kv_begin < 0) return ARC_ERR_INVALID_ARG;
+        if ((int64_t)q.q_begin + q.n_q > a->n_tok || (int64_t)q.kv_begin + q.n_kv > a->n_cells)
+            return ARC_ERR_INVALID_ARG;
+        if (G * q.n_q > 16) return ARC_ERR_UNSUPPORTED;
+    }
+    if (need_ptrs && a->n_seq > 0 && a->n_tok > 0) {
+        if (!a->q || !a->o || !a->lse || !a->k_cache || !a->v_cache) return ARC_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(a->k_cache) | reinterpret_cast<uintptr_t>(a->v_cache)) & 7u)
+            return ARC_ERR_INVALID_ARG;
+        if ((reinterpret_cast<uintptr_t>(a->q) | reinterpret_cast<uintptr_t>(a->o)) & 7u) return ARC_ERR_INVALID_ARG;
+    }
+    return ARC_OK;
+}
+
+DecodePlan plan_decode(const arc_decode_args *a)
+{
+    DecodePlan pl;
+    pl.simple = (a->flags & ARC_FLAG_FORCE_SIMPLE) != 0;
+    for (int s = 0; s < a->n_seq; ++s) pl.max_kv = std::max(pl.max_kv, a->seqs[s].n_kv);
+    if (pl.simple || pl.max_kv == 0) return pl;
+    const int pairs = a->n_seq * a->Hkv;
+    const int smem = decode_smem_bytes(a->kv_type, a->D);
+    const int per_sm = std::max(1, std::min(4, (228 * 1024) / (smem + 1024)));
+    const int target = sm_count() * per_sm;
+    int splits = std::max(1, target / std::max(1, pairs));
+    int chunk = (pl.max_kv + splits - 1) / splits;
+    chunk = ((chunk + 127) / 128) * 128;
+    splits = (pl.max_kv + chunk - 1) / chunk;
+    pl.splits = splits;
+    pl.chunk = chunk;
+    pl.ws = (size_t)pairs * splits * 16 * (a->D + 2) * sizeof(float);
+    return pl;
+}
+
+}  // namespace
+
+// ====================================================================== ABI
+
+extern "C" {
+
+int32_t arc_abi_version(void) { return ARC_ABI_VERSION; }
+
+const char *arc_status_string(arc_status s)
+{
+    switch (s) {
+    case ARC_OK: return "ok";
+    case ARC_ERR_INVALID_ARG: return "invalid argument";
+    case ARC_ERR_UNSUPPORTED: return "unsupported shape or layout";
+    case ARC_ERR_CUDA: return "CUDA error";
+    case ARC_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case ARC_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+arc_status arc_attn_fwd(const arc_attn_args *a, void *stream)
+{
+    arc_status st = check_attn(a);
+    if (st != ARC_OK) return st;
+    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    AttnPlan pl = plan_attn(a);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pl.path == Path::None) return ARC_ERR_UNSUPPORTED;
+    cudaError_t e;
+    if (pl.path == Path::Simple) {
+        note_dispatch("simple_attn_kernel");
+        e = launch_simple_attn(simple_from_attn(a), s);
+    } else {
+        TcParams p;
+        memset(&p, 0, sizeof(p));
+        const uint64_t qd[3] = {(uint64_t)a->D, (uint64_t)a->H * a->Tq, (uint64_t)a->B};
+        const int64_t qs[2] = {a->q_strides[2], a->q_strides[0] ? a->q_strides[0] : (int64_t)a->H * a->Tq * a->q_strides[2]};
+        const uint64_t kd[4] = {(uint64_t)a->D, (uint64_t)a->Tk, (uint64_t)a->Hkv, (uint64_t)a->B};
+        const int64_t ks[3] = {a->k_strides[2], a->k_strides[1] ? a->k_strides[1] : (int64_t)a->Tk * a->k_strides[2],
+                               a->k_strides[0] ? a->k_strides[0] : (int64_t)a->Hkv * a->Tk * a->k_strides[2]};
+        const uint64_t vd[4] = {(uint64_t)a->Dv, (uint64_t)a->Tk, (uint64_t)a->Hkv, (uint64_t)a->B};
+        const int64_t vs[3] = {a->v_strides[2], a->v_strides[1] ? a->v_strides[1] : (int64_t)a->Tk * a->v_strides[2],
+                               a->v_strides[0] ? a->v_strides[0] : (int64_t)a->Hkv * a->Tk * a->v_strides[2]};
+        if (!make_map(&p.tm_q, a->q, 3, qd, qs, kTcBM) || !make_map(&p.tm_k, a->k, 4, kd, ks, kTcBN) ||
+            !make_map(&p.tm_v, a->v, 4, vd, vs, kTcBN))
+            return ARC_ERR_CUDA;
+        p.tm_q2 = p.tm_q;
+        p.tm_k2 = p.tm_k;
+        p.B = a->B, p.H = a->H, p.Hkv = a->Hkv, p.G = a->H / a->Hkv, p.Tq = a->Tq, p.Tk = a->Tk, p.Dv = a->Dv;
+        p.n_tiles = pl.n_tiles, p.n_slices = pl.n_slices, p.kc_first = a->D / 64, p.stages = pl.stages;
+        p.o = a->o;
+        for (int i = 0; i < 3; ++i) p.os[i] = a->o_strides[i];
+        p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = a->scale * kLog2e, p.causal = a->causal;
+        p.status = a->status;
+        order_tiles(p, pl.n_tiles);
+        note_dispatch("tc_attn_kernel");
+        e = launch_tc_attn(p, a->D, pl.dvs, false, pl.grid, s);
+    }
+    return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+arc_status arc_mla_fwd(const arc_mla_args *a, void *stream)
+{
+    arc_status st = check_mla(a);
+    if (st != ARC_OK) return st;
+    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    AttnPlan pl = plan_mla(a);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pl.path == Path::None) return ARC_ERR_UNSUPPORTED;
+    cudaError_t e;
+    if (pl.path == Path::Simple) {
+        SimpleParams p{};
+        p.mode = 1;
+        p.dtype = ARC_DTYPE_BF16;
+        p.B = a->B, p.H = a->H, p.Hkv = a->H, p.Tq = a->Tq, p.Tk = a->Tk, p.Dqk = a->Dn + a->Dr, p.Dv = a->Dv;
+        p.Dn = a->Dn;
+        p.q = a->q_nope, p.q2 = a->q_rope, p.k = a->k_nope, p.k2 = a->k_rope, p.v = a->v, p.o = a->o;
+        for (int i = 0; i < 3; ++i) {
+            p.qs[i] = a->q_nope_strides[i], p.q2s[i] = a->q_rope_strides[i], p.ks[i] = a->k_nope_strides[i];
+            p.vs[i] = a->v_strides[i], p.os[i] = a->o_strides[i];
+        }
+        p.k2s[0] = a->k_rope_strides[0], p.k2s[1] = a->k_rope_strides[1];
+        p.lse = a->lse, p.scale = a->scale, p.causal = a->causal, p.status = a->status;
+        note_dispatch("simple_attn_kernel");
+        e = launch_simple_attn(p, s);
+    } else {
+        TcParams p;
+        memset(&p, 0, sizeof(p));
+        auto nz = [](int64_t s_, int64_t dflt) { return s_ ? s_ : dflt; };
+        const uint64_t qnd[3] = {(uint64_t)a->Dn, (uint64_t)a->H * a->Tq, (uint64_t)a->B};
+        const int64_t qns[2] = {a->q_nope_strides[2], nz(a->q_nope_strides[0], (int64_t)a->H * a->Tq * a->q_nope_strides[2])};
+        const uint64_t qrd[3] = {(uint64_t)a->Dr, (uint64_t)a->H * a->Tq, (uint64_t)a->B};
+        const int64_t qrs[2] = {a->q_rope_strides[2], nz(a->q_rope_strides[0], (int64_t)a->H * a->Tq * a->q_rope_strides[2])};
+        const uint64_t knd[4] = {(uint64_t)a->Dn, (uint64_t)a->Tk, (uint64_t)a->H, (uint64_t)a->B};
+        const int64_t kns[3] = {a->k_nope_strides[2], nz(a->k_nope_strides[1], (int64_t)a->Tk * a->k_nope_strides[2]),
+                                nz(a->k_nope_strides[0], (int64_t)a->H * a->Tk * a->k_nope_strides[2])};
+        const uint64_t krd[3] = {(uint64_t)a->Dr, (uint64_t)a->Tk, (uint64_t)a->B};
+        const int64_t krs[2] = {a->k_rope_strides[1], nz(a->k_rope_strides[0], (int64_t)a->Tk * a->k_rope_strides[1])};
+        const uint64_t vd[4] = {(uint64_t)a->Dv, (uint64_t)a->Tk, (uint64_t)a->H, (uint64_t)a->B};
+        const int64_t vs[3] = {a->v_strides[2], nz(a->v_strides[1], (int64_t)a->Tk * a->v_strides[2]),
+                               nz(a->v_strides[0], (int64_t)a->H * a->Tk * a->v_strides[2])};
+        if (!make_map(&p.tm_q, a->q_nope, 3, qnd, qns, kTcBM) || !make_map(&p.tm_q2, a->q_rope, 3, qrd, qrs, kTcBM) ||
+            !make_map(&p.tm_k, a->k_nope, 4, knd, kns, kTcBN) || !make_map(&p.tm_k2, a->k_rope, 3, krd, krs, kTcBN) ||
+            !make_map(&p.tm_v, a->v, 4, vd, vs, kTcBN))
+            return ARC_ERR_CUDA;
+        p.B = a->B, p.H = a->H, p.Hkv = a->H, p.G = 1, p.Tq = a->Tq, p.Tk = a->Tk, p.Dv = a->Dv;
+        p.n_tiles = pl.n_tiles, p.n_slices = 1, p.kc_first = a->Dn / 64, p.stages = pl.stages;
+        p.o = a->o;
+        for (int i = 0; i < 3; ++i) p.os[i] = a->o_strides[i];
+        p.lse = a->lse, p.sinks = nullptr, p.scale_log2 = a->scale * kLog2e, p.causal = a->causal;
+        p.status = a->status;
+        order_tiles(p, pl.n_tiles);
+        note_dispatch("tc_attn_kernel<mla>");
+        e = launch_tc_attn(p, a->Dn + a->Dr, a->Dv, true, pl.grid, s);
+    }
+    return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+arc_status arc_sparse_mla_fwd(const arc_sparse_args *a, void *stream)
+{
+    arc_status st = check_sparse(a);
+    if (st != ARC_OK) return st;
+    if (a->Sq == 0) return ARC_OK;
+    SimpleParams p{};
+    p.mode = 2;
+    p.dtype = ARC_DTYPE_BF16;
+    p.B = 1, p.H = a->H, p.Hkv = 1, p.Tq = a->Sq, p.Tk = a->topk, p.Dqk = a->Dqk, p.Dv = a->Dv, p.Dn = a->Dqk;
+    p.q = a->q, p.k = a->kv, p.v = a->v, p.o = a->o;
+    p.qs[0] = a->q_strides[0], p.qs[1] = a->q_strides[1];
+    p.ks[0] = a->kv_stride, p.vs[0] = a->v_stride;
+    p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
+    p.lse = a->lse, p.sinks = a->sinks, p.scale = a->scale, p.causal = 0;
+    p.idx = a->idx, p.idx_stride = a->idx_stride, p.topk = a->topk, p.Skv = a->Skv, p.status = a->status;
+    note_dispatch("simple_attn_kernel<sparse>");
+    cudaError_t e = launch_simple_attn(p, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+size_t arc_decode_workspace_size(const arc_decode_args *a)
+{
+    if (check_decode(a, false) != ARC_OK) return 0;
+    return plan_decode(a).ws;
+}
+
+arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t ws_bytes, void *stream)
+{
+    arc_status st = check_decode(a);
+    if (st != ARC_OK) return st;
+    if (a->n_seq == 0 || a->n_tok == 0) return ARC_OK;
+    DecodePlan pl = plan_decode(a);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (pl.simple || pl.max_kv == 0) {
+        SimpleDecodeParams p{};
+        p.kv_type = a->kv_type, p.n_tok = a->n_tok, p.H = a->H, p.Hkv = a->Hkv, p.D = a->D;
+        p.n_cells = a->n_cells, p.n_seq = a->n_seq;
+        p.q = a->q, p.k_cache = static_cast<const uint8_t *>(a->k_cache);
+        p.v_cache = static_cast<const uint8_t *>(a->v_cache);
+        memcpy(p.seqs, a->seqs, sizeof(arc_seq) * a->n_seq);
+        p.o = a->o, p.lse = a->lse, p.scale = a->scale;
+        note_dispatch("simple_decode_kernel");
+        e = launch_simple_decode(p, s);
+    } else {
+        if (!workspace || ws_bytes < pl.ws || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return ARC_ERR_WORKSPACE;
+        DecodeParams p{};
+        p.kv_type = a->kv_type, p.n_tok = a->n_tok, p.H = a->H, p.Hkv = a->Hkv, p.D = a->D, p.n_seq = a->n_seq;
+        p.splits = pl.splits, p.chunk = pl.chunk;
+        p.q = a->q, p.k_cache = static_cast<const uint8_t *>(a->k_cache);
+        p.v_cache = static_cast<const uint8_t *>(a->v_cache);
+        memcpy(p.seqs, a->seqs, sizeof(arc_seq) * a->n_seq);
+        p.o = a->o, p.lse = a->lse;
+        const size_t parts = (size_t)a->n_seq * a->Hkv * pl.splits;
+        p.ws_o = static_cast<float *>(workspace);
+        p.ws_ml = p.ws_o + parts * 16 * a->D;
+        p.scale_log2 = a->scale * kLog2e;
+        p.status = a->status;
+        note_dispatch(a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
+        e = launch_decode(p, s);
+    }
+    return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
+{
+    if (!args || !out) return ARC_ERR_INVALID_ARG;
+    if (op == ARC_OP_ATTN) {
+        const arc_attn_args *a = static_cast<const arc_attn_args *>(args);
+        arc_status st = check_attn(a);
+        if (st != ARC_OK) return st;
+        AttnPlan pl = plan_attn(a);
+        if (a->B == 0 || a->Tq == 0) {
+            set_name(out, "none");
+            return ARC_OK;
+        }
+        if (pl.path == Path::None) return ARC_ERR_UNSUPPORTED;
+        if (pl.path == Path::Simple) {
+            set_name(out, "simple_attn_kernel");
+            out->tile_m = 4;
+            out->n_ctas = (int)(((int64_t)a->B * a->H * a->Tq + 3) / 4);
+        } else {
+            set_name(out, "tc_attn_kernel");
+            out->tensor_cores = 1;
+            out->tile_m = kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
+            out->smem_bytes = tc_smem_bytes(a->D, pl.stages), out->tmem_cols = 512;
+        }
+        out->launches = 1;
+        return ARC_OK;
+    }
+    if (op == ARC_OP_MLA) {
+        const arc_mla_args *a = static_cast<const arc_mla_args *>(args);
+        arc_status st = check_mla(a);
+        if (st != ARC_OK) return st;
+        AttnPlan pl = plan_mla(a);
+        if (a->B == 0 || a->Tq == 0) {
+            set_name(out, "none");
+            return ARC_OK;
+        }
+        if (pl.path == Path::None) return ARC_ERR_UNSUPPORTED;
+        if (pl.path == Path::Simple) {
+            set_name(out, "simple_attn_kernel");
+            out->tile_m = 4;
+        } else {
+            set_name(out, "tc_attn_kernel<mla>");
+            out->tensor_cores = 1;
+            out->tile_m = kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
+            out->smem_bytes = tc_smem_bytes(a->Dn + a->Dr, pl.stages), out->tmem_cols = 512;
+        }
+        out->launches = 1;
+        return ARC_OK;
+    }
+    if (op == ARC_OP_SPARSE) {
+        const arc_sparse_args *a = static_cast<const arc_sparse_args *>(args);
+        arc_status st = check_sparse(a);
+        if (st != ARC_OK) return st;
+        set_name(out, "simple_attn_kernel<sparse>");
+        out->tile_m = 4;
+        out->launches = 1;
+        return ARC_OK;
+    }
+    if (op == ARC_OP_DECODE) {
+        const arc_decode_args *a = static_cast<const arc_decode_args *>(args);
+        arc_status st = check_decode(a);
+        if (st != ARC_OK) return st;
+        DecodePlan pl = plan_decode(a);
+        if (pl.simple || pl.max_kv == 0) {
+            set_name(out, "simple_decode_kernel");
+            out->launches = 1;
+        } else {
+            set_name(out, a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
+            out->tensor_cores = 1;
+            out->tile_m = 16, out->tile_n = 32, out->d_slice = a->D;
+            out->splits = pl.splits, out->n_ctas = a->n_seq * a->Hkv * pl.splits;
+            out->smem_bytes = decode_smem_bytes(a->kv_type, a->D);
+            out->launches = 2;
+        }
+        return ARC_OK;
+    }
+    return ARC_ERR_INVALID_ARG;
+}
+
+arc_status arc_check_device_error(const uint32_t *status, void *stream)
+{
+    if (!status) return ARC_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ARC_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return ARC_ERR_CUDA;
+    return v ? ARC_ERR_DEVICE_TIMEOUT : ARC_OK;
+}
+
+arc_status arc_selftest_timeout(uint32_t *status, uint64_t timeout_ns, void *stream)
+{
+    if (!status) return ARC_ERR_INVALID_ARG;
+    return launch_selftest_timeout(status, timeout_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? ARC_OK
+               : ARC_ERR_CUDA;
+}
+
+}  // extern "C"

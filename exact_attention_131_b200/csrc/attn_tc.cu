@@ -1,0 +1,432 @@
+// attn_tc.cu -- fused attention forward on tcgen05 tensor cores (sm_100a):
+// dense / GQA-folded / MLA, bf16 in, fp32 accumulate, O and LSE out.
+//
+// One CTA owns a tile of 128 query rows of one (batch, kv head) group and one
+// slice of d_v columns.  The GQA fold is pure index math: the g*Tq query rows
+// that share kv head `kv` are the contiguous rows kv*g*Tq .. of q viewed as
+// [B, H*Tq, D] ("ArcFlash ... rung 0", Fold section), so a tile may straddle
+// two query heads and every row computes its own position t = r mod Tq for the
+// causal mask.  Query rows are independent softmaxes, so tiles never exchange
+// anything (same page, Tile section).
+//
+// Warp roles (256 threads):
+//   warp 0      TMA producer: Q once, then K and V tiles in 64-column chunks
+//               through a ring of shared-memory stages
+//   warp 1      TMEM owner and MMA issuer (one elected lane):
+//                 S[buf] = Q K^T      (M=128, N=128, K-major A and B)
+//                 O     += P V        (M=128, N=d_v slice, V read MN-major)
+//   warps 4-7   softmax: one thread per query row; read S from TMEM, mask,
+//               online max / sum in log2 units, rescale O in TMEM when the
+//               running max grows by more than 2^8, write P (bf16) to shared
+//               memory in the 128-byte-swizzled K-major layout, epilogue.
+// TMEM (512 columns): O slice at columns [0, DVS), S double buffer at 256, 384.
+// Every wait is bounded; a wait that runs out reports through p.status.
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace arc {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int CHUNK = BM * 128;     // bytes of one [128 rows x 64 bf16] swizzled chunk
+constexpr int NTHREADS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int S_COL = 256;
+constexpr int MAX_STAGES = 12;
+constexpr int SMEM_LIMIT = 232448;  // 227 KB opt-in maximum per block
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+struct Bars {
+    uint64_t q_full;
+    uint64_t s_full[2];
+    uint64_t s_free[2];
+    uint64_t p_full;
+    uint64_t o_done;
+    uint64_t drain;
+    uint64_t full[MAX_STAGES];
+    uint64_t empty[MAX_STAGES];
+    uint32_t tmem_base;
+};
+
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+template <int DQK, int DVS, bool MLA>
+__global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_constant__ TcParams p)
+{
+    constexpr int KC = DQK / 64;  // 64-column chunks of a Q / K row
+    constexpr int VC = DVS / 64;  // 64-column chunks of this CTA's V slice
+    static_assert(DQK % 64 == 0 && DVS % 64 == 0 && DVS <= 256, "tile shape");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;
+    uint8_t *sRing = sQ + KC * CHUNK;
+    const int R = p.stages;
+    uint8_t *sP = sRing + R * CHUNK;
+    Bars *bars = reinterpret_cast<Bars *>(sP + 2 * CHUNK);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- which tile this CTA owns
+    const int groups = p.B * p.Hkv * p.n_slices;
+    const int rank = blockIdx.x / groups;
+    const int rest = blockIdx.x % groups;
+    const int slice = rest % p.n_slices;
+    const int kv = (rest / p.n_slices) % p.Hkv;
+    const int b = rest / (p.n_slices * p.Hkv);
+    const int tile = rank < 1024 ? (int)p.tile_order[rank] : rank;
+    const int rows_in_group = p.G * p.Tq;
+    const int r0 = tile * BM;
+    const int dv0 = slice * DVS;
+    int nt;
+    {
+        const int r_last = min(r0 + BM, rows_in_group) - 1;
+        const int t_max = (r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
+        const int kv_last = p.causal ? min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
+        nt = kv_last < 0 ? 0 : kv_last / BN + 1;
+    }
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->s_free[i], 128);
+        }
+        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->o_done, 1);
+        mbar_init(&bars->drain, 1);
+        for (int i = 0; i < R; ++i) {
+            mbar_init(&bars->full[i], 1);
+            mbar_init(&bars->empty[i], 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // =============================== TMA producer
+        if (lane == 0 && nt > 0) {
+            tma_prefetch_desc(&p.tm_q);
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            const int qrow = kv * rows_in_group + r0;  // row in the [H*Tq] view
+            mbar_arrive_expect_tx(&bars->q_full, KC * CHUNK);
+            for (int c = 0; c < KC; ++c) {
+                if (!MLA || c < p.kc_first)
+                    tma_load_3d(sQ + c * CHUNK, &p.tm_q, &bars->q_full, c * 64, qrow, b);
+                else
+                    tma_load_3d(sQ + c * CHUNK, &p.tm_q2, &bars->q_full, (c - p.kc_first) * 64, qrow, b);
+            }
+            int stage = 0;
+            uint32_t ephase = 0;
+            int issued[MAX_STAGES];
+            for (int i = 0; i < MAX_STAGES; ++i) issued[i] = 0;
+            bool ok = true;
+            auto acquire = [&]() -> bool {
+                if (!mbar_wait(&bars->empty[stage], ephase ^ 1u)) return false;
+                mbar_arrive_expect_tx(&bars->full[stage], CHUNK);
+                issued[stage]++;
+                return true;
+            };
+            auto advance = [&]() {
+                if (++stage == R) {
+                    stage = 0;
+                    ephase ^= 1u;
+                }
+            };
+            auto load_k = [&](int j) -> bool {
+                for (int c = 0; c < KC; ++c) {
+                    if (!acquire()) return false;
+                    uint8_t *dst = sRing + stage * CHUNK;
+                    if (!MLA || c < p.kc_first)
+                        tma_load_4d(dst, &p.tm_k, &bars->full[stage], c * 64, j * BN, kv, b);
+                    else
+                        tma_load_3d(dst, &p.tm_k2, &bars->full[stage], (c - p.kc_first) * 64, j * BN, b);
+                    advance();
+                }
+                return true;
+            };
+            auto load_v = [&](int j) -> bool {
+                for (int c = 0; c < VC; ++c) {
+                    if (!acquire()) return false;
+                    tma_load_4d(sRing + stage * CHUNK, &p.tm_v, &bars->full[stage], dv0 + c * 64, j * BN, kv, b);
+                    advance();
+                }
+                return true;
+            };
+            ok = load_k(0);
+            for (int j = 0; ok && j < nt; ++j) {
+                if (j + 1 < nt) ok = load_k(j + 1);
+                if (ok) ok = load_v(j);
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_LOAD);
+            // Drain: every copy this thread issued has landed before the CTA exits.
+            for (int s = 0; s < R; ++s)
+                if (issued[s] > 0) mbar_wait(&bars->full[s], (uint32_t)((issued[s] - 1) & 1));
+            mbar_wait(&bars->q_full, 0);
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer
+        if (lane == 0 && nt > 0) {
+            const uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
+            const uint32_t q_base = smem_u32(sQ), ring_base = smem_u32(sRing), p_base = smem_u32(sP);
+            int stage = 0;
+            uint32_t fphase = 0;
+            bool ok = mbar_wait(&bars->q_full, 0);
+            tc_fence_after();
+            auto advance = [&]() {
+                if (++stage == R) {
+                    stage = 0;
+                    fphase ^= 1u;
+                }
+            };
+            auto issue_s = [&](int j) -> bool {
+                const int buf = j & 1;
+                if (j >= 2 && !mbar_wait(&bars->s_free[buf], (uint32_t)(((j - 2) >> 1) & 1))) return false;
+                tc_fence_after();
+                const uint32_t d = tmem + S_COL + buf * BN;
+                for (int c = 0; c < KC; ++c) {
+                    if (!mbar_wait(&bars->full[stage], fphase)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t a = sdesc_sw128(q_base + c * CHUNK + kk * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(ring_base + stage * CHUNK + kk * 32, 16, 1024);
+                        umma_bf16(d, a, bd, idesc_s, (c | kk) != 0);
+                    }
+                    umma_commit(&bars->empty[stage]);
+                    advance();
+                }
+                umma_commit(&bars->s_full[buf]);
+                return true;
+            };
+            auto issue_pv = [&](int j) -> bool {
+                if (!mbar_wait(&bars->p_full, (uint32_t)(j & 1))) return false;
+                int vst[VC];
+                for (int c = 0; c < VC; ++c) {
+                    if (!mbar_wait(&bars->full[stage], fphase)) return false;
+                    vst[c] = stage;
+                    advance();
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t a = sdesc_sw128(p_base + (kk >> 2) * CHUNK + (kk & 3) * 32, 16, 1024);
+                    int c = 0;
+                    while (c < VC) {
+                        int len = 1;
+                        while (c + len < VC && vst[c + len] == vst[c] + len) ++len;
+                        const uint64_t bd = sdesc_sw128(ring_base + vst[c] * CHUNK + kk * 2048, CHUNK, 1024);
+                        umma_bf16(tmem + c * 64, a, bd, idesc_bf16(BM, 64 * len, false, true), (j > 0 || kk > 0));
+                        c += len;
+                    }
+                }
+                for (int c = 0; c < VC; ++c) umma_commit(&bars->empty[vst[c]]);
+                umma_commit(&bars->o_done);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < nt; ++j) {
+                if (j + 1 < nt) ok = issue_s(j + 1);
+                if (ok) ok = issue_pv(j);
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_MMA);
+            // Drain: all MMAs issued by this thread complete before TMEM is freed.
+            umma_commit(&bars->drain);
+            mbar_wait(&bars->drain, 0);
+        }
+    } else if (warp >= 4) {
+        // =============================== softmax, correction, epilogue
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const int R_ = r0 + r;
+        const bool row_ok = R_ < rows_in_group;
+        const int t = R_ % p.Tq;
+        const int h = kv * p.G + R_ / p.Tq;
+        const int last = p.causal ? min(p.Tk - 1, t + p.Tk - p.Tq) : p.Tk - 1;
+        const float sl2 = p.scale_log2;
+        float m_use = -INFINITY, l = 0.f;
+        bool ok = true;
+        uint8_t *prow = sP + (r >> 3) * 1024 + (r & 7) * 128;
+
+        for (int j = 0; j < nt; ++j) {
+            const int buf = j & 1;
+            ok = warp_all(mbar_wait(&bars->s_full[buf], (uint32_t)((j >> 1) & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sv[BN];
+#pragma unroll
+            for (int i = 0; i < BN / 32; ++i)
+                tmem_ld32(tmem + lane_off + S_COL + buf * BN + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * i]));
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bars->s_free[buf]);
+
+            const int kbase = j * BN;
+            if (kbase + BN - 1 > last) {
+#pragma unroll
+                for (int i = 0; i < BN; ++i)
+                    if (kbase + i > last) sv[i] = __float_as_uint(-INFINITY);
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
+            mx *= sl2;
+            const bool need = mx > m_use + RESCALE_THRESHOLD;
+            float alpha = 1.f;
+            if (need) {
+                alpha = (m_use == -INFINITY) ? 0.f : fast_exp2(m_use - mx);
+                m_use = mx;
+            }
+            const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
+            float rowsum = 0.f;
+            uint32_t pk[BN / 2];
+#pragma unroll
+            for (int i = 0; i < BN / 2; ++i) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), sl2, -msafe));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -msafe));
+                rowsum += p0 + p1;
+                pk[i] = pack_bf16(p0, p1);
+            }
+            l = l * alpha + rowsum;
+
+            // PV(j-1) must be complete before O is rescaled or the P buffer reused.
+            if (j > 0) {
+                ok = warp_all(mbar_wait(&bars->o_done, (uint32_t)((j - 1) & 1)));
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                    for (int c = 0; c < DVS / 32; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(tmem + lane_off + 32 * c, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                        tmem_st32(tmem + lane_off + 32 * c, ov);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row -> shared memory, 128-byte swizzle: 16-byte unit u of row r sits at u ^ (r & 7).
+#pragma unroll
+            for (int cc = 0; cc < BN / 64; ++cc) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    uint4 val = make_uint4(pk[cc * 32 + u * 4 + 0], pk[cc * 32 + u * 4 + 1],
+                                           pk[cc * 32 + u * 4 + 2], pk[cc * 32 + u * 4 + 3]);
+                    *reinterpret_cast<uint4 *>(prow + cc * CHUNK + ((u ^ (r & 7)) << 4)) = val;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+        }
+        if (ok && nt > 0) {
+            ok = warp_all(mbar_wait(&bars->o_done, (uint32_t)((nt - 1) & 1)));
+            tc_fence_after();
+        }
+        if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
+
+        // ---- final normalisation; the sink joins the denominator only
+        float fac, lse;
+        if (p.sinks) {
+            const float sg = row_ok ? p.sinks[h] * LOG2E : 0.f;  // padding rows may lie past the last head
+            const float mf = fmaxf(m_use, sg);
+            const float a = (m_use == -INFINITY) ? 0.f : exp2f(m_use - mf);
+            const float lf = l * a + exp2f(sg - mf);
+            fac = a / lf;
+            lse = (mf + log2f(lf)) * LN2;
+        } else {
+            fac = l > 0.f ? 1.f / l : 0.f;
+            lse = l > 0.f ? (m_use + log2f(l)) * LN2 : -INFINITY;
+        }
+        __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] +
+                              (int64_t)t * p.os[2] + dv0;
+#pragma unroll 1
+        for (int c = 0; c < DVS / 32; ++c) {
+            uint32_t ov[32];
+            if (nt > 0 && ok) {
+                tmem_ld32(tmem + lane_off + 32 * c, ov);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ov[i] = 0u;
+            }
+            if (row_ok) {
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack_bf16(__uint_as_float(ov[2 * i]) * fac, __uint_as_float(ov[2 * i + 1]) * fac);
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+        if (row_ok && slice == 0) p.lse[((int64_t)b * p.H + h) * p.Tq + t] = lse;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+template <int DQK, int DVS, bool MLA>
+cudaError_t launch_one(const TcParams &p, int grid, cudaStream_t s)
+{
+    const int smem = tc_smem_bytes(DQK, p.stages);
+    auto kern = tc_attn_kernel<DQK, DVS, MLA>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NTHREADS, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+int tc_smem_bytes(int dqk, int stages) { return 1024 + (dqk / 64 + stages + 2) * CHUNK + (int)sizeof(Bars); }
+
+int tc_max_stages(int dqk)
+{
+    int st = (SMEM_LIMIT - 1024 - (int)sizeof(Bars) - (dqk / 64 + 2) * CHUNK) / CHUNK;
+    return st < MAX_STAGES ? st : MAX_STAGES;
+}
+
+cudaError_t launch_tc_attn(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s)
+{
+#define ARC_TC_CASE(Q, V, M) \
+    if (dqk == Q && dvs == V && mla == M) return launch_one<Q, V, M>(p, grid, s);
+    ARC_TC_CASE(64, 64, false)
+    ARC_TC_CASE(128, 64, false)
+    ARC_TC_CASE(128, 128, false)
+    ARC_TC_CASE(192, 128, false)
+    ARC_TC_CASE(256, 128, false)
+    ARC_TC_CASE(256, 256, false)
+    ARC_TC_CASE(512, 256, false)
+    ARC_TC_CASE(512, 128, false)
+    ARC_TC_CASE(128, 128, true)
+    ARC_TC_CASE(192, 128, true)
+    ARC_TC_CASE(192, 64, true)
+    ARC_TC_CASE(256, 128, true)
+    ARC_TC_CASE(256, 256, true)
+#undef ARC_TC_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace arc

@@ -1,0 +1,107 @@
+// internal.h -- launch interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/arc_attn.h"
+
+namespace arc {
+
+// ---------------------------------------------------------------- CUDA-core kernels
+// One warp per output row; lanes split the head dims; exact fp32 arithmetic.
+// Used for fp32 "reference mode" and as the control arm (ARC_FLAG_FORCE_SIMPLE).
+struct SimpleParams {
+    int mode;  // 0 dense, 1 MLA, 2 sparse
+    int dtype; // ARC_DTYPE_BF16 or ARC_DTYPE_F32
+    int B, H, Hkv, Tq, Tk, Dqk, Dv, Dn;
+    const void *q, *q2, *k, *k2, *v;
+    int64_t qs[3], q2s[3], ks[3], k2s[3], vs[3], os[3];
+    void *o;
+    float *lse;
+    const float *sinks;
+    float scale;
+    int causal;
+    const int32_t *idx;
+    int64_t idx_stride;
+    int topk, Skv;
+    uint32_t *status;
+};
+cudaError_t launch_simple_attn(const SimpleParams &p, cudaStream_t s);
+
+struct SimpleDecodeParams {
+    int kv_type, n_tok, H, Hkv, D, n_cells, n_seq;
+    const float *q;
+    const uint8_t *k_cache, *v_cache;
+    arc_seq seqs[ARC_DECODE_MAX_SEQ];
+    float *o, *lse;
+    float scale;
+};
+cudaError_t launch_simple_decode(const SimpleDecodeParams &p, cudaStream_t s);
+
+// ---------------------------------------------------------------- tcgen05 attention
+// Dense / GQA fold / MLA forward, M = 128 query rows per CTA, K/V tiles by TMA.
+struct TcParams {
+    CUtensorMap tm_q;   // q (dense) or q_nope (MLA): dims {D, H*Tq, B}
+    CUtensorMap tm_q2;  // q_rope: dims {Dr, H*Tq, B}
+    CUtensorMap tm_k;   // k (dense) or k_nope: dims {D, Tk, Hkv, B}
+    CUtensorMap tm_k2;  // k_rope: dims {Dr, Tk, B}
+    CUtensorMap tm_v;   // v: dims {Dv, Tk, Hkv, B}
+    int B, H, Hkv, G, Tq, Tk, Dv;
+    int n_tiles;        // query-row tiles per (b, kv) group
+    int n_slices;       // d_v slices
+    int kc_first;       // 64-column chunks of q/k taken from the first tensor (MLA: nope)
+    int stages;         // ring stages
+    void *o;
+    int64_t os[3];
+    float *lse;
+    const float *sinks;
+    float scale_log2;   // scale * log2(e)
+    int causal;
+    uint32_t *status;
+    uint16_t tile_order[1024];
+};
+int tc_smem_bytes(int dqk, int stages);
+int tc_max_stages(int dqk);
+cudaError_t launch_tc_attn(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s);
+
+// Sparse top-k forward, M = 64 heads of one query token per CTA, gathered rows.
+struct SparseTcParams {
+    int Sq, H, Skv, Dqk, Dv, topk;
+    const __nv_bfloat16 *q;
+    int64_t qs[2];
+    const __nv_bfloat16 *kv;
+    int64_t kv_stride;
+    const __nv_bfloat16 *v;
+    int64_t v_stride;
+    const int32_t *idx;
+    int64_t idx_stride;
+    __nv_bfloat16 *o;
+    int64_t os[2];
+    float *lse;
+    const float *sinks;
+    float scale_log2;
+    uint32_t *status;
+};
+int sparse_smem_bytes(int dqk, int bn);
+cudaError_t launch_sparse_tc(const SparseTcParams &p, cudaStream_t s);
+
+// ---------------------------------------------------------------- quantised decode
+struct DecodeParams {
+    int kv_type, n_tok, H, Hkv, D, n_seq, splits, chunk;
+    const float *q;
+    const uint8_t *k_cache, *v_cache;
+    arc_seq seqs[ARC_DECODE_MAX_SEQ];
+    float *o, *lse;
+    float *ws_o;     // [n_seq*Hkv*splits][16][D] partial outputs (unnormalised)
+    float *ws_ml;    // [n_seq*Hkv*splits][16][2] partial (max, sum)
+    float scale_log2;
+    uint32_t *status;
+};
+cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s);
+
+cudaError_t launch_selftest_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
+
+}  // namespace arc

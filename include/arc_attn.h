@@ -1,0 +1,273 @@
+/*
+ * arc_attn.h -- C ABI of a fused exact-attention forward library for B200 (sm_100a).
+ *
+ * Every call computes, for each output row, exact softmax attention
+ *
+ *     O   = softmax(scale * q K^T + mask [+ sink]) V        (a row of d_v values)
+ *     LSE = ln( sum_j exp(scale * q.k_j) [+ exp(sink)] )    (natural log, fp32)
+ *
+ * tiled over keys with an online softmax, so no score matrix is ever stored.
+ * The forward output plus a per-row log-sum-exp is the output pair of the FA4
+ * forward ("pith-train PR: FA4 b19 return arity", summary).  The arity of
+ * every call is fixed by its argument struct; nothing is returned as a tuple
+ * whose length could change between versions (the crash that page reports).
+ *
+ * Conventions shared by all calls
+ *   - Pointers marked "device" are CUDA device (or managed) memory owned by the
+ *     caller.  The library allocates no memory and keeps no mutable global
+ *     state; a call only reads its inputs and writes its outputs (and, for
+ *     decode, the caller's workspace).
+ *   - Strides are in ELEMENTS, int64.  The last dimension of every tensor is
+ *     contiguous (stride 1).
+ *   - `stream` is a cudaStream_t passed as void*.  NULL is the legacy default
+ *     stream and is a valid stream.  Launches are asynchronous on it.
+ *   - Arguments are validated on the host before anything is launched.  On
+ *     ARC_ERR_INVALID_ARG / ARC_ERR_UNSUPPORTED nothing is launched and no
+ *     output is written.  A failed launch returns ARC_ERR_CUDA.
+ *   - `status` (optional, device, one uint32 the caller zeroes): every wait
+ *     inside the kernels is bounded; a wait that runs out ORs a nonzero code
+ *     into *status and the kernel returns early.  arc_check_device_error()
+ *     reads it.  With status == NULL such an event is not reported.
+ *   - Causal masks are bottom-right aligned: query i of Tq sees keys
+ *     j <= i + (Tk - Tq).  A row with no visible key and no sink gets O = 0 and
+ *     LSE = -inf.
+ */
+#ifndef ARC_ATTN_H
+#define ARC_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ARC_ABI_VERSION 1
+
+typedef enum {
+    ARC_OK = 0,
+    ARC_ERR_INVALID_ARG = 1,   /* a shape, pointer, stride or alignment is wrong */
+    ARC_ERR_UNSUPPORTED = 2,   /* valid, but outside what the kernels implement */
+    ARC_ERR_CUDA = 3,          /* a CUDA launch or runtime call failed */
+    ARC_ERR_DEVICE_TIMEOUT = 4,/* a bounded device-side wait ran out (see status) */
+    ARC_ERR_WORKSPACE = 5      /* workspace missing or smaller than required */
+} arc_status;
+
+typedef enum { ARC_DTYPE_BF16 = 0, ARC_DTYPE_F32 = 1 } arc_dtype;
+
+/* Quantised KV block types; the values are the ggml type ids. */
+typedef enum { ARC_KV_Q4_0 = 2, ARC_KV_Q8_0 = 8 } arc_kv_type;
+
+typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE = 4 } arc_op;
+
+/* flags (all calls) */
+#define ARC_FLAG_FORCE_SIMPLE 1u   /* run the CUDA-core kernel instead of the tensor-core one */
+
+/* --------------------------------------------------------------------------
+ * arc_attn_fwd: dense attention with GQA / MQA and optional per-head sinks.
+ *
+ * Source: "ArcFlash - Arc's own attention kernel, rung 0", section "What rung 0
+ * does": query head h reads kv head h / g (g = H / Hkv; heads are kv-major, as
+ * repeat_kv lays them out), and the GQA expansion is a reshape of q[B,H,Tq,D]
+ * to [B,Hkv,g*Tq,D] with no copy of K or V; a sink is a per-head constant in
+ * each row's softmax denominator and never multiplies V.
+ *
+ *   q  [B,H,Tq,D]     dtype, device, strides q_strides = {batch, head, token}
+ *   k  [B,Hkv,Tk,D]   dtype, device
+ *   v  [B,Hkv,Tk,Dv]  dtype, device
+ *   o  [B,H,Tq,Dv]    dtype, device, written
+ *   lse [B,H,Tq]      fp32, device, contiguous, written
+ *   sinks [H]         fp32, device, or NULL for no sink; a raw logit (not scaled)
+ *
+ * dtype BF16: D in {64,128,192,256,512}, Dv in {64,128,256,512}; fp32
+ * accumulation; P is rounded to bf16 before P*V.  The tensor-core path needs
+ * each (b, kv) group of g*Tq query rows evenly spaced (head stride ==
+ * Tq * token stride), 16-byte aligned rows and base pointers; otherwise the
+ * call returns ARC_ERR_UNSUPPORTED unless ARC_FLAG_FORCE_SIMPLE is set.
+ * dtype F32 ("reference mode"): any D, Dv <= 512, a multiple of 32 up to 512;
+ * CUDA-core fp32 arithmetic, no TF32.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t dtype;
+    int32_t B, H, Hkv, Tq, Tk, D, Dv;
+    const void *q; int64_t q_strides[3];
+    const void *k; int64_t k_strides[3];
+    const void *v; int64_t v_strides[3];
+    void *o;       int64_t o_strides[3];
+    float *lse;
+    const float *sinks;
+    float scale;
+    int32_t causal;
+    uint32_t flags;
+    uint32_t *status;
+} arc_attn_args;
+
+arc_status arc_attn_fwd(const arc_attn_args *args, void *stream);
+
+/* --------------------------------------------------------------------------
+ * arc_mla_fwd: MLA attention with d_qk != d_v and the q/k concat done on load.
+ *
+ * Source: "pith-train PR: FA4 b19 return arity", MLA section: q = q_nope||q_rope
+ * and k = k_nope||k_rope are concatenated and fed to the attention kernel with
+ * head dims d_qk != d_v.  Here the concat is never materialised: the kernel
+ * stages both parts of each row side by side.  k_rope is one tensor shared by
+ * all heads.
+ *
+ *   q_nope [B,H,Tq,Dn]  bf16, device, strides {batch, head, token}
+ *   q_rope [B,H,Tq,Dr]  bf16, device
+ *   k_nope [B,H,Tk,Dn]  bf16, device
+ *   k_rope [B,Tk,Dr]    bf16, device, strides {batch, token}
+ *   v      [B,H,Tk,Dv]  bf16, device
+ *   o      [B,H,Tq,Dv]  bf16, device, written
+ *   lse    [B,H,Tq]     fp32, device, contiguous, written
+ * Dn, Dr multiples of 64 with Dn + Dr <= 256; Dv in {64,128,256}.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t B, H, Tq, Tk, Dn, Dr, Dv;
+    const void *q_nope; int64_t q_nope_strides[3];
+    const void *q_rope; int64_t q_rope_strides[3];
+    const void *k_nope; int64_t k_nope_strides[3];
+    const void *k_rope; int64_t k_rope_strides[2];
+    const void *v;      int64_t v_strides[3];
+    void *o;            int64_t o_strides[3];
+    float *lse;
+    float scale;
+    int32_t causal;
+    uint32_t flags;
+    uint32_t *status;
+} arc_mla_args;
+
+arc_status arc_mla_fwd(const arc_mla_args *args, void *stream);
+
+/* --------------------------------------------------------------------------
+ * arc_sparse_mla_fwd: attention over per-query top-k index lists.
+ *
+ * Source: "TensorRT-LLM: FlashMLA without -rdc", timing paragraph: sparse MLA
+ * forward over 13312 queries x 64 heads x 2176 top-k at d_qk 512.  All heads of
+ * a query token attend to the same gathered pool rows.  A slot whose index is
+ * outside [0, Skv) (e.g. -1 padding) is masked; a repeated index counts once
+ * per slot; no causal mask is applied (the index list encodes it).
+ *
+ *   q    [Sq,H,Dqk]   bf16, device, strides q_strides = {token, head}
+ *   kv   [Skv,Dqk]    bf16, device, row stride kv_stride
+ *   v    [Skv,Dv]     bf16, device, row stride v_stride; NULL means V is the
+ *                     first Dv columns of the same kv row (an MLA latent)
+ *   idx  [Sq,topk]    int32, device, row stride idx_stride
+ *   o    [Sq,H,Dv]    bf16, device, strides o_strides = {token, head}, written
+ *   lse  [Sq,H]       fp32, device, contiguous, written
+ *   sinks [H]         fp32, device, or NULL
+ * Dqk in {64,128,256,512}, Dv <= Dqk a multiple of 64.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t Sq, H, Skv, Dqk, Dv, topk;
+    const void *q;      int64_t q_strides[2];
+    const void *kv;     int64_t kv_stride;
+    const void *v;      int64_t v_stride;
+    const int32_t *idx; int64_t idx_stride;
+    void *o;            int64_t o_strides[2];
+    float *lse;
+    const float *sinks;
+    float scale;
+    uint32_t flags;
+    uint32_t *status;
+} arc_sparse_args;
+
+arc_status arc_sparse_mla_fwd(const arc_sparse_args *args, void *stream);
+
+/* --------------------------------------------------------------------------
+ * arc_attn_decode_q8: multi-sequence decode over one unified q8_0 / q4_0 cache,
+ * the K/V blocks dequantised in registers as each tile is loaded.
+ *
+ * Source: "unsloth llama.cpp: dequantize q4_0/q8_0 K/V tiles in the FA MMA
+ * kernel", summary paragraph: with a q4_0 / q8_0 KV cache and 3 to 16 tokens per
+ * batch across several sequences in one unified cache, K/V tiles are
+ * dequantised as they are loaded instead of converting the whole cache first.
+ *
+ * Block formats (32 values plus an fp16 scale d, little endian, d first):
+ *   q8_0: d, then 32 int8 q_j; value = d*q_j                          (34 bytes)
+ *   q4_0: d, then 16 bytes, byte j = n_j | n_{j+16}<<4; value = d*(n-8) (18 bytes)
+ *
+ *   q        [n_tok,H,D]            fp32, device, contiguous
+ *   k_cache  [n_cells,Hkv,D/32 blk] device, contiguous blocks, 8-byte aligned
+ *   v_cache  same layout and type as k_cache
+ *   seqs     [n_seq]                HOST array; sequence s owns query tokens
+ *            q_begin..q_begin+n_q-1 and cells kv_begin..kv_begin+n_kv-1, and its
+ *            n_q tokens are its last n_q cells: its token t (0-based) sees cells
+ *            kv_begin .. kv_begin + n_kv - n_q + t.
+ *   o        [n_tok,H,D]            fp32, device, written (rows of tokens that no
+ *            sequence owns are left untouched)
+ *   lse      [n_tok,H]              fp32, device, written likewise
+ * D in {64,128}; H % Hkv == 0; (H/Hkv) * n_q <= 16 for every sequence;
+ * n_seq <= ARC_DECODE_MAX_SEQ.
+ * workspace: device, at least arc_decode_workspace_size(args) bytes, 256-byte
+ * aligned; used for the split-KV partial results and overwritten.
+ * ------------------------------------------------------------------------ */
+#define ARC_DECODE_MAX_SEQ 64
+
+typedef struct {
+    int32_t q_begin, n_q, kv_begin, n_kv;
+} arc_seq;
+
+typedef struct {
+    int32_t kv_type;
+    int32_t n_tok, H, Hkv, D, n_cells, n_seq;
+    const float *q;
+    const void *k_cache;
+    const void *v_cache;
+    const arc_seq *seqs;
+    float *o;
+    float *lse;
+    float scale;
+    uint32_t flags;
+    uint32_t *status;
+} arc_decode_args;
+
+size_t arc_decode_workspace_size(const arc_decode_args *args);
+
+arc_status arc_attn_decode_q8(const arc_decode_args *args, void *workspace, size_t ws_bytes,
+                              void *stream);
+
+/* --------------------------------------------------------------------------
+ * Engagement record and helpers.
+ *
+ * arc_plan() answers, without launching anything, which kernel a call with
+ * these arguments launches and with what tiling -- the per-call engagement
+ * record ("ArcFlash ... rung 0", section D18: engagement is asserted, not
+ * inferred from correct numbers; "unsloth llama.cpp ...", review note that
+ * numerical equivalence is no proof the fast path ran).  It runs the same
+ * host planner as the launch itself.  `op` is an arc_op and `args` points to
+ * the matching args struct.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    char kernel[64];      /* name of the kernel the call launches */
+    int32_t tensor_cores; /* 1 if the hot loop runs on tcgen05 / mma tensor cores */
+    int32_t tile_m;       /* query rows per CTA tile */
+    int32_t tile_n;       /* keys per KV tile */
+    int32_t d_slice;      /* d_v columns one CTA accumulates */
+    int32_t n_ctas;       /* CTAs of the main launch */
+    int32_t splits;       /* decode: KV splits per (sequence, kv head) */
+    int32_t smem_bytes;   /* dynamic shared memory per CTA */
+    int32_t tmem_cols;    /* TMEM columns allocated per CTA (0 if none) */
+    int32_t launches;     /* kernels launched per call */
+} arc_plan_info;
+
+arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out);
+
+int32_t arc_abi_version(void);
+
+const char *arc_status_string(arc_status s);
+
+/* Synchronise `stream`, then read the device status word: ARC_OK if it is 0,
+ * ARC_ERR_DEVICE_TIMEOUT otherwise (the word is left as it is). */
+arc_status arc_check_device_error(const uint32_t *status, void *stream);
+
+/* Launch one tiny kernel whose only wait is on a barrier nothing ever
+ * arrives at, bounded by `timeout_ns`; it must report a timeout through
+ * *status.  Exercises the same bounded-wait code the attention kernels use. */
+arc_status arc_selftest_timeout(uint32_t *status, uint64_t timeout_ns, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARC_ATTN_H */

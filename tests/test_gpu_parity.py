@@ -1,0 +1,219 @@
+"""CUDA path vs the fp64 CPU oracle, element by element, through the C ABI.
+
+Small cases span several query-row tiles, several KV tiles and ragged tails;
+full-size cases (the five workload configurations) compare sampled rows that
+the oracle evaluates one by one, in the launch configuration bench.py times.
+Engagement is asserted separately: arc_plan names the tensor-core kernel for
+every bf16 case and the CUDA-core kernel only under ARC_FLAG_FORCE_SIMPLE.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+import exact_attention_131_b200 as arc
+from tests._util import TOL_LSE, TOL_O_BF16, TOL_O_F32, compare, dev, status_word
+
+pytestmark = pytest.mark.gpu
+
+
+def run_dense(c, flags=0, status=None):
+    q, k, v = dev(c.q), dev(c.k), dev(c.v)
+    s = dev(c.sinks) if c.sinks is not None else None
+    o, lse = arc.attn_fwd(q, k, v, scale=c.scale, causal=c.causal, sinks=s, flags=flags, status=status)
+    torch.cuda.synchronize()
+    return o, lse, (q, k, v, s)
+
+
+# ------------------------------------------------------------------ dense / GQA
+
+def test_config1_fp32_reference_mode():
+    c = W.config(1)
+    o, lse, _ = run_dense(c)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_F32)
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,Tk,D,Dv,causal,sinks", [
+    (1, 8, 2, 300, 300, 128, 128, True, False),     # ragged fold rows and KV tail
+    (2, 4, 4, 129, 129, 64, 64, True, True),        # one row past a tile
+    (1, 16, 2, 200, 200, 512, 512, True, True),     # d=512 with sinks: two d_v slices
+    (1, 8, 1, 100, 260, 256, 256, True, False),     # Tq < Tk: bottom-right causal
+    (1, 4, 2, 77, 333, 128, 64, False, True),       # non-causal, Dv < D
+    (1, 6, 3, 64, 40, 192, 128, True, False),       # Tq > Tk: first rows see nothing
+])
+def test_dense_bf16_small(B, H, Hkv, Tq, Tk, D, Dv, causal, sinks):
+    c = W.dense_case(B, H, Hkv, Tq, Tk, D, Dv, dtype="bf16", std=0.5, causal=causal, sinks=sinks, seed=31)
+    st = status_word()
+    o, lse, (q, k, v, s) = run_dense(c, status=st)
+    info = arc.plan_attn(q, k, v, o, lse, causal=causal, sinks=s)
+    assert info["kernel"] == "tc_attn_kernel" and info["tensor_cores"] == 1
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
+def test_dense_control_arm_runs_the_simple_kernel():
+    c = W.dense_case(1, 8, 2, 150, 150, 128, dtype="bf16", std=0.5, sinks=True, seed=32)
+    o, lse, (q, k, v, s) = run_dense(c, flags=arc.ARC_FLAG_FORCE_SIMPLE)
+    info = arc.plan_attn(q, k, v, o, lse, sinks=s, flags=arc.ARC_FLAG_FORCE_SIMPLE)
+    assert info["kernel"] == "simple_attn_kernel" and info["tensor_cores"] == 0
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+
+
+def sample_rows(T, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.choice(T, size=n - 4, replace=False).tolist()) | {0, 1, T - 2, T - 1}
+    return np.array(sorted(rows), dtype=np.int32)
+
+
+def test_config2_gqa_sinks_full_size_sampled_rows():
+    c = W.config(2)
+    st = status_word()
+    o, lse, (q, k, v, s) = run_dense(c, status=st)
+    info = arc.plan_attn(q, k, v, o, lse, sinks=s)
+    assert info["kernel"] == "tc_attn_kernel" and info["d_slice"] == 256
+    rows = sample_rows(c.Tq, 40, 2)
+    ro, rl = oracle.run_case(c, rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
+# ------------------------------------------------------------------ MLA
+
+def run_mla(c, flags=0, status=None):
+    t = [dev(x) for x in (c.q_nope, c.q_rope, c.k_nope, c.k_rope, c.v)]
+    o, lse = arc.mla_fwd(*t, scale=c.scale, causal=c.causal, flags=flags, status=status)
+    torch.cuda.synchronize()
+    return o, lse, t
+
+
+@pytest.mark.parametrize("B,H,T,Dn,Dr,Dv", [(1, 3, 300, 128, 64, 128), (2, 2, 130, 128, 64, 64),
+                                             (1, 2, 257, 64, 64, 128)])
+def test_mla_small(B, H, T, Dn, Dr, Dv):
+    c = W.mla_case(B, H, T, T, Dn, Dr, Dv, seed=33)
+    st = status_word()
+    o, lse, t = run_mla(c, status=st)
+    info = arc.plan_mla(*t, o, lse)
+    assert info["kernel"] == "tc_attn_kernel<mla>"
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
+def test_config3_mla_full_size_sampled_rows():
+    c = W.config(3)
+    o, lse, t = run_mla(c)
+    rows = sample_rows(c.Tq, 24, 3)
+    ro, rl = oracle.run_case(c, rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], ro, rl, TOL_O_BF16)
+
+
+# ------------------------------------------------------------------ sparse
+
+def run_sparse(c, flags=0, status=None):
+    q, kv, idx = dev(c.q), dev(c.kv), dev(c.idx)
+    v = dev(c.v) if c.v is not None else None
+    o, lse = arc.sparse_mla_fwd(q, kv, idx, Dv=c.Dv, v=v, scale=c.scale, flags=flags, status=status)
+    torch.cuda.synchronize()
+    return o, lse, (q, kv, idx, v)
+
+
+@pytest.mark.parametrize("Sq,H,Skv,D,Dv,topk,pad_mode,sep_v", [
+    (37, 64, 5000, 512, 512, 300, "random", False),
+    (20, 64, 3000, 512, 512, 250, "tail", False),
+    (9, 16, 700, 128, 64, 130, "random", True),
+])
+def test_sparse_small(Sq, H, Skv, D, Dv, topk, pad_mode, sep_v):
+    c = W.sparse_case(Sq, H, Skv, D, Dv, topk, pad_mode=pad_mode, separate_v=sep_v, seed=34)
+    o, lse, _ = run_sparse(c)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+
+
+def test_config4_sparse_full_size_sampled_queries():
+    c = W.config(4)
+    o, lse, _ = run_sparse(c)
+    rows = sample_rows(c.Sq, 24, 4)
+    ro, rl = oracle.run_case(c, rows=rows)
+    compare(o[rows], lse[rows], ro, rl, TOL_O_BF16)
+
+
+# ------------------------------------------------------------------ decode
+
+def run_decode(c, flags=0, status=None):
+    q, kc, vc = dev(c.q), dev(c.k_cache), dev(c.v_cache)
+    o, lse = arc.attn_decode_q8(q, kc, vc, kv_type=c.kv_type, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q,
+                                kv_begin=c.kv_begin, n_kv=c.n_kv, scale=c.scale, flags=flags, status=status)
+    torch.cuda.synchronize()
+    return o, lse, (q, kc, vc)
+
+
+@pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
+def test_config5_decode_full(kv_type):
+    c = W.config(5, kv_type=kv_type)
+    st = status_word()
+    o, lse, (q, kc, vc) = run_decode(c, status=st)
+    info = arc.plan_decode(kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                           n_kv=c.n_kv)
+    assert info["kernel"].startswith("decode_split_kernel") and info["splits"] > 1
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
+@pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
+def test_decode_ragged_sequences(kv_type):
+    c = W.decode_case(5, 0, 0, 16, 4, 128, kv_type=kv_type, seed=35, n_q_list=[4, 1, 3, 2, 4],
+                      n_kv_list=[1000, 17, 3, 333, 4])
+    o, lse, _ = run_decode(c)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+
+
+def test_decode_head_dim_64_and_control_arm():
+    c = W.decode_case(2, 3, 500, 8, 2, 64, kv_type=W.KV_Q8_0, seed=36)
+    o, lse, _ = run_decode(c)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    o2, lse2, (q, kc, vc) = run_decode(c, flags=arc.ARC_FLAG_FORCE_SIMPLE)
+    info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q,
+                           kv_begin=c.kv_begin, n_kv=c.n_kv, flags=arc.ARC_FLAG_FORCE_SIMPLE)
+    assert info["kernel"] == "simple_decode_kernel"
+    compare(o2, lse2, ro, rl, TOL_O_BF16)
+
+
+# ------------------------------------------------------------------ edge cases and failure reporting
+
+def test_empty_and_degenerate_shapes():
+    # Tq = 0: nothing to do.  Tk = 0: every row sees nothing -> O = 0, LSE = -inf (or the sink).
+    c = W.dense_case(1, 4, 2, 0, 10, 64, dtype="bf16", seed=37)
+    o, lse, _ = run_dense(c)
+    assert o.numel() == 0
+    c = W.dense_case(1, 4, 2, 5, 0, 64, dtype="bf16", sinks=True, seed=38)
+    o, lse, _ = run_dense(c)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+
+
+def test_bounded_wait_reports_a_timeout():
+    st = status_word()
+    assert arc.selftest_timeout(st, 2_000_000) == arc.ARC_OK     # 2 ms bound
+    assert arc.check_device_error(st) == arc.ARC_ERR_DEVICE_TIMEOUT
+    # The context stays usable afterwards.
+    c = W.dense_case(1, 2, 2, 64, 64, 64, dtype="bf16", seed=39)
+    o, lse, _ = run_dense(c)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+
+
+def test_invalid_arguments_launch_nothing():
+    q = torch.zeros(1, 3, 8, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((1, 3, 8, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(arc.ArcError) as e:
+        arc.attn_fwd(q, k, k, out=out)
+    assert e.value.status == arc.ARC_ERR_INVALID_ARG
+    assert torch.all(out == 7.0)
