@@ -137,7 +137,7 @@ def _dev(t, name, dtype=None):
         raise ValueError(f"{name} must be a CUDA tensor")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
-    if t.dim() > 0 and t.stride(-1) != 1:
+    if t.numel() > 0 and t.dim() > 0 and t.stride(-1) != 1 and t.shape[-1] > 1:
         raise ValueError(f"{name} must have a contiguous last dimension")
     return t
 
