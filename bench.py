@@ -131,15 +131,15 @@ def build_call(case, torch, arc, status):
         q, kc, vc = U.to_dev(case.q), U.to_dev(case.k_cache), U.to_dev(case.v_cache)
         o = torch.empty(case.n_tok, case.H, case.D, dtype=torch.float32, device="cuda")
         lse = torch.empty(case.n_tok, case.H, dtype=torch.float32, device="cuda")
-        kw = dict(kv_type=case.kv_type, Hkv=case.Hkv, q_begin=case.q_begin, n_q=case.n_q,
-                  kv_begin=case.kv_begin, n_kv=case.n_kv)
+        kw = dict(Hkv=case.Hkv, q_begin=case.q_begin, n_q=case.n_q, kv_begin=case.kv_begin, n_kv=case.n_kv)
         ws_n = arc.decode_workspace_size(case.kv_type, q, case.Hkv, case.n_cells, case.q_begin, case.n_q,
                                          case.kv_begin, case.n_kv)
         ws = torch.empty(max(ws_n, 256), dtype=torch.uint8, device="cuda")
         info = arc.plan_decode(case.kv_type, q, kc, vc, **kw)
 
         def call():
-            arc.attn_decode_q8(q, kc, vc, scale=case.scale, workspace=ws, out=o, lse=lse, status=status, **kw)
+            arc.attn_decode_q8(q, kc, vc, kv_type=case.kv_type, scale=case.scale, workspace=ws, out=o, lse=lse,
+                               status=status, **kw)
         return call, {"q": q, "k_cache": kc, "v_cache": vc}, [o, lse], info
     raise TypeError(type(case))
 
@@ -247,8 +247,8 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
             spent += time.perf_counter() - t0
             Dqk = case.D if isinstance(case, W.DenseCase) else case.Dn + case.Dr
             heads = case.B * case.H
-            vis = sum(min(case.Tk, r + case.Tk - case.Tq + 1) if case.causal else case.Tk for r in rows)
-            done_units += heads * vis * (2 * Dqk + 2 * case.Dv)
+            vis = sum(min(case.Tk, int(r) + case.Tk - case.Tq + 1) if case.causal else case.Tk for r in rows)
+            done_units += int(heads) * int(vis) * (2 * Dqk + 2 * case.Dv)
             n_rows += batch
             if spent > budget_s[1]:
                 break
@@ -263,7 +263,7 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
             oracle.run_case(case, rows=rows)
             spent += time.perf_counter() - t0
             valid = int(((case.idx[rows] >= 0) & (case.idx[rows] < case.Skv)).sum())
-            done_units += valid * case.H * (2 * case.Dqk + 2 * case.Dv)
+            done_units += int(valid) * case.H * (2 * case.Dqk + 2 * case.Dv)
             n_rows += batch
             if spent > budget_s[1]:
                 break
@@ -410,7 +410,7 @@ def run_reference(args, spec, case):
         if isinstance(case, (W.DenseCase, W.MlaCase)):
             rows = np.sort(rng.choice(case.Tq, size=2, replace=False)).astype(np.int32)
             Dqk = case.D if isinstance(case, W.DenseCase) else case.Dn + case.Dr
-            vis = sum(min(case.Tk, r + case.Tk - case.Tq + 1) if case.causal else case.Tk for r in rows)
+            vis = sum(min(case.Tk, int(r) + case.Tk - case.Tq + 1) if case.causal else case.Tk for r in rows)
             u = case.B * case.H * vis * (2 * Dqk + 2 * case.Dv)
             t0 = time.perf_counter()
             oracle.run_case(case, rows=rows)
