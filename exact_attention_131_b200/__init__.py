@@ -75,7 +75,7 @@ class PlanInfo(ctypes.Structure):
 
 EXPORTS = ["arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
            "arc_decode_workspace_size", "arc_plan", "arc_abi_version", "arc_status_string",
-           "arc_check_device_error", "arc_selftest_timeout"]
+           "arc_check_device_error", "arc_selftest_timeout", "arc_attn_decode_q8_noalloc"]
 
 
 class ArcError(RuntimeError):
@@ -96,6 +96,7 @@ def lib():
         L.arc_mla_fwd.argtypes = [ctypes.POINTER(MlaArgs), _vp]
         L.arc_sparse_mla_fwd.argtypes = [ctypes.POINTER(SparseArgs), _vp]
         L.arc_attn_decode_q8.argtypes = [ctypes.POINTER(DecodeArgs), _vp, ctypes.c_size_t, _vp]
+        L.arc_attn_decode_q8_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         L.arc_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]
         L.arc_decode_workspace_size.restype = ctypes.c_size_t
         L.arc_plan.argtypes = [_i32, _vp, ctypes.POINTER(PlanInfo)]
@@ -103,7 +104,8 @@ def lib():
         L.arc_status_string.restype = ctypes.c_char_p
         L.arc_check_device_error.argtypes = [_vp, _vp]
         L.arc_selftest_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
-        for f in ("arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8", "arc_plan",
+        for f in ("arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
+                  "arc_attn_decode_q8_noalloc", "arc_plan",
                   "arc_check_device_error", "arc_selftest_timeout", "arc_abi_version"):
             getattr(L, f).restype = _i32
         _lib = L
@@ -322,6 +324,33 @@ def attn_decode_q8(q, k_cache, v_cache, *, kv_type, Hkv, q_begin, n_q, kv_begin,
     ws_ptr = _p(workspace) if workspace is not None else None
     ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check(lib().arc_attn_decode_q8(ctypes.byref(a), ws_ptr, ws_len, _stream(stream)), "arc_attn_decode_q8")
+    return out, lse
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def attn_decode_q8_noalloc(q, k_cache, v_cache, *, kv_type, Hkv, q_begin, n_q, kv_begin, n_kv, scale=None,
+                           out=None, lse=None, flags=0, status=None, stream=None):
+    """arc_attn_decode_q8_noalloc: the decode with the library's own 8 MiB static scratch.
+
+    For callers that must not allocate device memory: no workspace is passed and
+    the library allocates nothing.  (This wrapper still creates `out` / `lse`
+    with torch when they are not given; pass them to keep the call allocation-free.)
+    Calls on unordered streams race on the shared scratch.
+    """
+    torch = _torch()
+    _dev(q, "q", torch.float32), _dev(k_cache, "k_cache", torch.uint8), _dev(v_cache, "v_cache", torch.uint8)
+    n_tok, H, D = q.shape
+    seqs = make_seqs(q_begin, n_q, kv_begin, n_kv)
+    if out is None:
+        out = torch.empty(n_tok, H, D, dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty(n_tok, H, dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    a = _decode_args(kv_type, q, k_cache, v_cache, seqs, len(q_begin), Hkv, k_cache.shape[0], out, lse, scale,
+                     flags, status)
+    _check(lib().arc_attn_decode_q8_noalloc(ctypes.byref(a), _stream(stream)), "arc_attn_decode_q8_noalloc")
     return out, lse
 
 

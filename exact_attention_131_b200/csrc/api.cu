@@ -504,6 +504,38 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
 
+// Library-owned scratch for arc_attn_decode_q8_noalloc.  In host code the
+// symbol is only a stand-in; its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[ARC_DECODE_NOALLOC_SCRATCH_BYTES];
+
+static arc_status noalloc_scratch_address(void **out)
+{
+    static std::mutex mu;
+    static void *addr[256] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return ARC_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || !p) return ARC_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return ARC_OK;
+}
+
+arc_status arc_attn_decode_q8_noalloc(const arc_decode_args *a, void *stream)
+{
+    arc_status st = check_decode(a);
+    if (st != ARC_OK) return st;
+    if (a->n_seq == 0 || a->n_tok == 0) return ARC_OK;
+    if (plan_decode(a).ws > ARC_DECODE_NOALLOC_SCRATCH_BYTES) return ARC_ERR_WORKSPACE;
+    void *scratch = nullptr;
+    if ((st = noalloc_scratch_address(&scratch)) != ARC_OK) return st;
+    return arc_attn_decode_q8(a, scratch, ARC_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
 {
     if (!args || !out) return ARC_ERR_INVALID_ARG;

@@ -228,6 +228,35 @@ arc_status arc_attn_decode_q8(const arc_decode_args *args, void *workspace, size
                               void *stream);
 
 /* --------------------------------------------------------------------------
+ * arc_attn_decode_q8_noalloc: the same decode, for callers that cannot
+ * allocate device memory.
+ *
+ * The pages have no counterpart to this call; it exists for hosts that must
+ * not call cudaMalloc at all -- an engine whose memory planner owns every
+ * device byte, a process that runs with a fixed memory budget, or code that
+ * must stay out of the allocator while other work is in flight -- and so
+ * cannot hand arc_attn_decode_q8 a workspace.  It takes the same arguments
+ * minus the workspace and launches the same kernels, with the split-KV
+ * partial results kept in a library-owned buffer: a file-scope __device__
+ * array of ARC_DECODE_NOALLOC_SCRATCH_BYTES (8 MiB) that every GPU which loads
+ * the library holds until the process exits.  The caller still passes all
+ * inputs and outputs.
+ *   - A call whose partial results would need more than that buffer returns
+ *     ARC_ERR_WORKSPACE and launches nothing (arc_decode_workspace_size()
+ *     gives the bytes a call needs).
+ *   - The first call on a device (that device current) looks up the buffer's
+ *     device address once; make that first call before any stream capture.
+ *   - All calls share the one buffer and it keeps the last call's contents
+ *     (nothing in it needs to start at zero).  Calls that may overlap on the
+ *     GPU -- on different streams without ordering between them -- race on it;
+ *     serialise them.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ * ------------------------------------------------------------------------ */
+#define ARC_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+arc_status arc_attn_decode_q8_noalloc(const arc_decode_args *args, void *stream);
+
+/* --------------------------------------------------------------------------
  * Engagement record and helpers.
  *
  * arc_plan() answers, without launching anything, which kernel a call with
