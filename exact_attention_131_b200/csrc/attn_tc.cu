@@ -16,10 +16,13 @@
 //                 S[buf] = Q K^T      (M=128, N=128, K-major A and B)
 //                 O     += P V        (M=128, N=d_v slice, V read MN-major)
 //   warps 4-7   softmax: one thread per query row; read S from TMEM, mask,
-//               online max / sum in log2 units, rescale O in TMEM when the
-//               running max grows by more than 2^8, write P (bf16) to shared
-//               memory in the 128-byte-swizzled K-major layout, epilogue.
-// TMEM (512 columns): O slice at columns [0, DVS), S double buffer at 256, 384.
+//               online max / sum in log2 units, write P (bf16, two per 32-bit
+//               column) back over the S columns it came from, rescale O in
+//               TMEM when the running max grows by more than 2^8, epilogue.
+// TMEM (512 columns): O slice at columns [0, DVS), S/P double buffer at 256, 384.
+// P is the TMEM A operand of O += P V, so P never touches shared memory; S of
+// tile j+2 reuses the buffer only after O += P_j V_j, which the tensor core
+// executes in issue order.
 // Every wait is bounded; a wait that runs out reports through p.status.
 #include <math.h>
 
@@ -44,7 +47,6 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 struct Bars {
     uint64_t q_full;
     uint64_t s_full[2];
-    uint64_t s_free[2];
     uint64_t p_full;
     uint64_t o_done;
     uint64_t drain;
@@ -67,8 +69,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
     uint8_t *sQ = smem;
     uint8_t *sRing = sQ + KC * CHUNK;
     const int R = p.stages;
-    uint8_t *sP = sRing + R * CHUNK;
-    Bars *bars = reinterpret_cast<Bars *>(sP + 2 * CHUNK);
+    Bars *bars = reinterpret_cast<Bars *>(sRing + R * CHUNK);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -93,10 +94,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->s_free[i], 128);
-        }
+        for (int i = 0; i < 2; ++i) mbar_init(&bars->s_full[i], 1);
         mbar_init(&bars->p_full, 128);
         mbar_init(&bars->o_done, 1);
         mbar_init(&bars->drain, 1);
@@ -131,13 +129,12 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
             }
             int stage = 0;
             uint32_t ephase = 0;
-            int issued[MAX_STAGES];
-            for (int i = 0; i < MAX_STAGES; ++i) issued[i] = 0;
+            int total = 0;  // chunk loads issued so far (stage of load i is i % R)
             bool ok = true;
             auto acquire = [&]() -> bool {
                 if (!mbar_wait(&bars->empty[stage], ephase ^ 1u)) return false;
                 mbar_arrive_expect_tx(&bars->full[stage], CHUNK);
-                issued[stage]++;
+                ++total;
                 return true;
             };
             auto advance = [&]() {
@@ -173,15 +170,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
             }
             if (!ok) report(p.status, ST_TIMEOUT_LOAD);
             // Drain: every copy this thread issued has landed before the CTA exits.
-            for (int s = 0; s < R; ++s)
-                if (issued[s] > 0) mbar_wait(&bars->full[s], (uint32_t)((issued[s] - 1) & 1));
+            for (int s = 0; s < R && s < total; ++s) {
+                const int loads = (total - s + R - 1) / R;  // loads that went to stage s
+                mbar_wait(&bars->full[s], (uint32_t)((loads - 1) & 1));
+            }
             mbar_wait(&bars->q_full, 0);
         }
     } else if (warp == 1) {
         // =============================== MMA issuer
+        // Kept lean on purpose: one thread issues every MMA, so descriptors are
+        // precomputed and advanced by constants, four K steps go out per issue block,
+        // and nothing here touches local memory.
         if (lane == 0 && nt > 0) {
+            constexpr uint32_t kChunkUnits = CHUNK >> 4;     // descriptor units per ring stage
             const uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
-            const uint32_t q_base = smem_u32(sQ), ring_base = smem_u32(sRing), p_base = smem_u32(sP);
+            const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t kd0 = sdesc_sw128(smem_u32(sRing), 16, 1024);
+            const uint64_t vd0 = sdesc_sw128(smem_u32(sRing), CHUNK, 1024);
             int stage = 0;
             uint32_t fphase = 0;
             bool ok = mbar_wait(&bars->q_full, 0);
@@ -193,47 +198,45 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
                 }
             };
             auto issue_s = [&](int j) -> bool {
-                const int buf = j & 1;
-                if (j >= 2 && !mbar_wait(&bars->s_free[buf], (uint32_t)(((j - 2) >> 1) & 1))) return false;
-                tc_fence_after();
-                const uint32_t d = tmem + S_COL + buf * BN;
+                const uint32_t d = tmem + S_COL + (j & 1) * BN;
+#pragma unroll 1
                 for (int c = 0; c < KC; ++c) {
                     if (!mbar_wait(&bars->full[stage], fphase)) return false;
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t a = sdesc_sw128(q_base + c * CHUNK + kk * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(ring_base + stage * CHUNK + kk * 32, 16, 1024);
-                        umma_bf16(d, a, bd, idesc_s, (c | kk) != 0);
-                    }
+                    umma_ss_k64(d, qd0 + (uint64_t)(c * kChunkUnits), kd0 + (uint64_t)(stage * kChunkUnits), idesc_s,
+                                c > 0);
                     umma_commit(&bars->empty[stage]);
                     advance();
                 }
-                umma_commit(&bars->s_full[buf]);
+                umma_commit(&bars->s_full[j & 1]);
                 return true;
             };
             auto issue_pv = [&](int j) -> bool {
                 if (!mbar_wait(&bars->p_full, (uint32_t)(j & 1))) return false;
-                int vst[VC];
+                const int s0 = stage;
+#pragma unroll 1
                 for (int c = 0; c < VC; ++c) {
                     if (!mbar_wait(&bars->full[stage], fphase)) return false;
-                    vst[c] = stage;
                     advance();
                 }
                 tc_fence_after();
+                const uint32_t p_tm = tmem + S_COL + (j & 1) * BN;
+                // V chunks sit in stages s0.. (wrapping at R): at most two contiguous runs.
+                const int n1 = (s0 + VC <= R) ? VC : R - s0;
+                const uint32_t idesc1 = idesc_bf16(BM, 64 * n1, false, true);
+                const uint64_t b1 = vd0 + (uint64_t)(s0 * kChunkUnits);
+                const uint32_t acc = j > 0;
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t a = sdesc_sw128(p_base + (kk >> 2) * CHUNK + (kk & 3) * 32, 16, 1024);
-                    int c = 0;
-                    while (c < VC) {
-                        int len = 1;
-                        while (c + len < VC && vst[c + len] == vst[c] + len) ++len;
-                        const uint64_t bd = sdesc_sw128(ring_base + vst[c] * CHUNK + kk * 2048, CHUNK, 1024);
-                        umma_bf16(tmem + c * 64, a, bd, idesc_bf16(BM, 64 * len, false, true), (j > 0 || kk > 0));
-                        c += len;
-                    }
+                for (int k4 = 0; k4 < BN / 64; ++k4)
+                    umma_ts_k64(tmem, p_tm + k4 * 32, b1 + (uint64_t)(k4 * 512), 128, idesc1, acc | k4);
+                if (n1 < VC) {
+                    const uint32_t idesc2 = idesc_bf16(BM, 64 * (VC - n1), false, true);
+#pragma unroll
+                    for (int k4 = 0; k4 < BN / 64; ++k4)
+                        umma_ts_k64(tmem + n1 * 64, p_tm + k4 * 32, vd0 + (uint64_t)(k4 * 512), 128, idesc2, acc | k4);
                 }
-                for (int c = 0; c < VC; ++c) umma_commit(&bars->empty[vst[c]]);
+#pragma unroll 1
+                for (int c = 0; c < VC; ++c) umma_commit(&bars->empty[(s0 + c) % R]);
                 umma_commit(&bars->o_done);
                 return true;
             };
@@ -260,20 +263,18 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
         const float sl2 = p.scale_log2;
         float m_use = -INFINITY, l = 0.f;
         bool ok = true;
-        uint8_t *prow = sP + (r >> 3) * 1024 + (r & 7) * 128;
 
         for (int j = 0; j < nt; ++j) {
             const int buf = j & 1;
+            const uint32_t s_tmem = tmem + lane_off + S_COL + buf * BN;
             ok = warp_all(mbar_wait(&bars->s_full[buf], (uint32_t)((j >> 1) & 1)));
             if (!ok) break;
             tc_fence_after();
             uint32_t sv[BN];
 #pragma unroll
             for (int i = 0; i < BN / 32; ++i)
-                tmem_ld32(tmem + lane_off + S_COL + buf * BN + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * i]));
+                tmem_ld32(s_tmem + 32 * i, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * i]));
             tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&bars->s_free[buf]);
 
             const int kbase = j * BN;
             if (kbase + BN - 1 > last) {
@@ -293,17 +294,28 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
             }
             const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
             float rowsum = 0.f;
-            uint32_t pk[BN / 2];
+            uint32_t pk0[32], pk1[32];
 #pragma unroll
-            for (int i = 0; i < BN / 2; ++i) {
+            for (int i = 0; i < 32; ++i) {
                 const float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * i]), sl2, -msafe));
                 const float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * i + 1]), sl2, -msafe));
                 rowsum += p0 + p1;
-                pk[i] = pack_bf16(p0, p1);
+                pk0[i] = pack_bf16(p0, p1);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(sv[64 + 2 * i]), sl2, -msafe));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(sv[64 + 2 * i + 1]), sl2, -msafe));
+                rowsum += p0 + p1;
+                pk1[i] = pack_bf16(p0, p1);
             }
             l = l * alpha + rowsum;
+            // P (bf16 pairs) over the first half of the S columns it came from.
+            tmem_st32(s_tmem, pk0);
+            tmem_st32(s_tmem + 32, pk1);
 
-            // PV(j-1) must be complete before O is rescaled or the P buffer reused.
+            // O += P(j-1) V(j-1) must be complete before O is rescaled; waiting on
+            // every tile keeps this thread's view of o_done in step with its phases.
             if (j > 0) {
                 ok = warp_all(mbar_wait(&bars->o_done, (uint32_t)((j - 1) & 1)));
                 if (!ok) break;
@@ -318,20 +330,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
                         for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
                         tmem_st32(tmem + lane_off + 32 * c, ov);
                     }
-                    tmem_wait_st();
                 }
             }
-            // P row -> shared memory, 128-byte swizzle: 16-byte unit u of row r sits at u ^ (r & 7).
-#pragma unroll
-            for (int cc = 0; cc < BN / 64; ++cc) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    uint4 val = make_uint4(pk[cc * 32 + u * 4 + 0], pk[cc * 32 + u * 4 + 1],
-                                           pk[cc * 32 + u * 4 + 2], pk[cc * 32 + u * 4 + 3]);
-                    *reinterpret_cast<uint4 *>(prow + cc * CHUNK + ((u ^ (r & 7)) << 4)) = val;
-                }
-            }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bars->p_full);
         }
@@ -400,11 +401,11 @@ cudaError_t launch_one(const TcParams &p, int grid, cudaStream_t s)
 
 }  // namespace
 
-int tc_smem_bytes(int dqk, int stages) { return 1024 + (dqk / 64 + stages + 2) * CHUNK + (int)sizeof(Bars); }
+int tc_smem_bytes(int dqk, int stages) { return 1024 + (dqk / 64 + stages) * CHUNK + (int)sizeof(Bars); }
 
 int tc_max_stages(int dqk)
 {
-    int st = (SMEM_LIMIT - 1024 - (int)sizeof(Bars) - (dqk / 64 + 2) * CHUNK) / CHUNK;
+    int st = (SMEM_LIMIT - 1024 - (int)sizeof(Bars) - (dqk / 64) * CHUNK) / CHUNK;
     return st < MAX_STAGES ? st : MAX_STAGES;
 }
 

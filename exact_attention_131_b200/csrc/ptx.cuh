@@ -149,6 +149,52 @@ ARC_DEV void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16.  A (M rows x 16 bf16) sits in
+// TMEM: one row per data-path lane, two bf16 per 32-bit column (8 columns per K step).
+ARC_DEV void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Four consecutive K=16 steps of an SS MMA in one issue block: A and B advance by
+// 32 bytes (2 descriptor units) per step inside a 128-byte swizzle row.  The first
+// step accumulates iff acc != 0, the other three always accumulate.
+ARC_DEV void umma_ss_k64(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, %4, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %9, %10, %3, q;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "l"(a + 2), "l"(b + 2), "l"(a + 4), "l"(b + 4), "l"(a + 6), "l"(b + 6)
+        : "memory");
+}
+
+// Four consecutive K=16 steps of a TS MMA: A in TMEM advances 8 columns per step,
+// B advances b_step descriptor units per step.
+ARC_DEV void umma_ts_k64(uint32_t d, uint32_t a_tm, uint64_t b, uint32_t b_step, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, %4, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %3, q;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%9], %10, %3, q;\n\t}" ::"r"(d),
+        "r"(a_tm), "l"(b), "r"(idesc), "r"(acc), "r"(a_tm + 8), "l"(b + b_step), "r"(a_tm + 16),
+        "l"(b + 2 * b_step), "r"(a_tm + 24), "l"(b + 3 * b_step)
+        : "memory");
+}
+
 // Arrive (once) on *bar when every tcgen05.mma this thread issued so far has completed.
 ARC_DEV void umma_commit(uint64_t *bar)
 {
