@@ -267,6 +267,20 @@ arc_status check_sparse(const arc_sparse_args *a)
     return ARC_OK;
 }
 
+// Tensor-core sparse path: instantiated head dims, 16-byte aligned rows.
+bool plan_sparse_tc(const arc_sparse_args *a)
+{
+    if (a->flags & ARC_FLAG_FORCE_SIMPLE) return false;
+    const bool sepv = a->v != nullptr;
+    if (!sparse_tc_supported(a->Dqk, a->Dv, sepv)) return false;
+    if (!aligned16(a->q) || !aligned16(a->kv) || !aligned16(a->o) || (sepv && !aligned16(a->v))) return false;
+    auto al = [](int64_t s) { return (s * 2) % 16 == 0; };
+    if (!al(a->q_strides[0]) || !al(a->q_strides[1]) || !al(a->kv_stride) || !al(a->o_strides[0]) ||
+        !al(a->o_strides[1]) || (sepv && !al(a->v_stride)))
+        return false;
+    return true;
+}
+
 // ------------------------------------------------------------------ decode
 
 struct DecodePlan {
@@ -445,18 +459,33 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *a, void *stream)
     arc_status st = check_sparse(a);
     if (st != ARC_OK) return st;
     if (a->Sq == 0) return ARC_OK;
-    SimpleParams p{};
-    p.mode = 2;
-    p.dtype = ARC_DTYPE_BF16;
-    p.B = 1, p.H = a->H, p.Hkv = 1, p.Tq = a->Sq, p.Tk = a->topk, p.Dqk = a->Dqk, p.Dv = a->Dv, p.Dn = a->Dqk;
-    p.q = a->q, p.k = a->kv, p.v = a->v, p.o = a->o;
-    p.qs[0] = a->q_strides[0], p.qs[1] = a->q_strides[1];
-    p.ks[0] = a->kv_stride, p.vs[0] = a->v_stride;
-    p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
-    p.lse = a->lse, p.sinks = a->sinks, p.scale = a->scale, p.causal = 0;
-    p.idx = a->idx, p.idx_stride = a->idx_stride, p.topk = a->topk, p.Skv = a->Skv, p.status = a->status;
-    note_dispatch("simple_attn_kernel<sparse>");
-    cudaError_t e = launch_simple_attn(p, static_cast<cudaStream_t>(stream));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (plan_sparse_tc(a)) {
+        SparseTcParams p{};
+        p.Sq = a->Sq, p.H = a->H, p.Skv = a->Skv, p.Dqk = a->Dqk, p.Dv = a->Dv, p.topk = a->topk;
+        p.q = static_cast<const __nv_bfloat16 *>(a->q), p.qs[0] = a->q_strides[0], p.qs[1] = a->q_strides[1];
+        p.kv = static_cast<const __nv_bfloat16 *>(a->kv), p.kv_stride = a->kv_stride;
+        p.v = static_cast<const __nv_bfloat16 *>(a->v), p.v_stride = a->v_stride;
+        p.idx = a->idx, p.idx_stride = a->idx_stride;
+        p.o = static_cast<__nv_bfloat16 *>(a->o), p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
+        p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = a->scale * kLog2e, p.status = a->status;
+        note_dispatch("sparse_tc_kernel");
+        e = launch_sparse_tc(p, s);
+    } else {
+        SimpleParams p{};
+        p.mode = 2;
+        p.dtype = ARC_DTYPE_BF16;
+        p.B = 1, p.H = a->H, p.Hkv = 1, p.Tq = a->Sq, p.Tk = a->topk, p.Dqk = a->Dqk, p.Dv = a->Dv, p.Dn = a->Dqk;
+        p.q = a->q, p.k = a->kv, p.v = a->v, p.o = a->o;
+        p.qs[0] = a->q_strides[0], p.qs[1] = a->q_strides[1];
+        p.ks[0] = a->kv_stride, p.vs[0] = a->v_stride;
+        p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
+        p.lse = a->lse, p.sinks = a->sinks, p.scale = a->scale, p.causal = 0;
+        p.idx = a->idx, p.idx_stride = a->idx_stride, p.topk = a->topk, p.Skv = a->Skv, p.status = a->status;
+        note_dispatch("simple_attn_kernel<sparse>");
+        e = launch_simple_attn(p, s);
+    }
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
 
@@ -588,8 +617,16 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
         const arc_sparse_args *a = static_cast<const arc_sparse_args *>(args);
         arc_status st = check_sparse(a);
         if (st != ARC_OK) return st;
-        set_name(out, "simple_attn_kernel<sparse>");
-        out->tile_m = 4;
+        if (a->Sq > 0 && plan_sparse_tc(a)) {
+            set_name(out, "sparse_tc_kernel");
+            out->tensor_cores = 1;
+            out->tile_m = 64, out->tile_n = 64, out->d_slice = a->Dv;
+            out->n_ctas = a->Sq * ((a->H + 63) / 64);
+            out->smem_bytes = sparse_smem_bytes(a->Dqk, a->Dv, a->v != nullptr), out->tmem_cols = 512;
+        } else {
+            set_name(out, "simple_attn_kernel<sparse>");
+            out->tile_m = 4;
+        }
         out->launches = 1;
         return ARC_OK;
     }

@@ -85,7 +85,8 @@ struct SparseTcParams {
     float scale_log2;
     uint32_t *status;
 };
-int sparse_smem_bytes(int dqk, int bn);
+int sparse_smem_bytes(int dqk, int dv, bool sepv);
+bool sparse_tc_supported(int dqk, int dv, bool sepv);
 cudaError_t launch_sparse_tc(const SparseTcParams &p, cudaStream_t s);
 
 // ---------------------------------------------------------------- quantised decode

@@ -128,9 +128,24 @@ def run_sparse(c, flags=0, status=None):
 ])
 def test_sparse_small(Sq, H, Skv, D, Dv, topk, pad_mode, sep_v):
     c = W.sparse_case(Sq, H, Skv, D, Dv, topk, pad_mode=pad_mode, separate_v=sep_v, seed=34)
-    o, lse, _ = run_sparse(c)
+    st = status_word()
+    o, lse, (q, kv, idx, v) = run_sparse(c, status=st)
+    info = arc.plan_sparse(q, kv, idx, o, lse, Dv=Dv, v=v)
+    assert info["kernel"] == "sparse_tc_kernel" and info["tensor_cores"] == 1
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
+def test_sparse_more_than_64_heads_and_control_arm():
+    c = W.sparse_case(7, 96, 900, 256, 256, 200, seed=43)
+    o, lse, (q, kv, idx, v) = run_sparse(c)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    o2, lse2, _ = run_sparse(c, flags=arc.ARC_FLAG_FORCE_SIMPLE)
+    assert arc.plan_sparse(q, kv, idx, o2, lse2, flags=arc.ARC_FLAG_FORCE_SIMPLE)["kernel"] == \
+        "simple_attn_kernel<sparse>"
+    compare(o2, lse2, ro, rl, TOL_O_BF16)
 
 
 def test_config4_sparse_full_size_sampled_queries():
