@@ -11,8 +11,9 @@
 //               16-byte cp.async per lane (a warp reads 512 contiguous bytes of
 //               one pool row), written straight into the 128-byte-swizzled
 //               K-major layout the tensor core reads; an index outside
-//               [0, Skv) writes zeros (the softmax masks that slot from the
-//               same index list).
+//               [0, Skv) writes zeros and clears its bit in the tile's validity
+//               mask.  A tile's 64 indices are read once per warp and the next
+//               tile's are fetched while this tile's rows are in flight.
 //               Two tile buffers alternate.
 //   warp 8      TMEM owner and MMA issuer:
 //                 S[buf] = Q K^T       M=64, N=64 keys,  A and B K-major
@@ -50,6 +51,7 @@ struct SparseBars {
     uint64_t p_full[2];
     uint64_t o_done;
     uint64_t drain;
+    uint32_t mask[2][2];  // validity of the 64 slots of each tile buffer
     uint32_t tmem_base;
 };
 
@@ -120,6 +122,19 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
         mbar_arrive(&bars->q_full);
 
         const int32_t *idx_row = p.idx + (int64_t)tok * p.idx_stride;
+        // Lane i < 16 of warp w holds the index of tile row w + 4i; warp 0 also holds
+        // one index per lane for each half of the tile, for the validity mask.
+        auto fetch = [&](int j, int32_t &mine, int32_t &m0, int32_t &m1) {
+            const int slot = j * SBN + warp + 4 * (lane & 15);
+            mine = (lane < 16 && slot < p.topk) ? idx_row[slot] : -1;
+            if (warp == 0) {
+                const int s0 = j * SBN + lane, s1 = s0 + 32;
+                m0 = s0 < p.topk ? idx_row[s0] : -1;
+                m1 = s1 < p.topk ? idx_row[s1] : -1;
+            }
+        };
+        int32_t mine = -1, m0 = -1, m1 = -1;
+        if (nt > 0) fetch(0, mine, m0, m1);
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             const int b = j & 1;
@@ -128,11 +143,10 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                 if (!ok) break;
             }
             uint8_t *tile = sKV + b * L::TILE_BYTES;
-            // each warp takes rows w, w+4, ...; a row is KC*8 16-byte units, 32 per instruction
-#pragma unroll 1
-            for (int r = warp; r < SBN; r += 4) {
-                const int slot = j * SBN + r;
-                int32_t key = slot < p.topk ? idx_row[slot] : -1;
+#pragma unroll 4
+            for (int i = 0; i < SBN / 4; ++i) {
+                const int r = warp + 4 * i;
+                int32_t key = __shfl_sync(0xffffffffu, mine, i);
                 const bool valid = key >= 0 && key < p.Skv;
                 if (!valid) key = 0;
                 const __nv_bfloat16 *krow = p.kv + (int64_t)key * p.kv_stride;
@@ -151,6 +165,15 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                 }
             }
             cp_async_commit_group();
+            if (warp == 0) {
+                const uint32_t b0 = __ballot_sync(0xffffffffu, m0 >= 0 && m0 < p.Skv);
+                const uint32_t b1 = __ballot_sync(0xffffffffu, m1 >= 0 && m1 < p.Skv);
+                if (lane == 0) {
+                    bars->mask[b][0] = b0;
+                    bars->mask[b][1] = b1;
+                }
+            }
+            if (j + 1 < nt) fetch(j + 1, mine, m0, m1);  // next tile's indices fly with this tile's rows
             cp_async_wait_all();
             fence_proxy_async_smem();
             mbar_arrive(&bars->kv_full[b]);
@@ -216,7 +239,6 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
         const uint32_t o_lanes = (uint32_t)(q4 * 32) << 16;
         const uint32_t s_lanes = (uint32_t)(q4 * 32 + 16) << 16;
         const float sl2 = p.scale_log2;
-        const int32_t *idx_row = p.idx + (int64_t)tok * p.idx_stride;
         float m_use = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
@@ -227,16 +249,11 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
             uint32_t sv[32];
             tmem_ld16x2_32(tmem + s_lanes + b * SBN, sv);
             tmem_wait_ld();
-            // validity of this thread's 32 keys: one index per lane, two ballots
-            uint32_t bits;
-            {
-                const int slot0 = j * SBN + lane, slot1 = slot0 + 32;
-                const int32_t k0 = slot0 < p.topk ? idx_row[slot0] : -1;
-                const int32_t k1 = slot1 < p.topk ? idx_row[slot1] : -1;
-                const uint32_t b0 = __ballot_sync(0xffffffffu, k0 >= 0 && k0 < p.Skv);
-                const uint32_t b1 = __ballot_sync(0xffffffffu, k1 >= 0 && k1 < p.Skv);
-                bits = half ? b1 : b0;
-            }
+            // validity of this thread's 32 keys, published with the tile (kv_full is
+            // already complete here; waiting on it orders the mask read after its write)
+            ok = warp_all_sparse(mbar_wait(&bars->kv_full[b], (uint32_t)((j >> 1) & 1)));
+            if (!ok) break;
+            const uint32_t bits = bars->mask[b][half];
             float mx = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
