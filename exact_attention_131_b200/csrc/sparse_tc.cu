@@ -220,9 +220,10 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                 umma_commit(&bars->o_done);
                 return true;
             };
-            if (ok && nt > 0) ok = issue_s(0);
+            // S(j) then O += P(j) V(j): the gather of tile j+1 (free once P(j-1) V(j-1) is
+            // done) then has a whole tile of tensor-core work to hide behind.
             for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt) ok = issue_s(j + 1);
+                ok = issue_s(j);
                 if (ok) ok = issue_pv(j);
             }
             if (!ok) report(p.status, ST_TIMEOUT_MMA);
