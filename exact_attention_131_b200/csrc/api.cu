@@ -325,7 +325,7 @@ DecodePlan plan_decode(const arc_decode_args *a)
     const int smem = decode_smem_bytes(a->kv_type, a->D);
     const int per_sm = std::max(1, std::min(4, (228 * 1024) / (smem + 1024)));
     const int target = sm_count() * per_sm;
-    int splits = std::max(1, target / std::max(1, pairs));
+    int splits = std::min(256, std::max(1, target / std::max(1, pairs)));
     int chunk = (pl.max_kv + splits - 1) / splits;
     chunk = ((chunk + 127) / 128) * 128;
     splits = (pl.max_kv + chunk - 1) / chunk;

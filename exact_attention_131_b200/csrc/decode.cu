@@ -1,25 +1,29 @@
 // decode.cu -- multi-sequence decode over a unified q8_0 / q4_0 KV cache.
 //
-// The quantised K/V blocks are never converted as a whole: each warp copies the
-// raw bytes of a 32-key tile into shared memory (cp.async) and dequantises them
-// into tensor-core fragments in registers right before each mma.sync
-// ("unsloth llama.cpp: dequantize q4_0/q8_0 K/V tiles in the FA MMA kernel",
-// summary: tiles are dequantised as they are loaded instead of a whole-cache
-// f16 conversion per layer per step).
+// The quantised K/V blocks are never converted as a whole: each CTA copies the
+// raw bytes of a 64-key tile into shared memory (cp.async, two stages in
+// flight), and one cooperative pass turns that tile into f16 right before the
+// tensor cores read it ("unsloth llama.cpp: dequantize q4_0/q8_0 K/V tiles in
+// the FA MMA kernel", summary: tiles are dequantised as they are loaded
+// instead of a whole-cache f16 conversion per layer per step).  Each element
+// is dequantised exactly once; the f16 tile is read with ldmatrix (K) and
+// ldmatrix.trans (V) into mma.sync fragments.
 //
 // Work split.  For one sequence and one kv head the g query heads x n_q new
 // tokens fold into M = g*n_q <= 16 rows (fold row r = rep*n_q + t, query head
 // kv*g + rep), one m16n8k16 tile high.  The sequence's cells are cut into
-// `splits` chunks; one CTA of 4 warps takes one (sequence, kv head, chunk), each
-// warp walking 32-key tiles of the chunk with its own online softmax.  The CTA
-// merges its warps and writes one partial (max, sum, unnormalised O) per row;
-// a second kernel merges the chunks by their log-sum-exp weights (the output
-// merge of "TransformerEngine: FA4 in context-parallel attention", flowchart).
+// `splits` chunks; one CTA of 4 warps takes one (sequence, kv head, chunk),
+// each warp taking 16 keys of every 64-key tile with its own online softmax.
+// The CTA merges its warps and writes one partial (max, sum, unnormalised O)
+// per row; a second kernel, launched as a programmatic dependent of the first,
+// merges the chunks by their log-sum-exp weights (the output merge of
+// "TransformerEngine: FA4 in context-parallel attention", flowchart).
 //
 // Scores are kept in log2 units: Q is pre-multiplied by scale*log2(e) before it
 // is rounded to f16.  Integer -> f16 conversion places the byte or nibble in
 // the mantissa of 1024.0 (0x6400) and subtracts the offset, which is exact for
-// every value a q8_0 byte or q4_0 nibble can hold.
+// every value a q8_0 byte or q4_0 nibble can hold; the block scale multiplies
+// afterwards.
 #include <math.h>
 
 #include "internal.h"
@@ -29,7 +33,7 @@ namespace arc {
 namespace {
 
 constexpr int WARPS = 4;
-constexpr int SUB = 32;  // keys per warp step
+constexpr int DT = 64;             // keys per CTA tile (16 per warp)
 constexpr float LN2 = 0.6931471805599453f;
 
 template <int KVT>
@@ -43,6 +47,18 @@ struct Fmt<ARC_KV_Q4_0> {
     static constexpr int BB = 18;
 };
 
+template <int KVT, int D>
+struct DecLayout {
+    static constexpr int ROWB = (D / 32) * Fmt<KVT>::BB;       // raw bytes of one head row
+    static constexpr int RAW = DT * ROWB;                      // raw bytes of one K (or V) tile
+    static constexpr int HSTRIDE = D + 8;                      // f16 tile row stride (elements), breaks bank conflicts
+    static constexpr int HBYTES = DT * HSTRIDE * 2;
+    static constexpr int MERGE = WARPS * 16 * (D + 2) * 4;
+    static constexpr int MAIN = 2 * 2 * RAW + 2 * HBYTES;      // 2 stages x (K,V) raw + f16 K,V
+    static constexpr int BYTES = MAIN > MERGE ? MAIN : MERGE;
+    static constexpr int PIECE = (ROWB % 8 == 0) ? 8 : 4;      // cp.async granule
+};
+
 ARC_DEV void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
     asm volatile(
@@ -52,109 +68,101 @@ ARC_DEV void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+ARC_DEV void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
+ARC_DEV void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+
 ARC_DEV uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t *>(&h); }
 ARC_DEV __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2 *>(&u); }
 
-// Bytes 0 and 1 of x (signed int8) -> half2 of the same integers.
-ARC_DEV __half2 s8x2_to_h2(uint32_t x)
+ARC_DEV uint32_t lds_u32(const uint8_t *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+// Four signed bytes of w -> two half2 of the same integers (exact).
+ARC_DEV void s8x4_to_h2x2(uint32_t w, __half2 &lo, __half2 &hi)
 {
-    const uint32_t v = __byte_perm(x ^ 0x8080u, 0x64646464u, 0x4140u);
-    return __hsub2(bits_h2(v), bits_h2(0x64806480u));  // 1024 + 128
+    const uint32_t t = w ^ 0x80808080u;
+    lo = __hsub2(bits_h2(__byte_perm(t, 0x64646464u, 0x4140u)), bits_h2(0x64806480u));  // 1024 + 128
+    hi = __hsub2(bits_h2(__byte_perm(t, 0x64646464u, 0x4342u)), bits_h2(0x64806480u));
 }
 
-// Bytes 0 and 1 of x, each holding a value 0..15 -> half2 of (n - 8).
-ARC_DEV __half2 u4x2_to_h2(uint32_t x)
+// Four values 0..15 (one per byte of w) -> two half2 of (n - 8) (exact).
+ARC_DEV void u4x4_to_h2x2(uint32_t w, __half2 &lo, __half2 &hi)
 {
-    const uint32_t v = __byte_perm(x, 0x64646464u, 0x4140u);
-    return __hsub2(bits_h2(v), bits_h2(0x64086408u));  // 1024 + 8
+    lo = __hsub2(bits_h2(__byte_perm(w, 0x64646464u, 0x4140u)), bits_h2(0x64086408u));  // 1024 + 8
+    hi = __hsub2(bits_h2(__byte_perm(w, 0x64646464u, 0x4342u)), bits_h2(0x64086408u));
 }
 
-ARC_DEV uint32_t lds_u16(const uint8_t *p) { return *reinterpret_cast<const uint16_t *>(p); }
-ARC_DEV __half lds_h(const uint8_t *p) { return *reinterpret_cast<const __half *>(p); }
+// Eight bytes starting at byte offset `off` of a 4-byte-aligned row, as two words.
+// Blocks are 34 or 18 bytes, so `off` is 2 mod 4 for even blocks: three aligned
+// loads and a byte permute realign it without a branch.
+ARC_DEV void ld8_unaligned(const uint8_t *row, int off, uint32_t &a, uint32_t &b)
+{
+    const uint8_t *base = row + (off & ~3);
+    const uint32_t w0 = lds_u32(base), w1 = lds_u32(base + 4), w2 = lds_u32(base + 8);
+    const uint32_t sel = (off & 2) ? 0x5432u : 0x3210u;
+    a = __byte_perm(w0, w1, sel);
+    b = __byte_perm(w1, w2, sel);
+}
 
-// K fragment (B operand of S = Q K^T): key row `row`, dims ks*16 + {2tq,2tq+1} and +8.
+// Dequantise 8 consecutive elements (group grp = dims 8*grp .. 8*grp+7) of one raw
+// head row into four half2 words.
 template <int KVT>
-ARC_DEV void k_frag(const uint8_t *row, int ks, int tq, uint32_t &b0, uint32_t &b1)
+ARC_DEV uint4 dequant8(const uint8_t *row, int grp)
 {
-    const int blk = ks >> 1;
-    const uint8_t *bp = row + blk * Fmt<KVT>::BB;
-    const __half2 sc = __half2half2(lds_h(bp));
+    const int blk = grp >> 2, e0 = (grp & 3) * 8;
+    const int boff = blk * Fmt<KVT>::BB;
+    const __half2 sc = __half2half2(*reinterpret_cast<const __half *>(row + boff));
+    uint32_t a, b;
+    __half2 h0, h1, h2, h3;
     if constexpr (KVT == ARC_KV_Q8_0) {
-        const int e0 = (ks & 1) * 16 + 2 * tq;
-        b0 = h2_bits(__hmul2(s8x2_to_h2(lds_u16(bp + 2 + e0)), sc));
-        b1 = h2_bits(__hmul2(s8x2_to_h2(lds_u16(bp + 2 + e0 + 8)), sc));
+        ld8_unaligned(row, boff + 2 + e0, a, b);
+        s8x4_to_h2x2(a, h0, h1);
+        s8x4_to_h2x2(b, h2, h3);
     } else {
-        const uint32_t x0 = lds_u16(bp + 2 + 2 * tq), x1 = lds_u16(bp + 2 + 2 * tq + 8);
-        const int sh = (ks & 1) * 4;  // elements 16..31 sit in the high nibbles
-        b0 = h2_bits(__hmul2(u4x2_to_h2((x0 >> sh) & 0x0F0Fu), sc));
-        b1 = h2_bits(__hmul2(u4x2_to_h2((x1 >> sh) & 0x0F0Fu), sc));
+        // elements 0..15 are the low nibbles of bytes 0..15, elements 16..31 the high ones
+        ld8_unaligned(row, boff + 2 + (e0 & 15), a, b);
+        const int sh = e0 >= 16 ? 4 : 0;
+        u4x4_to_h2x2((a >> sh) & 0x0F0F0F0Fu, h0, h1);
+        u4x4_to_h2x2((b >> sh) & 0x0F0F0F0Fu, h2, h3);
     }
-}
-
-// One dequantised element d of a row, as raw integer byte (in bits 0..7) and scale.
-template <int KVT>
-ARC_DEV uint32_t v_code(const uint8_t *row, int d)
-{
-    const uint8_t *bp = row + (d >> 5) * Fmt<KVT>::BB;
-    const int e = d & 31;
-    if constexpr (KVT == ARC_KV_Q8_0) {
-        return bp[2 + e];
-    } else {
-        const uint32_t byte = bp[2 + (e & 15)];
-        return (e < 16) ? (byte & 15u) : (byte >> 4);
-    }
-}
-
-template <int KVT>
-ARC_DEV __half v_scale(const uint8_t *row, int d)
-{
-    return lds_h(row + (d >> 5) * Fmt<KVT>::BB);
-}
-
-// V fragment (B operand of O += P V): keys k0, k0+1 (b0) and k0+8, k0+9 (b1), dim d.
-template <int KVT>
-ARC_DEV void v_frag(const uint8_t *sv, int rowb, int k0, int d, uint32_t &b0, uint32_t &b1)
-{
-    const uint8_t *r0 = sv + (k0)*rowb, *r1 = sv + (k0 + 1) * rowb;
-    const uint8_t *r8 = sv + (k0 + 8) * rowb, *r9 = sv + (k0 + 9) * rowb;
-    const uint32_t x01 = v_code<KVT>(r0, d) | (v_code<KVT>(r1, d) << 8);
-    const uint32_t x89 = v_code<KVT>(r8, d) | (v_code<KVT>(r9, d) << 8);
-    const __half2 s01 = __halves2half2(v_scale<KVT>(r0, d), v_scale<KVT>(r1, d));
-    const __half2 s89 = __halves2half2(v_scale<KVT>(r8, d), v_scale<KVT>(r9, d));
-    if constexpr (KVT == ARC_KV_Q8_0) {
-        b0 = h2_bits(__hmul2(s8x2_to_h2(x01), s01));
-        b1 = h2_bits(__hmul2(s8x2_to_h2(x89), s89));
-    } else {
-        b0 = h2_bits(__hmul2(u4x2_to_h2(x01), s01));
-        b1 = h2_bits(__hmul2(u4x2_to_h2(x89), s89));
-    }
+    return make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)), h2_bits(__hmul2(h2, sc)),
+                      h2_bits(__hmul2(h3, sc)));
 }
 
 template <int BYTES>
-ARC_DEV void cp_async(void *dst, const void *src)
+ARC_DEV void cp_async_n(void *dst, const void *src)
 {
     asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(smem_u32(dst)), "l"(src), "n"(BYTES) : "memory");
 }
-ARC_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
-ARC_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+ARC_DEV void cp_async_wait_n() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int KVT, int D>
 __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_constant__ DecodeParams p)
 {
-    constexpr int ROWB = (D / 32) * Fmt<KVT>::BB;   // bytes of one head row
-    constexpr int TILE = SUB * ROWB;                 // bytes of one 32-key raw tile
-    constexpr int KS = D / 16;                       // k-steps of S
-    constexpr int NT_O = D / 8;                      // n-tiles of O
-    constexpr int PIECE = (ROWB % 8 == 0) ? 8 : 4;   // cp.async granule (rows are 4-byte multiples)
-    static_assert(ROWB % 4 == 0, "rows are copied in 4- or 8-byte pieces");
+    using L = DecLayout<KVT, D>;
+    constexpr int KS = D / 16;    // k-steps of S
+    constexpr int NT_O = D / 8;   // n-tiles of O
 
     extern __shared__ __align__(16) uint8_t smem[];
+    uint8_t *raw = smem;                                   // [2 stages][K, V][RAW]
+    __half *kh = reinterpret_cast<__half *>(smem + 4 * L::RAW);
+    __half *vh = kh + DT * L::HSTRIDE;
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
 
-    const int per_seq = p.Hkv * p.splits;
-    const int s = blockIdx.x / per_seq;
+    const int s = blockIdx.x / (p.Hkv * p.splits);
     const int kvh = (blockIdx.x / p.splits) % p.Hkv;
     const int sp = blockIdx.x % p.splits;
     const arc_seq sq = p.seqs[s];
@@ -166,7 +174,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
 
     // ---- Q fragments (16 rows x D), pre-scaled into log2 units, f16
     uint32_t qa[KS][4];
-    int row_t[2];  // token index within the sequence for rows g and g+8 (-1: padding row)
+    int row_t[2];
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
         const int r = g + 8 * hr;
@@ -175,16 +183,16 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
-        for (int part_i = 0; part_i < 4; ++part_i) {
-            const int r = g + 8 * (part_i & 1);
-            const int d = ks * 16 + 2 * tq + 8 * (part_i >> 1);
+        for (int pi = 0; pi < 4; ++pi) {
+            const int r = g + 8 * (pi & 1);
+            const int d = ks * 16 + 2 * tq + 8 * (pi >> 1);
             float2 v = make_float2(0.f, 0.f);
             if (r < M) {
                 const int h = kvh * G + r / sq.n_q;
                 const int tok = sq.q_begin + r % sq.n_q;
                 v = *reinterpret_cast<const float2 *>(p.q + ((int64_t)tok * p.H + h) * D + d);
             }
-            qa[ks][part_i] = h2_bits(__floats2half2_rn(v.x * p.scale_log2, v.y * p.scale_log2));
+            qa[ks][pi] = h2_bits(__floats2half2_rn(v.x * p.scale_log2, v.y * p.scale_log2));
         }
     }
 
@@ -193,52 +201,67 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
     for (int i = 0; i < NT_O; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
 
-    uint8_t *wbuf = smem + warp * (4 * TILE);  // [stage 2][K,V] tiles of this warp
-    const int n_steps = c_end > c_begin ? (c_end - c_begin + SUB - 1) / SUB : 0;
-    const int my_steps = n_steps > warp ? (n_steps - warp + WARPS - 1) / WARPS : 0;
-    const uint8_t *kbase = p.k_cache + (int64_t)kvh * ROWB;
-    const uint8_t *vbase = p.v_cache + (int64_t)kvh * ROWB;
-    const int64_t cell_stride = (int64_t)p.Hkv * ROWB;
+    const int n_tiles = c_end > c_begin ? (c_end - c_begin + DT - 1) / DT : 0;
+    const uint8_t *kbase = p.k_cache + (int64_t)kvh * L::ROWB;
+    const uint8_t *vbase = p.v_cache + (int64_t)kvh * L::ROWB;
+    const int64_t cell_stride = (int64_t)p.Hkv * L::ROWB;
 
-    auto issue = [&](int i, int stage) {
-        const int key0 = c_begin + (warp + i * WARPS) * SUB;
-        uint8_t *dk = wbuf + stage * 2 * TILE;
-        uint8_t *dv = dk + TILE;
-        for (int x = lane; x < SUB * (ROWB / PIECE); x += 32) {
-            const int kr = x / (ROWB / PIECE), off = (x % (ROWB / PIECE)) * PIECE;
-            const int key = min(key0 + kr, c_end - 1);  // rows past the chunk repeat a valid row; masked
-            const int64_t cell = sq.kv_begin + key;
-            cp_async<PIECE>(dk + kr * ROWB + off, kbase + cell * cell_stride + off);
-            cp_async<PIECE>(dv + kr * ROWB + off, vbase + cell * cell_stride + off);
+    auto issue = [&](int i) {
+        uint8_t *dk = raw + (i & 1) * 2 * L::RAW;
+        uint8_t *dv = dk + L::RAW;
+        const int key0 = c_begin + i * DT;
+        constexpr int PR = L::ROWB / L::PIECE;  // pieces per row (<= 32): one lane each
+        static_assert(PR <= 32, "a head row must fit one warp instruction");
+        if (lane < PR) {
+            const int off = lane * L::PIECE;
+#pragma unroll 4
+            for (int kr = warp; kr < DT; kr += WARPS) {
+                const int key = min(key0 + kr, c_end - 1);  // rows past the chunk repeat a valid row; masked
+                const int64_t cell = sq.kv_begin + key;
+                cp_async_n<L::PIECE>(dk + kr * L::ROWB + off, kbase + cell * cell_stride + off);
+                cp_async_n<L::PIECE>(dv + kr * L::ROWB + off, vbase + cell * cell_stride + off);
+            }
         }
-        cp_async_commit();
+        asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
-    if (my_steps > 0) issue(0, 0);
-    for (int i = 0; i < my_steps; ++i) {
-        const int stage = i & 1;
-        if (i + 1 < my_steps) {
-            issue(i + 1, stage ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+    if (n_tiles > 0) issue(0);
+    if (n_tiles > 1) issue(1);
+    const uint32_t kh_s = smem_u32(kh), vh_s = smem_u32(vh);
+    for (int i = 0; i < n_tiles; ++i) {
+        if (i + 1 < n_tiles)
+            cp_async_wait_n<1>();
+        else
+            cp_async_wait_n<0>();
+        __syncthreads();  // raw tile i visible; every warp is done with the f16 tiles of tile i-1
+        {
+            const uint8_t *rk = raw + (i & 1) * 2 * L::RAW;
+            const uint8_t *rv = rk + L::RAW;
+            constexpr int GROUPS = DT * (D / 8);
+#pragma unroll 2
+            for (int x = threadIdx.x; x < GROUPS; x += WARPS * 32) {
+                const int r = x / (D / 8), grp = x % (D / 8);  // D / 8 is a power of two
+                *reinterpret_cast<uint4 *>(kh + r * L::HSTRIDE + grp * 8) = dequant8<KVT>(rk + r * L::ROWB, grp);
+                *reinterpret_cast<uint4 *>(vh + r * L::HSTRIDE + grp * 8) = dequant8<KVT>(rv + r * L::ROWB, grp);
+            }
         }
-        __syncwarp();
-        const uint8_t *sk = wbuf + stage * 2 * TILE;
-        const uint8_t *sv = sk + TILE;
-        const int key0 = c_begin + (warp + i * WARPS) * SUB;
+        __syncthreads();  // f16 tiles ready; raw stage (i & 1) is free again
+        if (i + 2 < n_tiles) issue(i + 2);
 
-        // ---- S = Q K^T for 32 keys: 4 n-tiles of 8 keys
-        float sacc[4][4];
+        const int kw = warp * 16;                      // this warp's 16 keys of the tile
+        const int key0 = c_begin + i * DT + kw;
+        // ---- S = Q K^T, 16 rows x 16 keys (two n-tiles of 8)
+        float sacc[2][4];
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
+        for (int nt = 0; nt < 2; ++nt) {
             sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-            const uint8_t *krow = sk + (nt * 8 + g) * ROWB;
+            const int krow = kw + nt * 8 + (lane & 7);
 #pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                uint32_t b0, b1;
-                k_frag<KVT>(krow, ks, tq, b0, b1);
+            for (int ks = 0; ks < KS; ks += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kh_s + (krow * L::HSTRIDE + ks * 16 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
                 mma16816(sacc[nt], qa[ks], b0, b1);
+                mma16816(sacc[nt], qa[ks + 1], b2, b3);
             }
         }
         // ---- mask: key index vs. the chunk end and each row's causal limit
@@ -246,7 +269,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
         for (int hr = 0; hr < 2; ++hr) {
             const int lim = row_t[hr] < 0 ? -1 : sq.n_kv - sq.n_q + row_t[hr];
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     const int key = key0 + nt * 8 + 2 * tq + e;
@@ -254,51 +277,38 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
                 }
         }
         // ---- online softmax for rows g and g+8 (a row is spread over the 4 lanes of a quad)
-        uint32_t pa[2][4];
+        uint32_t pa[4];
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) mx = fmaxf(mx, fmaxf(sacc[nt][2 * hr], sacc[nt][2 * hr + 1]));
+            float mx = fmaxf(fmaxf(sacc[0][2 * hr], sacc[0][2 * hr + 1]), fmaxf(sacc[1][2 * hr], sacc[1][2 * hr + 1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             const float m_new = fmaxf(m_r[hr], mx);
             const float msafe = (m_new == -INFINITY) ? 0.f : m_new;
             const float alpha = (m_r[hr] == -INFINITY) ? 0.f : fast_exp2(m_r[hr] - msafe);
             m_r[hr] = m_new;
-            float rs = 0.f;
-            float pv[4][2];
+            const float p00 = fast_exp2(sacc[0][2 * hr] - msafe), p01 = fast_exp2(sacc[0][2 * hr + 1] - msafe);
+            const float p10 = fast_exp2(sacc[1][2 * hr] - msafe), p11 = fast_exp2(sacc[1][2 * hr + 1] - msafe);
+            l_r[hr] = l_r[hr] * alpha + (p00 + p01 + p10 + p11);
+            if (alpha != 1.f) {
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    pv[nt][e] = fast_exp2(sacc[nt][2 * hr + e] - msafe);
-                    rs += pv[nt][e];
+                for (int i2 = 0; i2 < NT_O; ++i2) {
+                    o[i2][2 * hr] *= alpha;
+                    o[i2][2 * hr + 1] *= alpha;
                 }
-            l_r[hr] = l_r[hr] * alpha + rs;
-#pragma unroll
-            for (int i2 = 0; i2 < NT_O; ++i2) {
-                o[i2][2 * hr] *= alpha;
-                o[i2][2 * hr + 1] *= alpha;
             }
-            // A fragments of P for the two 16-key k-steps
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-                pa[kk][hr] = h2_bits(__floats2half2_rn(pv[2 * kk][0], pv[2 * kk][1]));
-                pa[kk][2 + hr] = h2_bits(__floats2half2_rn(pv[2 * kk + 1][0], pv[2 * kk + 1][1]));
-            }
+            pa[hr] = h2_bits(__floats2half2_rn(p00, p01));       // row g / g+8, keys 2tq..  (n-tile 0)
+            pa[2 + hr] = h2_bits(__floats2half2_rn(p10, p11));   // keys 8 + 2tq..           (n-tile 1)
         }
-        // ---- O += P V
+        // ---- O += P V: V fragments by ldmatrix.trans from the f16 tile
+        const int vrow = kw + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-#pragma unroll
-            for (int nd = 0; nd < NT_O; ++nd) {
-                uint32_t b0, b1;
-                v_frag<KVT>(sv, ROWB, kk * 16 + 2 * tq, nd * 8 + g, b0, b1);
-                mma16816(o[nd], pa[kk], b0, b1);
-            }
+        for (int nd = 0; nd < NT_O; nd += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vh_s + (vrow * L::HSTRIDE + nd * 8 + (lane >> 4) * 8) * 2, b0, b1, b2, b3);
+            mma16816(o[nd], pa, b0, b1);
+            mma16816(o[nd + 1], pa, b2, b3);
         }
-        __syncwarp();
     }
 
     // ---- merge the 4 warps of this CTA in shared memory
@@ -307,7 +317,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
         l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 1);
         l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 2);
     }
-    __syncthreads();  // all warps are done with their raw tiles
+    __syncthreads();
     float *so = reinterpret_cast<float *>(smem);       // [WARPS][16][D]
     float *sml = so + WARPS * 16 * D;                   // [WARPS][16][2]
 #pragma unroll
@@ -346,6 +356,8 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
             p.ws_ml[(part * 16 + r) * 2 + 1] = ll;
         }
     }
+    // Let the merge kernel start its prologue; it waits for this grid's writes.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Merge the chunk partials of one (sequence, kv head, fold row) by their
@@ -353,6 +365,8 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant__ DecodeParams p)
 {
+    __shared__ float s_w[256];     // per-split weight exp2(m_sp - m)
+    __shared__ float s_red[2];
     const int s = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv, r = blockIdx.y;
     const arc_seq sq = p.seqs[s];
     const int G = p.H / p.Hkv;
@@ -360,17 +374,26 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
     const int h = kvh * G + r / sq.n_q, tok = sq.q_begin + r % sq.n_q;
     const int d = threadIdx.x;
     const int64_t part0 = ((int64_t)s * p.Hkv + kvh) * p.splits;
-    float mm = -INFINITY;
-    for (int sp = 0; sp < p.splits; ++sp) mm = fmaxf(mm, p.ws_ml[((part0 + sp) * 16 + r) * 2]);
-    const float ms = (mm == -INFINITY) ? 0.f : mm;
-    float acc = 0.f, ll = 0.f;
-    for (int sp = 0; sp < p.splits; ++sp) {
-        const float mw = p.ws_ml[((part0 + sp) * 16 + r) * 2];
-        if (mw == -INFINITY) continue;
-        const float f = exp2f(mw - ms);
-        acc += f * p.ws_o[((part0 + sp) * 16 + r) * D + d];
-        ll += f * p.ws_ml[((part0 + sp) * 16 + r) * 2 + 1];
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the split kernel are complete
+    if (d == 0) {
+        float mm = -INFINITY;
+        for (int sp = 0; sp < p.splits; ++sp) mm = fmaxf(mm, p.ws_ml[((part0 + sp) * 16 + r) * 2]);
+        const float ms = (mm == -INFINITY) ? 0.f : mm;
+        float ll = 0.f;
+        for (int sp = 0; sp < p.splits; ++sp) {
+            const float mw = p.ws_ml[((part0 + sp) * 16 + r) * 2];
+            const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - ms);
+            s_w[sp] = f;
+            ll += f * p.ws_ml[((part0 + sp) * 16 + r) * 2 + 1];
+        }
+        s_red[0] = mm;
+        s_red[1] = ll;
     }
+    __syncthreads();
+    const float mm = s_red[0], ll = s_red[1];
+    float acc = 0.f;
+#pragma unroll 4
+    for (int sp = 0; sp < p.splits; ++sp) acc += s_w[sp] * p.ws_o[((part0 + sp) * 16 + r) * D + d];
     p.o[((int64_t)tok * p.H + h) * D + d] = ll > 0.f ? acc / ll : 0.f;
     if (d == 0) p.lse[(int64_t)tok * p.H + h] = ll > 0.f ? (mm + log2f(ll)) * LN2 : -INFINITY;
 }
@@ -378,33 +401,40 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
 template <int KVT, int D>
 cudaError_t launch_t(const DecodeParams &p, cudaStream_t s)
 {
-    constexpr int ROWB = (D / 32) * Fmt<KVT>::BB;
-    const int tiles = WARPS * 4 * SUB * ROWB;
-    const int merge = WARPS * 16 * (D + 2) * 4;
-    const int smem = tiles > merge ? tiles : merge;
+    using L = DecLayout<KVT, D>;
     auto k1 = decode_split_kernel<KVT, D>;
-    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
     const int grid = p.n_seq * p.Hkv * p.splits;
     if (grid == 0) return cudaSuccess;
-    k1<<<grid, WARPS * 32, smem, s>>>(p);
+    k1<<<grid, WARPS * 32, L::BYTES, s>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    decode_combine_kernel<D><<<dim3(p.n_seq * p.Hkv, 16), D, 0, s>>>(p);
-    return cudaGetLastError();
+    // The merge launches as a programmatic dependent: its launch overlaps the
+    // split kernel's tail and it waits (griddepcontrol.wait) for the partials.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.n_seq * p.Hkv, 16);
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
 }
 
 }  // namespace
 
 int decode_smem_bytes(int kv_type, int D)
 {
-    const int bb = kv_type == ARC_KV_Q8_0 ? 34 : 18;
-    const int tiles = WARPS * 4 * SUB * (D / 32) * bb;
-    const int merge = WARPS * 16 * (D + 2) * 4;
-    return tiles > merge ? tiles : merge;
+    if (kv_type == ARC_KV_Q8_0) return D == 64 ? DecLayout<ARC_KV_Q8_0, 64>::BYTES : DecLayout<ARC_KV_Q8_0, 128>::BYTES;
+    return D == 64 ? DecLayout<ARC_KV_Q4_0, 64>::BYTES : DecLayout<ARC_KV_Q4_0, 128>::BYTES;
 }
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s)
 {
+    if (p.splits > 256) return cudaErrorInvalidValue;
     if (p.kv_type == ARC_KV_Q8_0) {
         if (p.D == 64) return launch_t<ARC_KV_Q8_0, 64>(p, s);
         if (p.D == 128) return launch_t<ARC_KV_Q8_0, 128>(p, s);
