@@ -108,7 +108,7 @@ bool tma_strides_ok(std::initializer_list<int64_t> strides_el)
 }
 
 // Tile order: heavier tiles (more KV tiles under the causal mask) first.
-void order_tiles(TcParams &p, int n_tiles)
+void order_tiles(TcParams &p, int n_tiles, int rows_per_item = kTcBM)
 {
     if (n_tiles > 1024) {
         for (int i = 0; i < 1024; ++i) p.tile_order[i] = (uint16_t)i;
@@ -117,7 +117,7 @@ void order_tiles(TcParams &p, int n_tiles)
     std::vector<std::pair<int, int>> w(n_tiles);
     const int rows = p.G * p.Tq;
     for (int t = 0; t < n_tiles; ++t) {
-        const int r0 = t * kTcBM, r_last = std::min(r0 + kTcBM, rows) - 1;
+        const int r0 = t * rows_per_item, r_last = std::min(r0 + rows_per_item, rows) - 1;
         const int t_max = (r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
         const int last = p.causal ? std::min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
         w[t] = {last < 0 ? 0 : last / kTcBN + 1, t};
@@ -163,8 +163,34 @@ enum class Path { None, Simple, Tc };
 
 struct AttnPlan {
     Path path = Path::None;
+    bool two = false;  // two query tiles per CTA (d_v <= 128)
     int dvs = 0, n_slices = 0, n_tiles = 0, grid = 0, stages = 0;
 };
+
+bool tc2_pair_supported(int dqk, int dvs, bool mla)
+{
+    static const int dense[][2] = {{64, 64}, {128, 64}, {128, 128}, {192, 128}, {256, 128}};
+    static const int mlas[][2] = {{128, 128}, {192, 128}, {192, 64}, {256, 128}};
+    if (mla) {
+        for (auto &x : mlas)
+            if (x[0] == dqk && x[1] == dvs) return true;
+    } else {
+        for (auto &x : dense)
+            if (x[0] == dqk && x[1] == dvs) return true;
+    }
+    return false;
+}
+
+// Switch a planned one-tile launch to the two-tile kernel when it applies.
+void maybe_two(AttnPlan &pl, int dqk, bool mla, int groups)
+{
+    if (pl.dvs > 128 || pl.n_slices != 1 || !tc2_pair_supported(dqk, pl.dvs, mla)) return;
+    const int st = tc2_max_stages(dqk);
+    if (st < dqk / 64 + pl.dvs / 64) return;
+    pl.two = true;
+    pl.stages = st;
+    pl.grid = ((pl.n_tiles + 1) / 2) * groups;
+}
 
 AttnPlan plan_attn(const arc_attn_args *a)
 {
@@ -192,6 +218,7 @@ AttnPlan plan_attn(const arc_attn_args *a)
     pl.n_tiles = (a->H / a->Hkv * a->Tq + kTcBM - 1) / kTcBM;
     pl.grid = pl.n_tiles * a->B * a->Hkv * pl.n_slices;
     pl.stages = tc_max_stages(a->D);
+    maybe_two(pl, a->D, false, a->B * a->Hkv);
     return pl;
 }
 
@@ -251,6 +278,7 @@ AttnPlan plan_mla(const arc_mla_args *a)
     pl.n_tiles = (a->Tq + kTcBM - 1) / kTcBM;
     pl.grid = pl.n_tiles * a->B * a->H;
     pl.stages = tc_max_stages(dqk);
+    maybe_two(pl, dqk, true, a->B * a->H);
     return pl;
 }
 
@@ -390,9 +418,15 @@ arc_status arc_attn_fwd(const arc_attn_args *a, void *stream)
         for (int i = 0; i < 3; ++i) p.os[i] = a->o_strides[i];
         p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = a->scale * kLog2e, p.causal = a->causal;
         p.status = a->status;
-        order_tiles(p, pl.n_tiles);
-        note_dispatch("tc_attn_kernel");
-        e = launch_tc_attn(p, a->D, pl.dvs, false, pl.grid, s);
+        if (pl.two) {
+            order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
+            note_dispatch("tc_attn2_kernel");
+            e = launch_tc_attn2(p, a->D, pl.dvs, false, pl.grid, s);
+        } else {
+            order_tiles(p, pl.n_tiles);
+            note_dispatch("tc_attn_kernel");
+            e = launch_tc_attn(p, a->D, pl.dvs, false, pl.grid, s);
+        }
     }
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
@@ -447,9 +481,15 @@ arc_status arc_mla_fwd(const arc_mla_args *a, void *stream)
         for (int i = 0; i < 3; ++i) p.os[i] = a->o_strides[i];
         p.lse = a->lse, p.sinks = nullptr, p.scale_log2 = a->scale * kLog2e, p.causal = a->causal;
         p.status = a->status;
-        order_tiles(p, pl.n_tiles);
-        note_dispatch("tc_attn_kernel<mla>");
-        e = launch_tc_attn(p, a->Dn + a->Dr, a->Dv, true, pl.grid, s);
+        if (pl.two) {
+            order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
+            note_dispatch("tc_attn2_kernel<mla>");
+            e = launch_tc_attn2(p, a->Dn + a->Dr, a->Dv, true, pl.grid, s);
+        } else {
+            order_tiles(p, pl.n_tiles);
+            note_dispatch("tc_attn_kernel<mla>");
+            e = launch_tc_attn(p, a->Dn + a->Dr, a->Dv, true, pl.grid, s);
+        }
     }
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
@@ -583,10 +623,11 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             out->tile_m = 4;
             out->n_ctas = (int)(((int64_t)a->B * a->H * a->Tq + 3) / 4);
         } else {
-            set_name(out, "tc_attn_kernel");
+            set_name(out, pl.two ? "tc_attn2_kernel" : "tc_attn_kernel");
             out->tensor_cores = 1;
-            out->tile_m = kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
-            out->smem_bytes = tc_smem_bytes(a->D, pl.stages), out->tmem_cols = 512;
+            out->tile_m = pl.two ? 2 * kTcBM : kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
+            out->smem_bytes = pl.two ? tc2_smem_bytes(a->D, pl.stages) : tc_smem_bytes(a->D, pl.stages);
+            out->tmem_cols = 512;
         }
         out->launches = 1;
         return ARC_OK;
@@ -605,10 +646,11 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             set_name(out, "simple_attn_kernel");
             out->tile_m = 4;
         } else {
-            set_name(out, "tc_attn_kernel<mla>");
+            set_name(out, pl.two ? "tc_attn2_kernel<mla>" : "tc_attn_kernel<mla>");
             out->tensor_cores = 1;
-            out->tile_m = kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
-            out->smem_bytes = tc_smem_bytes(a->Dn + a->Dr, pl.stages), out->tmem_cols = 512;
+            out->tile_m = pl.two ? 2 * kTcBM : kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
+            out->smem_bytes = pl.two ? tc2_smem_bytes(a->Dn + a->Dr, pl.stages) : tc_smem_bytes(a->Dn + a->Dr, pl.stages);
+            out->tmem_cols = 512;
         }
         out->launches = 1;
         return ARC_OK;

@@ -388,6 +388,373 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
     }
 }
 
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA (d_v <= 128).  Tiles A and B are 128 consecutive fold
+// rows each of the same (batch, kv head) group, so every K/V tile the producer
+// brings in feeds both: half the shared-memory and L2 traffic per FLOP of the
+// one-tile kernel.  TMEM: O_A [0,128), S/P_A [128,256), O_B [256,384),
+// S/P_B [384,512).  MMA order per KV tile j (steady state):
+//     O_A += P_A(j) V(j),  S_A(j+1),  O_B += P_B(j) V(j),  S_B(j+1)
+// so softmax A(j+1) overlaps the B-side MMAs and softmax B(j+1) the A side.
+// Softmax warps 4-7 serve tile A, warps 8-11 tile B; each reads its S twice
+// (max pass, then exp pass writing P over the columns already read) to stay
+// within the register budget of 384 threads.
+constexpr int NTHREADS2 = 384;
+
+template <int DQK, int DVS, bool MLA>
+__global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_constant__ TcParams p)
+{
+    constexpr int KC = DQK / 64;
+    constexpr int VC = DVS / 64;
+    static_assert(DQK % 64 == 0 && DVS % 64 == 0 && DVS <= 128, "tile shape");
+    // TMEM columns of tile t: O at 256*t, S/P at 128 + 256*t
+#define O_COL(t) (256u * (uint32_t)(t))
+#define S_COL2(t) (128u + 256u * (uint32_t)(t))
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem;                       // [2 tiles][KC chunks]
+    uint8_t *sRing = sQ + 2 * KC * CHUNK;
+    const int R = p.stages;
+    struct Bars2 {
+        uint64_t q_full;
+        uint64_t s_full[2];
+        uint64_t p_full[2];
+        uint64_t o_done[2];
+        uint64_t drain;
+        uint64_t full[MAX_STAGES];
+        uint64_t empty[MAX_STAGES];
+        uint32_t tmem_base;
+    };
+    Bars2 *bars = reinterpret_cast<Bars2 *>(sRing + R * CHUNK);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int groups = p.B * p.Hkv;
+    const int rank = blockIdx.x / groups;
+    const int rest = blockIdx.x % groups;
+    const int kv = rest % p.Hkv;
+    const int b = rest / p.Hkv;
+    const int pair = rank < 1024 ? (int)p.tile_order[rank] : rank;
+    const int rows_in_group = p.G * p.Tq;
+    const int r0 = pair * 2 * BM;
+    int nt;  // KV tiles covering both query tiles
+    {
+        const int r_last = min(r0 + 2 * BM, rows_in_group) - 1;
+        const int t_max = (r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
+        const int kv_last = p.causal ? min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
+        nt = kv_last < 0 ? 0 : kv_last / BN + 1;
+    }
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 128);
+            mbar_init(&bars->o_done[i], 1);
+        }
+        mbar_init(&bars->drain, 1);
+        for (int i = 0; i < R; ++i) {
+            mbar_init(&bars->full[i], 1);
+            mbar_init(&bars->empty[i], 1);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // =============================== TMA producer: Q_A, Q_B, then K(0), V(0), K(1), V(1), ...
+        if (lane == 0 && nt > 0) {
+            tma_prefetch_desc(&p.tm_q);
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            const int qrow = kv * rows_in_group + r0;
+            mbar_arrive_expect_tx(&bars->q_full, 2 * KC * CHUNK);
+            for (int t = 0; t < 2; ++t)
+                for (int c = 0; c < KC; ++c) {
+                    uint8_t *dst = sQ + (t * KC + c) * CHUNK;
+                    if (!MLA || c < p.kc_first)
+                        tma_load_3d(dst, &p.tm_q, &bars->q_full, c * 64, qrow + t * BM, b);
+                    else
+                        tma_load_3d(dst, &p.tm_q2, &bars->q_full, (c - p.kc_first) * 64, qrow + t * BM, b);
+                }
+            int stage = 0, total = 0;
+            uint32_t ephase = 0;
+            bool ok = true;
+            auto acquire = [&]() -> bool {
+                if (!mbar_wait(&bars->empty[stage], ephase ^ 1u)) return false;
+                mbar_arrive_expect_tx(&bars->full[stage], CHUNK);
+                ++total;
+                return true;
+            };
+            auto advance = [&]() {
+                if (++stage == R) {
+                    stage = 0;
+                    ephase ^= 1u;
+                }
+            };
+            for (int j = 0; ok && j < nt; ++j) {
+                for (int c = 0; ok && c < KC; ++c) {
+                    if (!(ok = acquire())) break;
+                    uint8_t *dst = sRing + stage * CHUNK;
+                    if (!MLA || c < p.kc_first)
+                        tma_load_4d(dst, &p.tm_k, &bars->full[stage], c * 64, j * BN, kv, b);
+                    else
+                        tma_load_3d(dst, &p.tm_k2, &bars->full[stage], (c - p.kc_first) * 64, j * BN, b);
+                    advance();
+                }
+                for (int c = 0; ok && c < VC; ++c) {
+                    if (!(ok = acquire())) break;
+                    tma_load_4d(sRing + stage * CHUNK, &p.tm_v, &bars->full[stage], c * 64, j * BN, kv, b);
+                    advance();
+                }
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_LOAD);
+            for (int s = 0; s < R && s < total; ++s) {
+                const int loads = (total - s + R - 1) / R;
+                mbar_wait(&bars->full[s], (uint32_t)((loads - 1) & 1));
+            }
+            mbar_wait(&bars->q_full, 0);
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer
+        if (lane == 0 && nt > 0) {
+            constexpr uint32_t kChunkUnits = CHUNK >> 4;
+            const uint32_t idesc_s = idesc_bf16(BM, BN, false, false);
+            const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t kd0 = sdesc_sw128(smem_u32(sRing), 16, 1024);
+            const uint64_t vd0 = sdesc_sw128(smem_u32(sRing), CHUNK, 1024);
+            int stage = 0;
+            uint32_t fphase = 0;
+            bool ok = mbar_wait(&bars->q_full, 0);
+            tc_fence_after();
+            auto advance = [&]() {
+                if (++stage == R) {
+                    stage = 0;
+                    fphase ^= 1u;
+                }
+            };
+            // First use of the next KC (or VC) ring stages: wait for each and return the first.
+            auto take = [&](int n, int &first) -> bool {
+                first = stage;
+                for (int c = 0; c < n; ++c) {
+                    if (!mbar_wait(&bars->full[stage], fphase)) return false;
+                    advance();
+                }
+                tc_fence_after();
+                return true;
+            };
+            auto issue_s = [&](int t, int k0) {
+                const uint32_t d = tmem + S_COL2(t);
+#pragma unroll
+                for (int c = 0; c < KC; ++c)
+                    umma_ss_k64(d, qd0 + (uint64_t)((t * KC + c) * kChunkUnits),
+                                kd0 + (uint64_t)(((k0 + c) % R) * kChunkUnits), idesc_s, c > 0);
+                umma_commit(&bars->s_full[t]);
+            };
+            auto issue_pv = [&](int t, int j, int v0) {
+                const uint32_t p_tm = tmem + S_COL2(t);
+                const int n1 = (v0 + VC <= R) ? VC : R - v0;
+                const uint32_t idesc1 = idesc_bf16(BM, 64 * n1, false, true);
+#pragma unroll
+                for (int k4 = 0; k4 < BN / 64; ++k4)
+                    umma_ts_k64(tmem + O_COL(t), p_tm + k4 * 32, vd0 + (uint64_t)(v0 * kChunkUnits + k4 * 512), 128,
+                                idesc1, (j > 0) | k4);
+                if (n1 < VC) {
+                    const uint32_t idesc2 = idesc_bf16(BM, 64 * (VC - n1), false, true);
+#pragma unroll
+                    for (int k4 = 0; k4 < BN / 64; ++k4)
+                        umma_ts_k64(tmem + O_COL(t) + n1 * 64, p_tm + k4 * 32, vd0 + (uint64_t)(k4 * 512), 128, idesc2,
+                                    (j > 0) | k4);
+                }
+                umma_commit(&bars->o_done[t]);
+            };
+            auto release = [&](int first, int n) {
+                for (int c = 0; c < n; ++c) umma_commit(&bars->empty[(first + c) % R]);
+            };
+            int k0 = 0, v0 = 0;
+            if (ok) ok = take(KC, k0);
+            if (ok) {
+                issue_s(0, k0);
+                issue_s(1, k0);
+                release(k0, KC);
+            }
+            for (int j = 0; ok && j < nt; ++j) {
+                if (!(ok = take(VC, v0))) break;
+                if (!(ok = mbar_wait(&bars->p_full[0], (uint32_t)(j & 1)))) break;
+                tc_fence_after();
+                issue_pv(0, j, v0);
+                const bool more = j + 1 < nt;
+                if (more) {
+                    if (!(ok = take(KC, k0))) break;
+                    issue_s(0, k0);
+                }
+                if (!(ok = mbar_wait(&bars->p_full[1], (uint32_t)(j & 1)))) break;
+                tc_fence_after();
+                issue_pv(1, j, v0);
+                release(v0, VC);
+                if (more) {
+                    issue_s(1, k0);
+                    release(k0, KC);
+                }
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_MMA);
+            umma_commit(&bars->drain);
+            mbar_wait(&bars->drain, 0);
+        }
+    } else if (warp >= 4) {
+        // =============================== softmax (warps 4-7: tile A, 8-11: tile B) and epilogue
+        const int t = (warp - 4) >> 2;
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const int R_ = r0 + t * BM + r;
+        const bool row_ok = R_ < rows_in_group;
+        const int tpos = R_ % p.Tq;
+        const int h = kv * p.G + R_ / p.Tq;
+        const int last = p.causal ? min(p.Tk - 1, tpos + p.Tk - p.Tq) : p.Tk - 1;
+        const float sl2 = p.scale_log2;
+        const uint32_t s_tmem = tmem + lane_off + S_COL2(t);
+        const uint32_t o_tmem = tmem + lane_off + O_COL(t);
+        float m_use = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            ok = warp_all(mbar_wait(&bars->s_full[t], (uint32_t)(j & 1)));
+            if (!ok) break;
+            tc_fence_after();
+            const int kbase = j * BN;
+            const bool partial = kbase + BN - 1 > last;
+            // pass 1: row max
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t sv[32];
+                tmem_ld32(s_tmem + 32 * c, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float x = (partial && kbase + 32 * c + i > last) ? -INFINITY : __uint_as_float(sv[i]);
+                    mx = fmaxf(mx, x);
+                }
+            }
+            mx *= sl2;
+            const bool need = mx > m_use + RESCALE_THRESHOLD;
+            float alpha = 1.f;
+            if (need) {
+                alpha = (m_use == -INFINITY) ? 0.f : fast_exp2(m_use - mx);
+                m_use = mx;
+            }
+            const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
+            // pass 2: P = exp2(s*scale*log2e - m), written over S columns already read
+            float rowsum = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t sv[32], pk[16];
+                tmem_ld32(s_tmem + 32 * c, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int k0i = kbase + 32 * c + 2 * i;
+                    const float s0 = (partial && k0i > last) ? -INFINITY : __uint_as_float(sv[2 * i]);
+                    const float s1 = (partial && k0i + 1 > last) ? -INFINITY : __uint_as_float(sv[2 * i + 1]);
+                    const float p0 = fast_exp2(fmaf(s0, sl2, -msafe));
+                    const float p1 = fast_exp2(fmaf(s1, sl2, -msafe));
+                    rowsum += p0 + p1;
+                    pk[i] = pack_bf16(p0, p1);
+                }
+                tmem_st16(s_tmem + 16 * c, pk);
+            }
+            l = l * alpha + rowsum;
+            if (j > 0) {
+                ok = warp_all(mbar_wait(&bars->o_done[t], (uint32_t)((j - 1) & 1)));
+                if (!ok) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+                    for (int c = 0; c < DVS / 32; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(o_tmem + 32 * c, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                        tmem_st32(o_tmem + 32 * c, ov);
+                    }
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full[t]);
+        }
+        if (ok && nt > 0) {
+            ok = warp_all(mbar_wait(&bars->o_done[t], (uint32_t)((nt - 1) & 1)));
+            tc_fence_after();
+        }
+        if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
+        float fac, lse;
+        if (p.sinks) {
+            const float sg = row_ok ? p.sinks[h] * LOG2E : 0.f;
+            const float mf = fmaxf(m_use, sg);
+            const float a = (m_use == -INFINITY) ? 0.f : exp2f(m_use - mf);
+            const float lf = l * a + exp2f(sg - mf);
+            fac = a / lf;
+            lse = (mf + log2f(lf)) * LN2;
+        } else {
+            fac = l > 0.f ? 1.f / l : 0.f;
+            lse = l > 0.f ? (m_use + log2f(l)) * LN2 : -INFINITY;
+        }
+        __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] +
+                              (int64_t)tpos * p.os[2];
+#pragma unroll 1
+        for (int c = 0; c < DVS / 32; ++c) {
+            uint32_t ov[32];
+            if (nt > 0 && ok) {
+                tmem_ld32(o_tmem + 32 * c, ov);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) ov[i] = 0u;
+            }
+            if (row_ok) {
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack_bf16(__uint_as_float(ov[2 * i]) * fac, __uint_as_float(ov[2 * i + 1]) * fac);
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+        if (row_ok) p.lse[((int64_t)b * p.H + h) * p.Tq + tpos] = lse;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+#undef O_COL
+#undef S_COL2
+
+template <int DQK, int DVS, bool MLA>
+cudaError_t launch_two(const TcParams &p, int grid, cudaStream_t s)
+{
+    const int smem = tc2_smem_bytes(DQK, p.stages);
+    auto kern = tc_attn2_kernel<DQK, DVS, MLA>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, NTHREADS2, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
 template <int DQK, int DVS, bool MLA>
 cudaError_t launch_one(const TcParams &p, int grid, cudaStream_t s)
 {
@@ -400,6 +767,31 @@ cudaError_t launch_one(const TcParams &p, int grid, cudaStream_t s)
 }
 
 }  // namespace
+
+int tc2_smem_bytes(int dqk, int stages) { return 1024 + (2 * (dqk / 64) + stages) * CHUNK + 512; }
+
+int tc2_max_stages(int dqk)
+{
+    int st = (SMEM_LIMIT - 1024 - 512 - 2 * (dqk / 64) * CHUNK) / CHUNK;
+    return st < MAX_STAGES ? st : MAX_STAGES;
+}
+
+cudaError_t launch_tc_attn2(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s)
+{
+#define ARC_TC2_CASE(Q, V, M) \
+    if (dqk == Q && dvs == V && mla == M) return launch_two<Q, V, M>(p, grid, s);
+    ARC_TC2_CASE(64, 64, false)
+    ARC_TC2_CASE(128, 64, false)
+    ARC_TC2_CASE(128, 128, false)
+    ARC_TC2_CASE(192, 128, false)
+    ARC_TC2_CASE(256, 128, false)
+    ARC_TC2_CASE(128, 128, true)
+    ARC_TC2_CASE(192, 128, true)
+    ARC_TC2_CASE(192, 64, true)
+    ARC_TC2_CASE(256, 128, true)
+#undef ARC_TC2_CASE
+    return cudaErrorInvalidValue;
+}
 
 int tc_smem_bytes(int dqk, int stages) { return 1024 + (dqk / 64 + stages) * CHUNK + (int)sizeof(Bars); }
 

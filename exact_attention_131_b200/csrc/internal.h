@@ -66,6 +66,10 @@ struct TcParams {
 int tc_smem_bytes(int dqk, int stages);
 int tc_max_stages(int dqk);
 cudaError_t launch_tc_attn(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s);
+// Two query tiles per CTA sharing every K/V tile (d_v <= 128).
+int tc2_smem_bytes(int dqk, int stages);
+int tc2_max_stages(int dqk);
+cudaError_t launch_tc_attn2(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s);
 
 // Sparse top-k forward, M = 64 heads of one query token per CTA, gathered rows.
 struct SparseTcParams {

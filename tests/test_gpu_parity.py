@@ -48,7 +48,8 @@ def test_dense_bf16_small(B, H, Hkv, Tq, Tk, D, Dv, causal, sinks):
     st = status_word()
     o, lse, (q, k, v, s) = run_dense(c, status=st)
     info = arc.plan_attn(q, k, v, o, lse, causal=causal, sinks=s)
-    assert info["kernel"] == "tc_attn_kernel" and info["tensor_cores"] == 1
+    # d_v <= 128: two query tiles per CTA; wider d_v: one tile per d_v slice
+    assert info["kernel"] == ("tc_attn2_kernel" if Dv <= 128 else "tc_attn_kernel") and info["tensor_cores"] == 1
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
     assert arc.check_device_error(st) == arc.ARC_OK
@@ -97,7 +98,7 @@ def test_mla_small(B, H, T, Dn, Dr, Dv):
     st = status_word()
     o, lse, t = run_mla(c, status=st)
     info = arc.plan_mla(*t, o, lse)
-    assert info["kernel"] == "tc_attn_kernel<mla>"
+    assert info["kernel"] == "tc_attn2_kernel<mla>"
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
     assert arc.check_device_error(st) == arc.ARC_OK
