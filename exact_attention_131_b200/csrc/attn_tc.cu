@@ -396,10 +396,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
 // S/P_B [384,512).  MMA order per KV tile j (steady state):
 //     O_A += P_A(j) V(j),  S_A(j+1),  O_B += P_B(j) V(j),  S_B(j+1)
 // so softmax A(j+1) overlaps the B-side MMAs and softmax B(j+1) the A side.
-// Softmax warps 4-7 serve tile A, warps 8-11 tile B; each reads its S twice
-// (max pass, then exp pass writing P over the columns already read) to stay
-// within the register budget of 384 threads.
-constexpr int NTHREADS2 = 384;
+// Softmax warps 2-5 serve tile A, warps 6-9 tile B (a warp reads TMEM lanes
+// 32*(warp % 4) .. +31); each loads its whole S row, then writes P over it.
+constexpr int NTHREADS2 = 320;  // producer, MMA, two softmax warpgroups
 
 template <int DQK, int DVS, bool MLA>
 __global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_constant__ TcParams p)
@@ -608,9 +607,9 @@ __global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_con
             umma_commit(&bars->drain);
             mbar_wait(&bars->drain, 0);
         }
-    } else if (warp >= 4) {
-        // =============================== softmax (warps 4-7: tile A, 8-11: tile B) and epilogue
-        const int t = (warp - 4) >> 2;
+    } else {
+        // =============================== softmax (warps 2-5: tile A, 6-9: tile B) and epilogue
+        const int t = (warp - 2) >> 2;
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -629,20 +628,20 @@ __global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_con
             if (!ok) break;
             tc_fence_after();
             const int kbase = j * BN;
-            const bool partial = kbase + BN - 1 > last;
-            // pass 1: row max
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t sv[32];
-                tmem_ld32(s_tmem + 32 * c, sv);
-                tmem_wait_ld();
+            // All of S in one go (four loads, one wait), then P written over it in place.
+            uint32_t sv[BN];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float x = (partial && kbase + 32 * c + i > last) ? -INFINITY : __uint_as_float(sv[i]);
-                    mx = fmaxf(mx, x);
-                }
+            for (int c = 0; c < BN / 32; ++c)
+                tmem_ld32(s_tmem + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * c]));
+            tmem_wait_ld();
+            if (kbase + BN - 1 > last) {
+#pragma unroll
+                for (int i = 0; i < BN; ++i)
+                    if (kbase + i > last) sv[i] = __float_as_uint(-INFINITY);
             }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < BN; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
             mx *= sl2;
             const bool need = mx > m_use + RESCALE_THRESHOLD;
             float alpha = 1.f;
@@ -651,24 +650,18 @@ __global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_con
                 m_use = mx;
             }
             const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
-            // pass 2: P = exp2(s*scale*log2e - m), written over S columns already read
             float rowsum = 0.f;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t sv[32], pk[16];
-                tmem_ld32(s_tmem + 32 * c, sv);
-                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int k0i = kbase + 32 * c + 2 * i;
-                    const float s0 = (partial && k0i > last) ? -INFINITY : __uint_as_float(sv[2 * i]);
-                    const float s1 = (partial && k0i + 1 > last) ? -INFINITY : __uint_as_float(sv[2 * i + 1]);
-                    const float p0 = fast_exp2(fmaf(s0, sl2, -msafe));
-                    const float p1 = fast_exp2(fmaf(s1, sl2, -msafe));
+            for (int c = 0; c < BN / 8; ++c) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float p0 = fast_exp2(fmaf(__uint_as_float(sv[8 * c + 2 * i]), sl2, -msafe));
+                    const float p1 = fast_exp2(fmaf(__uint_as_float(sv[8 * c + 2 * i + 1]), sl2, -msafe));
                     rowsum += p0 + p1;
                     pk[i] = pack_bf16(p0, p1);
                 }
-                tmem_st16(s_tmem + 16 * c, pk);
+                tmem_st4(s_tmem + 4 * c, pk[0], pk[1], pk[2], pk[3]);
             }
             l = l * alpha + rowsum;
             if (j > 0) {

@@ -291,6 +291,13 @@ ARC_DEV void cp_async16(void *dst, const void *src, uint32_t src_bytes)
 ARC_DEV void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 ARC_DEV void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+ARC_DEV void tmem_st4(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2),
+                 "r"(r3)
+                 : "memory");
+}
+
 ARC_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16])
 {
     asm volatile(
