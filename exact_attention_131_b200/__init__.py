@@ -26,6 +26,7 @@ ARC_DTYPE_BF16, ARC_DTYPE_F32 = 0, 1
 ARC_KV_Q4_0, ARC_KV_Q8_0 = 2, 8
 ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE = 1, 2, 3, 4
 ARC_FLAG_FORCE_SIMPLE = 1
+ARC_FLAG_SINGLE_CTA = 2
 ARC_DECODE_MAX_SEQ = 64
 
 _i32, _i64, _u32, _f32, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float, ctypes.c_void_p

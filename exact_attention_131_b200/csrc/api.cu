@@ -163,7 +163,8 @@ enum class Path { None, Simple, Tc };
 
 struct AttnPlan {
     Path path = Path::None;
-    bool two = false;  // two query tiles per CTA (d_v <= 128)
+    bool two = false;   // two query tiles per CTA (d_v <= 128)
+    bool pair = false;  // CTA pair, M = 256 (d_qk 256 / 512, d_v slice 256)
     int dvs = 0, n_slices = 0, n_tiles = 0, grid = 0, stages = 0;
 };
 
@@ -219,6 +220,11 @@ AttnPlan plan_attn(const arc_attn_args *a)
     pl.grid = pl.n_tiles * a->B * a->Hkv * pl.n_slices;
     pl.stages = tc_max_stages(a->D);
     maybe_two(pl, a->D, false, a->B * a->Hkv);
+    if (!pl.two && !(a->flags & ARC_FLAG_SINGLE_CTA) && pair_supported(a->D, pl.dvs)) {
+        pl.pair = true;
+        pl.stages = pair_max_stages(a->D);
+        pl.grid = ((pl.n_tiles + 1) / 2) * a->B * a->Hkv * pl.n_slices * 2;
+    }
     return pl;
 }
 
@@ -407,8 +413,9 @@ arc_status arc_attn_fwd(const arc_attn_args *a, void *stream)
         const uint64_t vd[4] = {(uint64_t)a->Dv, (uint64_t)a->Tk, (uint64_t)a->Hkv, (uint64_t)a->B};
         const int64_t vs[3] = {a->v_strides[2], a->v_strides[1] ? a->v_strides[1] : (int64_t)a->Tk * a->v_strides[2],
                                a->v_strides[0] ? a->v_strides[0] : (int64_t)a->Hkv * a->Tk * a->v_strides[2]};
-        if (!make_map(&p.tm_q, a->q, 3, qd, qs, kTcBM) || !make_map(&p.tm_k, a->k, 4, kd, ks, kTcBN) ||
-            !make_map(&p.tm_v, a->v, 4, vd, vs, kTcBN))
+        const uint32_t kv_box = pl.pair ? 64 : kTcBN;  // a CTA of a pair stages half of each key tile
+        if (!make_map(&p.tm_q, a->q, 3, qd, qs, kTcBM) || !make_map(&p.tm_k, a->k, 4, kd, ks, kv_box) ||
+            !make_map(&p.tm_v, a->v, 4, vd, vs, kv_box))
             return ARC_ERR_CUDA;
         p.tm_q2 = p.tm_q;
         p.tm_k2 = p.tm_k;
@@ -422,6 +429,10 @@ arc_status arc_attn_fwd(const arc_attn_args *a, void *stream)
             order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
             note_dispatch("tc_attn2_kernel");
             e = launch_tc_attn2(p, a->D, pl.dvs, false, pl.grid, s);
+        } else if (pl.pair) {
+            order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
+            note_dispatch("tc_attn_pair_kernel");
+            e = launch_tc_attn_pair(p, a->D, pl.dvs, pl.grid, s);
         } else {
             order_tiles(p, pl.n_tiles);
             note_dispatch("tc_attn_kernel");
@@ -623,10 +634,12 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             out->tile_m = 4;
             out->n_ctas = (int)(((int64_t)a->B * a->H * a->Tq + 3) / 4);
         } else {
-            set_name(out, pl.two ? "tc_attn2_kernel" : "tc_attn_kernel");
+            set_name(out, pl.two ? "tc_attn2_kernel" : (pl.pair ? "tc_attn_pair_kernel" : "tc_attn_kernel"));
             out->tensor_cores = 1;
-            out->tile_m = pl.two ? 2 * kTcBM : kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
-            out->smem_bytes = pl.two ? tc2_smem_bytes(a->D, pl.stages) : tc_smem_bytes(a->D, pl.stages);
+            out->tile_m = (pl.two || pl.pair) ? 2 * kTcBM : kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs;
+            out->n_ctas = pl.grid;
+            out->smem_bytes = pl.two ? tc2_smem_bytes(a->D, pl.stages)
+                                     : (pl.pair ? pair_smem_bytes(a->D, pl.stages) : tc_smem_bytes(a->D, pl.stages));
             out->tmem_cols = 512;
         }
         out->launches = 1;

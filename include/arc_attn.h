@@ -62,6 +62,7 @@ typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE
 
 /* flags (all calls) */
 #define ARC_FLAG_FORCE_SIMPLE 1u   /* run the CUDA-core kernel instead of the tensor-core one */
+#define ARC_FLAG_SINGLE_CTA 2u     /* do not use the CTA-pair (cta_group::2) kernel */
 
 /* --------------------------------------------------------------------------
  * arc_attn_fwd: dense attention with GQA / MQA and optional per-head sinks.

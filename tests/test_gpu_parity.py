@@ -48,11 +48,37 @@ def test_dense_bf16_small(B, H, Hkv, Tq, Tk, D, Dv, causal, sinks):
     st = status_word()
     o, lse, (q, k, v, s) = run_dense(c, status=st)
     info = arc.plan_attn(q, k, v, o, lse, causal=causal, sinks=s)
-    # d_v <= 128: two query tiles per CTA; wider d_v: one tile per d_v slice
-    assert info["kernel"] == ("tc_attn2_kernel" if Dv <= 128 else "tc_attn_kernel") and info["tensor_cores"] == 1
+    assert info["kernel"] == expected_dense_kernel(D, Dv) and info["tensor_cores"] == 1
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
     assert arc.check_device_error(st) == arc.ARC_OK
+
+
+def expected_dense_kernel(D, Dv):
+    # d_v <= 128: two query tiles per CTA; d_qk 256 / 512 with a 256-wide d_v
+    # slice: a CTA pair (M = 256); otherwise one tile per d_v slice
+    if Dv <= 128:
+        return "tc_attn2_kernel"
+    if D in (256, 512) and Dv in (256, 512):
+        return "tc_attn_pair_kernel"
+    return "tc_attn_kernel"
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,Tk,D,causal,sinks", [
+    (1, 16, 2, 200, 200, 512, True, True),     # odd tile count: the last pair's second CTA has no rows
+    (2, 8, 1, 190, 450, 256, True, False),      # Tq < Tk, two batches
+    (1, 4, 4, 300, 300, 512, False, True),      # non-causal, G = 1
+])
+def test_dense_pair_and_single_cta_agree_with_oracle(B, H, Hkv, Tq, Tk, D, causal, sinks):
+    c = W.dense_case(B, H, Hkv, Tq, Tk, D, D, dtype="bf16", std=0.5, causal=causal, sinks=sinks, seed=34)
+    ro, rl = oracle.run_case(c)
+    for flags, name in ((0, "tc_attn_pair_kernel"), (arc.ARC_FLAG_SINGLE_CTA, "tc_attn_kernel")):
+        st = status_word()
+        o, lse, (q, k, v, s) = run_dense(c, flags=flags, status=st)
+        info = arc.plan_attn(q, k, v, o, lse, causal=causal, sinks=s, flags=flags)
+        assert info["kernel"] == name
+        compare(o, lse, ro, rl, TOL_O_BF16)
+        assert arc.check_device_error(st) == arc.ARC_OK
 
 
 def test_dense_control_arm_runs_the_simple_kernel():
@@ -75,7 +101,7 @@ def test_config2_gqa_sinks_full_size_sampled_rows():
     st = status_word()
     o, lse, (q, k, v, s) = run_dense(c, status=st)
     info = arc.plan_attn(q, k, v, o, lse, sinks=s)
-    assert info["kernel"] == "tc_attn_kernel" and info["d_slice"] == 256
+    assert info["kernel"] == "tc_attn_pair_kernel" and info["d_slice"] == 256 and info["tile_m"] == 256
     rows = sample_rows(c.Tq, 40, 2)
     ro, rl = oracle.run_case(c, rows=rows)
     compare(o[:, :, rows], lse[:, :, rows], ro, rl, TOL_O_BF16)
