@@ -100,6 +100,22 @@ bool make_map(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, 
     return r == CUDA_SUCCESS;
 }
 
+// Same with an explicit box (one entry per dimension, innermost first).
+bool make_map_box(CUtensorMap *m, const void *base, int rank, const uint64_t *dims, const int64_t *strides_el,
+                  const uint32_t *box_in)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[5], gstr[4];
+    cuuint32_t box[5], estr[5];
+    for (int i = 0; i < rank; ++i) gdim[i] = dims[i], estr[i] = 1, box[i] = box_in[i];
+    for (int i = 0; i < rank - 1; ++i) gstr[i] = (cuuint64_t)strides_el[i] * 2;
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gdim, gstr, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool tma_strides_ok(std::initializer_list<int64_t> strides_el)
 {
     for (int64_t s : strides_el)
@@ -118,7 +134,7 @@ void order_tiles(TcParams &p, int n_tiles, int rows_per_item = kTcBM)
     const int rows = p.G * p.Tq;
     for (int t = 0; t < n_tiles; ++t) {
         const int r0 = t * rows_per_item, r_last = std::min(r0 + rows_per_item, rows) - 1;
-        const int t_max = (r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
+        const int t_max = p.tmajor ? r_last / p.G : ((r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq);
         const int last = p.causal ? std::min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
         w[t] = {last < 0 ? 0 : last / kTcBN + 1, t};
     }
@@ -414,8 +430,22 @@ arc_status arc_attn_fwd(const arc_attn_args *a, void *stream)
         const int64_t vs[3] = {a->v_strides[2], a->v_strides[1] ? a->v_strides[1] : (int64_t)a->Tk * a->v_strides[2],
                                a->v_strides[0] ? a->v_strides[0] : (int64_t)a->Hkv * a->Tk * a->v_strides[2]};
         const uint32_t kv_box = pl.pair ? 64 : kTcBN;  // a CTA of a pair stages half of each key tile
-        if (!make_map(&p.tm_q, a->q, 3, qd, qs, kTcBM) || !make_map(&p.tm_k, a->k, 4, kd, ks, kv_box) ||
-            !make_map(&p.tm_v, a->v, 4, vd, vs, kv_box))
+        const int G = a->H / a->Hkv;
+        // The pair kernel visits the fold rows of a kv head t-major (row = t*G + head in group)
+        // when G divides the 128-row box: a tile then spans 128/G positions of every head of
+        // the group, so under the causal mask all its rows need nearly the same key tiles.
+        p.tmajor = pl.pair && G > 1 && kTcBM % G == 0;
+        bool ok_q;
+        if (p.tmajor) {
+            const int64_t hs = a->q_strides[1] ? a->q_strides[1] : (int64_t)a->Tq * a->q_strides[2];
+            const uint64_t qd5[5] = {(uint64_t)a->D, (uint64_t)G, (uint64_t)a->Tq, (uint64_t)a->Hkv, (uint64_t)a->B};
+            const int64_t qs5[4] = {hs, a->q_strides[2], hs * G, qs[1]};
+            const uint32_t box5[5] = {64, (uint32_t)G, (uint32_t)(kTcBM / G), 1, 1};
+            ok_q = make_map_box(&p.tm_q, a->q, 5, qd5, qs5, box5);
+        } else {
+            ok_q = make_map(&p.tm_q, a->q, 3, qd, qs, kTcBM);
+        }
+        if (!ok_q || !make_map(&p.tm_k, a->k, 4, kd, ks, kv_box) || !make_map(&p.tm_v, a->v, 4, vd, vs, kv_box))
             return ARC_ERR_CUDA;
         p.tm_q2 = p.tm_q;
         p.tm_k2 = p.tm_k;

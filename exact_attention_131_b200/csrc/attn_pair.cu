@@ -31,6 +31,8 @@ namespace {
 constexpr int PBM = 128;           // query rows per CTA
 constexpr int PBN = 128;           // keys per KV tile (64 staged by each CTA)
 constexpr int PCH = 64 * 128;      // bytes of one [64 rows x 64 bf16] swizzled box
+constexpr int BPS = 4;             // boxes per ring stage (one barrier hand-off per 32 KB)
+constexpr int PST = BPS * PCH;     // bytes of one ring stage
 constexpr int P_THREADS = 256;
 constexpr int P_TMEM = 512;
 constexpr int P_SCOL = 256;        // S/P double buffer at columns 256, 384
@@ -71,9 +73,12 @@ __device__ __forceinline__ void cluster_sync_all()
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+// Arrive on the leader's barrier from the other CTA of the pair.  The data this
+// orders is in TMEM and is ordered by the tcgen05 fences around the arrive and
+// the wait; a release at cluster scope (which costs ~1-2k clk here) is not needed.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // 2-SM bulk tensor loads: data lands in this CTA's shared memory, the
@@ -95,6 +100,16 @@ __device__ __forceinline__ void tma2_load_4d(void *dst, const CUtensorMap *map, 
         "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
         "l"(map), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma2_load_5d(void *dst, const CUtensorMap *map, uint32_t mbar_cluster, int c0, int c1,
+                                             int c2, int c3, int c4)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(mbar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
         : "memory");
 }
 
@@ -170,13 +185,14 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
     constexpr int KC = DQK / 64;     // 64-column chunks of a Q / K row
     constexpr int VG = DVS / 128;    // 128-column MMA groups of the d_v slice
     static_assert(DQK % 64 == 0 && DVS % 128 == 0 && DVS <= 256, "tile shape");
+    static_assert(KC % BPS == 0 && (2 * VG) % BPS == 0, "K and V tiles fill whole ring stages");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem;                          // KC chunks of [128 rows x 64]
-    uint8_t *sRing = sQ + KC * 2 * PCH;          // R stages of [64 rows x 64]
+    uint8_t *sRing = sQ + KC * 2 * PCH;          // R stages of BPS boxes of [64 rows x 64]
     const int R = p.stages;
-    PairBars *bars = reinterpret_cast<PairBars *>(sRing + R * PCH);
+    PairBars *bars = reinterpret_cast<PairBars *>(sRing + R * PST);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -198,7 +214,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
     int nt;
     {
         const int r_last = min(rp + 2 * PBM, rows_in_group) - 1;
-        const int t_max = (rp / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
+        const int t_max = p.tmajor ? r_last / p.G : ((rp / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq);
         const int kv_last = p.causal ? min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
         nt = kv_last < 0 ? 0 : kv_last / PBN + 1;
     }
@@ -235,14 +251,21 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             tma_prefetch_desc(&p.tm_v);
             const uint32_t q_full_l = mapa(smem_u32(&bars->q_full), 0);
             if (leader) mbar_arrive_expect_tx_u32(smem_u32(&bars->q_full), 2 * KC * 2 * PCH);
-            const int qrow = kv * rows_in_group + r0;
-            for (int c = 0; c < KC; ++c) tma2_load_3d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, qrow, b);
+            if (p.tmajor) {
+                // box {64, G, 128/G}: smem row = (t - t0) * G + head in group
+                for (int c = 0; c < KC; ++c) tma2_load_5d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, 0, r0 / p.G, kv, b);
+            } else {
+                const int qrow = kv * rows_in_group + r0;
+                for (int c = 0; c < KC; ++c) tma2_load_3d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, qrow, b);
+            }
             int stage = 0;
             uint32_t ephase = 0;
             bool ok = true;
+            // Each barrier round trip costs this thread a few hundred clocks, so a
+            // stage carries BPS boxes: one wait and one expect_tx per 32 KB.
             auto acquire = [&]() -> bool {
                 if (!mbar_wait(&bars->empty[stage], ephase ^ 1u)) return false;
-                if (leader) mbar_arrive_expect_tx_u32(smem_u32(&bars->full[stage]), 2 * PCH);
+                if (leader) mbar_arrive_expect_tx_u32(smem_u32(&bars->full[stage]), 2 * PST);
                 return true;
             };
             auto advance = [&]() {
@@ -253,21 +276,28 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             };
             auto full_l = [&]() { return mapa(smem_u32(&bars->full[stage]), 0); };
             auto load_k = [&](int j) -> bool {
-                for (int c = 0; c < KC; ++c) {
+                for (int c0 = 0; c0 < KC; c0 += BPS) {
                     if (!acquire()) return false;
-                    tma2_load_4d(sRing + stage * PCH, &p.tm_k, full_l(), c * 64, j * PBN + (int)rank * 64, kv, b);
+                    const uint32_t fl = full_l();
+                    for (int q = 0; q < BPS; ++q)
+                        tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_k, fl, (c0 + q) * 64,
+                                     j * PBN + (int)rank * 64, kv, b);
                     advance();
                 }
                 return true;
             };
+            // V box q of a stage: 128-column group q / 2, key half q % 2
             auto load_v = [&](int j) -> bool {
-                for (int g = 0; g < VG; ++g)
-                    for (int hh = 0; hh < 2; ++hh) {
-                        if (!acquire()) return false;
-                        tma2_load_4d(sRing + stage * PCH, &p.tm_v, full_l(), dv0 + g * 128 + (int)rank * 64,
+                for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
+                    if (!acquire()) return false;
+                    const uint32_t fl = full_l();
+                    for (int q = 0; q < BPS; ++q) {
+                        const int g = (q0 + q) >> 1, hh = (q0 + q) & 1;
+                        tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_v, fl, dv0 + g * 128 + (int)rank * 64,
                                      j * PBN + hh * 64, kv, b);
-                        advance();
                     }
+                    advance();
+                }
                 return true;
             };
             ok = load_k(0);
@@ -296,13 +326,34 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                     fphase ^= 1u;
                 }
             };
+            // A shared-memory access by this thread after a tcgen05.commit waits
+            // until the committed MMAs have completed, so every barrier wait here
+            // empties the tensor pipe (measured: ~230 clk of idle pipe per wait).
+            // The issuer therefore waits once for a whole operand tile (all K
+            // boxes of S, or P plus all V boxes of PV) and then issues the tile's
+            // MMAs back to back; ring boxes are still released one by one.
+            auto wait_boxes = [&](int n) -> bool {
+                int st = stage;
+                uint32_t ph = fphase;
+                for (int i = 0; i < n; ++i) {
+                    if (!mbar_wait(&bars->full[st], ph)) return false;
+                    if (++st == R) {
+                        st = 0;
+                        ph ^= 1u;
+                    }
+                }
+                return true;
+            };
             auto issue_s = [&](int j) -> bool {
                 const uint32_t d = tmem + P_SCOL + (j & 1) * PBN;
+                if (!wait_boxes(KC / BPS)) return false;
+                tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < KC; ++c) {
-                    if (!mbar_wait(&bars->full[stage], fphase)) return false;
-                    tc_fence_after();
-                    umma2_ss_k64(d, qd0 + (uint64_t)(c * 2 * kBox), kd0 + (uint64_t)(stage * kBox), idesc_s, c > 0);
+                for (int c0 = 0; c0 < KC; c0 += BPS) {
+#pragma unroll
+                    for (int q = 0; q < BPS; ++q)
+                        umma2_ss_k64(d, qd0 + (uint64_t)((c0 + q) * 2 * kBox), kd0 + (uint64_t)((stage * BPS + q) * kBox),
+                                     idesc_s, (c0 + q) > 0);
                     umma2_commit_both(&bars->empty[stage]);
                     advance();
                 }
@@ -311,18 +362,20 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             };
             auto issue_pv = [&](int j) -> bool {
                 if (!mbar_wait_cluster(&bars->p_full, (uint32_t)(j & 1))) return false;
+                if (!wait_boxes(2 * VG / BPS)) return false;
+                tc_fence_after();
                 const uint32_t p_tm = tmem + P_SCOL + (j & 1) * PBN;
 #pragma unroll 1
-                for (int g = 0; g < VG; ++g)
-#pragma unroll 1
-                    for (int hh = 0; hh < 2; ++hh) {
-                        if (!mbar_wait(&bars->full[stage], fphase)) return false;
-                        tc_fence_after();
-                        umma2_ts_k64(tmem + g * 128, p_tm + hh * 32, vd0 + (uint64_t)(stage * kBox), idesc_pv,
+                for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
+#pragma unroll
+                    for (int q = 0; q < BPS; ++q) {
+                        const int g = (q0 + q) >> 1, hh = (q0 + q) & 1;
+                        umma2_ts_k64(tmem + g * 128, p_tm + hh * 32, vd0 + (uint64_t)((stage * BPS + q) * kBox), idesc_pv,
                                      (j > 0) | hh);
-                        umma2_commit_both(&bars->empty[stage]);
-                        advance();
                     }
+                    umma2_commit_both(&bars->empty[stage]);
+                    advance();
+                }
                 umma2_commit_both(&bars->o_done);
                 return true;
             };
@@ -341,8 +394,8 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const int R_ = r0 + r;
         const bool row_ok = R_ < rows_in_group;
-        const int t = R_ % p.Tq;
-        const int h = kv * p.G + R_ / p.Tq;
+        const int t = p.tmajor ? R_ / p.G : R_ % p.Tq;
+        const int h = kv * p.G + (p.tmajor ? R_ % p.G : R_ / p.Tq);
         const int last = p.causal ? min(p.Tk - 1, t + p.Tk - p.Tq) : p.Tk - 1;
         const float sl2 = p.scale_log2;
         const uint32_t p_full_l = mapa(smem_u32(&bars->p_full), 0);
@@ -408,7 +461,10 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive_cluster(p_full_l);
+            if (leader)
+                mbar_arrive(&bars->p_full);
+            else
+                mbar_arrive_remote(p_full_l);
         }
         if (ok && nt > 0) {
             ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((nt - 1) & 1)));
@@ -491,11 +547,11 @@ cudaError_t launch_p(const TcParams &p, int grid, cudaStream_t s)
 
 }  // namespace
 
-int pair_smem_bytes(int dqk, int stages) { return 1024 + (dqk / 64) * 2 * PCH + stages * PCH + (int)sizeof(PairBars); }
+int pair_smem_bytes(int dqk, int stages) { return 1024 + (dqk / 64) * 2 * PCH + stages * PST + (int)sizeof(PairBars); }
 
 int pair_max_stages(int dqk)
 {
-    int st = (P_SMEM_LIMIT - 1024 - (int)sizeof(PairBars) - (dqk / 64) * 2 * PCH) / PCH;
+    int st = (P_SMEM_LIMIT - 1024 - (int)sizeof(PairBars) - (dqk / 64) * 2 * PCH) / PST;
     return st < P_MAX_STAGES ? st : P_MAX_STAGES;
 }
 

@@ -44,7 +44,7 @@ cudaError_t launch_simple_decode(const SimpleDecodeParams &p, cudaStream_t s);
 // ---------------------------------------------------------------- tcgen05 attention
 // Dense / GQA fold / MLA forward, M = 128 query rows per CTA, K/V tiles by TMA.
 struct TcParams {
-    CUtensorMap tm_q;   // q (dense) or q_nope (MLA): dims {D, H*Tq, B}
+    CUtensorMap tm_q;   // q (dense) or q_nope (MLA): dims {D, H*Tq, B}; t-major: {D, G, Tq, Hkv, B}
     CUtensorMap tm_q2;  // q_rope: dims {Dr, H*Tq, B}
     CUtensorMap tm_k;   // k (dense) or k_nope: dims {D, Tk, Hkv, B}
     CUtensorMap tm_k2;  // k_rope: dims {Dr, Tk, B}
@@ -60,6 +60,7 @@ struct TcParams {
     const float *sinks;
     float scale_log2;   // scale * log2(e)
     int causal;
+    int tmajor;         // fold rows visited t-major (row = t*G + head-in-group); tm_q is then 5-d
     uint32_t *status;
     uint16_t tile_order[1024];
 };
