@@ -239,7 +239,7 @@ AttnPlan plan_attn(const arc_attn_args *a)
     if (!pl.two && !(a->flags & ARC_FLAG_SINGLE_CTA) && pair_supported(a->D, pl.dvs)) {
         pl.pair = true;
         pl.stages = pair_max_stages(a->D);
-        pl.grid = ((pl.n_tiles + 1) / 2) * a->B * a->Hkv * pl.n_slices * 2;
+        pl.grid = ((pl.n_tiles + 1) / 2) * a->B * a->Hkv * 2;  // each pair runs every d_v slice
     }
     return pl;
 }

@@ -199,18 +199,19 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
     const bool leader = rank == 0;
 
     // ---- which rows this pair owns
+    // A pair computes every d_v slice of its rows in turn with Q resident: work
+    // item `it` is (slice it / nt, key tile it % nt).
     const int cl = blockIdx.x >> 1;
-    const int groups = p.B * p.Hkv * p.n_slices;
+    const int groups = p.B * p.Hkv;
     const int prank = cl / groups;
     const int rest = cl % groups;
-    const int slice = rest % p.n_slices;
-    const int kv = (rest / p.n_slices) % p.Hkv;
-    const int b = rest / (p.n_slices * p.Hkv);
+    const int kv = rest % p.Hkv;
+    const int b = rest / p.Hkv;
+    const int NSL = p.n_slices;
     const int pair = prank < 1024 ? (int)p.tile_order[prank] : prank;
     const int rows_in_group = p.G * p.Tq;
     const int rp = pair * 2 * PBM;               // first row of the pair
     const int r0 = rp + (int)rank * PBM;         // first row of this CTA
-    const int dv0 = slice * DVS;
     int nt;
     {
         const int r_last = min(rp + 2 * PBM, rows_in_group) - 1;
@@ -218,6 +219,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
         const int kv_last = p.causal ? min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
         nt = kv_last < 0 ? 0 : kv_last / PBN + 1;
     }
+    const int NI = nt * NSL;                     // work items of the pair
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
@@ -287,7 +289,8 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 return true;
             };
             // V box q of a stage: 128-column group q / 2, key half q % 2
-            auto load_v = [&](int j) -> bool {
+            auto load_v = [&](int it) -> bool {
+                const int j = it % nt, dv0 = (it / nt) * DVS;
                 for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
                     if (!acquire()) return false;
                     const uint32_t fl = full_l();
@@ -301,9 +304,9 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 return true;
             };
             ok = load_k(0);
-            for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt) ok = load_k(j + 1);
-                if (ok) ok = load_v(j);
+            for (int it = 0; ok && it < NI; ++it) {
+                if (it + 1 < NI) ok = load_k((it + 1) % nt);
+                if (ok) ok = load_v(it);
             }
             if (!ok) report(p.status, ST_TIMEOUT_LOAD);
         }
@@ -344,8 +347,8 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 }
                 return true;
             };
-            auto issue_s = [&](int j) -> bool {
-                const uint32_t d = tmem + P_SCOL + (j & 1) * PBN;
+            auto issue_s = [&](int it) -> bool {
+                const uint32_t d = tmem + P_SCOL + (it & 1) * PBN;
                 if (!wait_boxes(KC / BPS)) return false;
                 tc_fence_after();
 #pragma unroll 1
@@ -357,21 +360,22 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                     umma2_commit_both(&bars->empty[stage]);
                     advance();
                 }
-                umma2_commit_both(&bars->s_full[j & 1]);
+                umma2_commit_both(&bars->s_full[it & 1]);
                 return true;
             };
-            auto issue_pv = [&](int j) -> bool {
-                if (!mbar_wait_cluster(&bars->p_full, (uint32_t)(j & 1))) return false;
+            auto issue_pv = [&](int it) -> bool {
+                const int first = (it % nt) == 0;     // first key tile of a slice overwrites O
+                if (!mbar_wait_cluster(&bars->p_full, (uint32_t)(it & 1))) return false;
                 if (!wait_boxes(2 * VG / BPS)) return false;
                 tc_fence_after();
-                const uint32_t p_tm = tmem + P_SCOL + (j & 1) * PBN;
+                const uint32_t p_tm = tmem + P_SCOL + (it & 1) * PBN;
 #pragma unroll 1
                 for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
 #pragma unroll
                     for (int q = 0; q < BPS; ++q) {
                         const int g = (q0 + q) >> 1, hh = (q0 + q) & 1;
                         umma2_ts_k64(tmem + g * 128, p_tm + hh * 32, vd0 + (uint64_t)((stage * BPS + q) * kBox), idesc_pv,
-                                     (j > 0) | hh);
+                                     (first ? 0 : 1) | hh);
                     }
                     umma2_commit_both(&bars->empty[stage]);
                     advance();
@@ -380,9 +384,9 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 return true;
             };
             if (ok) ok = issue_s(0);
-            for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt) ok = issue_s(j + 1);
-                if (ok) ok = issue_pv(j);
+            for (int it = 0; ok && it < NI; ++it) {
+                if (it + 1 < NI) ok = issue_s(it + 1);
+                if (ok) ok = issue_pv(it);
             }
             if (!ok) report(p.status, ST_TIMEOUT_MMA);
             umma2_commit_both(&bars->drain);
@@ -399,12 +403,15 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
         const int last = p.causal ? min(p.Tk - 1, t + p.Tk - p.Tq) : p.Tk - 1;
         const float sl2 = p.scale_log2;
         const uint32_t p_full_l = mapa(smem_u32(&bars->p_full), 0);
-        float m_use = -INFINITY, l = 0.f;
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
-            const int buf = j & 1;
+        for (int slice = 0; slice < NSL; ++slice) {
+        const int dv0 = slice * DVS;
+        float m_use = -INFINITY, l = 0.f;
+        for (int j = 0; ok && j < nt; ++j) {
+            const int it = slice * nt + j;
+            const int buf = it & 1;
             const uint32_t s_tmem = tmem + lane_off + P_SCOL + buf * PBN;
-            ok = warp_all_pair(mbar_wait(&bars->s_full[buf], (uint32_t)((j >> 1) & 1)));
+            ok = warp_all_pair(mbar_wait(&bars->s_full[buf], (uint32_t)((it >> 1) & 1)));
             if (!ok) break;
             tc_fence_after();
             uint32_t sv[PBN];
@@ -444,7 +451,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             }
             l = l * alpha + rowsum;
             if (j > 0) {
-                ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((j - 1) & 1)));
+                ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((it - 1) & 1)));
                 if (!ok) break;
                 tc_fence_after();
                 if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -467,10 +474,9 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 mbar_arrive_remote(p_full_l);
         }
         if (ok && nt > 0) {
-            ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((nt - 1) & 1)));
+            ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((slice * nt + nt - 1) & 1)));
             tc_fence_after();
         }
-        if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
         float fac, lse;
         if (p.sinks) {
             const float sg = row_ok ? p.sinks[h] * P_LOG2E : 0.f;
@@ -506,6 +512,8 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             }
         }
         if (row_ok && slice == 0) p.lse[((int64_t)b * p.H + h) * p.Tq + t] = lse;
+        }
+        if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
     }
 
     // Drain: the leader's last MMAs have finished (they write both CTAs' TMEM)
