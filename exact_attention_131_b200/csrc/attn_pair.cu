@@ -179,6 +179,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
 
 __device__ __forceinline__ bool warp_all_pair(bool ok) { return __all_sync(0xffffffffu, ok); }
 
+// One 32-byte global store (a whole sector); dst must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void *dst, const uint32_t *w)
+{
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                 "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                 : "memory");
+}
+
 template <int DQK, int DVS>
 __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid_constant__ TcParams p)
 {
@@ -491,24 +499,39 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
         }
         __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.o) + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] +
                               (int64_t)t * p.os[2] + dv0;
+        // Four 32-column TMEM loads in flight per wait; each 32-column piece of
+        // the row leaves as two 32-byte stores (whole sectors).
+        const bool st32 = (reinterpret_cast<uintptr_t>(orow) & 31) == 0;
 #pragma unroll 1
-        for (int c = 0; c < DVS / 32; ++c) {
-            uint32_t ov[32];
+        for (int c0 = 0; c0 < DVS / 32; c0 += 4) {
+            uint32_t ov[4][32];
             if (nt > 0 && ok) {
-                tmem_ld32(tmem + lane_off + 32 * c, ov);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) tmem_ld32(tmem + lane_off + 32 * (c0 + u), ov[u]);
                 tmem_wait_ld();
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) ov[i] = 0u;
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[u][i] = 0u;
             }
             if (row_ok) {
-                uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    w[i] = pack_bf16(__uint_as_float(ov[2 * i]) * fac, __uint_as_float(ov[2 * i + 1]) * fac);
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + 32 * c);
+                for (int u = 0; u < 4; ++u) {
+                    uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack_bf16(__uint_as_float(ov[u][2 * i]) * fac, __uint_as_float(ov[u][2 * i + 1]) * fac);
+                    __nv_bfloat16 *dst = orow + 32 * (c0 + u);
+                    if (st32) {
+                        st_global_v8(dst, w);
+                        st_global_v8(dst + 16, w + 8);
+                    } else {
+                        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) d4[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                    }
+                }
             }
         }
         if (row_ok && slice == 0) p.lse[((int64_t)b * p.H + h) * p.Tq + t] = lse;
