@@ -17,7 +17,8 @@
 using namespace arc;
 
 namespace arc {
-int decode_smem_bytes(int kv_type, int D);
+int decode_smem_bytes(int kv_type, int D, bool tma);
+int decode_box_bytes(int kv_type, int D);
 }
 
 namespace {
@@ -112,6 +113,19 @@ bool make_map_box(CUtensorMap *m, const void *base, int rank, const uint64_t *di
     for (int i = 0; i < rank - 1; ++i) gstr[i] = (cuuint64_t)strides_el[i] * 2;
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), gdim, gstr, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Byte tensor {width bytes, rows}, row stride = width, no swizzle; box {box_w bytes, box_rows}.
+bool make_map_bytes(CUtensorMap *m, const void *base, uint64_t width, uint64_t rows, uint32_t box_w, uint32_t box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[2] = {width, rows}, gstr[1] = {width};
+    cuuint32_t box[2] = {box_w, box_rows}, estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), gdim, gstr, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -335,6 +349,7 @@ bool plan_sparse_tc(const arc_sparse_args *a)
 
 struct DecodePlan {
     bool simple = false;
+    bool tma = false;   // shape allows the TMA ring (cell stride a multiple of 16 bytes)
     int splits = 0, chunk = 0, max_kv = 0;
     size_t ws = 0;
 };
@@ -372,7 +387,9 @@ DecodePlan plan_decode(const arc_decode_args *a)
     for (int s = 0; s < a->n_seq; ++s) pl.max_kv = std::max(pl.max_kv, a->seqs[s].n_kv);
     if (pl.simple || pl.max_kv == 0) return pl;
     const int pairs = a->n_seq * a->Hkv;
-    const int smem = decode_smem_bytes(a->kv_type, a->D);
+    const int64_t cell_bytes = (int64_t)a->Hkv * (a->D / 32) * (a->kv_type == ARC_KV_Q8_0 ? 34 : 18);
+    pl.tma = cell_bytes % 16 == 0;
+    const int smem = decode_smem_bytes(a->kv_type, a->D, pl.tma);
     const int per_sm = std::max(1, std::min(4, (228 * 1024) / (smem + 1024)));
     const int target = sm_count() * per_sm;
     int splits = std::min(256, std::max(1, target / std::max(1, pairs)));
@@ -608,6 +625,16 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
         p.ws_ml = p.ws_o + parts * 16 * a->D;
         p.scale_log2 = a->scale * kLog2e;
         p.status = a->status;
+        // K/V tiles by TMA when the cache rows allow it: a byte tensor {cell bytes, n_cells} per cache.
+        p.tma = pl.tma && (reinterpret_cast<uintptr_t>(a->k_cache) & 15) == 0 &&
+                (reinterpret_cast<uintptr_t>(a->v_cache) & 15) == 0;
+        if (p.tma) {
+            const int64_t cell_bytes = (int64_t)a->Hkv * (a->D / 32) * (a->kv_type == ARC_KV_Q8_0 ? 34 : 18);
+            const uint32_t box_w = (uint32_t)decode_box_bytes(a->kv_type, a->D);
+            if (!make_map_bytes(&p.tm_kc, a->k_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64) ||
+                !make_map_bytes(&p.tm_vc, a->v_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64))
+                return ARC_ERR_CUDA;
+        }
         note_dispatch(a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
         e = launch_decode(p, s);
     }
@@ -728,7 +755,7 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             out->tensor_cores = 1;
             out->tile_m = 16, out->tile_n = 32, out->d_slice = a->D;
             out->splits = pl.splits, out->n_ctas = a->n_seq * a->Hkv * pl.splits;
-            out->smem_bytes = decode_smem_bytes(a->kv_type, a->D);
+            out->smem_bytes = decode_smem_bytes(a->kv_type, a->D, pl.tma);
             out->launches = 2;
         }
         return ARC_OK;

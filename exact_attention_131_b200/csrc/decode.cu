@@ -47,15 +47,22 @@ struct Fmt<ARC_KV_Q4_0> {
     static constexpr int BB = 18;
 };
 
-template <int KVT, int D>
+constexpr int gcd16(int x) { return (x & 15) == 0 ? 16 : ((x & 7) == 0 ? 8 : ((x & 3) == 0 ? 4 : ((x & 1) == 0 ? 2 : 1))); }
+
+// TMA: the head row of kv head h starts at byte ROWB*h of a cell, which is not
+// 16-byte aligned in general; the box starts at the boundary below it (at most
+// 16 - gcd(ROWB, 16) bytes earlier) and is wide enough to cover the row.
+template <int KVT, int D, bool TMA>
 struct DecLayout {
     static constexpr int ROWB = (D / 32) * Fmt<KVT>::BB;       // raw bytes of one head row
-    static constexpr int RAW = DT * ROWB;                      // raw bytes of one K (or V) tile
+    static constexpr int RS = TMA ? ((ROWB + 16 - gcd16(ROWB) + 15) / 16) * 16 : ROWB;  // raw row stride in smem
+    static constexpr int RAW = DT * RS;                        // raw bytes of one K (or V) tile
+    static constexpr int NST = TMA ? (KVT == ARC_KV_Q8_0 ? 2 : 4) : 2;  // raw stages in flight
     static constexpr int HSTRIDE = D + 8;                      // f16 tile row stride (elements), breaks bank conflicts
     static constexpr int HBYTES = DT * HSTRIDE * 2;
     static constexpr int MERGE = WARPS * 16 * (D + 2) * 4;
-    static constexpr int MAIN = 2 * 2 * RAW + 2 * HBYTES;      // 2 stages x (K,V) raw + f16 K,V
-    static constexpr int BYTES = MAIN > MERGE ? MAIN : MERGE;
+    static constexpr int MAIN = NST * 2 * RAW + 2 * HBYTES;    // stages x (K,V) raw + f16 K,V
+    static constexpr int BYTES = (MAIN > MERGE ? MAIN : MERGE) + 64 + 128;  // + stage barriers, alignment
     static constexpr int PIECE = (ROWB % 8 == 0) ? 8 : 4;      // cp.async granule
 };
 
@@ -147,17 +154,20 @@ ARC_DEV void cp_async_n(void *dst, const void *src)
 template <int N>
 ARC_DEV void cp_async_wait_n() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int KVT, int D>
+template <int KVT, int D, bool TMA>
 __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_constant__ DecodeParams p)
 {
-    using L = DecLayout<KVT, D>;
+    using L = DecLayout<KVT, D, TMA>;
     constexpr int KS = D / 16;    // k-steps of S
     constexpr int NT_O = D / 8;   // n-tiles of O
 
-    extern __shared__ __align__(16) uint8_t smem[];
-    uint8_t *raw = smem;                                   // [2 stages][K, V][RAW]
-    __half *kh = reinterpret_cast<__half *>(smem + 4 * L::RAW);
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // TMA destinations 128-byte aligned (every tile size below is a multiple of 128)
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *raw = smem;                                   // [NST stages][K, V][RAW]
+    __half *kh = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW);
     __half *vh = kh + DT * L::HSTRIDE;
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BYTES - 128 - 64);   // TMA stage barriers
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
@@ -205,13 +215,34 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
     const uint8_t *kbase = p.k_cache + (int64_t)kvh * L::ROWB;
     const uint8_t *vbase = p.v_cache + (int64_t)kvh * L::ROWB;
     const int64_t cell_stride = (int64_t)p.Hkv * L::ROWB;
+    const int pad = TMA ? (L::ROWB * kvh) & 15 : 0;       // head row offset inside a smem row
+    const int x0 = L::ROWB * kvh - pad;                    // 16-byte aligned box start (bytes)
 
+    if (TMA) {
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < L::NST; ++i) mbar_init(&full[i], 1);
+            fence_mbar_init();
+        }
+        __syncthreads();
+    }
+    // Tile i: TMA into stage i % NST (thread 0), completion on full[i % NST].
+    auto issue_tma = [&](int i) {
+        if (threadIdx.x == 0) {
+            const int st = i % L::NST;
+            uint8_t *dk = raw + st * 2 * L::RAW;
+            mbar_arrive_expect_tx(&full[st], 2 * L::RAW);
+            const int row = sq.kv_begin + c_begin + i * DT;
+            tma_load_2d(dk, &p.tm_kc, &full[st], x0, row);
+            tma_load_2d(dk + L::RAW, &p.tm_vc, &full[st], x0, row);
+        }
+    };
     auto issue = [&](int i) {
         uint8_t *dk = raw + (i & 1) * 2 * L::RAW;
         uint8_t *dv = dk + L::RAW;
         const int key0 = c_begin + i * DT;
         constexpr int PR = L::ROWB / L::PIECE;  // pieces per row (<= 32): one lane each
         static_assert(PR <= 32, "a head row must fit one warp instruction");
+        static_assert(!TMA || L::RAW % 128 == 0, "TMA tiles keep 128-byte alignment");
         if (lane < PR) {
             const int off = lane * L::PIECE;
 #pragma unroll 4
@@ -225,28 +256,47 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
-    if (n_tiles > 0) issue(0);
-    if (n_tiles > 1) issue(1);
+    if (TMA) {
+        for (int i = 0; i < L::NST && i < n_tiles; ++i) issue_tma(i);
+    } else {
+        if (n_tiles > 0) issue(0);
+        if (n_tiles > 1) issue(1);
+    }
+    bool ok = true;
     const uint32_t kh_s = smem_u32(kh), vh_s = smem_u32(vh);
     for (int i = 0; i < n_tiles; ++i) {
-        if (i + 1 < n_tiles)
-            cp_async_wait_n<1>();
-        else
-            cp_async_wait_n<0>();
+        if (TMA) {
+            ok = mbar_wait(&full[i % L::NST], (uint32_t)((i / L::NST) & 1)) && ok;
+        } else {
+            if (i + 1 < n_tiles)
+                cp_async_wait_n<1>();
+            else
+                cp_async_wait_n<0>();
+        }
         __syncthreads();  // raw tile i visible; every warp is done with the f16 tiles of tile i-1
         {
-            const uint8_t *rk = raw + (i & 1) * 2 * L::RAW;
+            const uint8_t *rk = raw + (TMA ? (i % L::NST) : (i & 1)) * 2 * L::RAW + pad;
             const uint8_t *rv = rk + L::RAW;
+            const int valid = c_end - (c_begin + i * DT);     // rows of this tile inside the chunk
             constexpr int GROUPS = DT * (D / 8);
 #pragma unroll 2
             for (int x = threadIdx.x; x < GROUPS; x += WARPS * 32) {
                 const int r = x / (D / 8), grp = x % (D / 8);  // D / 8 is a power of two
-                *reinterpret_cast<uint4 *>(kh + r * L::HSTRIDE + grp * 8) = dequant8<KVT>(rk + r * L::ROWB, grp);
-                *reinterpret_cast<uint4 *>(vh + r * L::HSTRIDE + grp * 8) = dequant8<KVT>(rv + r * L::ROWB, grp);
+                uint4 kq = make_uint4(0, 0, 0, 0), vq = kq;
+                if (!TMA || r < valid) {  // a TMA box may run past the chunk into unused cells: zeros there
+                    kq = dequant8<KVT>(rk + r * L::RS, grp);
+                    vq = dequant8<KVT>(rv + r * L::RS, grp);
+                }
+                *reinterpret_cast<uint4 *>(kh + r * L::HSTRIDE + grp * 8) = kq;
+                *reinterpret_cast<uint4 *>(vh + r * L::HSTRIDE + grp * 8) = vq;
             }
         }
-        __syncthreads();  // f16 tiles ready; raw stage (i & 1) is free again
-        if (i + 2 < n_tiles) issue(i + 2);
+        __syncthreads();  // f16 tiles ready; the raw stage of tile i is free again
+        if (TMA) {
+            if (i + L::NST < n_tiles) issue_tma(i + L::NST);
+        } else {
+            if (i + 2 < n_tiles) issue(i + 2);
+        }
 
         const int kw = warp * 16;                      // this warp's 16 keys of the tile
         const int key0 = c_begin + i * DT + kw;
@@ -356,6 +406,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
             p.ws_ml[(part * 16 + r) * 2 + 1] = ll;
         }
     }
+    if (!ok && threadIdx.x == 0) report(p.status, ST_TIMEOUT_LOAD);
     // Let the merge kernel start its prologue; it waits for this grid's writes.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -398,11 +449,11 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
     if (d == 0) p.lse[(int64_t)tok * p.H + h] = ll > 0.f ? (mm + log2f(ll)) * LN2 : -INFINITY;
 }
 
-template <int KVT, int D>
+template <int KVT, int D, bool TMA>
 cudaError_t launch_t(const DecodeParams &p, cudaStream_t s)
 {
-    using L = DecLayout<KVT, D>;
-    auto k1 = decode_split_kernel<KVT, D>;
+    using L = DecLayout<KVT, D, TMA>;
+    auto k1 = decode_split_kernel<KVT, D, TMA>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
     const int grid = p.n_seq * p.Hkv * p.splits;
@@ -424,25 +475,42 @@ cudaError_t launch_t(const DecodeParams &p, cudaStream_t s)
     return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
 }
 
+template <bool TMA>
+int smem_t(int kv_type, int D)
+{
+    if (kv_type == ARC_KV_Q8_0)
+        return D == 64 ? DecLayout<ARC_KV_Q8_0, 64, TMA>::BYTES : DecLayout<ARC_KV_Q8_0, 128, TMA>::BYTES;
+    return D == 64 ? DecLayout<ARC_KV_Q4_0, 64, TMA>::BYTES : DecLayout<ARC_KV_Q4_0, 128, TMA>::BYTES;
+}
+
+template <bool TMA>
+cudaError_t launch_k(const DecodeParams &p, cudaStream_t s)
+{
+    if (p.kv_type == ARC_KV_Q8_0) {
+        if (p.D == 64) return launch_t<ARC_KV_Q8_0, 64, TMA>(p, s);
+        if (p.D == 128) return launch_t<ARC_KV_Q8_0, 128, TMA>(p, s);
+    } else {
+        if (p.D == 64) return launch_t<ARC_KV_Q4_0, 64, TMA>(p, s);
+        if (p.D == 128) return launch_t<ARC_KV_Q4_0, 128, TMA>(p, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
-int decode_smem_bytes(int kv_type, int D)
+int decode_smem_bytes(int kv_type, int D, bool tma) { return tma ? smem_t<true>(kv_type, D) : smem_t<false>(kv_type, D); }
+
+// Box width in bytes of the TMA path (covers a head row from the 16-byte boundary below it).
+int decode_box_bytes(int kv_type, int D)
 {
-    if (kv_type == ARC_KV_Q8_0) return D == 64 ? DecLayout<ARC_KV_Q8_0, 64>::BYTES : DecLayout<ARC_KV_Q8_0, 128>::BYTES;
-    return D == 64 ? DecLayout<ARC_KV_Q4_0, 64>::BYTES : DecLayout<ARC_KV_Q4_0, 128>::BYTES;
+    if (kv_type == ARC_KV_Q8_0) return D == 64 ? DecLayout<ARC_KV_Q8_0, 64, true>::RS : DecLayout<ARC_KV_Q8_0, 128, true>::RS;
+    return D == 64 ? DecLayout<ARC_KV_Q4_0, 64, true>::RS : DecLayout<ARC_KV_Q4_0, 128, true>::RS;
 }
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s)
 {
     if (p.splits > 256) return cudaErrorInvalidValue;
-    if (p.kv_type == ARC_KV_Q8_0) {
-        if (p.D == 64) return launch_t<ARC_KV_Q8_0, 64>(p, s);
-        if (p.D == 128) return launch_t<ARC_KV_Q8_0, 128>(p, s);
-    } else {
-        if (p.D == 64) return launch_t<ARC_KV_Q4_0, 64>(p, s);
-        if (p.D == 128) return launch_t<ARC_KV_Q4_0, 128>(p, s);
-    }
-    return cudaErrorInvalidValue;
+    return p.tma ? launch_k<true>(p, s) : launch_k<false>(p, s);
 }
 
 }  // namespace arc

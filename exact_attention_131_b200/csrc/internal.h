@@ -102,6 +102,9 @@ cudaError_t launch_sparse_tc(const SparseTcParams &p, cudaStream_t s);
 
 // ---------------------------------------------------------------- quantised decode
 struct DecodeParams {
+    CUtensorMap tm_kc;  // k_cache as bytes {Hkv*row bytes, n_cells}, box {row span, 64 cells} (tma != 0)
+    CUtensorMap tm_vc;  // v_cache likewise
+    int tma;            // 1: K/V tiles arrive by TMA through a multi-stage ring; 0: cp.async
     int kv_type, n_tok, H, Hkv, D, n_seq, splits, chunk;
     const float *q;
     const uint8_t *k_cache, *v_cache;
