@@ -411,6 +411,300 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Warp-specialised split kernel (TMA path).  Warp 4 streams raw K/V tiles of 64
+// cells into a ring of NST stages; each of warps 0-3 owns 16 cells of every
+// tile: it dequantises just those rows into its own f16 buffers, releases the
+// raw stage (one arrive per warp on empty[stage]) and runs its MMAs.  No
+// CTA-wide barrier inside the loop, so the four warps drift independently and
+// hide one another's latencies.
+constexpr int WS_WARPS = 5;
+
+template <int KVT, int D>
+struct WsLayout {
+    static constexpr int ROWB = (D / 32) * Fmt<KVT>::BB;
+    static constexpr int RS = ((ROWB + 16 - gcd16(ROWB) + 15) / 16) * 16;   // smem row stride of a raw tile
+    static constexpr int RAW = DT * RS;
+    static constexpr int NST = KVT == ARC_KV_Q8_0 ? 2 : 3;          // three CTAs per SM fit
+    static constexpr int WROWS = DT / WARPS;                                  // cells per consumer warp
+    static constexpr int HSTRIDE = D + 8;
+    static constexpr int HW = WROWS * HSTRIDE * 2;                            // one f16 buffer (K or V) of a warp
+    static constexpr int QB = 16 * HSTRIDE * 2;                               // Q tile (f16, pre-scaled)
+    static constexpr int MAIN = NST * 2 * RAW + WARPS * 2 * HW + QB;
+    static constexpr int MERGE = WARPS * 16 * (D + 2) * 4;
+    static constexpr int BYTES = (MAIN > MERGE ? MAIN : MERGE) + 128 + 128;  // + barriers, alignment
+};
+
+// Dequantise one whole block (32 values) of a raw row into 32 halves at dst
+// (16-byte aligned).  `row` is 4-byte aligned; the block starts at byte
+// blk*BB, which is 2 bytes off a word boundary for even blocks: the words are
+// read aligned and realigned with one byte permute each.
+template <int KVT>
+ARC_DEV void dequant_block(const uint8_t *row, int blk, __half *dst)
+{
+    constexpr int BB = Fmt<KVT>::BB;
+    constexpr int NW = (BB + 2 + 3) / 4 + 1;          // aligned words covering the block (9 or 5)
+    const int off = blk * BB;
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + (off & ~3));
+    const bool odd = (off & 2) != 0;                  // block starts 2 bytes into a word
+    uint32_t W[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) W[k] = w[k];
+    const uint32_t sel = odd ? 0x7654u : 0x5432u;     // data word k = bytes 2+4k .. of the block
+    const __half2 sc = bits_h2(__byte_perm(W[0], 0u, odd ? 0x3232u : 0x1010u));
+    uint4 *out = reinterpret_cast<uint4 *>(dst);
+    if constexpr (KVT == ARC_KV_Q8_0) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {                 // 8 values per 16-byte store
+            __half2 h0, h1, h2, h3;
+            s8x4_to_h2x2(__byte_perm(W[2 * q], W[2 * q + 1], sel), h0, h1);
+            s8x4_to_h2x2(__byte_perm(W[2 * q + 1], W[2 * q + 2], sel), h2, h3);
+            out[q] = make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)), h2_bits(__hmul2(h2, sc)),
+                                h2_bits(__hmul2(h3, sc)));
+        }
+    } else {
+        uint32_t d[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) d[k] = __byte_perm(W[k], W[k + 1], sel);
+#pragma unroll
+        for (int half = 0; half < 2; ++half)          // low nibbles: values 0..15, high: 16..31
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const uint32_t a = half ? (d[2 * q] >> 4) & 0x0F0F0F0Fu : d[2 * q] & 0x0F0F0F0Fu;
+                const uint32_t b = half ? (d[2 * q + 1] >> 4) & 0x0F0F0F0Fu : d[2 * q + 1] & 0x0F0F0F0Fu;
+                __half2 h0, h1, h2, h3;
+                u4x4_to_h2x2(a, h0, h1);
+                u4x4_to_h2x2(b, h2, h3);
+                out[half * 2 + q] = make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)),
+                                               h2_bits(__hmul2(h2, sc)), h2_bits(__hmul2(h3, sc)));
+            }
+    }
+}
+
+template <int KVT, int D>
+__global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __grid_constant__ DecodeParams p)
+{
+    using L = WsLayout<KVT, D>;
+    constexpr int KS = D / 16;
+    constexpr int NT_O = D / 8;
+    constexpr int NB = D / 32;                        // blocks per row
+
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *raw = smem;                                            // [NST][K, V][RAW]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BYTES - 256);
+    uint64_t *empty = full + L::NST;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, tq = lane & 3;
+    const int s = blockIdx.x / (p.Hkv * p.splits);
+    const int kvh = (blockIdx.x / p.splits) % p.Hkv;
+    const int sp = blockIdx.x % p.splits;
+    const arc_seq sq = p.seqs[s];
+    const int G = p.H / p.Hkv;
+    const int M = G * sq.n_q;
+    const int c_begin = sp * p.chunk;
+    const int c_end = min(c_begin + p.chunk, sq.n_kv);
+    const int n_tiles = c_end > c_begin ? (c_end - c_begin + DT - 1) / DT : 0;
+    const int pad = (L::ROWB * kvh) & 15;
+    const int x0 = L::ROWB * kvh - pad;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < L::NST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], WARPS);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    float o[NT_O][4];
+#pragma unroll
+    for (int i = 0; i < NT_O; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
+    bool ok = true;
+
+    if (warp == WARPS) {
+        // =============================== producer
+        if (lane == 0) {
+            for (int i = 0; i < n_tiles && ok; ++i) {
+                const int st = i % L::NST;
+                if (i >= L::NST) ok = mbar_wait(&empty[st], (uint32_t)((i / L::NST - 1) & 1));
+                if (!ok) break;
+                uint8_t *dk = raw + st * 2 * L::RAW;
+                mbar_arrive_expect_tx(&full[st], 2 * L::RAW);
+                const int row = sq.kv_begin + c_begin + i * DT;
+                tma_load_2d(dk, &p.tm_kc, &full[st], x0, row);
+                tma_load_2d(dk + L::RAW, &p.tm_vc, &full[st], x0, row);
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_LOAD);
+        }
+    } else {
+        // =============================== consumer warp: 16 cells of each tile
+        __half *kb = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW + warp * 2 * L::HW);
+        __half *vb = kb + L::WROWS * L::HSTRIDE;
+        __half *qs = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW + WARPS * 2 * L::HW);
+        const uint32_t kb_s = smem_u32(kb), vb_s = smem_u32(vb), qs_s = smem_u32(qs);
+        int row_t[2];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int r = g + 8 * hr;
+            row_t[hr] = (r < M) ? r % sq.n_q : -1;
+        }
+        // Q tile, shared by the four warps: 16 fold rows x D, scaled into log2 units, f16.
+        for (int x = threadIdx.x; x < 16 * D / 2; x += WARPS * 32) {
+            const int r = x / (D / 2), d = (x % (D / 2)) * 2;
+            float2 v = make_float2(0.f, 0.f);
+            if (r < M) {
+                const int h = kvh * G + r / sq.n_q;
+                const int tok = sq.q_begin + r % sq.n_q;
+                v = *reinterpret_cast<const float2 *>(p.q + ((int64_t)tok * p.H + h) * D + d);
+            }
+            *reinterpret_cast<__half2 *>(qs + r * L::HSTRIDE + d) = __floats2half2_rn(v.x * p.scale_log2, v.y * p.scale_log2);
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32) : "memory");   // consumer warps only
+        for (int i = 0; i < n_tiles; ++i) {
+            const int st = i % L::NST;
+            ok = mbar_wait(&full[st], (uint32_t)((i / L::NST) & 1)) && ok;
+            const int kw0 = i * DT + warp * L::WROWS;              // first cell (chunk-relative) of this warp
+            const int valid = c_end - c_begin - kw0;               // rows of this warp inside the chunk
+            {
+                const uint8_t *rk = raw + st * 2 * L::RAW + warp * L::WROWS * L::RS + pad;
+                // 2 x 16 rows x NB blocks; lanes 0-15 take rows 0-15 of one block, 16-31 the next
+#pragma unroll
+                for (int k = 0; k < 2 * NB * L::WROWS / 32; ++k) {
+                    const int J = k * 32 + lane;
+                    const int which = J / (NB * L::WROWS);         // 0: K, 1: V
+                    const int rem = J % (NB * L::WROWS);
+                    const int b = rem / L::WROWS, rr = rem % L::WROWS;
+                    __half *dst = (which ? vb : kb) + rr * L::HSTRIDE + b * 32;
+                    if (rr < valid) {
+                        dequant_block<KVT>(rk + which * L::RAW + rr * L::RS, b, dst);
+                    } else {
+                        uint4 *z = reinterpret_cast<uint4 *>(dst);
+                        z[0] = z[1] = z[2] = z[3] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);                // this warp is done with the raw stage
+
+            const int key0 = c_begin + kw0;
+            float sacc[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+                const int krow = nt * 8 + (lane & 7);
+#pragma unroll
+                for (int ks = 0; ks < KS; ks += 2) {
+                    uint32_t b0, b1, b2, b3, qa0[4], qa1[4];
+                    ldsm_x4(kb_s + (krow * L::HSTRIDE + ks * 16 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
+                    ldsm_x4(qs_s + ((lane & 15) * L::HSTRIDE + ks * 16 + (lane >> 4) * 8) * 2, qa0[0], qa0[1], qa0[2],
+                            qa0[3]);
+                    ldsm_x4(qs_s + ((lane & 15) * L::HSTRIDE + (ks + 1) * 16 + (lane >> 4) * 8) * 2, qa1[0], qa1[1],
+                            qa1[2], qa1[3]);
+                    mma16816(sacc[nt], qa0, b0, b1);
+                    mma16816(sacc[nt], qa1, b2, b3);
+                }
+            }
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int lim = row_t[hr] < 0 ? -1 : sq.n_kv - sq.n_q + row_t[hr];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int key = key0 + nt * 8 + 2 * tq + e;
+                        if (key >= c_end || key > lim) sacc[nt][2 * hr + e] = -INFINITY;
+                    }
+            }
+            uint32_t pa[4];
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                float mx = fmaxf(fmaxf(sacc[0][2 * hr], sacc[0][2 * hr + 1]), fmaxf(sacc[1][2 * hr], sacc[1][2 * hr + 1]));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                const float m_new = fmaxf(m_r[hr], mx);
+                const float msafe = (m_new == -INFINITY) ? 0.f : m_new;
+                const float alpha = (m_r[hr] == -INFINITY) ? 0.f : fast_exp2(m_r[hr] - msafe);
+                m_r[hr] = m_new;
+                const float p00 = fast_exp2(sacc[0][2 * hr] - msafe), p01 = fast_exp2(sacc[0][2 * hr + 1] - msafe);
+                const float p10 = fast_exp2(sacc[1][2 * hr] - msafe), p11 = fast_exp2(sacc[1][2 * hr + 1] - msafe);
+                l_r[hr] = l_r[hr] * alpha + (p00 + p01 + p10 + p11);
+                if (alpha != 1.f) {
+#pragma unroll
+                    for (int i2 = 0; i2 < NT_O; ++i2) {
+                        o[i2][2 * hr] *= alpha;
+                        o[i2][2 * hr + 1] *= alpha;
+                    }
+                }
+                pa[hr] = h2_bits(__floats2half2_rn(p00, p01));
+                pa[2 + hr] = h2_bits(__floats2half2_rn(p10, p11));
+            }
+            const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int nd = 0; nd < NT_O; nd += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vb_s + (vrow * L::HSTRIDE + nd * 8 + (lane >> 4) * 8) * 2, b0, b1, b2, b3);
+                mma16816(o[nd], pa, b0, b1);
+                mma16816(o[nd + 1], pa, b2, b3);
+            }
+            __syncwarp();   // every lane's ldmatrix of this warp's buffers is done before the next dequant
+        }
+        if (!ok && lane == 0) report(p.status, ST_TIMEOUT_LOAD);
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 1);
+            l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 2);
+        }
+    }
+
+    // ---- merge the 4 consumer warps (the raw ring and f16 buffers are idle now)
+    __syncthreads();
+    float *so = reinterpret_cast<float *>(smem);
+    float *sml = so + WARPS * 16 * D;
+    if (warp < WARPS) {
+#pragma unroll
+        for (int nd = 0; nd < NT_O; ++nd)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                float *dst = so + ((warp * 16) + g + 8 * hr) * D + nd * 8 + 2 * tq;
+                dst[0] = o[nd][2 * hr];
+                dst[1] = o[nd][2 * hr + 1];
+            }
+        if (tq == 0) {
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                sml[(warp * 16 + g + 8 * hr) * 2 + 0] = m_r[hr];
+                sml[(warp * 16 + g + 8 * hr) * 2 + 1] = l_r[hr];
+            }
+        }
+    }
+    __syncthreads();
+    const int64_t part = (int64_t)blockIdx.x;
+    for (int x = threadIdx.x; x < 16 * D; x += WS_WARPS * 32) {
+        const int r = x / D, d = x % D;
+        float mm = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) mm = fmaxf(mm, sml[(w * 16 + r) * 2]);
+        const float ms = (mm == -INFINITY) ? 0.f : mm;
+        float acc = 0.f, ll = 0.f;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) {
+            const float mw = sml[(w * 16 + r) * 2];
+            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - ms);
+            acc += f * so[(w * 16 + r) * D + d];
+            ll += f * sml[(w * 16 + r) * 2 + 1];
+        }
+        p.ws_o[(part * 16 + r) * D + d] = acc;
+        if (d == 0) {
+            p.ws_ml[(part * 16 + r) * 2 + 0] = mm;
+            p.ws_ml[(part * 16 + r) * 2 + 1] = ll;
+        }
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Merge the chunk partials of one (sequence, kv head, fold row) by their
 // log-sum-exp weights, normalise, write O and LSE.
 template <int D>
@@ -452,13 +746,20 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
 template <int KVT, int D, bool TMA>
 cudaError_t launch_t(const DecodeParams &p, cudaStream_t s)
 {
-    using L = DecLayout<KVT, D, TMA>;
-    auto k1 = decode_split_kernel<KVT, D, TMA>;
-    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
-    if (e != cudaSuccess) return e;
     const int grid = p.n_seq * p.Hkv * p.splits;
     if (grid == 0) return cudaSuccess;
-    k1<<<grid, WARPS * 32, L::BYTES, s>>>(p);
+    cudaError_t e;
+    if (TMA) {
+        auto k1 = decode_ws_kernel<KVT, D>;
+        const int bytes = WsLayout<KVT, D>::BYTES;
+        if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+        k1<<<grid, WS_WARPS * 32, bytes, s>>>(p);
+    } else {
+        auto k1 = decode_split_kernel<KVT, D, false>;
+        const int bytes = DecLayout<KVT, D, false>::BYTES;
+        if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+        k1<<<grid, WARPS * 32, bytes, s>>>(p);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // The merge launches as a programmatic dependent: its launch overlaps the
     // split kernel's tail and it waits (griddepcontrol.wait) for the partials.
@@ -478,9 +779,13 @@ cudaError_t launch_t(const DecodeParams &p, cudaStream_t s)
 template <bool TMA>
 int smem_t(int kv_type, int D)
 {
+    if (TMA) {
+        if (kv_type == ARC_KV_Q8_0) return D == 64 ? WsLayout<ARC_KV_Q8_0, 64>::BYTES : WsLayout<ARC_KV_Q8_0, 128>::BYTES;
+        return D == 64 ? WsLayout<ARC_KV_Q4_0, 64>::BYTES : WsLayout<ARC_KV_Q4_0, 128>::BYTES;
+    }
     if (kv_type == ARC_KV_Q8_0)
-        return D == 64 ? DecLayout<ARC_KV_Q8_0, 64, TMA>::BYTES : DecLayout<ARC_KV_Q8_0, 128, TMA>::BYTES;
-    return D == 64 ? DecLayout<ARC_KV_Q4_0, 64, TMA>::BYTES : DecLayout<ARC_KV_Q4_0, 128, TMA>::BYTES;
+        return D == 64 ? DecLayout<ARC_KV_Q8_0, 64, false>::BYTES : DecLayout<ARC_KV_Q8_0, 128, false>::BYTES;
+    return D == 64 ? DecLayout<ARC_KV_Q4_0, 64, false>::BYTES : DecLayout<ARC_KV_Q4_0, 128, false>::BYTES;
 }
 
 template <bool TMA>
