@@ -210,7 +210,7 @@ def kernel_source_hash(kernel):
              "sparse_tc_kernel": "sparse_tc.cu", "simple_attn_kernel<sparse>": "simple_kernels.cu",
              "simple_attn_kernel": "simple_kernels.cu"}
     f = files.get(kernel)
-    if kernel.startswith("decode_split_kernel"):
+    if kernel.startswith("decode_split_kernel") or kernel.startswith("decode_ws_kernel"):
         f = "decode.cu"
     if not f:
         return None

@@ -635,7 +635,10 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
                 !make_map_bytes(&p.tm_vc, a->v_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64))
                 return ARC_ERR_CUDA;
         }
-        note_dispatch(a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
+        if (p.tma)
+            note_dispatch(a->kv_type == ARC_KV_Q8_0 ? "decode_ws_kernel<q8_0>" : "decode_ws_kernel<q4_0>");
+        else
+            note_dispatch(a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
         e = launch_decode(p, s);
     }
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
@@ -751,11 +754,17 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             set_name(out, "simple_decode_kernel");
             out->launches = 1;
         } else {
-            set_name(out, a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
+            // the TMA kernel needs 16-byte aligned caches; arc_plan reports the shape's choice
+            const bool tma = pl.tma && (reinterpret_cast<uintptr_t>(a->k_cache) & 15) == 0 &&
+                             (reinterpret_cast<uintptr_t>(a->v_cache) & 15) == 0;
+            if (tma)
+                set_name(out, a->kv_type == ARC_KV_Q8_0 ? "decode_ws_kernel<q8_0>" : "decode_ws_kernel<q4_0>");
+            else
+                set_name(out, a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
             out->tensor_cores = 1;
             out->tile_m = 16, out->tile_n = 32, out->d_slice = a->D;
             out->splits = pl.splits, out->n_ctas = a->n_seq * a->Hkv * pl.splits;
-            out->smem_bytes = decode_smem_bytes(a->kv_type, a->D, pl.tma);
+            out->smem_bytes = decode_smem_bytes(a->kv_type, a->D, tma);
             out->launches = 2;
         }
         return ARC_OK;

@@ -200,7 +200,8 @@ def test_config5_decode_full(kv_type):
     o, lse, (q, kc, vc) = run_decode(c, status=st)
     info = arc.plan_decode(kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
                            n_kv=c.n_kv)
-    assert info["kernel"].startswith("decode_split_kernel") and info["splits"] > 1
+    # 16-byte aligned caches with a 16-byte multiple cell stride take the TMA kernel
+    assert info["kernel"].startswith("decode_ws_kernel") and info["splits"] > 1
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
     assert arc.check_device_error(st) == arc.ARC_OK
@@ -213,6 +214,23 @@ def test_decode_ragged_sequences(kv_type):
     o, lse, _ = run_decode(c)
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
+
+
+@pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
+@pytest.mark.parametrize("H,Hkv,D,kernel", [
+    (6, 3, 128, "decode_split_kernel"),   # cell = 3 head rows (408 / 216 bytes): no TMA, cp.async path
+    (16, 4, 64, "decode_ws_kernel"),      # cell = 4 rows of 68 / 36 bytes = 272 / 144: TMA path at D = 64
+])
+def test_decode_both_load_paths(kv_type, H, Hkv, D, kernel):
+    c = W.decode_case(3, 2, 700, H, Hkv, D, kv_type=kv_type, seed=40)
+    st = status_word()
+    o, lse, (q, kc, vc) = run_decode(c, status=st)
+    info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                           n_kv=c.n_kv)
+    assert info["kernel"].startswith(kernel)
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
 
 
 def test_decode_head_dim_64_and_control_arm():
