@@ -283,6 +283,23 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
     raise TypeError(type(case))
 
 
+def max_over_ranks(x, world, device):
+    """The largest x over all ranks; every rank takes this collective step."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step, world, steps, total_ms, unit_kind):
+    """Whole-job rate: the units all ranks processed over the slowest rank's time."""
+    scale = 1e12 if unit_kind == "flop" else 1e9
+    return units_per_step * world * steps / (total_ms * 1e-3) / scale
+
+
 def run_ours(args, spec, case):
     import torch
     import torch.distributed as dist
@@ -327,10 +344,7 @@ def run_ours(args, spec, case):
     times_ms = [a.elapsed_time(b) for a, b in ev]
     mean_ms = sum(times_ms) / len(times_ms)
     total_ms = sum(times_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, "cuda")
     assert arc.check_device_error(status) == arc.ARC_OK, "a device-side wait timed out"
 
     # ---- end to end through the public API with host buffers: H2D of the inputs from
@@ -357,7 +371,7 @@ def run_ours(args, spec, case):
 
     peaks = load_peaks()
     if unit_kind == "flop":
-        value = units * world * args.steps / (total_ms * 1e-3) / 1e12
+        value = job_throughput(units, world, args.steps, total_ms, unit_kind)
         unit = "TFLOP/s"
         achieved = units / (mean_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -365,7 +379,7 @@ def run_ours(args, spec, case):
                 "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None}
         e2e_val = units / (e2e_mean * 1e-3) / 1e12
     else:
-        value = units * world * args.steps / (total_ms * 1e-3) / 1e9
+        value = job_throughput(units, world, args.steps, total_ms, unit_kind)
         unit = "GB/s"
         achieved = units / (mean_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
