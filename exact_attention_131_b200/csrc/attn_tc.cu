@@ -469,57 +469,60 @@ __global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_con
 
     if (warp == 0) {
         // =============================== TMA producer: Q_A, Q_B, then K(0), V(0), K(1), V(1), ...
-        if (lane == 0 && nt > 0) {
-            tma_prefetch_desc(&p.tm_q);
-            tma_prefetch_desc(&p.tm_k);
-            tma_prefetch_desc(&p.tm_v);
-            const int qrow = kv * rows_in_group + r0;
-            mbar_arrive_expect_tx(&bars->q_full, 2 * KC * CHUNK);
-            for (int t = 0; t < 2; ++t)
-                for (int c = 0; c < KC; ++c) {
-                    uint8_t *dst = sQ + (t * KC + c) * CHUNK;
-                    if (!MLA || c < p.kc_first)
-                        tma_load_3d(dst, &p.tm_q, &bars->q_full, c * 64, qrow + t * BM, b);
-                    else
-                        tma_load_3d(dst, &p.tm_q2, &bars->q_full, (c - p.kc_first) * 64, qrow + t * BM, b);
-                }
-            int stage = 0, total = 0;
-            uint32_t ephase = 0;
+        // A barrier round trip costs the issuing thread a few hundred clocks, so the
+        // KC + VC chunks of a tile are handled by that many lanes at once: each lane
+        // waits for its own ring slot and issues its own load.
+        if (nt > 0) {
+            if (lane == 0) {
+                tma_prefetch_desc(&p.tm_q);
+                tma_prefetch_desc(&p.tm_k);
+                tma_prefetch_desc(&p.tm_v);
+                const int qrow = kv * rows_in_group + r0;
+                mbar_arrive_expect_tx(&bars->q_full, 2 * KC * CHUNK);
+                for (int t = 0; t < 2; ++t)
+                    for (int c = 0; c < KC; ++c) {
+                        uint8_t *dst = sQ + (t * KC + c) * CHUNK;
+                        if (!MLA || c < p.kc_first)
+                            tma_load_3d(dst, &p.tm_q, &bars->q_full, c * 64, qrow + t * BM, b);
+                        else
+                            tma_load_3d(dst, &p.tm_q2, &bars->q_full, (c - p.kc_first) * 64, qrow + t * BM, b);
+                    }
+            }
+            __syncwarp();
+            constexpr int PER = KC + VC;   // chunks per KV tile (<= 32: one lane each)
+            static_assert(PER <= 32, "one lane per chunk of a tile");
+            const int total = nt * PER;
             bool ok = true;
-            auto acquire = [&]() -> bool {
-                if (!mbar_wait(&bars->empty[stage], ephase ^ 1u)) return false;
-                mbar_arrive_expect_tx(&bars->full[stage], CHUNK);
-                ++total;
-                return true;
-            };
-            auto advance = [&]() {
-                if (++stage == R) {
-                    stage = 0;
-                    ephase ^= 1u;
-                }
-            };
             for (int j = 0; ok && j < nt; ++j) {
-                for (int c = 0; ok && c < KC; ++c) {
-                    if (!(ok = acquire())) break;
-                    uint8_t *dst = sRing + stage * CHUNK;
-                    if (!MLA || c < p.kc_first)
-                        tma_load_4d(dst, &p.tm_k, &bars->full[stage], c * 64, j * BN, kv, b);
-                    else
-                        tma_load_3d(dst, &p.tm_k2, &bars->full[stage], (c - p.kc_first) * 64, j * BN, b);
-                    advance();
+                bool mine = true;
+                if (lane < PER) {
+                    const int n = j * PER + lane;                 // chunk index in the load sequence
+                    const int st = n % R;
+                    mine = mbar_wait(&bars->empty[st], (uint32_t)(((n / R) & 1) ^ 1));
+                    if (mine) {
+                        mbar_arrive_expect_tx(&bars->full[st], CHUNK);
+                        uint8_t *dst = sRing + st * CHUNK;
+                        if (lane < KC) {
+                            const int c = lane;
+                            if (!MLA || c < p.kc_first)
+                                tma_load_4d(dst, &p.tm_k, &bars->full[st], c * 64, j * BN, kv, b);
+                            else
+                                tma_load_3d(dst, &p.tm_k2, &bars->full[st], (c - p.kc_first) * 64, j * BN, b);
+                        } else {
+                            tma_load_4d(dst, &p.tm_v, &bars->full[st], (lane - KC) * 64, j * BN, kv, b);
+                        }
+                    }
                 }
-                for (int c = 0; ok && c < VC; ++c) {
-                    if (!(ok = acquire())) break;
-                    tma_load_4d(sRing + stage * CHUNK, &p.tm_v, &bars->full[stage], c * 64, j * BN, kv, b);
-                    advance();
+                ok = __all_sync(0xffffffffu, mine);
+            }
+            if (lane == 0) {
+                if (!ok) report(p.status, ST_TIMEOUT_LOAD);
+                for (int s = 0; s < R && s < total; ++s) {
+                    const int loads = (total - s + R - 1) / R;
+                    mbar_wait(&bars->full[s], (uint32_t)((loads - 1) & 1));
                 }
+                mbar_wait(&bars->q_full, 0);
             }
-            if (!ok) report(p.status, ST_TIMEOUT_LOAD);
-            for (int s = 0; s < R && s < total; ++s) {
-                const int loads = (total - s + R - 1) / R;
-                mbar_wait(&bars->full[s], (uint32_t)((loads - 1) & 1));
-            }
-            mbar_wait(&bars->q_full, 0);
         }
     } else if (warp == 1) {
         // =============================== MMA issuer
