@@ -253,7 +253,9 @@ AttnPlan plan_attn(const arc_attn_args *a)
     if (!pl.two && !(a->flags & ARC_FLAG_SINGLE_CTA) && pair_supported(a->D, pl.dvs)) {
         pl.pair = true;
         pl.stages = pair_max_stages(a->D);
-        pl.grid = ((pl.n_tiles + 1) / 2) * a->B * a->Hkv * 2;  // each pair runs every d_v slice
+        // persistent: at most one resident cluster per two SMs walks the list of row-tile pairs
+        const int items = ((pl.n_tiles + 1) / 2) * a->B * a->Hkv;
+        pl.grid = 2 * std::min(items, std::max(1, sm_count() / 2));
     }
     return pl;
 }

@@ -22,6 +22,8 @@
 // Every mbarrier wait is bounded and reports through p.status.
 #include <math.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -44,6 +46,7 @@ constexpr float P_RESCALE = 8.0f;
 
 struct PairBars {
     uint64_t q_full;
+    uint64_t q_empty;   // the last S of a row tile has read Q: the next tile's Q may land
     uint64_t s_full[2];
     uint64_t p_full;
     uint64_t o_done;
@@ -179,6 +182,34 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
 
 __device__ __forceinline__ bool warp_all_pair(bool ok) { return __all_sync(0xffffffffu, ok); }
 
+// The k-th item of cluster c out of C: items are ordered by decreasing work, and
+// round k hands them out left to right on even rounds and right to left on odd
+// ones, which evens out the clusters' totals.  Increases with k for every c.
+__device__ __forceinline__ int snake_item(int k, int c, int C) { return k * C + ((k & 1) ? C - 1 - c : c); }
+
+// One work item of the persistent pair kernel: 256 consecutive fold rows (rp ..)
+// of kv head kv of batch b, and the number of 128-key tiles they need.
+struct PairItem {
+    int b, kv, rp, nt;
+};
+
+__device__ __forceinline__ PairItem pair_item(const TcParams &p, int item)
+{
+    const int groups = p.B * p.Hkv;
+    const int prank = item / groups, rest = item % groups;
+    PairItem w;
+    w.kv = rest % p.Hkv;
+    w.b = rest / p.Hkv;
+    const int pair = prank < 1024 ? (int)p.tile_order[prank] : prank;
+    const int rows_in_group = p.G * p.Tq;
+    w.rp = pair * 2 * PBM;
+    const int r_last = min(w.rp + 2 * PBM, rows_in_group) - 1;
+    const int t_max = p.tmajor ? r_last / p.G : ((w.rp / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq);
+    const int kv_last = p.causal ? min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
+    w.nt = kv_last < 0 ? 0 : kv_last / PBN + 1;
+    return w;
+}
+
 // One 32-byte global store (a whole sector); dst must be 32-byte aligned.
 __device__ __forceinline__ void st_global_v8(void *dst, const uint32_t *w)
 {
@@ -206,31 +237,19 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
 
-    // ---- which rows this pair owns
-    // A pair computes every d_v slice of its rows in turn with Q resident: work
-    // item `it` is (slice it / nt, key tile it % nt).
-    const int cl = blockIdx.x >> 1;
-    const int groups = p.B * p.Hkv;
-    const int prank = cl / groups;
-    const int rest = cl % groups;
-    const int kv = rest % p.Hkv;
-    const int b = rest / p.Hkv;
+    // ---- persistent schedule: cluster c takes one item per round of a list ordered by
+    // decreasing work (snake order, see snake_item).  Within an item the pair computes every d_v slice
+    // of its rows in turn with Q resident: unit u of the item is (slice u / nt, key
+    // tile u % nt); units are numbered globally across items (S buffer u & 1 and
+    // the barrier parities follow the global number).
+    const int C = gridDim.x >> 1, c0 = blockIdx.x >> 1;
+    const int n_items = ((p.n_tiles + 1) / 2) * p.B * p.Hkv;
     const int NSL = p.n_slices;
-    const int pair = prank < 1024 ? (int)p.tile_order[prank] : prank;
     const int rows_in_group = p.G * p.Tq;
-    const int rp = pair * 2 * PBM;               // first row of the pair
-    const int r0 = rp + (int)rank * PBM;         // first row of this CTA
-    int nt;
-    {
-        const int r_last = min(rp + 2 * PBM, rows_in_group) - 1;
-        const int t_max = p.tmajor ? r_last / p.G : ((rp / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq);
-        const int kv_last = p.causal ? min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
-        nt = kv_last < 0 ? 0 : kv_last / PBN + 1;
-    }
-    const int NI = nt * NSL;                     // work items of the pair
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
+        mbar_init(&bars->q_empty, 1);
         for (int i = 0; i < 2; ++i) mbar_init(&bars->s_full[i], 1);
         mbar_init(&bars->p_full, 256);
         mbar_init(&bars->o_done, 1);
@@ -255,20 +274,12 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
 
     if (warp == 0) {
         // =============================== TMA producer (both CTAs, each its half)
-        if (lane == 0 && nt > 0) {
+        if (lane == 0) {
             tma_prefetch_desc(&p.tm_q);
             tma_prefetch_desc(&p.tm_k);
             tma_prefetch_desc(&p.tm_v);
             const uint32_t q_full_l = mapa(smem_u32(&bars->q_full), 0);
-            if (leader) mbar_arrive_expect_tx_u32(smem_u32(&bars->q_full), 2 * KC * 2 * PCH);
-            if (p.tmajor) {
-                // box {64, G, 128/G}: smem row = (t - t0) * G + head in group
-                for (int c = 0; c < KC; ++c) tma2_load_5d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, 0, r0 / p.G, kv, b);
-            } else {
-                const int qrow = kv * rows_in_group + r0;
-                for (int c = 0; c < KC; ++c) tma2_load_3d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, qrow, b);
-            }
-            int stage = 0;
+            int stage = 0, qn = 0;
             uint32_t ephase = 0;
             bool ok = true;
             // Each barrier round trip costs this thread a few hundred clocks, so a
@@ -285,52 +296,69 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 }
             };
             auto full_l = [&]() { return mapa(smem_u32(&bars->full[stage]), 0); };
-            auto load_k = [&](int j) -> bool {
-                for (int c0 = 0; c0 < KC; c0 += BPS) {
-                    if (!acquire()) return false;
-                    const uint32_t fl = full_l();
-                    for (int q = 0; q < BPS; ++q)
-                        tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_k, fl, (c0 + q) * 64,
-                                     j * PBN + (int)rank * 64, kv, b);
-                    advance();
+            for (int k = 0; ok && snake_item(k, c0, C) < n_items; ++k) {
+                const PairItem w = pair_item(p, snake_item(k, c0, C));
+                if (w.nt == 0) continue;
+                const int nt = w.nt, NI = nt * NSL, kv = w.kv, b = w.b;
+                const int r0 = w.rp + (int)rank * PBM;
+                // Q of this item replaces the previous item's once its last S has run
+                if (qn > 0 && !(ok = mbar_wait(&bars->q_empty, (uint32_t)((qn - 1) & 1)))) break;
+                if (leader) mbar_arrive_expect_tx_u32(smem_u32(&bars->q_full), 2 * KC * 2 * PCH);
+                if (p.tmajor) {
+                    // box {64, G, 128/G}: smem row = (t - t0) * G + head in group
+                    for (int c = 0; c < KC; ++c)
+                        tma2_load_5d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, 0, r0 / p.G, kv, b);
+                } else {
+                    const int qrow = kv * rows_in_group + r0;
+                    for (int c = 0; c < KC; ++c) tma2_load_3d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, qrow, b);
                 }
-                return true;
-            };
-            // V box q of a stage: 128-column group q / 2, key half q % 2
-            auto load_v = [&](int it) -> bool {
-                const int j = it % nt, dv0 = (it / nt) * DVS;
-                for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
-                    if (!acquire()) return false;
-                    const uint32_t fl = full_l();
-                    for (int q = 0; q < BPS; ++q) {
-                        const int g = (q0 + q) >> 1, hh = (q0 + q) & 1;
-                        tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_v, fl, dv0 + g * 128 + (int)rank * 64,
-                                     j * PBN + hh * 64, kv, b);
+                ++qn;
+                auto load_k = [&](int j) -> bool {
+                    for (int cc = 0; cc < KC; cc += BPS) {
+                        if (!acquire()) return false;
+                        const uint32_t fl = full_l();
+                        for (int q = 0; q < BPS; ++q)
+                            tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_k, fl, (cc + q) * 64,
+                                         j * PBN + (int)rank * 64, kv, b);
+                        advance();
                     }
-                    advance();
+                    return true;
+                };
+                // V box q of a stage: 128-column group q / 2, key half q % 2
+                auto load_v = [&](int it) -> bool {
+                    const int j = it % nt, dv0 = (it / nt) * DVS;
+                    for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
+                        if (!acquire()) return false;
+                        const uint32_t fl = full_l();
+                        for (int q = 0; q < BPS; ++q) {
+                            const int g = (q0 + q) >> 1, hh = (q0 + q) & 1;
+                            tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_v, fl, dv0 + g * 128 + (int)rank * 64,
+                                         j * PBN + hh * 64, kv, b);
+                        }
+                        advance();
+                    }
+                    return true;
+                };
+                ok = load_k(0);
+                for (int it = 0; ok && it < NI; ++it) {
+                    if (it + 1 < NI) ok = load_k((it + 1) % nt);
+                    if (ok) ok = load_v(it);
                 }
-                return true;
-            };
-            ok = load_k(0);
-            for (int it = 0; ok && it < NI; ++it) {
-                if (it + 1 < NI) ok = load_k((it + 1) % nt);
-                if (ok) ok = load_v(it);
             }
             if (!ok) report(p.status, ST_TIMEOUT_LOAD);
         }
     } else if (warp == 1) {
         // =============================== MMA issuer (leader only)
-        if (leader && lane == 0 && nt > 0) {
+        if (leader && lane == 0) {
             constexpr uint32_t kBox = PCH >> 4;       // descriptor units per 8 KB box
             const uint32_t idesc_s = idesc_bf16(2 * PBM, PBN, false, false);
             const uint32_t idesc_pv = idesc_bf16(2 * PBM, 128, false, true);
             const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t kd0 = sdesc_sw128(smem_u32(sRing), 16, 1024);
             const uint64_t vd0 = sdesc_sw128(smem_u32(sRing), 16, 1024);
-            int stage = 0;
+            int stage = 0, qn = 0, gu = 0;
             uint32_t fphase = 0;
-            bool ok = mbar_wait(&bars->q_full, 0);
-            tc_fence_after();
+            bool ok = true;
             auto advance = [&]() {
                 if (++stage == R) {
                     stage = 0;
@@ -371,8 +399,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 umma2_commit_both(&bars->s_full[it & 1]);
                 return true;
             };
-            auto issue_pv = [&](int it) -> bool {
-                const int first = (it % nt) == 0;     // first key tile of a slice overwrites O
+            auto issue_pv = [&](int it, bool first) -> bool {   // first key tile of a slice overwrites O
                 if (!mbar_wait_cluster(&bars->p_full, (uint32_t)(it & 1))) return false;
                 if (!wait_boxes(2 * VG / BPS)) return false;
                 tc_fence_after();
@@ -391,10 +418,24 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 umma2_commit_both(&bars->o_done);
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            for (int it = 0; ok && it < NI; ++it) {
-                if (it + 1 < NI) ok = issue_s(it + 1);
-                if (ok) ok = issue_pv(it);
+            for (int k = 0; ok && snake_item(k, c0, C) < n_items; ++k) {
+                const PairItem w = pair_item(p, snake_item(k, c0, C));
+                if (w.nt == 0) continue;
+                const int nt = w.nt, NI = nt * NSL;
+                if (!(ok = mbar_wait(&bars->q_full, (uint32_t)(qn & 1)))) break;
+                tc_fence_after();
+                ++qn;
+                // units gu .. gu + NI - 1; the last S of the item frees Q for the next one
+                ok = issue_s(gu);
+                if (ok && NI == 1) umma2_commit_both(&bars->q_empty);
+                for (int it = 0; ok && it < NI; ++it) {
+                    if (it + 1 < NI) {
+                        ok = issue_s(gu + it + 1);
+                        if (ok && it + 2 == NI) umma2_commit_both(&bars->q_empty);
+                    }
+                    if (ok) ok = issue_pv(gu + it, (it % nt) == 0);
+                }
+                gu += NI;
             }
             if (!ok) report(p.status, ST_TIMEOUT_MMA);
             umma2_commit_both(&bars->drain);
@@ -404,19 +445,23 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
         const int wq = warp & 3;
         const int r = wq * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        const int R_ = r0 + r;
+        const float sl2 = p.scale_log2;
+        const uint32_t p_full_l = mapa(smem_u32(&bars->p_full), 0);
+        bool ok = true;
+        int gu = 0;
+        for (int k = 0; ok && snake_item(k, c0, C) < n_items; ++k) {
+        const PairItem w = pair_item(p, snake_item(k, c0, C));
+        const int nt = w.nt, kv = w.kv, b = w.b;
+        const int R_ = w.rp + (int)rank * PBM + r;
         const bool row_ok = R_ < rows_in_group;
         const int t = p.tmajor ? R_ / p.G : R_ % p.Tq;
         const int h = kv * p.G + (p.tmajor ? R_ % p.G : R_ / p.Tq);
         const int last = p.causal ? min(p.Tk - 1, t + p.Tk - p.Tq) : p.Tk - 1;
-        const float sl2 = p.scale_log2;
-        const uint32_t p_full_l = mapa(smem_u32(&bars->p_full), 0);
-        bool ok = true;
-        for (int slice = 0; slice < NSL; ++slice) {
+        for (int slice = 0; ok && slice < NSL; ++slice) {
         const int dv0 = slice * DVS;
         float m_use = -INFINITY, l = 0.f;
         for (int j = 0; ok && j < nt; ++j) {
-            const int it = slice * nt + j;
+            const int it = gu + slice * nt + j;
             const int buf = it & 1;
             const uint32_t s_tmem = tmem + lane_off + P_SCOL + buf * PBN;
             ok = warp_all_pair(mbar_wait(&bars->s_full[buf], (uint32_t)((it >> 1) & 1)));
@@ -482,7 +527,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 mbar_arrive_remote(p_full_l);
         }
         if (ok && nt > 0) {
-            ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((slice * nt + nt - 1) & 1)));
+            ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((gu + slice * nt + nt - 1) & 1)));
             tc_fence_after();
         }
         float fac, lse;
@@ -536,6 +581,8 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
         }
         if (row_ok && slice == 0) p.lse[((int64_t)b * p.H + h) * p.Tq + t] = lse;
         }
+        gu += nt * NSL;
+        }
         if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
     }
 
@@ -543,7 +590,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
     // and their final commit has reached this CTA's barriers before either CTA
     // leaves; then release TMEM.
     __syncwarp();
-    if (warp == 1 && lane == 0 && nt > 0) mbar_wait(&bars->drain, 0);
+    if (warp == 1 && lane == 0) mbar_wait(&bars->drain, 0);
     __syncwarp();
     tc_fence_before();
     cluster_sync_all();
@@ -562,7 +609,6 @@ cudaError_t launch_p(const TcParams &p, int grid, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(P_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
@@ -573,6 +619,15 @@ cudaError_t launch_p(const TcParams &p, int grid, cudaStream_t s)
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    // Persistent: as many clusters as can be resident at once (each walks the item list).
+    cfg.gridDim = dim3(2);
+    int resident = 0;
+    if (cudaOccupancyMaxActiveClusters(&resident, kern, &cfg) != cudaSuccess || resident <= 0) {
+        cudaGetLastError();
+        resident = grid / 2;
+    }
+    const int clusters = std::max(1, std::min(grid / 2, resident));
+    cfg.gridDim = dim3(2 * clusters);
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 

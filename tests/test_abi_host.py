@@ -137,7 +137,9 @@ def test_plan_names_the_tensor_core_kernels(arc):
     a.o_strides = (arc._i64 * 3)(64 * 1400 * 512, 1400 * 512, 512)
     info = arc.plan(arc.ARC_OP_ATTN, a)
     assert info["kernel"] == "tc_attn_pair_kernel" and info["d_slice"] == 256 and info["tmem_cols"] == 512
-    assert info["n_ctas"] == 2 * 44 * 8            # 2 CTAs x ceil(8*1400/256) pairs x 8 kv heads (slices run in turn)
+    # persistent: one cluster per two SMs (148 on B200; the planner's default without a GPU)
+    # walks the 44 x 8 row-tile pairs, running both d_v slices of each in turn
+    assert info["n_ctas"] == 2 * min(44 * 8, 148 // 2)
     assert info["tile_m"] == 256
     a.flags = arc.ARC_FLAG_SINGLE_CTA
     info = arc.plan(arc.ARC_OP_ATTN, a)
