@@ -435,39 +435,44 @@ struct WsLayout {
     static constexpr int BYTES = (MAIN > MERGE ? MAIN : MERGE) + 128 + 128;  // + barriers, alignment
 };
 
-// Dequantise one whole block (32 values) of a raw row into 32 halves at dst
-// (16-byte aligned).  `row` is 4-byte aligned; the block starts at byte
-// blk*BB, which is 2 bytes off a word boundary for even blocks: the words are
-// read aligned and realigned with one byte permute each.
+// Dequantise the block that starts `off` bytes into a 16-byte-aligned raw row:
+// three (q8_0) or two (q4_0) aligned 16-byte loads cover it wherever it starts,
+// which with the 144 / 80-byte smem row stride touches 8 rows in distinct banks.
+// `off` is a compile-time constant at every call (unrolled loops, template pad),
+// so all byte positions below fold away.
 template <int KVT>
-ARC_DEV void dequant_block(const uint8_t *row, int blk, __half *dst)
+ARC_DEV void dequant_block16(const uint8_t *row, int off, __half *dst)
 {
-    constexpr int BB = Fmt<KVT>::BB;
-    constexpr int NW = (BB + 2 + 3) / 4 + 1;          // aligned words covering the block (9 or 5)
-    const int off = blk * BB;
-    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + (off & ~3));
-    const bool odd = (off & 2) != 0;                  // block starts 2 bytes into a word
-    uint32_t W[NW];
+    constexpr int N4 = KVT == ARC_KV_Q8_0 ? 3 : 2;
+    const uint4 *w4 = reinterpret_cast<const uint4 *>(row + (off & ~15));
+    const int o = off & 15;
+    uint32_t W[4 * N4];
 #pragma unroll
-    for (int k = 0; k < NW; ++k) W[k] = w[k];
-    const uint32_t sel = odd ? 0x7654u : 0x5432u;     // data word k = bytes 2+4k .. of the block
-    const __half2 sc = bits_h2(__byte_perm(W[0], 0u, odd ? 0x3232u : 0x1010u));
+    for (int i = 0; i < N4; ++i) {
+        const uint4 t = w4[i];
+        W[4 * i] = t.x, W[4 * i + 1] = t.y, W[4 * i + 2] = t.z, W[4 * i + 3] = t.w;
+    }
+    const __half2 sc = bits_h2(__byte_perm(W[o >> 2], 0u, (o & 2) ? 0x3232u : 0x1010u));
+    auto word = [&](int j) -> uint32_t {   // data bytes 4j .. 4j+3 of the block
+        const int b0 = o + 2 + 4 * j;
+        return (b0 & 3) ? __byte_perm(W[b0 >> 2], W[(b0 >> 2) + 1], 0x5432u) : W[b0 >> 2];
+    };
     uint4 *out = reinterpret_cast<uint4 *>(dst);
     if constexpr (KVT == ARC_KV_Q8_0) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {                 // 8 values per 16-byte store
+        for (int q = 0; q < 4; ++q) {
             __half2 h0, h1, h2, h3;
-            s8x4_to_h2x2(__byte_perm(W[2 * q], W[2 * q + 1], sel), h0, h1);
-            s8x4_to_h2x2(__byte_perm(W[2 * q + 1], W[2 * q + 2], sel), h2, h3);
+            s8x4_to_h2x2(word(2 * q), h0, h1);
+            s8x4_to_h2x2(word(2 * q + 1), h2, h3);
             out[q] = make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)), h2_bits(__hmul2(h2, sc)),
                                 h2_bits(__hmul2(h3, sc)));
         }
     } else {
         uint32_t d[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) d[k] = __byte_perm(W[k], W[k + 1], sel);
+        for (int k = 0; k < 4; ++k) d[k] = word(k);
 #pragma unroll
-        for (int half = 0; half < 2; ++half)          // low nibbles: values 0..15, high: 16..31
+        for (int half = 0; half < 2; ++half)
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
                 const uint32_t a = half ? (d[2 * q] >> 4) & 0x0F0F0F0Fu : d[2 * q] & 0x0F0F0F0Fu;
@@ -478,6 +483,26 @@ ARC_DEV void dequant_block(const uint8_t *row, int blk, __half *dst)
                 out[half * 2 + q] = make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)),
                                                h2_bits(__hmul2(h2, sc)), h2_bits(__hmul2(h3, sc)));
             }
+    }
+}
+
+// One consumer warp's 16 rows of a raw K/V tile (kvh's head row starts PAD bytes
+// into each 16-byte-aligned smem row) into its f16 buffers: at step k every lane
+// takes block k, lanes 0-15 of K rows 0-15 and lanes 16-31 of V rows 0-15.
+template <int KVT, int D, int PAD>
+ARC_DEV void dequant_warp_rows(const uint8_t *rk, int raw_bytes, int rs, int valid, __half *kb, __half *vb, int hstride)
+{
+    const int lane = threadIdx.x & 31, which = lane >> 4, rr = lane & 15;
+    const uint8_t *rowp = rk + which * raw_bytes + rr * rs;
+    __half *dst = (which ? vb : kb) + rr * hstride;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+        if (rr < valid) {
+            dequant_block16<KVT>(rowp, PAD + k * Fmt<KVT>::BB, dst + k * 32);
+        } else {
+            uint4 *z = reinterpret_cast<uint4 *>(dst + k * 32);
+            z[0] = z[1] = z[2] = z[3] = make_uint4(0, 0, 0, 0);
+        }
     }
 }
 
@@ -569,21 +594,12 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
             const int kw0 = i * DT + warp * L::WROWS;              // first cell (chunk-relative) of this warp
             const int valid = c_end - c_begin - kw0;               // rows of this warp inside the chunk
             {
-                const uint8_t *rk = raw + st * 2 * L::RAW + warp * L::WROWS * L::RS + pad;
-                // 2 x 16 rows x NB blocks; lanes 0-15 take rows 0-15 of one block, 16-31 the next
-#pragma unroll
-                for (int k = 0; k < 2 * NB * L::WROWS / 32; ++k) {
-                    const int J = k * 32 + lane;
-                    const int which = J / (NB * L::WROWS);         // 0: K, 1: V
-                    const int rem = J % (NB * L::WROWS);
-                    const int b = rem / L::WROWS, rr = rem % L::WROWS;
-                    __half *dst = (which ? vb : kb) + rr * L::HSTRIDE + b * 32;
-                    if (rr < valid) {
-                        dequant_block<KVT>(rk + which * L::RAW + rr * L::RS, b, dst);
-                    } else {
-                        uint4 *z = reinterpret_cast<uint4 *>(dst);
-                        z[0] = z[1] = z[2] = z[3] = make_uint4(0, 0, 0, 0);
-                    }
+                const uint8_t *rk = raw + st * 2 * L::RAW + warp * L::WROWS * L::RS;   // 16-byte aligned rows
+                switch (pad) {   // CTA-uniform
+                case 0: dequant_warp_rows<KVT, D, 0>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
+                case 4: dequant_warp_rows<KVT, D, 4>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
+                case 8: dequant_warp_rows<KVT, D, 8>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
+                default: dequant_warp_rows<KVT, D, 12>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
                 }
             }
             __syncwarp();
