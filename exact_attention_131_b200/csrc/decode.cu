@@ -1,13 +1,17 @@
 // decode.cu -- multi-sequence decode over a unified q8_0 / q4_0 KV cache.
 //
 // The quantised K/V blocks are never converted as a whole: each CTA copies the
-// raw bytes of a 64-key tile into shared memory (cp.async, two stages in
-// flight), and one cooperative pass turns that tile into f16 right before the
-// tensor cores read it ("unsloth llama.cpp: dequantize q4_0/q8_0 K/V tiles in
-// the FA MMA kernel", summary: tiles are dequantised as they are loaded
-// instead of a whole-cache f16 conversion per layer per step).  Each element
-// is dequantised exactly once; the f16 tile is read with ldmatrix (K) and
-// ldmatrix.trans (V) into mma.sync fragments.
+// raw bytes of a 64-key tile into shared memory and dequantises them right
+// before the tensor cores use them ("unsloth llama.cpp: dequantize q4_0/q8_0
+// K/V tiles in the FA MMA kernel", summary: tiles are dequantised as they are
+// loaded instead of a whole-cache f16 conversion per layer per step).  Each
+// element is dequantised exactly once.  Two kernels do this:
+//   decode_ws_kernel (TMA path, cache rows at 16-byte multiples): a producer
+//     warp streams raw tiles by TMA; the consumer warps build their mma.sync
+//     operands in registers straight from the raw bytes (no f16 tile in shared
+//     memory), in a dim order matched to the block layout.
+//   decode_split_kernel (any cell stride): cp.async copies, one cooperative
+//     pass into an f16 tile, ldmatrix (K) and ldmatrix.trans (V) fragments.
 //
 // Work split.  For one sequence and one kv head the g query heads x n_q new
 // tokens fold into M = g*n_q <= 16 rows (fold row r = rep*n_q + t, query head
@@ -25,6 +29,8 @@
 // every value a q8_0 byte or q4_0 nibble can hold; the block scale multiplies
 // afterwards.
 #include <math.h>
+
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -49,6 +55,16 @@ struct Fmt<ARC_KV_Q4_0> {
 
 constexpr int gcd16(int x) { return (x & 15) == 0 ? 16 : ((x & 7) == 0 ? 8 : ((x & 3) == 0 ? 4 : ((x & 1) == 0 ? 2 : 1))); }
 
+// Shared memory of the in-CTA merge of the WARPS consumer warps: per-warp O
+// partials with a padded row stride (D + 8 floats: the fragment stores of the 8
+// row groups of a warp land in distinct banks), per-warp row max / sum, the
+// merge weights and the merged row max / sum.
+template <int D>
+struct MergeLayout {
+    static constexpr int OS = D + 8;
+    static constexpr int BYTES = (WARPS * 16 * OS + WARPS * 16 * 2 + WARPS * 16 + 16 * 2) * 4;
+};
+
 // TMA: the head row of kv head h starts at byte ROWB*h of a cell, which is not
 // 16-byte aligned in general; the box starts at the boundary below it (at most
 // 16 - gcd(ROWB, 16) bytes earlier) and is wide enough to cover the row.
@@ -60,7 +76,7 @@ struct DecLayout {
     static constexpr int NST = TMA ? (KVT == ARC_KV_Q8_0 ? 2 : 4) : 2;  // raw stages in flight
     static constexpr int HSTRIDE = D + 8;                      // f16 tile row stride (elements), breaks bank conflicts
     static constexpr int HBYTES = DT * HSTRIDE * 2;
-    static constexpr int MERGE = WARPS * 16 * (D + 2) * 4;
+    static constexpr int MERGE = MergeLayout<D>::BYTES;
     static constexpr int MAIN = NST * 2 * RAW + 2 * HBYTES;    // stages x (K,V) raw + f16 K,V
     static constexpr int BYTES = (MAIN > MERGE ? MAIN : MERGE) + 64 + 128;  // + stage barriers, alignment
     static constexpr int PIECE = (ROWB % 8 == 0) ? 8 : 4;      // cp.async granule
@@ -144,6 +160,101 @@ ARC_DEV uint4 dequant8(const uint8_t *row, int grp)
     }
     return make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)), h2_bits(__hmul2(h2, sc)),
                       h2_bits(__hmul2(h3, sc)));
+}
+
+// Merge the consumer warps of this CTA (each holding an online-softmax partial of
+// 16 fold rows: unnormalised O fragments, row max, row sum) into the CTA's one
+// partial in the workspace, weighting each warp by exp2(m_warp - m) as in the
+// log-sum-exp merge of split attention.  Called by all NTHR threads of the CTA
+// after the main loop; `consumer` marks the threads that hold fragments.
+//
+// PERM = false: fragment n-tile nd, column c holds dim 8*nd + c (the plain
+// m16n8k16 layout).  PERM = true: the B operand of P V was loaded with a
+// permuted dim order (lane group g takes the D/8 consecutive dims D/8*g ...), so
+// column c of n-tile nd holds dim D/8*c + nd.  In shared memory dim d then sits
+// at column d + 2*(d / (D/4)): the skew spreads the four lanes of a quad, whose
+// dims are D/4 apart, over different banks.
+template <int D, int NTHR, bool PERM>
+ARC_DEV void write_cta_partial(const float (&o)[D / 8][4], const float (&m_r)[2], const float (&l_r)[2], bool consumer,
+                               uint8_t *smem, const DecodeParams &p, int64_t part)
+{
+    using ML = MergeLayout<D>;
+    constexpr int ND = D / 8;
+    float *so = reinterpret_cast<float *>(smem);        // [WARPS][16][OS]
+    float *sml = so + WARPS * 16 * ML::OS;              // [WARPS][16][2]
+    float *swt = sml + WARPS * 16 * 2;                  // [WARPS][16]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    __syncthreads();   // every warp is past its last read of the tile buffers this overlays
+    if (consumer) {
+#pragma unroll
+        for (int nd = 0; nd < ND; ++nd)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                float *row = so + (warp * 16 + g + 8 * hr) * ML::OS;
+                if constexpr (PERM) {
+                    // dims 2*ND*tq + nd and 2*ND*tq + ND + nd, skewed by 2*tq
+                    row[2 * ND * tq + nd + 2 * tq] = o[nd][2 * hr];
+                    row[2 * ND * tq + ND + nd + 2 * tq] = o[nd][2 * hr + 1];
+                } else {
+                    *reinterpret_cast<float2 *>(row + nd * 8 + 2 * tq) = make_float2(o[nd][2 * hr], o[nd][2 * hr + 1]);
+                }
+            }
+        if (tq == 0) {
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                sml[(warp * 16 + g + 8 * hr) * 2 + 0] = m_r[hr];
+                sml[(warp * 16 + g + 8 * hr) * 2 + 1] = l_r[hr];
+            }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < 16) {
+        const int r = threadIdx.x;
+        float mm = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) mm = fmaxf(mm, sml[(w * 16 + r) * 2]);
+        const float ms = (mm == -INFINITY) ? 0.f : mm;
+        float ll = 0.f;
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) {
+            const float mw = sml[(w * 16 + r) * 2];
+            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - ms);
+            swt[w * 16 + r] = f;
+            ll += f * sml[(w * 16 + r) * 2 + 1];
+        }
+        *reinterpret_cast<float2 *>(p.ws_ml + (part * 16 + r) * 2) = make_float2(mm, ll);
+    }
+    __syncthreads();
+    if constexpr (PERM) {
+        constexpr int D2 = D / 2;
+#pragma unroll
+        for (int x = threadIdx.x; x < 16 * D2; x += NTHR) {
+            const int r = x / D2, d = (x % D2) * 2;
+            const int col = d + 2 * (d / (D / 4));
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < WARPS; ++w) {
+                const float f = swt[w * 16 + r];
+                const float2 v = *reinterpret_cast<const float2 *>(so + (w * 16 + r) * ML::OS + col);
+                acc.x += f * v.x, acc.y += f * v.y;
+            }
+            *reinterpret_cast<float2 *>(p.ws_o + (part * 16 + r) * D + d) = acc;
+        }
+    } else {
+        constexpr int D4 = D / 4;
+#pragma unroll
+        for (int x = threadIdx.x; x < 16 * D4; x += NTHR) {
+            const int r = x / D4, d = (x % D4) * 4;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w = 0; w < WARPS; ++w) {
+                const float f = swt[w * 16 + r];
+                const float4 v = *reinterpret_cast<const float4 *>(so + (w * 16 + r) * ML::OS + d);
+                acc.x += f * v.x, acc.y += f * v.y, acc.z += f * v.z, acc.w += f * v.w;
+            }
+            *reinterpret_cast<float4 *>(p.ws_o + (part * 16 + r) * D + d) = acc;
+        }
+    }
 }
 
 template <int BYTES>
@@ -367,45 +478,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
         l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 1);
         l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 2);
     }
-    __syncthreads();
-    float *so = reinterpret_cast<float *>(smem);       // [WARPS][16][D]
-    float *sml = so + WARPS * 16 * D;                   // [WARPS][16][2]
-#pragma unroll
-    for (int nd = 0; nd < NT_O; ++nd)
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            float *dst = so + ((warp * 16) + g + 8 * hr) * D + nd * 8 + 2 * tq;
-            dst[0] = o[nd][2 * hr];
-            dst[1] = o[nd][2 * hr + 1];
-        }
-    if (tq == 0) {
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            sml[(warp * 16 + g + 8 * hr) * 2 + 0] = m_r[hr];
-            sml[(warp * 16 + g + 8 * hr) * 2 + 1] = l_r[hr];
-        }
-    }
-    __syncthreads();
-    for (int x = threadIdx.x; x < 16 * D; x += WARPS * 32) {
-        const int r = x / D, d = x % D;
-        float mm = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < WARPS; ++w) mm = fmaxf(mm, sml[(w * 16 + r) * 2]);
-        const float ms = (mm == -INFINITY) ? 0.f : mm;
-        float acc = 0.f, ll = 0.f;
-#pragma unroll
-        for (int w = 0; w < WARPS; ++w) {
-            const float mw = sml[(w * 16 + r) * 2];
-            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - ms);
-            acc += f * so[(w * 16 + r) * D + d];
-            ll += f * sml[(w * 16 + r) * 2 + 1];
-        }
-        p.ws_o[(part * 16 + r) * D + d] = acc;
-        if (d == 0) {
-            p.ws_ml[(part * 16 + r) * 2 + 0] = mm;
-            p.ws_ml[(part * 16 + r) * 2 + 1] = ll;
-        }
-    }
+    write_cta_partial<D, WARPS * 32, false>(o, m_r, l_r, true, smem, p, part);
     if (!ok && threadIdx.x == 0) report(p.status, ST_TIMEOUT_LOAD);
     // Let the merge kernel start its prologue; it waits for this grid's writes.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -414,105 +487,114 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
 // ---------------------------------------------------------------------------
 // Warp-specialised split kernel (TMA path).  Warp 4 streams raw K/V tiles of 64
 // cells into a ring of NST stages; each of warps 0-3 owns 16 cells of every
-// tile: it dequantises just those rows into its own f16 buffers, releases the
-// raw stage (one arrive per warp on empty[stage]) and runs its MMAs.  No
-// CTA-wide barrier inside the loop, so the four warps drift independently and
-// hide one another's latencies.
+// tile and builds its mma.sync operands straight from the raw bytes, in
+// registers: no f16 copy of the tile is ever written, so shared memory carries
+// only the TMA writes, one read of each raw byte and the Q fragments.
+//
+// Dim permutations.  A dot product does not change when the same permutation
+// is applied to the head dim of both operands, so S = Q K^T takes the k-step
+// order that suits the q8_0 / q4_0 block layout: in k-step j (block b = j/2,
+// half hh = j%2) the lane with quad index t holds the four consecutive dims
+// 32b + 16hh + 4t .. +3 (k positions 2t, 2t+1, 2t+8, 2t+9 of the fragment).
+// Those are four consecutive bytes of one block (q8_0), or the low / high
+// nibbles of four consecutive bytes (q4_0), so each B fragment register pair
+// comes from one 32-bit word; the Q fragments are read from shared memory in
+// the same order.  For O += P V the n index is the output dim: lane group g
+// loads dims D/8*g .. D/8*g + D/8 - 1 (consecutive bytes again) and n-tile nd
+// column c accumulates dim D/8*c + nd, which write_cta_partial<.., true> undoes.
 constexpr int WS_WARPS = 5;
 
 template <int KVT, int D>
 struct WsLayout {
-    static constexpr int ROWB = (D / 32) * Fmt<KVT>::BB;
+    static constexpr int BB = Fmt<KVT>::BB;
+    static constexpr int ROWB = (D / 32) * BB;
     static constexpr int RS = ((ROWB + 16 - gcd16(ROWB) + 15) / 16) * 16;   // smem row stride of a raw tile
     static constexpr int RAW = DT * RS;
-    static constexpr int NST = KVT == ARC_KV_Q8_0 ? 2 : 3;          // three CTAs per SM fit
-    static constexpr int WROWS = DT / WARPS;                                  // cells per consumer warp
-    static constexpr int HSTRIDE = D + 8;
-    static constexpr int HW = WROWS * HSTRIDE * 2;                            // one f16 buffer (K or V) of a warp
-    static constexpr int QB = 16 * HSTRIDE * 2;                               // Q tile (f16, pre-scaled)
-    static constexpr int MAIN = NST * 2 * RAW + WARPS * 2 * HW + QB;
-    static constexpr int MERGE = WARPS * 16 * (D + 2) * 4;
+    static constexpr int NST = KVT == ARC_KV_Q8_0 ? 3 : 4;          // stages in flight; three CTAs per SM fit
+    static constexpr int QS = D + 16;                                 // Q row stride (halfs): 8-byte fragment reads hit distinct banks
+    static constexpr int QB = 16 * QS * 2;                            // Q tile (f16, pre-scaled)
+    static constexpr int MAIN = NST * 2 * RAW + QB;
+    static constexpr int MERGE = MergeLayout<D>::BYTES;
     static constexpr int BYTES = (MAIN > MERGE ? MAIN : MERGE) + 128 + 128;  // + barriers, alignment
 };
 
-// Dequantise the block that starts `off` bytes into a 16-byte-aligned raw row:
-// three (q8_0) or two (q4_0) aligned 16-byte loads cover it wherever it starts,
-// which with the 144 / 80-byte smem row stride touches 8 rows in distinct banks.
-// `off` is a compile-time constant at every call (unrolled loops, template pad),
-// so all byte positions below fold away.
-template <int KVT>
-ARC_DEV void dequant_block16(const uint8_t *row, int off, __half *dst)
+ARC_DEV uint2 lds_u64(const void *p) { return *reinterpret_cast<const uint2 *>(p); }
+
+// The 32-bit word of a raw row at byte offset OFF (OFF % 4 is 0 or 2; the row
+// pointer is 4-byte aligned).
+template <int OFF>
+ARC_DEV uint32_t raw_word(const uint8_t *row)
 {
-    constexpr int N4 = KVT == ARC_KV_Q8_0 ? 3 : 2;
-    const uint4 *w4 = reinterpret_cast<const uint4 *>(row + (off & ~15));
-    const int o = off & 15;
-    uint32_t W[4 * N4];
-#pragma unroll
-    for (int i = 0; i < N4; ++i) {
-        const uint4 t = w4[i];
-        W[4 * i] = t.x, W[4 * i + 1] = t.y, W[4 * i + 2] = t.z, W[4 * i + 3] = t.w;
-    }
-    const __half2 sc = bits_h2(__byte_perm(W[o >> 2], 0u, (o & 2) ? 0x3232u : 0x1010u));
-    auto word = [&](int j) -> uint32_t {   // data bytes 4j .. 4j+3 of the block
-        const int b0 = o + 2 + 4 * j;
-        return (b0 & 3) ? __byte_perm(W[b0 >> 2], W[(b0 >> 2) + 1], 0x5432u) : W[b0 >> 2];
-    };
-    uint4 *out = reinterpret_cast<uint4 *>(dst);
-    if constexpr (KVT == ARC_KV_Q8_0) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            __half2 h0, h1, h2, h3;
-            s8x4_to_h2x2(word(2 * q), h0, h1);
-            s8x4_to_h2x2(word(2 * q + 1), h2, h3);
-            out[q] = make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)), h2_bits(__hmul2(h2, sc)),
-                                h2_bits(__hmul2(h3, sc)));
-        }
+    if constexpr ((OFF & 3) == 0) {
+        return lds_u32(row + OFF);
     } else {
-        uint32_t d[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) d[k] = word(k);
-#pragma unroll
-        for (int half = 0; half < 2; ++half)
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const uint32_t a = half ? (d[2 * q] >> 4) & 0x0F0F0F0Fu : d[2 * q] & 0x0F0F0F0Fu;
-                const uint32_t b = half ? (d[2 * q + 1] >> 4) & 0x0F0F0F0Fu : d[2 * q + 1] & 0x0F0F0F0Fu;
-                __half2 h0, h1, h2, h3;
-                u4x4_to_h2x2(a, h0, h1);
-                u4x4_to_h2x2(b, h2, h3);
-                out[half * 2 + q] = make_uint4(h2_bits(__hmul2(h0, sc)), h2_bits(__hmul2(h1, sc)),
-                                               h2_bits(__hmul2(h2, sc)), h2_bits(__hmul2(h3, sc)));
-            }
+        return __byte_perm(lds_u32(row + (OFF & ~3)), lds_u32(row + (OFF & ~3) + 4), 0x5432u);
     }
 }
 
-// One consumer warp's 16 rows of a raw K/V tile (kvh's head row starts PAD bytes
-// into each 16-byte-aligned smem row) into its f16 buffers: at step k every lane
-// takes block k, lanes 0-15 of K rows 0-15 and lanes 16-31 of V rows 0-15.
-template <int KVT, int D, int PAD>
-ARC_DEV void dequant_warp_rows(const uint8_t *rk, int raw_bytes, int rs, int valid, __half *kb, __half *vb, int hstride)
+// The scale of block B of a raw row, replicated into both halves of a half2.
+template <int KVT, int B>
+ARC_DEV __half2 raw_scale(const uint8_t *row)
 {
-    const int lane = threadIdx.x & 31, which = lane >> 4, rr = lane & 15;
-    const uint8_t *rowp = rk + which * raw_bytes + rr * rs;
-    __half *dst = (which ? vb : kb) + rr * hstride;
+    constexpr int OFF = B * Fmt<KVT>::BB;
+    return bits_h2(__byte_perm(lds_u32(row + (OFF & ~3)), 0u, (OFF & 2) ? 0x3232u : 0x1010u));
+}
+
+// The B fragments of K block B for the lane with quad index t: kf[hh] = {b0, b1}
+// of k-step 2B + hh (dims 32B + 16hh + 4t .. +3 of this cell).
+template <int KVT, int B>
+ARC_DEV void k_block_frags(const uint8_t *row, int t, uint32_t (&kf)[2][2])
+{
+    const __half2 sc = raw_scale<KVT, B>(row);
+    const uint8_t *rt = row + 4 * t;
+    __half2 lo, hi;
+    if constexpr (KVT == ARC_KV_Q8_0) {
 #pragma unroll
-    for (int k = 0; k < D / 32; ++k) {
-        if (rr < valid) {
-            dequant_block16<KVT>(rowp, PAD + k * Fmt<KVT>::BB, dst + k * 32);
-        } else {
-            uint4 *z = reinterpret_cast<uint4 *>(dst + k * 32);
-            z[0] = z[1] = z[2] = z[3] = make_uint4(0, 0, 0, 0);
+        for (int hh = 0; hh < 2; ++hh) {
+            s8x4_to_h2x2(hh ? raw_word<B * 34 + 2 + 16>(rt) : raw_word<B * 34 + 2>(rt), lo, hi);
+            kf[hh][0] = h2_bits(__hmul2(lo, sc));
+            kf[hh][1] = h2_bits(__hmul2(hi, sc));
         }
+    } else {
+        const uint32_t w = raw_word<B * 18 + 2>(rt);     // low nibbles: dims +0..3, high nibbles: dims +16..19
+        u4x4_to_h2x2(w & 0x0F0F0F0Fu, lo, hi);
+        kf[0][0] = h2_bits(__hmul2(lo, sc));
+        kf[0][1] = h2_bits(__hmul2(hi, sc));
+        u4x4_to_h2x2((w >> 4) & 0x0F0F0F0Fu, lo, hi);
+        kf[1][0] = h2_bits(__hmul2(lo, sc));
+        kf[1][1] = h2_bits(__hmul2(hi, sc));
     }
+}
+
+// One V cell as this lane needs it: the D/8 dims starting at D/8*g (NW data
+// words, realigned) and the word holding that block's scale (0 past the end of
+// the chunk, which zeroes the cell: its data bytes are finite integers).
+template <int KVT, int D>
+struct VCell {
+    static constexpr int NW = D / 32;   // D/8 bytes (q8_0) or nibbles in D/8 bytes' halves (q4_0), as words
+    uint32_t d[NW];
+    uint32_t sw;
+};
+
+template <int KVT, int D>
+ARC_DEV void load_vcell(const uint8_t *row, int vbase, uint32_t vsel, int soff4, bool valid, VCell<KVT, D> &c)
+{
+    const uint8_t *b = row + vbase;
+    uint32_t w[VCell<KVT, D>::NW + 1];
+#pragma unroll
+    for (int i = 0; i <= VCell<KVT, D>::NW; ++i) w[i] = lds_u32(b + 4 * i);
+#pragma unroll
+    for (int i = 0; i < VCell<KVT, D>::NW; ++i) c.d[i] = __byte_perm(w[i], w[i + 1], vsel);
+    c.sw = valid ? lds_u32(row + soff4) : 0u;
 }
 
 template <int KVT, int D>
 __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __grid_constant__ DecodeParams p)
 {
     using L = WsLayout<KVT, D>;
-    constexpr int KS = D / 16;
-    constexpr int NT_O = D / 8;
     constexpr int NB = D / 32;                        // blocks per row
+    constexpr int ND = D / 8;                         // P V n-tiles = dims per lane group
+    constexpr int NW = VCell<KVT, D>::NW;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -534,27 +616,46 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
     const int pad = (L::ROWB * kvh) & 15;
     const int x0 = L::ROWB * kvh - pad;
 
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < L::NST; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], WARPS);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
-
-    float o[NT_O][4];
+    // Q tile loads, all in flight before anything waits on them: 16 fold rows x D
+    // fp32, QI float2 per consumer thread.
+    constexpr int QI = 16 * D / 2 / (WARPS * 32);
+    static_assert(QI * WARPS * 32 == 16 * D / 2, "Q tile split");
+    float2 qv[QI];
 #pragma unroll
-    for (int i = 0; i < NT_O; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    for (int j = 0; j < QI; ++j) {
+        const int x = threadIdx.x + j * WARPS * 32;
+        const int r = x / (D / 2), d = (x % (D / 2)) * 2;
+        qv[j] = make_float2(0.f, 0.f);
+        if (warp < WARPS && r < M) {
+            const int h = kvh * G + r / sq.n_q;
+            const int tok = sq.q_begin + r % sq.n_q;
+            qv[j] = __ldg(reinterpret_cast<const float2 *>(p.q + ((int64_t)tok * p.H + h) * D + d));
+        }
+    }
+
+    float o[ND][4];
+#pragma unroll
+    for (int i = 0; i < ND; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
     bool ok = true;
 
     if (warp == WARPS) {
         // =============================== producer
+        // It initialises the stage barriers itself and only signals the consumers
+        // (bar.arrive), so its first loads go out without waiting for the Q tile.
+        if (lane == 0) {
+            for (int i = 0; i < L::NST; ++i) {
+                mbar_init(&full[i], 1);
+                mbar_init(&empty[i], WARPS);
+            }
+            fence_mbar_init();
+        }
+        __syncwarp();
+        asm volatile("bar.arrive 2, %0;" ::"n"(WS_WARPS * 32) : "memory");
         if (lane == 0) {
             for (int i = 0; i < n_tiles && ok; ++i) {
                 const int st = i % L::NST;
-                if (i >= L::NST) ok = mbar_wait(&empty[st], (uint32_t)((i / L::NST - 1) & 1));
+                if (i >= L::NST) ok = mbar_wait_sleep(&empty[st], (uint32_t)((i / L::NST - 1) & 1));
                 if (!ok) break;
                 uint8_t *dk = raw + st * 2 * L::RAW;
                 mbar_arrive_expect_tx(&full[st], 2 * L::RAW);
@@ -566,106 +667,153 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
         }
     } else {
         // =============================== consumer warp: 16 cells of each tile
-        __half *kb = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW + warp * 2 * L::HW);
-        __half *vb = kb + L::WROWS * L::HSTRIDE;
-        __half *qs = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW + WARPS * 2 * L::HW);
-        const uint32_t kb_s = smem_u32(kb), vb_s = smem_u32(vb), qs_s = smem_u32(qs);
+        __half *qs = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW);
         int row_t[2];
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
             const int r = g + 8 * hr;
             row_t[hr] = (r < M) ? r % sq.n_q : -1;
         }
+        // This lane's V dims D/8*g .. : block vb, first element ve of that block.  Offsets
+        // are from the head row's first byte (the row pointers below include the pad,
+        // a multiple of 4, so the word alignment of each offset is its own).
+        const int vb = (ND * g) / 32, ve = (ND * g) % 32;
+        const int voff = vb * L::BB + 2 + (KVT == ARC_KV_Q8_0 ? ve : (ve & 15));   // first data byte
+        const int vbase = voff & ~3;
+        const uint32_t vsel = (voff & 2) ? 0x5432u : 0x3210u;
+        const int soff = vb * L::BB;                                              // the block's scale
+        const int soff4 = soff & ~3;
+        const uint32_t spair = (soff & 2) ? 0x7632u : 0x5410u;     // {scale of cell A, scale of cell B}
+        const int vsh = (KVT == ARC_KV_Q4_0 && ve >= 16) ? 4 : 0;  // q4_0: high nibbles hold elements 16..31
+
+        asm volatile("bar.sync 2, %0;" ::"n"(WS_WARPS * 32) : "memory");   // stage barriers initialised
         // Q tile, shared by the four warps: 16 fold rows x D, scaled into log2 units, f16.
-        for (int x = threadIdx.x; x < 16 * D / 2; x += WARPS * 32) {
+#pragma unroll
+        for (int j = 0; j < QI; ++j) {
+            const int x = threadIdx.x + j * WARPS * 32;
             const int r = x / (D / 2), d = (x % (D / 2)) * 2;
-            float2 v = make_float2(0.f, 0.f);
-            if (r < M) {
-                const int h = kvh * G + r / sq.n_q;
-                const int tok = sq.q_begin + r % sq.n_q;
-                v = *reinterpret_cast<const float2 *>(p.q + ((int64_t)tok * p.H + h) * D + d);
-            }
-            *reinterpret_cast<__half2 *>(qs + r * L::HSTRIDE + d) = __floats2half2_rn(v.x * p.scale_log2, v.y * p.scale_log2);
+            *reinterpret_cast<__half2 *>(qs + r * L::QS + d) =
+                __floats2half2_rn(qv[j].x * p.scale_log2, qv[j].y * p.scale_log2);
         }
         asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32) : "memory");   // consumer warps only
+        const __half *q0 = qs + g * L::QS + 4 * tq, *q1 = q0 + 8 * L::QS;
+
         for (int i = 0; i < n_tiles; ++i) {
             const int st = i % L::NST;
             ok = mbar_wait(&full[st], (uint32_t)((i / L::NST) & 1)) && ok;
-            const int kw0 = i * DT + warp * L::WROWS;              // first cell (chunk-relative) of this warp
-            const int valid = c_end - c_begin - kw0;               // rows of this warp inside the chunk
-            {
-                const uint8_t *rk = raw + st * 2 * L::RAW + warp * L::WROWS * L::RS;   // 16-byte aligned rows
-                switch (pad) {   // CTA-uniform
-                case 0: dequant_warp_rows<KVT, D, 0>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
-                case 4: dequant_warp_rows<KVT, D, 4>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
-                case 8: dequant_warp_rows<KVT, D, 8>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
-                default: dequant_warp_rows<KVT, D, 12>(rk, L::RAW, L::RS, valid, kb, vb, L::HSTRIDE); break;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);                // this warp is done with the raw stage
+            const int kw0 = i * DT + warp * 16;                    // first cell (chunk-relative) of this warp
+            const int valid = c_end - c_begin - kw0;               // cells of this warp inside the chunk
+            const uint8_t *kt = raw + st * 2 * L::RAW + warp * 16 * L::RS + pad;   // this warp's 16 K rows
+            const uint8_t *vt = kt + L::RAW;
 
-            const int key0 = c_begin + kw0;
+            // ---- V words for cells 2t, 2t+1, 2t+8, 2t+9 (loaded early; used after the softmax)
+            VCell<KVT, D> vc[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int cell = 2 * tq + (c & 1) + 8 * (c >> 1);
+                load_vcell<KVT, D>(vt + cell * L::RS, vbase, vsel, soff4, cell < valid, vc[c]);
+            }
+
+            // ---- S = Q K^T over the permuted k order; cells g and g+8
             float sacc[2][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-                const int krow = nt * 8 + (lane & 7);
+            for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+            const uint8_t *k0 = kt + g * L::RS, *k1 = k0 + 8 * L::RS;
+            auto kstep = [&](auto bc) {
+                constexpr int B = decltype(bc)::value;
+                uint32_t kf0[2][2], kf1[2][2];
+                k_block_frags<KVT, B>(k0, tq, kf0);
+                k_block_frags<KVT, B>(k1, tq, kf1);
 #pragma unroll
-                for (int ks = 0; ks < KS; ks += 2) {
-                    uint32_t b0, b1, b2, b3, qa0[4], qa1[4];
-                    ldsm_x4(kb_s + (krow * L::HSTRIDE + ks * 16 + (lane >> 3) * 8) * 2, b0, b1, b2, b3);
-                    ldsm_x4(qs_s + ((lane & 15) * L::HSTRIDE + ks * 16 + (lane >> 4) * 8) * 2, qa0[0], qa0[1], qa0[2],
-                            qa0[3]);
-                    ldsm_x4(qs_s + ((lane & 15) * L::HSTRIDE + (ks + 1) * 16 + (lane >> 4) * 8) * 2, qa1[0], qa1[1],
-                            qa1[2], qa1[3]);
-                    mma16816(sacc[nt], qa0, b0, b1);
-                    mma16816(sacc[nt], qa1, b2, b3);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint2 a0 = lds_u64(q0 + 32 * B + 16 * hh), a1 = lds_u64(q1 + 32 * B + 16 * hh);
+                    const uint32_t a[4] = {a0.x, a1.x, a0.y, a1.y};
+                    mma16816(sacc[0], a, kf0[hh][0], kf0[hh][1]);
+                    mma16816(sacc[1], a, kf1[hh][0], kf1[hh][1]);
+                }
+            };
+            kstep(std::integral_constant<int, 0>{});
+            kstep(std::integral_constant<int, 1>{});
+            if constexpr (NB > 2) {
+                kstep(std::integral_constant<int, (NB > 2 ? 2 : 0)>{});
+                kstep(std::integral_constant<int, (NB > 2 ? 3 : 0)>{});
+            }
+
+            // Mask only where a key can fall past the chunk end or a row's causal
+            // limit (the last n_q - 1 keys of the sequence); the test is warp-uniform.
+            // Fold-padding rows (r >= M, zero Q) are then unmasked in most tiles: their
+            // partials stay finite and are never read.
+            const int key0 = c_begin + kw0;
+            if (key0 + 16 > c_end || key0 + 15 > sq.n_kv - sq.n_q) {
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int lim = row_t[hr] < 0 ? -1 : sq.n_kv - sq.n_q + row_t[hr];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int key = key0 + nt * 8 + 2 * tq + e;
+                            if (key >= c_end || key > lim) sacc[nt][2 * hr + e] = -INFINITY;
+                        }
                 }
             }
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                const int lim = row_t[hr] < 0 ? -1 : sq.n_kv - sq.n_q + row_t[hr];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int key = key0 + nt * 8 + 2 * tq + e;
-                        if (key >= c_end || key > lim) sacc[nt][2 * hr + e] = -INFINITY;
-                    }
-            }
+            // Online softmax with a lazy rescale: the running max m_r moves (and O, l
+            // are rescaled) only when a tile raises it by more than kLazy (log2 units);
+            // otherwise p = exp2(s - m_r) <= 2^kLazy, which f16 and the f32 sums hold.
+            // (m_r, l_r, O) stay one consistent partial either way.
+            constexpr float kLazy = 8.f;
             uint32_t pa[4];
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
                 float mx = fmaxf(fmaxf(sacc[0][2 * hr], sacc[0][2 * hr + 1]), fmaxf(sacc[1][2 * hr], sacc[1][2 * hr + 1]));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float m_new = fmaxf(m_r[hr], mx);
-                const float msafe = (m_new == -INFINITY) ? 0.f : m_new;
-                const float alpha = (m_r[hr] == -INFINITY) ? 0.f : fast_exp2(m_r[hr] - msafe);
-                m_r[hr] = m_new;
-                const float p00 = fast_exp2(sacc[0][2 * hr] - msafe), p01 = fast_exp2(sacc[0][2 * hr + 1] - msafe);
-                const float p10 = fast_exp2(sacc[1][2 * hr] - msafe), p11 = fast_exp2(sacc[1][2 * hr + 1] - msafe);
-                l_r[hr] = l_r[hr] * alpha + (p00 + p01 + p10 + p11);
-                if (alpha != 1.f) {
+                if (mx > m_r[hr] + kLazy) {   // also the first finite max (m_r = -inf)
+                    const float alpha = (m_r[hr] == -INFINITY) ? 0.f : fast_exp2(m_r[hr] - mx);
+                    m_r[hr] = mx;
+                    l_r[hr] *= alpha;
 #pragma unroll
-                    for (int i2 = 0; i2 < NT_O; ++i2) {
+                    for (int i2 = 0; i2 < ND; ++i2) {
                         o[i2][2 * hr] *= alpha;
                         o[i2][2 * hr + 1] *= alpha;
                     }
                 }
+                const float msafe = (m_r[hr] == -INFINITY) ? 0.f : m_r[hr];
+                const float p00 = fast_exp2(sacc[0][2 * hr] - msafe), p01 = fast_exp2(sacc[0][2 * hr + 1] - msafe);
+                const float p10 = fast_exp2(sacc[1][2 * hr] - msafe), p11 = fast_exp2(sacc[1][2 * hr + 1] - msafe);
+                l_r[hr] += (p00 + p01) + (p10 + p11);
                 pa[hr] = h2_bits(__floats2half2_rn(p00, p01));
                 pa[2 + hr] = h2_bits(__floats2half2_rn(p10, p11));
             }
-            const int vrow = (lane & 7) + ((lane >> 3) & 1) * 8;
+
+            // ---- O += P V: b0 from cells (2t, 2t+1), b1 from (2t+8, 2t+9), dims D/8*g + nd
+            const __half2 s01 = bits_h2(__byte_perm(vc[0].sw, vc[1].sw, spair));
+            const __half2 s89 = bits_h2(__byte_perm(vc[2].sw, vc[3].sw, spair));
 #pragma unroll
-            for (int nd = 0; nd < NT_O; nd += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(vb_s + (vrow * L::HSTRIDE + nd * 8 + (lane >> 4) * 8) * 2, b0, b1, b2, b3);
-                mma16816(o[nd], pa, b0, b1);
-                mma16816(o[nd + 1], pa, b2, b3);
+            for (int w = 0; w < NW; ++w) {
+                uint32_t x01 = vc[0].d[w], y01 = vc[1].d[w], x89 = vc[2].d[w], y89 = vc[3].d[w];
+                if constexpr (KVT == ARC_KV_Q4_0) {
+                    x01 = (x01 >> vsh) & 0x0F0F0F0Fu, y01 = (y01 >> vsh) & 0x0F0F0F0Fu;
+                    x89 = (x89 >> vsh) & 0x0F0F0F0Fu, y89 = (y89 >> vsh) & 0x0F0F0F0Fu;
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const uint32_t sel = half ? 0x7362u : 0x5140u;   // bytes 2,3 or 0,1 of both cells, interleaved
+                    __half2 a0, a1, c0, c1;
+                    if constexpr (KVT == ARC_KV_Q8_0) {
+                        s8x4_to_h2x2(__byte_perm(x01, y01, sel), a0, a1);
+                        s8x4_to_h2x2(__byte_perm(x89, y89, sel), c0, c1);
+                    } else {
+                        u4x4_to_h2x2(__byte_perm(x01, y01, sel), a0, a1);
+                        u4x4_to_h2x2(__byte_perm(x89, y89, sel), c0, c1);
+                    }
+                    const int nd = 4 * w + 2 * half;
+                    mma16816(o[nd], pa, h2_bits(__hmul2(a0, s01)), h2_bits(__hmul2(c0, s89)));
+                    mma16816(o[nd + 1], pa, h2_bits(__hmul2(a1, s01)), h2_bits(__hmul2(c1, s89)));
+                }
             }
-            __syncwarp();   // every lane's ldmatrix of this warp's buffers is done before the next dequant
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);                // this warp is done with the raw stage
         }
         if (!ok && lane == 0) report(p.status, ST_TIMEOUT_LOAD);
 #pragma unroll
@@ -675,49 +823,8 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
         }
     }
 
-    // ---- merge the 4 consumer warps (the raw ring and f16 buffers are idle now)
-    __syncthreads();
-    float *so = reinterpret_cast<float *>(smem);
-    float *sml = so + WARPS * 16 * D;
-    if (warp < WARPS) {
-#pragma unroll
-        for (int nd = 0; nd < NT_O; ++nd)
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                float *dst = so + ((warp * 16) + g + 8 * hr) * D + nd * 8 + 2 * tq;
-                dst[0] = o[nd][2 * hr];
-                dst[1] = o[nd][2 * hr + 1];
-            }
-        if (tq == 0) {
-#pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                sml[(warp * 16 + g + 8 * hr) * 2 + 0] = m_r[hr];
-                sml[(warp * 16 + g + 8 * hr) * 2 + 1] = l_r[hr];
-            }
-        }
-    }
-    __syncthreads();
-    const int64_t part = (int64_t)blockIdx.x;
-    for (int x = threadIdx.x; x < 16 * D; x += WS_WARPS * 32) {
-        const int r = x / D, d = x % D;
-        float mm = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < WARPS; ++w) mm = fmaxf(mm, sml[(w * 16 + r) * 2]);
-        const float ms = (mm == -INFINITY) ? 0.f : mm;
-        float acc = 0.f, ll = 0.f;
-#pragma unroll
-        for (int w = 0; w < WARPS; ++w) {
-            const float mw = sml[(w * 16 + r) * 2];
-            const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - ms);
-            acc += f * so[(w * 16 + r) * D + d];
-            ll += f * sml[(w * 16 + r) * 2 + 1];
-        }
-        p.ws_o[(part * 16 + r) * D + d] = acc;
-        if (d == 0) {
-            p.ws_ml[(part * 16 + r) * 2 + 0] = mm;
-            p.ws_ml[(part * 16 + r) * 2 + 1] = ll;
-        }
-    }
+    // ---- merge the 4 consumer warps (the raw ring is idle now)
+    write_cta_partial<D, WS_WARPS * 32, true>(o, m_r, l_r, warp < WARPS, smem, p, (int64_t)blockIdx.x);
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
@@ -727,6 +834,7 @@ template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant__ DecodeParams p)
 {
     __shared__ float s_w[256];     // per-split weight exp2(m_sp - m)
+    __shared__ float s_m[256], s_l[256];
     __shared__ float s_red[2];
     const int s = blockIdx.x / p.Hkv, kvh = blockIdx.x % p.Hkv, r = blockIdx.y;
     const arc_seq sq = p.seqs[s];
@@ -736,25 +844,38 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
     const int d = threadIdx.x;
     const int64_t part0 = ((int64_t)s * p.Hkv + kvh) * p.splits;
     asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the split kernel are complete
-    if (d == 0) {
+    // every split's (max, sum) loaded at once; warp 0 reduces them
+    const int nsp = p.splits;
+    for (int sp = d; sp < nsp; sp += D) {
+        const float2 ml = *reinterpret_cast<const float2 *>(p.ws_ml + ((part0 + sp) * 16 + r) * 2);
+        s_m[sp] = ml.x;
+        s_l[sp] = ml.y;
+    }
+    __syncthreads();
+    if (d < 32) {
         float mm = -INFINITY;
-        for (int sp = 0; sp < p.splits; ++sp) mm = fmaxf(mm, p.ws_ml[((part0 + sp) * 16 + r) * 2]);
+        for (int sp = d; sp < nsp; sp += 32) mm = fmaxf(mm, s_m[sp]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mm = fmaxf(mm, __shfl_xor_sync(0xffffffffu, mm, o));
         const float ms = (mm == -INFINITY) ? 0.f : mm;
         float ll = 0.f;
-        for (int sp = 0; sp < p.splits; ++sp) {
-            const float mw = p.ws_ml[((part0 + sp) * 16 + r) * 2];
-            const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - ms);
+        for (int sp = d; sp < nsp; sp += 32) {
+            const float f = (s_m[sp] == -INFINITY) ? 0.f : exp2f(s_m[sp] - ms);
             s_w[sp] = f;
-            ll += f * p.ws_ml[((part0 + sp) * 16 + r) * 2 + 1];
+            ll += f * s_l[sp];
         }
-        s_red[0] = mm;
-        s_red[1] = ll;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
+        if (d == 0) {
+            s_red[0] = mm;
+            s_red[1] = ll;
+        }
     }
     __syncthreads();
     const float mm = s_red[0], ll = s_red[1];
     float acc = 0.f;
 #pragma unroll 4
-    for (int sp = 0; sp < p.splits; ++sp) acc += s_w[sp] * p.ws_o[((part0 + sp) * 16 + r) * D + d];
+    for (int sp = 0; sp < nsp; ++sp) acc += s_w[sp] * p.ws_o[((part0 + sp) * 16 + r) * D + d];
     p.o[((int64_t)tok * p.H + h) * D + d] = ll > 0.f ? acc / ll : 0.f;
     if (d == 0) p.lse[(int64_t)tok * p.H + h] = ll > 0.f ? (mm + log2f(ll)) * LN2 : -INFINITY;
 }
