@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
     static_assert(KC % BPS == 0 && (2 * VG) % BPS == 0, "K and V tiles fill whole ring stages");
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align_smem<1024>(smem_raw);
     uint8_t *sQ = smem;                          // KC chunks of [128 rows x 64]
     uint8_t *sRing = sQ + KC * 2 * PCH;          // R stages of BPS boxes of [64 rows x 64]
     const int R = p.stages;

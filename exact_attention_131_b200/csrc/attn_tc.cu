@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
     static_assert(DQK % 64 == 0 && DVS % 64 == 0 && DVS <= 256, "tile shape");
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align_smem<1024>(smem_raw);
     uint8_t *sQ = smem;
     uint8_t *sRing = sQ + KC * CHUNK;
     const int R = p.stages;
@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_con
 #define S_COL2(t) (128u + 256u * (uint32_t)(t))
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align_smem<1024>(smem_raw);
     uint8_t *sQ = smem;                       // [2 tiles][KC chunks]
     uint8_t *sRing = sQ + 2 * KC * CHUNK;
     const int R = p.stages;

@@ -274,7 +274,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     // TMA destinations 128-byte aligned (every tile size below is a multiple of 128)
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *smem = align_smem<128>(smem_raw);
     uint8_t *raw = smem;                                   // [NST stages][K, V][RAW]
     __half *kh = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW);
     __half *vh = kh + DT * L::HSTRIDE;
@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
     constexpr int NW = VCell<KVT, D>::NW;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    uint8_t *smem = align_smem<128>(smem_raw);
     uint8_t *raw = smem;                                            // [NST][K, V][RAW]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BYTES - 256);
     uint64_t *empty = full + L::NST;

@@ -113,6 +113,16 @@ ARC_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns = kWait
     }
 }
 
+// The first ALIGN-byte aligned byte of the dynamic shared memory.  The offset is
+// added to the __shared__ array itself (no integer round trip), so the compiler
+// still knows every pointer derived from it is shared memory and emits shared
+// loads and stores with 32-bit addresses rather than generic ones.
+template <int ALIGN>
+ARC_DEV uint8_t *align_smem(uint8_t *smem_raw)
+{
+    return smem_raw + ((ALIGN - (smem_u32(smem_raw) & (ALIGN - 1))) & (ALIGN - 1));
+}
+
 // ------------------------------------------------------------------ proxies
 
 // Make this thread's generic-proxy shared-memory writes visible to the async

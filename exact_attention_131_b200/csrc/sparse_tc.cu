@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
 {
     using L = SparseLayout<KC, VC, SEPV>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *smem = align_smem<1024>(smem_raw);
     uint8_t *sQ = smem;
     uint8_t *sKV = sQ + L::Q_BYTES;               // 2 tile buffers
     uint8_t *sP = sKV + 2 * L::TILE_BYTES;        // 2 P buffers
