@@ -74,6 +74,20 @@ ARC_DEV bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test of a phase (test_wait never suspends the thread).
+ARC_DEV bool mbar_test(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // try_wait with a suspend-time hint: a thread whose phase is not complete sleeps
 // until it completes or about hint_ns pass, instead of returning at once.
 ARC_DEV bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns)

@@ -192,9 +192,8 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
             const uint64_t pd0 = sdesc_sw128(smem_u32(sP), 16, 1024);
             bool ok = mbar_wait(&bars->q_full, 0);
             tc_fence_after();
-            auto issue_s = [&](int j) -> bool {
+            auto issue_s = [&](int j) {
                 const int b = j & 1;
-                if (!mbar_wait(&bars->kv_full[b], (uint32_t)((j >> 1) & 1))) return false;
                 tc_fence_after();
                 const uint32_t d = tmem + (16u << 16) + b * SBN;
 #pragma unroll
@@ -202,11 +201,9 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                     umma_ss_k64(d, qd0 + (uint64_t)(c * kChunkUnits),
                                 kvd0 + (uint64_t)((b * L::TILE_CHUNKS + c) * kChunkUnits), idesc_s, c > 0);
                 umma_commit(&bars->s_full[b]);
-                return true;
             };
-            auto issue_pv = [&](int j) -> bool {
+            auto issue_pv = [&](int j) {
                 const int b = j & 1;
-                if (!mbar_wait(&bars->p_full[b], (uint32_t)((j >> 1) & 1))) return false;
                 tc_fence_after();
                 const uint64_t a = pd0 + (uint64_t)(b * kChunkUnits);
                 const int vfirst = b * L::TILE_CHUNKS + (SEPV ? KC : 0);
@@ -218,13 +215,26 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                 }
                 umma_commit(&bars->kv_empty[b]);
                 umma_commit(&bars->o_done);
-                return true;
             };
-            // S(j) then O += P(j) V(j): the gather of tile j+1 (free once P(j-1) V(j-1) is
-            // done) then has a whole tile of tensor-core work to hide behind.
-            for (int j = 0; ok && j < nt; ++j) {
-                ok = issue_s(j);
-                if (ok) ok = issue_pv(j);
+            // Out-of-order issue between two in-order streams: S(js) as soon as its tile
+            // is gathered (and its TMEM buffer is free: S may run at most one tile ahead
+            // of P V, the softmax of tile js-2 being done once P(js-2) was posted), else
+            // O += P(jp) V(jp) as soon as P(jp) is posted.  The softmax of tile j then
+            // runs under S(j+1) instead of leaving the tensor pipe idle, while P V never
+            // waits behind a gather it does not need.  Bounded: no progress for
+            // kWaitLimitNs ends the loop with an error.
+            int js = 0, jp = 0;
+            uint64_t t_last = globaltimer_ns();
+            while (ok && jp < nt) {
+                if (js < nt && js <= jp + 1 && mbar_test(&bars->kv_full[js & 1], (uint32_t)((js >> 1) & 1))) {
+                    issue_s(js++);
+                    t_last = globaltimer_ns();
+                } else if (jp < js && mbar_test(&bars->p_full[jp & 1], (uint32_t)((jp >> 1) & 1))) {
+                    issue_pv(jp++);
+                    t_last = globaltimer_ns();
+                } else if (globaltimer_ns() - t_last > kWaitLimitNs) {
+                    ok = false;
+                }
             }
             if (!ok) report(p.status, ST_TIMEOUT_MMA);
             umma_commit(&bars->drain);
