@@ -844,10 +844,16 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
     const int d = threadIdx.x;
     const int64_t part0 = ((int64_t)s * p.Hkv + kvh) * p.splits;
     asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the split kernel are complete
-    // every split's (max, sum) loaded at once; warp 0 reduces them
+    // This thread's column of the first KV32 splits goes out at once, with every
+    // split's (max, sum); warp 0 reduces the latter while those loads fly.
+    constexpr int KV32 = 32;
     const int nsp = p.splits;
+    float v[KV32];
+#pragma unroll
+    for (int sp = 0; sp < KV32; ++sp)
+        v[sp] = sp < nsp ? __ldcg(p.ws_o + ((part0 + sp) * 16 + r) * D + d) : 0.f;
     for (int sp = d; sp < nsp; sp += D) {
-        const float2 ml = *reinterpret_cast<const float2 *>(p.ws_ml + ((part0 + sp) * 16 + r) * 2);
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.ws_ml + ((part0 + sp) * 16 + r) * 2));
         s_m[sp] = ml.x;
         s_l[sp] = ml.y;
     }
@@ -874,8 +880,10 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
     __syncthreads();
     const float mm = s_red[0], ll = s_red[1];
     float acc = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < KV32; ++sp) acc += s_w[sp < nsp ? sp : 0] * v[sp];   // v is 0 past nsp
 #pragma unroll 4
-    for (int sp = 0; sp < nsp; ++sp) acc += s_w[sp] * p.ws_o[((part0 + sp) * 16 + r) * D + d];
+    for (int sp = KV32; sp < nsp; ++sp) acc += s_w[sp] * __ldcg(p.ws_o + ((part0 + sp) * 16 + r) * D + d);
     p.o[((int64_t)tok * p.H + h) * D + d] = ll > 0.f ? acc / ll : 0.f;
     if (d == 0) p.lse[(int64_t)tok * p.H + h] = ll > 0.f ? (mm + log2f(ll)) * LN2 : -INFINITY;
 }

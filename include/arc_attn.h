@@ -201,7 +201,9 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *args, void *stream);
  * D in {64,128}; H % Hkv == 0; (H/Hkv) * n_q <= 16 for every sequence;
  * n_seq <= ARC_DECODE_MAX_SEQ.
  * workspace: device, at least arc_decode_workspace_size(args) bytes, 256-byte
- * aligned; used for the split-KV partial results and overwritten.
+ * aligned; used for the split-KV partial results and overwritten.  Its
+ * contents need no initialisation (every byte read is first written by the
+ * same call).  Two calls in flight at once need two workspaces.
  * ------------------------------------------------------------------------ */
 #define ARC_DECODE_MAX_SEQ 64
 

@@ -233,6 +233,44 @@ def test_decode_both_load_paths(kv_type, H, Hkv, D, kernel):
     assert arc.check_device_error(st) == arc.ARC_OK
 
 
+def _decode_into(c, q, kc, vc, ws, o, lse):
+    arc.attn_decode_q8(q, kc, vc, kv_type=c.kv_type, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                       n_kv=c.n_kv, scale=c.scale, workspace=ws, out=o, lse=lse)
+
+
+def test_decode_workspace_garbage_reuse_and_graph_replay():
+    """The workspace needs no initialisation (stale bytes are never read before they
+    are written), may be reused call after call, and a captured launch (split kernel
+    plus its programmatic-dependent combine) replays correctly."""
+    c = W.decode_case(2, 4, 3000, 16, 4, 128, kv_type=W.KV_Q8_0, seed=43)
+    q, kc, vc = dev(c.q), dev(c.k_cache), dev(c.v_cache)
+    n = arc.decode_workspace_size(c.kv_type, q, c.Hkv, c.k_cache.shape[0], c.q_begin, c.n_q, c.kv_begin, c.n_kv)
+    ws = torch.full((n,), 0xFF, dtype=torch.uint8, device="cuda")
+    o = torch.empty(c.n_tok, c.H, c.D, dtype=torch.float32, device="cuda")
+    lse = torch.empty(c.n_tok, c.H, dtype=torch.float32, device="cuda")
+    ro, rl = oracle.run_case(c)
+    for _ in range(3):
+        o.fill_(float("nan"))
+        _decode_into(c, q, kc, vc, ws, o, lse)
+        torch.cuda.synchronize()
+        compare(o, lse, ro, rl, TOL_O_BF16)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        _decode_into(c, q, kc, vc, ws, o, lse)   # warm-up on the capture stream
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            _decode_into(c, q, kc, vc, ws, o, lse)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        o.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        compare(o, lse, ro, rl, TOL_O_BF16)
+    del g
+
+
 def test_decode_head_dim_64_and_control_arm():
     c = W.decode_case(2, 3, 500, 8, 2, 64, kv_type=W.KV_Q8_0, seed=36)
     o, lse, _ = run_decode(c)
