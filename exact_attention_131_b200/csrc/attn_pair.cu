@@ -24,6 +24,8 @@
 
 #include <algorithm>
 
+#include <type_traits>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -457,9 +459,13 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
         const int t = p.tmajor ? R_ / p.G : R_ % p.Tq;
         const int h = kv * p.G + (p.tmajor ? R_ % p.G : R_ / p.Tq);
         const int last = p.causal ? min(p.Tk - 1, t + p.Tk - p.Tq) : p.Tk - 1;
+        // The row max and sum come from the first d_v slice; later slices recompute
+        // the same S and reuse them: with the lazy max fixed, p = exp2(s - m_use) <= 2^8,
+        // so no running max, row sum or O rescale is needed there.
+        float m_use = -INFINITY, l = 0.f;
         for (int slice = 0; ok && slice < NSL; ++slice) {
         const int dv0 = slice * DVS;
-        float m_use = -INFINITY, l = 0.f;
+        const bool first = slice == 0;
         for (int j = 0; ok && j < nt; ++j) {
             const int it = gu + slice * nt + j;
             const int buf = it & 1;
@@ -478,31 +484,39 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 for (int i = 0; i < PBN; ++i)
                     if (kbase + i > last) sv[i] = __float_as_uint(-INFINITY);
             }
-            float mx = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < PBN; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
-            mx *= sl2;
-            const bool need = mx > m_use + P_RESCALE;
             float alpha = 1.f;
-            if (need) {
-                alpha = (m_use == -INFINITY) ? 0.f : fast_exp2(m_use - mx);
-                m_use = mx;
+            if (first) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < PBN; ++i) mx = fmaxf(mx, __uint_as_float(sv[i]));
+                mx *= sl2;
+                if (mx > m_use + P_RESCALE) {
+                    alpha = (m_use == -INFINITY) ? 0.f : fast_exp2(m_use - mx);
+                    m_use = mx;
+                }
             }
             const float msafe = (m_use == -INFINITY) ? 0.f : m_use;
-            float rowsum = 0.f;
+            // P = exp2(S*scale - m) as bf16 over S in place; the row sum only in the first slice
+            auto p_tile = [&](auto with_sum) {
+                float rowsum = 0.f;
 #pragma unroll
-            for (int c = 0; c < PBN / 8; ++c) {
-                uint32_t pk[4];
+                for (int c = 0; c < PBN / 8; ++c) {
+                    uint32_t pk[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float p0 = fast_exp2(fmaf(__uint_as_float(sv[8 * c + 2 * i]), sl2, -msafe));
-                    const float p1 = fast_exp2(fmaf(__uint_as_float(sv[8 * c + 2 * i + 1]), sl2, -msafe));
-                    rowsum += p0 + p1;
-                    pk[i] = pack_bf16(p0, p1);
+                    for (int i = 0; i < 4; ++i) {
+                        const float p0 = fast_exp2(fmaf(__uint_as_float(sv[8 * c + 2 * i]), sl2, -msafe));
+                        const float p1 = fast_exp2(fmaf(__uint_as_float(sv[8 * c + 2 * i + 1]), sl2, -msafe));
+                        if constexpr (decltype(with_sum)::value) rowsum += p0 + p1;
+                        pk[i] = pack_bf16(p0, p1);
+                    }
+                    tmem_st4(s_tmem + 4 * c, pk[0], pk[1], pk[2], pk[3]);
                 }
-                tmem_st4(s_tmem + 4 * c, pk[0], pk[1], pk[2], pk[3]);
-            }
-            l = l * alpha + rowsum;
+                return rowsum;
+            };
+            if (first)
+                l = l * alpha + p_tile(std::true_type{});
+            else
+                p_tile(std::false_type{});
             if (j > 0) {
                 ok = warp_all_pair(mbar_wait(&bars->o_done, (uint32_t)((it - 1) & 1)));
                 if (!ok) break;
