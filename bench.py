@@ -206,6 +206,7 @@ def load_peaks():
 
 def kernel_source_hash(kernel):
     files = {"tc_attn_kernel": "attn_tc.cu", "tc_attn_kernel<mla>": "attn_tc.cu", "tc_attn_pair_kernel": "attn_pair.cu",
+             "tc_attn_pair_kernel<mla>": "attn_pair.cu",
              "tc_attn2_kernel": "attn_tc.cu", "tc_attn2_kernel<mla>": "attn_tc.cu",
              "sparse_tc_kernel": "sparse_tc.cu", "simple_attn_kernel<sparse>": "simple_kernels.cu",
              "simple_attn_kernel": "simple_kernels.cu"}

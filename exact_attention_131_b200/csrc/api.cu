@@ -250,7 +250,7 @@ AttnPlan plan_attn(const arc_attn_args *a)
     pl.grid = pl.n_tiles * a->B * a->Hkv * pl.n_slices;
     pl.stages = tc_max_stages(a->D);
     maybe_two(pl, a->D, false, a->B * a->Hkv);
-    if (!pl.two && !(a->flags & ARC_FLAG_SINGLE_CTA) && pair_supported(a->D, pl.dvs)) {
+    if (!pl.two && !(a->flags & ARC_FLAG_SINGLE_CTA) && pair_supported(a->D, pl.dvs, false)) {
         pl.pair = true;
         pl.stages = pair_max_stages(a->D);
         // persistent: at most one resident cluster per two SMs walks the list of row-tile pairs
@@ -317,6 +317,14 @@ AttnPlan plan_mla(const arc_mla_args *a)
     pl.grid = pl.n_tiles * a->B * a->H;
     pl.stages = tc_max_stages(dqk);
     maybe_two(pl, dqk, true, a->B * a->H);
+    if (!(a->flags & ARC_FLAG_SINGLE_CTA) && pair_supported(dqk, a->Dv, true)) {
+        // CTA pair (M = 256), persistent like the dense pair path
+        pl.two = false;
+        pl.pair = true;
+        pl.stages = pair_max_stages(dqk);
+        const int items = ((pl.n_tiles + 1) / 2) * a->B * a->H;
+        pl.grid = 2 * std::min(items, std::max(1, sm_count() / 2));
+    }
     return pl;
 }
 
@@ -481,7 +489,7 @@ arc_status arc_attn_fwd(const arc_attn_args *a, void *stream)
         } else if (pl.pair) {
             order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
             note_dispatch("tc_attn_pair_kernel");
-            e = launch_tc_attn_pair(p, a->D, pl.dvs, pl.grid, s);
+            e = launch_tc_attn_pair(p, a->D, pl.dvs, false, pl.grid, s);
         } else {
             order_tiles(p, pl.n_tiles);
             note_dispatch("tc_attn_kernel");
@@ -531,9 +539,10 @@ arc_status arc_mla_fwd(const arc_mla_args *a, void *stream)
         const uint64_t vd[4] = {(uint64_t)a->Dv, (uint64_t)a->Tk, (uint64_t)a->H, (uint64_t)a->B};
         const int64_t vs[3] = {a->v_strides[2], nz(a->v_strides[1], (int64_t)a->Tk * a->v_strides[2]),
                                nz(a->v_strides[0], (int64_t)a->H * a->Tk * a->v_strides[2])};
+        const uint32_t kv_box = pl.pair ? 64 : kTcBN;   // a CTA of a pair stages half of each key tile
         if (!make_map(&p.tm_q, a->q_nope, 3, qnd, qns, kTcBM) || !make_map(&p.tm_q2, a->q_rope, 3, qrd, qrs, kTcBM) ||
-            !make_map(&p.tm_k, a->k_nope, 4, knd, kns, kTcBN) || !make_map(&p.tm_k2, a->k_rope, 3, krd, krs, kTcBN) ||
-            !make_map(&p.tm_v, a->v, 4, vd, vs, kTcBN))
+            !make_map(&p.tm_k, a->k_nope, 4, knd, kns, kv_box) || !make_map(&p.tm_k2, a->k_rope, 3, krd, krs, kv_box) ||
+            !make_map(&p.tm_v, a->v, 4, vd, vs, kv_box))
             return ARC_ERR_CUDA;
         p.B = a->B, p.H = a->H, p.Hkv = a->H, p.G = 1, p.Tq = a->Tq, p.Tk = a->Tk, p.Dv = a->Dv;
         p.n_tiles = pl.n_tiles, p.n_slices = 1, p.kc_first = a->Dn / 64, p.stages = pl.stages;
@@ -541,7 +550,11 @@ arc_status arc_mla_fwd(const arc_mla_args *a, void *stream)
         for (int i = 0; i < 3; ++i) p.os[i] = a->o_strides[i];
         p.lse = a->lse, p.sinks = nullptr, p.scale_log2 = a->scale * kLog2e, p.causal = a->causal;
         p.status = a->status;
-        if (pl.two) {
+        if (pl.pair) {
+            order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
+            note_dispatch("tc_attn_pair_kernel<mla>");
+            e = launch_tc_attn_pair(p, a->Dn + a->Dr, a->Dv, true, pl.grid, s);
+        } else if (pl.two) {
             order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
             note_dispatch("tc_attn2_kernel<mla>");
             e = launch_tc_attn2(p, a->Dn + a->Dr, a->Dv, true, pl.grid, s);
@@ -721,10 +734,13 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             set_name(out, "simple_attn_kernel");
             out->tile_m = 4;
         } else {
-            set_name(out, pl.two ? "tc_attn2_kernel<mla>" : "tc_attn_kernel<mla>");
+            set_name(out, pl.pair ? "tc_attn_pair_kernel<mla>" : (pl.two ? "tc_attn2_kernel<mla>" : "tc_attn_kernel<mla>"));
             out->tensor_cores = 1;
-            out->tile_m = pl.two ? 2 * kTcBM : kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs, out->n_ctas = pl.grid;
-            out->smem_bytes = pl.two ? tc2_smem_bytes(a->Dn + a->Dr, pl.stages) : tc_smem_bytes(a->Dn + a->Dr, pl.stages);
+            out->tile_m = (pl.two || pl.pair) ? 2 * kTcBM : kTcBM, out->tile_n = kTcBN, out->d_slice = pl.dvs,
+            out->n_ctas = pl.grid;
+            out->smem_bytes = pl.pair ? pair_smem_bytes(a->Dn + a->Dr, pl.stages)
+                                      : (pl.two ? tc2_smem_bytes(a->Dn + a->Dr, pl.stages)
+                                                : tc_smem_bytes(a->Dn + a->Dr, pl.stages));
             out->tmem_cols = 512;
         }
         out->launches = 1;

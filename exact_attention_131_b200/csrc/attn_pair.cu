@@ -1,6 +1,11 @@
 // attn_pair.cu -- attention forward on a pair of CTAs (cta_group::2), for
 // head dims where one CTA's shared memory is mostly taken by its Q tile
-// (d_qk = 512: 128 query rows x 512 = 128 KB).
+// (d_qk = 512: 128 query rows x 512 = 128 KB), and for MLA prefill
+// (d_qk 128 + 64, d_v 128: one d_v pass, Q and K concatenated on load from
+// the nope and the shared rope tensors).  With M = 256 each CTA reads only half
+// of every B operand from its shared memory, which keeps the S = Q K^T MMAs of
+// the small head dims below the shared-memory bandwidth (an M = 128, N = 128
+// SS MMA reads 8 KB per 64 clk, all of it).
 //
 // A cluster of two CTAs owns 256 consecutive fold rows of one (batch, kv head)
 // group and one d_v slice; each CTA keeps its own 128 rows of Q and of O.  The
@@ -220,13 +225,17 @@ __device__ __forceinline__ void st_global_v8(void *dst, const uint32_t *w)
                  : "memory");
 }
 
-template <int DQK, int DVS>
+template <int DQK, int DVS, bool MLA>
 __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid_constant__ TcParams p)
 {
     constexpr int KC = DQK / 64;     // 64-column chunks of a Q / K row
     constexpr int VG = DVS / 128;    // 128-column MMA groups of the d_v slice
+    // Boxes per ring stage: BPS when a tile's boxes are a multiple of it, else the
+    // whole tile in one partly filled stage (d_qk 192: 3 K boxes; d_v 128: 2 V boxes).
+    constexpr int KB = (KC % BPS == 0) ? BPS : KC;
+    constexpr int VB = ((2 * VG) % BPS == 0) ? BPS : 2 * VG;
     static_assert(DQK % 64 == 0 && DVS % 128 == 0 && DVS <= 256, "tile shape");
-    static_assert(KC % BPS == 0 && (2 * VG) % BPS == 0, "K and V tiles fill whole ring stages");
+    static_assert(KB <= BPS && KC % KB == 0 && VB <= BPS && (2 * VG) % VB == 0, "K and V tiles fill ring stages");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem<1024>(smem_raw);
@@ -286,9 +295,9 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             bool ok = true;
             // Each barrier round trip costs this thread a few hundred clocks, so a
             // stage carries BPS boxes: one wait and one expect_tx per 32 KB.
-            auto acquire = [&]() -> bool {
+            auto acquire = [&](int boxes) -> bool {
                 if (!mbar_wait(&bars->empty[stage], ephase ^ 1u)) return false;
-                if (leader) mbar_arrive_expect_tx_u32(smem_u32(&bars->full[stage]), 2 * PST);
+                if (leader) mbar_arrive_expect_tx_u32(smem_u32(&bars->full[stage]), 2 * boxes * PCH);
                 return true;
             };
             auto advance = [&]() {
@@ -312,16 +321,27 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                         tma2_load_5d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, 0, r0 / p.G, kv, b);
                 } else {
                     const int qrow = kv * rows_in_group + r0;
-                    for (int c = 0; c < KC; ++c) tma2_load_3d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, qrow, b);
+                    for (int c = 0; c < KC; ++c) {
+                        if (!MLA || c < p.kc_first)
+                            tma2_load_3d(sQ + c * 2 * PCH, &p.tm_q, q_full_l, c * 64, qrow, b);
+                        else   // MLA: the rope columns of q
+                            tma2_load_3d(sQ + c * 2 * PCH, &p.tm_q2, q_full_l, (c - p.kc_first) * 64, qrow, b);
+                    }
                 }
                 ++qn;
                 auto load_k = [&](int j) -> bool {
-                    for (int cc = 0; cc < KC; cc += BPS) {
-                        if (!acquire()) return false;
+                    for (int cc = 0; cc < KC; cc += KB) {
+                        if (!acquire(KB)) return false;
                         const uint32_t fl = full_l();
-                        for (int q = 0; q < BPS; ++q)
-                            tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_k, fl, (cc + q) * 64,
-                                         j * PBN + (int)rank * 64, kv, b);
+                        for (int q = 0; q < KB; ++q) {
+                            const int c = cc + q;
+                            if (!MLA || c < p.kc_first)
+                                tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_k, fl, c * 64,
+                                             j * PBN + (int)rank * 64, kv, b);
+                            else   // MLA: the rope columns, shared by every head
+                                tma2_load_3d(sRing + stage * PST + q * PCH, &p.tm_k2, fl, (c - p.kc_first) * 64,
+                                             j * PBN + (int)rank * 64, b);
+                        }
                         advance();
                     }
                     return true;
@@ -329,10 +349,10 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
                 // V box q of a stage: 128-column group q / 2, key half q % 2
                 auto load_v = [&](int it) -> bool {
                     const int j = it % nt, dv0 = (it / nt) * DVS;
-                    for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
-                        if (!acquire()) return false;
+                    for (int q0 = 0; q0 < 2 * VG; q0 += VB) {
+                        if (!acquire(VB)) return false;
                         const uint32_t fl = full_l();
-                        for (int q = 0; q < BPS; ++q) {
+                        for (int q = 0; q < VB; ++q) {
                             const int g = (q0 + q) >> 1, hh = (q0 + q) & 1;
                             tma2_load_4d(sRing + stage * PST + q * PCH, &p.tm_v, fl, dv0 + g * 128 + (int)rank * 64,
                                          j * PBN + hh * 64, kv, b);
@@ -387,12 +407,12 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             };
             auto issue_s = [&](int it) -> bool {
                 const uint32_t d = tmem + P_SCOL + (it & 1) * PBN;
-                if (!wait_boxes(KC / BPS)) return false;
+                if (!wait_boxes(KC / KB)) return false;
                 tc_fence_after();
 #pragma unroll 1
-                for (int c0 = 0; c0 < KC; c0 += BPS) {
+                for (int c0 = 0; c0 < KC; c0 += KB) {
 #pragma unroll
-                    for (int q = 0; q < BPS; ++q)
+                    for (int q = 0; q < KB; ++q)
                         umma2_ss_k64(d, qd0 + (uint64_t)((c0 + q) * 2 * kBox), kd0 + (uint64_t)((stage * BPS + q) * kBox),
                                      idesc_s, (c0 + q) > 0);
                     umma2_commit_both(&bars->empty[stage]);
@@ -403,13 +423,13 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
             };
             auto issue_pv = [&](int it, bool first) -> bool {   // first key tile of a slice overwrites O
                 if (!mbar_wait_cluster(&bars->p_full, (uint32_t)(it & 1))) return false;
-                if (!wait_boxes(2 * VG / BPS)) return false;
+                if (!wait_boxes(2 * VG / VB)) return false;
                 tc_fence_after();
                 const uint32_t p_tm = tmem + P_SCOL + (it & 1) * PBN;
 #pragma unroll 1
-                for (int q0 = 0; q0 < 2 * VG; q0 += BPS) {
+                for (int q0 = 0; q0 < 2 * VG; q0 += VB) {
 #pragma unroll
-                    for (int q = 0; q < BPS; ++q) {
+                    for (int q = 0; q < VB; ++q) {
                         const int g = (q0 + q) >> 1, hh = (q0 + q) & 1;
                         umma2_ts_k64(tmem + g * 128, p_tm + hh * 32, vd0 + (uint64_t)((stage * BPS + q) * kBox), idesc_pv,
                                      (first ? 0 : 1) | hh);
@@ -615,11 +635,11 @@ __global__ void __launch_bounds__(P_THREADS, 1) tc_attn_pair_kernel(const __grid
     cluster_sync_all();
 }
 
-template <int DQK, int DVS>
+template <int DQK, int DVS, bool MLA>
 cudaError_t launch_p(const TcParams &p, int grid, cudaStream_t s)
 {
     const int smem = pair_smem_bytes(DQK, p.stages);
-    auto kern = tc_attn_pair_kernel<DQK, DVS>;
+    auto kern = tc_attn_pair_kernel<DQK, DVS, MLA>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -655,12 +675,16 @@ int pair_max_stages(int dqk)
     return st < P_MAX_STAGES ? st : P_MAX_STAGES;
 }
 
-bool pair_supported(int dqk, int dvs) { return (dqk == 512 || dqk == 256) && dvs == 256; }
-
-cudaError_t launch_tc_attn_pair(const TcParams &p, int dqk, int dvs, int grid, cudaStream_t s)
+bool pair_supported(int dqk, int dvs, bool mla)
 {
-    if (dqk == 512 && dvs == 256) return launch_p<512, 256>(p, grid, s);
-    if (dqk == 256 && dvs == 256) return launch_p<256, 256>(p, grid, s);
+    return mla ? (dqk == 192 && dvs == 128) : ((dqk == 512 || dqk == 256) && dvs == 256);
+}
+
+cudaError_t launch_tc_attn_pair(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s)
+{
+    if (!mla && dqk == 512 && dvs == 256) return launch_p<512, 256, false>(p, grid, s);
+    if (!mla && dqk == 256 && dvs == 256) return launch_p<256, 256, false>(p, grid, s);
+    if (mla && dqk == 192 && dvs == 128) return launch_p<192, 128, true>(p, grid, s);
     return cudaErrorInvalidValue;
 }
 

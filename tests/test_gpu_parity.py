@@ -124,15 +124,31 @@ def test_mla_small(B, H, T, Dn, Dr, Dv):
     st = status_word()
     o, lse, t = run_mla(c, status=st)
     info = arc.plan_mla(*t, o, lse)
-    assert info["kernel"] == "tc_attn2_kernel<mla>"
+    # d_qk 128 + 64 with d_v 128 runs on a CTA pair (M = 256); other shapes on two tiles per CTA
+    assert info["kernel"] == ("tc_attn_pair_kernel<mla>" if (Dn + Dr, Dv) == (192, 128) else "tc_attn2_kernel<mla>")
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
     assert arc.check_device_error(st) == arc.ARC_OK
 
 
+@pytest.mark.parametrize("B,H,T,causal", [(1, 2, 700, True),    # 3 row tiles: the last pair's second CTA is empty
+                                          (2, 3, 520, False),
+                                          (1, 1, 1000, True)])
+def test_mla_pair_and_two_tile_agree_with_oracle(B, H, T, causal):
+    c = W.mla_case(B, H, T, T, 128, 64, 128, causal=causal, seed=34)
+    ro, rl = oracle.run_case(c)
+    for flags, name in ((0, "tc_attn_pair_kernel<mla>"), (arc.ARC_FLAG_SINGLE_CTA, "tc_attn2_kernel<mla>")):
+        st = status_word()
+        o, lse, t = run_mla(c, flags=flags, status=st)
+        assert arc.plan_mla(*t, o, lse, causal=causal, flags=flags)["kernel"] == name
+        compare(o, lse, ro, rl, TOL_O_BF16)
+        assert arc.check_device_error(st) == arc.ARC_OK
+
+
 def test_config3_mla_full_size_sampled_rows():
     c = W.config(3)
     o, lse, t = run_mla(c)
+    assert arc.plan_mla(*t, o, lse)["kernel"] == "tc_attn_pair_kernel<mla>"
     rows = sample_rows(c.Tq, 24, 3)
     ro, rl = oracle.run_case(c, rows=rows)
     compare(o[:, :, rows], lse[:, :, rows], ro, rl, TOL_O_BF16)
