@@ -194,7 +194,7 @@ enum class Path { None, Simple, Tc };
 struct AttnPlan {
     Path path = Path::None;
     bool two = false;   // two query tiles per CTA (d_v <= 128)
-    bool pair = false;  // CTA pair, M = 256 (d_qk 256 / 512, d_v slice 256)
+    bool pair = false;  // CTA pair, M = 256 (see pair_supported)
     int dvs = 0, n_slices = 0, n_tiles = 0, grid = 0, stages = 0;
 };
 
@@ -249,7 +249,7 @@ AttnPlan plan_attn(const arc_attn_args *a)
     pl.n_tiles = (a->H / a->Hkv * a->Tq + kTcBM - 1) / kTcBM;
     pl.grid = pl.n_tiles * a->B * a->Hkv * pl.n_slices;
     pl.stages = tc_max_stages(a->D);
-    maybe_two(pl, a->D, false, a->B * a->Hkv);
+    if ((a->flags & ARC_FLAG_SINGLE_CTA) || !pair_supported(a->D, pl.dvs, false)) maybe_two(pl, a->D, false, a->B * a->Hkv);
     if (!pl.two && !(a->flags & ARC_FLAG_SINGLE_CTA) && pair_supported(a->D, pl.dvs, false)) {
         pl.pair = true;
         pl.stages = pair_max_stages(a->D);

@@ -1,6 +1,7 @@
 // attn_pair.cu -- attention forward on a pair of CTAs (cta_group::2), for
 // head dims where one CTA's shared memory is mostly taken by its Q tile
-// (d_qk = 512: 128 query rows x 512 = 128 KB), and for MLA prefill
+// (d_qk = 512: 128 query rows x 512 = 128 KB), for d_qk 128-256 with d_v 128,
+// and for MLA prefill
 // (d_qk 128 + 64, d_v 128: one d_v pass, Q and K concatenated on load from
 // the nope and the shared rope tensors).  With M = 256 each CTA reads only half
 // of every B operand from its shared memory, which keeps the S = Q K^T MMAs of
@@ -677,13 +678,17 @@ int pair_max_stages(int dqk)
 
 bool pair_supported(int dqk, int dvs, bool mla)
 {
-    return mla ? (dqk == 192 && dvs == 128) : ((dqk == 512 || dqk == 256) && dvs == 256);
+    if (mla) return dqk == 192 && dvs == 128;
+    return ((dqk == 512 || dqk == 256) && dvs == 256) || ((dqk == 128 || dqk == 192 || dqk == 256) && dvs == 128);
 }
 
 cudaError_t launch_tc_attn_pair(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s)
 {
     if (!mla && dqk == 512 && dvs == 256) return launch_p<512, 256, false>(p, grid, s);
     if (!mla && dqk == 256 && dvs == 256) return launch_p<256, 256, false>(p, grid, s);
+    if (!mla && dqk == 256 && dvs == 128) return launch_p<256, 128, false>(p, grid, s);
+    if (!mla && dqk == 192 && dvs == 128) return launch_p<192, 128, false>(p, grid, s);
+    if (!mla && dqk == 128 && dvs == 128) return launch_p<128, 128, false>(p, grid, s);
     if (mla && dqk == 192 && dvs == 128) return launch_p<192, 128, true>(p, grid, s);
     return cudaErrorInvalidValue;
 }

@@ -73,7 +73,7 @@ int tc2_max_stages(int dqk);
 cudaError_t launch_tc_attn2(const TcParams &p, int dqk, int dvs, bool mla, int grid, cudaStream_t s);
 
 // Pair of CTAs (cta_group::2, M = 256): dense d_qk in {256, 512} with a 256-wide
-// d_v slice; MLA d_qk 192 (128 + 64) with d_v 128.
+// d_v slice or d_qk in {128, 192, 256} with d_v 128; MLA d_qk 192 (128 + 64), d_v 128.
 int pair_smem_bytes(int dqk, int stages);
 int pair_max_stages(int dqk);
 bool pair_supported(int dqk, int dvs, bool mla);

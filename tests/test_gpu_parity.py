@@ -55,8 +55,10 @@ def test_dense_bf16_small(B, H, Hkv, Tq, Tk, D, Dv, causal, sinks):
 
 
 def expected_dense_kernel(D, Dv):
-    # d_v <= 128: two query tiles per CTA; d_qk 256 / 512 with a 256-wide d_v
-    # slice: a CTA pair (M = 256); otherwise one tile per d_v slice
+    # a CTA pair (M = 256) for d_qk 128-256 with d_v 128 and for d_qk 256 / 512 with a
+    # 256-wide d_v slice; other d_v <= 128: two query tiles per CTA; else one tile per slice
+    if (D, Dv) in ((128, 128), (192, 128), (256, 128)):
+        return "tc_attn_pair_kernel"
     if Dv <= 128:
         return "tc_attn2_kernel"
     if D in (256, 512) and Dv in (256, 512):
@@ -73,6 +75,23 @@ def test_dense_pair_and_single_cta_agree_with_oracle(B, H, Hkv, Tq, Tk, D, causa
     c = W.dense_case(B, H, Hkv, Tq, Tk, D, D, dtype="bf16", std=0.5, causal=causal, sinks=sinks, seed=34)
     ro, rl = oracle.run_case(c)
     for flags, name in ((0, "tc_attn_pair_kernel"), (arc.ARC_FLAG_SINGLE_CTA, "tc_attn_kernel")):
+        st = status_word()
+        o, lse, (q, k, v, s) = run_dense(c, flags=flags, status=st)
+        info = arc.plan_attn(q, k, v, o, lse, causal=causal, sinks=s, flags=flags)
+        assert info["kernel"] == name
+        compare(o, lse, ro, rl, TOL_O_BF16)
+        assert arc.check_device_error(st) == arc.ARC_OK
+
+
+@pytest.mark.parametrize("B,H,Hkv,Tq,Tk,D,causal,sinks", [
+    (1, 8, 2, 300, 300, 128, True, True),      # G = 4: t-major fold
+    (2, 6, 3, 260, 400, 192, True, False),     # Tq < Tk, 3 row tiles: last pair half empty
+    (1, 4, 4, 200, 200, 256, False, True),     # non-causal, G = 1
+])
+def test_dense_small_d_pair_and_two_tile_agree_with_oracle(B, H, Hkv, Tq, Tk, D, causal, sinks):
+    c = W.dense_case(B, H, Hkv, Tq, Tk, D, 128, dtype="bf16", std=0.5, causal=causal, sinks=sinks, seed=35)
+    ro, rl = oracle.run_case(c)
+    for flags, name in ((0, "tc_attn_pair_kernel"), (arc.ARC_FLAG_SINGLE_CTA, "tc_attn2_kernel")):
         st = status_word()
         o, lse, (q, k, v, s) = run_dense(c, flags=flags, status=st)
         info = arc.plan_attn(q, k, v, o, lse, causal=causal, sinks=s, flags=flags)
