@@ -9,6 +9,7 @@ Names follow the C ABI:
     mla_fwd             -> arc_mla_fwd          q_nope||q_rope, d_qk != d_v
     sparse_mla_fwd      -> arc_sparse_mla_fwd   per-query top-k index lists
     attn_decode_q8      -> arc_attn_decode_q8   q8_0 / q4_0 cache, multi-sequence
+    attn_merge          -> arc_attn_merge       results over disjoint key sets -> the whole
     plan                -> arc_plan             engagement record, no launch
 """
 from __future__ import annotations
@@ -24,7 +25,8 @@ _lib = None
 ARC_OK, ARC_ERR_INVALID_ARG, ARC_ERR_UNSUPPORTED, ARC_ERR_CUDA, ARC_ERR_DEVICE_TIMEOUT, ARC_ERR_WORKSPACE = range(6)
 ARC_DTYPE_BF16, ARC_DTYPE_F32 = 0, 1
 ARC_KV_Q4_0, ARC_KV_Q8_0 = 2, 8
-ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE = 1, 2, 3, 4
+ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE, ARC_OP_MERGE = 1, 2, 3, 4, 5
+ARC_MERGE_MAX_PARTS = 16
 ARC_FLAG_FORCE_SIMPLE = 1
 ARC_FLAG_SINGLE_CTA = 2
 ARC_DECODE_MAX_SEQ = 64
@@ -68,6 +70,12 @@ class DecodeArgs(ctypes.Structure):
                 ("status", _vp)]
 
 
+class MergeArgs(ctypes.Structure):
+    _fields_ = [("n_parts", _i32), ("rows", _i32), ("dv", _i32), ("dtype", _i32),
+                ("o_parts", _vp * ARC_MERGE_MAX_PARTS), ("lse_parts", _vp * ARC_MERGE_MAX_PARTS),
+                ("sinks", _vp), ("sink_heads", _i32), ("sink_rows", _i32), ("o", _vp), ("lse", _vp)]
+
+
 class PlanInfo(ctypes.Structure):
     _fields_ = [("kernel", ctypes.c_char * 64), ("tensor_cores", _i32), ("tile_m", _i32), ("tile_n", _i32),
                 ("d_slice", _i32), ("n_ctas", _i32), ("splits", _i32), ("smem_bytes", _i32),
@@ -76,7 +84,7 @@ class PlanInfo(ctypes.Structure):
 
 EXPORTS = ["arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
            "arc_decode_workspace_size", "arc_plan", "arc_abi_version", "arc_status_string",
-           "arc_check_device_error", "arc_selftest_timeout", "arc_attn_decode_q8_noalloc"]
+           "arc_check_device_error", "arc_selftest_timeout", "arc_attn_decode_q8_noalloc", "arc_attn_merge"]
 
 
 class ArcError(RuntimeError):
@@ -98,6 +106,7 @@ def lib():
         L.arc_sparse_mla_fwd.argtypes = [ctypes.POINTER(SparseArgs), _vp]
         L.arc_attn_decode_q8.argtypes = [ctypes.POINTER(DecodeArgs), _vp, ctypes.c_size_t, _vp]
         L.arc_attn_decode_q8_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
+        L.arc_attn_merge.argtypes = [ctypes.POINTER(MergeArgs), _vp]
         L.arc_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]
         L.arc_decode_workspace_size.restype = ctypes.c_size_t
         L.arc_plan.argtypes = [_i32, _vp, ctypes.POINTER(PlanInfo)]
@@ -106,7 +115,7 @@ def lib():
         L.arc_check_device_error.argtypes = [_vp, _vp]
         L.arc_selftest_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
         for f in ("arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
-                  "arc_attn_decode_q8_noalloc", "arc_plan",
+                  "arc_attn_decode_q8_noalloc", "arc_attn_merge", "arc_plan",
                   "arc_check_device_error", "arc_selftest_timeout", "arc_abi_version"):
             getattr(L, f).restype = _i32
         _lib = L
@@ -355,6 +364,56 @@ def attn_decode_q8_noalloc(q, k_cache, v_cache, *, kv_type, Hkv, q_begin, n_q, k
     return out, lse
 
 
+def _merge_args(o_parts, lse_parts, o, lse, sinks, sink_rows):
+    n = len(o_parts)
+    if not 1 <= n <= ARC_MERGE_MAX_PARTS or len(lse_parts) != n:
+        raise ValueError(f"1..{ARC_MERGE_MAX_PARTS} parts, one LSE per O")
+    dv = int(o_parts[0].shape[-1])
+    rows = int(o_parts[0].numel() // dv) if dv else 0
+    a = MergeArgs()
+    a.n_parts, a.rows, a.dv = n, rows, dv
+    torch = _torch()
+    a.dtype = ARC_DTYPE_F32 if o_parts[0].dtype == torch.float32 else ARC_DTYPE_BF16
+    for i in range(n):
+        a.o_parts[i], a.lse_parts[i] = _p(o_parts[i]), _p(lse_parts[i])
+    a.sinks = _p(sinks)
+    a.sink_heads = int(sinks.numel()) if sinks is not None else 0
+    a.sink_rows = int(sink_rows) if sinks is not None else 0
+    a.o, a.lse = _p(o), _p(lse)
+    return a
+
+
+def attn_merge(o_parts, lse_parts, *, sinks=None, sink_rows=None, out=None, lse=None, stream=None):
+    """O, LSE = arc_attn_merge over parts computed on disjoint key sets.
+
+    o_parts: tensors of one shape [..., dv] (bf16 or fp32, contiguous); lse_parts: the
+    matching [...] fp32 log-sum-exps (natural log, -inf = empty part).  sinks: optional
+    [H] fp32 sink logits added once (parts computed without them); for [B, H, Tq, dv]
+    outputs pass sink_rows = Tq.
+    """
+    torch = _torch()
+    if not o_parts:
+        raise ValueError("at least one part")
+    shape, dt = o_parts[0].shape, o_parts[0].dtype
+    for i, (o_i, l_i) in enumerate(zip(o_parts, lse_parts)):
+        _dev(o_i, f"o_parts[{i}]", dt), _dev(l_i, f"lse_parts[{i}]", torch.float32)
+        if o_i.shape != shape or tuple(l_i.shape) != tuple(shape[:-1]):
+            raise ValueError("every part must have the shape of the first, and LSE its leading dims")
+        if not (o_i.is_contiguous() and l_i.is_contiguous()):
+            raise ValueError("parts must be contiguous")
+    if sinks is not None:
+        _dev(sinks, "sinks", torch.float32)
+        if sink_rows is None:
+            raise ValueError("sink_rows is needed with sinks (Tq for [B, H, Tq, dv] rows)")
+    if out is None:
+        out = torch.empty(shape, dtype=dt, device=o_parts[0].device)
+    if lse is None:
+        lse = torch.empty(shape[:-1], dtype=torch.float32, device=o_parts[0].device)
+    a = _merge_args(o_parts, lse_parts, out, lse, sinks, sink_rows)
+    _check(lib().arc_attn_merge(ctypes.byref(a), _stream(stream)), "arc_attn_merge")
+    return out, lse
+
+
 def plan(op: int, args) -> dict:
     """arc_plan on a filled args struct: which kernel a call launches, without launching it."""
     info = PlanInfo()
@@ -381,6 +440,10 @@ def plan_decode(kv_type, q, k_cache, v_cache, *, Hkv, q_begin, n_q, kv_begin, n_
     a = _decode_args(kv_type, q, k_cache, v_cache, seqs, len(q_begin), Hkv, k_cache.shape[0], q, q, 1.0,
                      flags, None)
     return plan(ARC_OP_DECODE, a)
+
+
+def plan_merge(o_parts, lse_parts, out, lse) -> dict:
+    return plan(ARC_OP_MERGE, _merge_args(o_parts, lse_parts, out, lse, None, None))
 
 
 def check_device_error(status, stream=None) -> int:

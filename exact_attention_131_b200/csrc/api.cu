@@ -691,6 +691,29 @@ arc_status arc_attn_decode_q8_noalloc(const arc_decode_args *a, void *stream)
     return arc_attn_decode_q8(a, scratch, ARC_DECODE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+arc_status arc_attn_merge(const arc_merge_args *a, void *stream)
+{
+    if (!a) return ARC_ERR_INVALID_ARG;
+    if (a->n_parts < 1 || a->n_parts > ARC_MERGE_MAX_PARTS || a->rows < 0 || a->dv <= 0 || (a->dv & 1))
+        return ARC_ERR_INVALID_ARG;
+    if (a->dv > 1024) return ARC_ERR_UNSUPPORTED;
+    if (a->dtype != ARC_DTYPE_F32 && a->dtype != ARC_DTYPE_BF16) return ARC_ERR_INVALID_ARG;
+    if (a->sinks && (a->sink_heads <= 0 || a->sink_rows <= 0)) return ARC_ERR_INVALID_ARG;
+    if (a->rows == 0) return ARC_OK;
+    auto bad = [](const void *ptr) { return !ptr || (reinterpret_cast<uintptr_t>(ptr) & 7u); };
+    if (bad(a->o) || bad(a->lse)) return ARC_ERR_INVALID_ARG;
+    for (int i = 0; i < a->n_parts; ++i)
+        if (bad(a->o_parts[i]) || !a->lse_parts[i] || (reinterpret_cast<uintptr_t>(a->lse_parts[i]) & 3u))
+            return ARC_ERR_INVALID_ARG;
+    MergeParams p{};
+    p.n_parts = a->n_parts, p.rows = a->rows, p.dv = a->dv, p.dtype = a->dtype;
+    for (int i = 0; i < a->n_parts; ++i) p.o_parts[i] = a->o_parts[i], p.lse_parts[i] = a->lse_parts[i];
+    p.sinks = a->sinks, p.sink_heads = a->sink_heads, p.sink_rows = a->sink_rows;
+    p.o = a->o, p.lse = a->lse;
+    note_dispatch("merge_kernel");
+    return launch_merge(p, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
 arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
 {
     if (!args || !out) return ARC_ERR_INVALID_ARG;
@@ -744,6 +767,15 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             out->tmem_cols = 512;
         }
         out->launches = 1;
+        return ARC_OK;
+    }
+    if (op == ARC_OP_MERGE) {
+        const arc_merge_args *a = static_cast<const arc_merge_args *>(args);
+        if (a->n_parts < 1 || a->n_parts > ARC_MERGE_MAX_PARTS || a->rows < 0 || a->dv <= 0 || (a->dv & 1))
+            return ARC_ERR_INVALID_ARG;
+        set_name(out, "merge_kernel");
+        out->n_ctas = (a->rows + 7) / 8;
+        out->launches = a->rows > 0 ? 1 : 0;
         return ARC_OK;
     }
     if (op == ARC_OP_SPARSE) {

@@ -120,4 +120,16 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s);
 
 cudaError_t launch_selftest_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
 
+// Merge of partial results over disjoint key sets (arc_attn_merge), one warp per row.
+struct MergeParams {
+    int n_parts, rows, dv, dtype;
+    const void *o_parts[ARC_MERGE_MAX_PARTS];
+    const float *lse_parts[ARC_MERGE_MAX_PARTS];
+    const float *sinks;
+    int sink_heads, sink_rows;
+    void *o;
+    float *lse;
+};
+cudaError_t launch_merge(const MergeParams &p, cudaStream_t s);
+
 }  // namespace arc

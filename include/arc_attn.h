@@ -58,7 +58,7 @@ typedef enum { ARC_DTYPE_BF16 = 0, ARC_DTYPE_F32 = 1 } arc_dtype;
 /* Quantised KV block types; the values are the ggml type ids. */
 typedef enum { ARC_KV_Q4_0 = 2, ARC_KV_Q8_0 = 8 } arc_kv_type;
 
-typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE = 4 } arc_op;
+typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE = 4, ARC_OP_MERGE = 5 } arc_op;
 
 /* flags (all calls) */
 #define ARC_FLAG_FORCE_SIMPLE 1u   /* run the CUDA-core kernel instead of the tensor-core one */
@@ -258,6 +258,49 @@ arc_status arc_attn_decode_q8(const arc_decode_args *args, void *workspace, size
 #define ARC_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 
 arc_status arc_attn_decode_q8_noalloc(const arc_decode_args *args, void *stream);
+
+/* --------------------------------------------------------------------------
+ * arc_attn_merge: the exact result over a union of disjoint key sets, from
+ * the results over each set.
+ *
+ * When the keys of every row are split over parts (context-parallel ranks,
+ * or the chunks of a long sequence), each part gives its own normalised
+ * output O_i and log-sum-exp LSE_i.  The merge is the output merge of
+ * "TransformerEngine: FA4 in context-parallel attention" (flowchart):
+ *
+ *     LSE = ln( sum_i exp(LSE_i) [+ exp(sink)] )
+ *     O   = sum_i exp(LSE_i - LSE) * O_i
+ *
+ * which equals attention over all the keys at once.  A per-head sink logit,
+ * if given, is added once here (the parts must then be computed without it).
+ * A part with LSE_i = -inf is empty and contributes nothing; a row whose
+ * parts are all empty gets O = 0 and LSE = -inf (or = sink).
+ *
+ *   n_parts        1 .. ARC_MERGE_MAX_PARTS
+ *   rows, dv       the parts and the output are [rows, dv], row stride dv
+ *                  (a [B,H,Tq,Dv] output with contiguous rows is rows = B*H*Tq);
+ *                  dv even, <= 1024
+ *   dtype          arc_dtype of every O_i and of o (fp32 arithmetic inside)
+ *   o_parts[i]     device, [rows, dv];   lse_parts[i]  device fp32, [rows]
+ *   sinks          device fp32 or NULL; row r uses sinks[(r / sink_rows) % sink_heads]
+ *                  (for [B,H,Tq] rows: sink_rows = Tq, sink_heads = H)
+ *   o, lse         device, written: [rows, dv] and [rows] fp32
+ * Pointers must be 8-byte aligned.  o may alias o_parts[0] and lse may alias
+ * lse_parts[0] (each row is read in full before it is written).
+ * ------------------------------------------------------------------------ */
+#define ARC_MERGE_MAX_PARTS 16
+
+typedef struct {
+    int32_t n_parts, rows, dv, dtype;
+    const void *o_parts[ARC_MERGE_MAX_PARTS];
+    const float *lse_parts[ARC_MERGE_MAX_PARTS];
+    const float *sinks;
+    int32_t sink_heads, sink_rows;
+    void *o;
+    float *lse;
+} arc_merge_args;
+
+arc_status arc_attn_merge(const arc_merge_args *args, void *stream);
 
 /* --------------------------------------------------------------------------
  * Engagement record and helpers.

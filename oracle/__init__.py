@@ -32,6 +32,7 @@ MUT_TILE_LOCAL_MASK = 2
 MUT_DROP_SINK = 3
 MUT_TOP_LEFT_CAUSAL = 4
 MUT_SWAP_NIBBLES = 5
+MUT_MERGE_UNWEIGHTED = 6
 
 _dp = ctypes.POINTER(ctypes.c_double)
 _ip = ctypes.POINTER(ctypes.c_int32)
@@ -64,10 +65,11 @@ def _load():
         lib.oracle_decode_q.argtypes = [I, I, _ip, _ip, _ip, _ip, I, I, I, I, _dp, I, _bp, _bp,
                                         D, _dp, _dp]
         lib.oracle_dequant_cache.argtypes = [I, I, I, I, _bp, _dp]
+        lib.oracle_merge.argtypes = [I, ctypes.c_long, I, _dp, _dp, _dp, _dp, _dp]
         lib.oracle_set_mutation.argtypes = [I]
         lib.oracle_set_num_threads.argtypes = [I]
         for f in ("oracle_attn", "oracle_attn_tiled", "oracle_attn_fold", "oracle_mla",
-                  "oracle_sparse", "oracle_decode_q", "oracle_dequant_cache"):
+                  "oracle_sparse", "oracle_decode_q", "oracle_dequant_cache", "oracle_merge"):
             getattr(lib, f).restype = ctypes.c_int
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -255,3 +257,23 @@ def run_case(case, rows=None):
     if isinstance(case, W.DecodeCase):
         return decode_q(case)
     raise TypeError(type(case))
+
+
+def merge(o_parts, lse_parts, *, sink_rows=None):
+    """Merge of results over disjoint key sets: o_parts, a list of [..., dv] outputs,
+    lse_parts the matching [...] natural-log LSEs (-inf = empty part); sink_rows,
+    optional [...] sink logits added once.  Returns (o, lse) over the union of the keys.
+    Follows the output merge of "TransformerEngine: FA4 in context-parallel attention"
+    (flowchart); see oracle_merge in arc_oracle.c."""
+    shape = np.shape(o_parts[0])
+    dv = shape[-1]
+    rows = int(np.prod(shape[:-1]))
+    op = _c(np.stack([widen(x).reshape(rows, dv) for x in o_parts]))
+    lp = _c(np.stack([widen(x).reshape(rows) for x in lse_parts]))
+    sr = None if sink_rows is None else _c(np.broadcast_to(widen(sink_rows), shape[:-1]).reshape(rows))
+    o = np.zeros((rows, dv))
+    lse = np.zeros(rows)
+    rc = _load().oracle_merge(len(o_parts), rows, dv, _ptr(op, _dp), _ptr(lp, _dp), _ptr(sr, _dp),
+                              _ptr(o, _dp), _ptr(lse, _dp))
+    _check(rc, "merge")
+    return o.reshape(shape), lse.reshape(shape[:-1])

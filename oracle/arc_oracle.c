@@ -53,6 +53,7 @@ enum {
     MUT_DROP_SINK = 3,        /* sink left out of the softmax denominator */
     MUT_TOP_LEFT_CAUSAL = 4,  /* causal mask aligned top-left instead of bottom-right */
     MUT_SWAP_NIBBLES = 5,     /* q4_0: low/high nibble roles swapped */
+    MUT_MERGE_UNWEIGHTED = 6, /* merge: plain mean of the parts, no log-sum-exp weights */
 };
 
 static int g_mutation = MUT_NONE;
@@ -490,4 +491,52 @@ int oracle_decode_q(int kv_type, int n_seq, const int32_t *q_begin, const int32_
         free(Vd);
     }
     return fail ? -1 : 0;
+}
+
+/*
+ * Merge of results over disjoint key sets ("TransformerEngine: FA4 in
+ * context-parallel attention", flowchart): when the keys of a row are split
+ * over parts and part i gives a normalised output O_i and log-sum-exp LSE_i
+ * over its own keys, then over all the keys
+ *
+ *   LSE = ln( sum_i exp(LSE_i) + exp(sigma) )      sigma = sink logit, or -inf
+ *   O   = sum_i exp(LSE_i - LSE) O_i
+ *
+ * (the sink enters once, here).  A part with LSE_i = -inf is empty.  A row
+ * with every part empty and no sink gets O = 0 and LSE = -inf.  The largest
+ * term is factored out of the sum only to keep exp finite.
+ *
+ * o_parts [n_parts][rows][dv], lse_parts [n_parts][rows], sink_row [rows] or NULL.
+ */
+int oracle_merge(int n_parts, long rows, int dv, const double *o_parts, const double *lse_parts,
+                 const double *sink_row, double *o, double *lse)
+{
+    if (n_parts < 1 || rows < 0 || dv < 1) return -1;
+#pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        const double sigma = sink_row ? sink_row[r] : -INFINITY;
+        double mx = sigma;
+        for (int i = 0; i < n_parts; ++i) mx = fmax(mx, lse_parts[(long)i * rows + r]);
+        double *orow = o + r * dv;
+        for (int d = 0; d < dv; ++d) orow[d] = 0.0;
+        if (mx == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double sum = (sigma == -INFINITY) ? 0.0 : exp(sigma - mx);
+        for (int i = 0; i < n_parts; ++i) {
+            const double li = lse_parts[(long)i * rows + r];
+            if (li != -INFINITY) sum += exp(li - mx);
+        }
+        const double L = mx + log(sum);
+        lse[r] = L;
+        for (int i = 0; i < n_parts; ++i) {
+            const double li = lse_parts[(long)i * rows + r];
+            if (li == -INFINITY) continue;
+            const double w = (g_mutation == MUT_MERGE_UNWEIGHTED) ? 1.0 / n_parts : exp(li - L);
+            const double *pr = o_parts + ((long)i * rows + r) * dv;
+            for (int d = 0; d < dv; ++d) orow[d] += w * pr[d];
+        }
+    }
+    return 0;
 }

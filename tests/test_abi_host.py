@@ -53,6 +53,7 @@ STRUCTS = {
     "arc_decode_args": ("DecodeArgs", ["q", "seqs", "o", "lse", "scale", "flags", "status"]),
     "arc_plan_info": ("PlanInfo", ["kernel", "tensor_cores", "splits", "launches"]),
     "arc_seq": ("Seq", ["q_begin", "n_kv"]),
+    "arc_merge_args": ("MergeArgs", ["dtype", "o_parts", "lse_parts", "sinks", "sink_rows", "o", "lse"]),
 }
 
 
@@ -123,6 +124,35 @@ def test_decode_validation_and_workspace_size(arc):
     wide = arc.make_seqs([0], [5], [0], [10])                # g * n_q = 20 > 16
     d.seqs, d.n_seq, d.H, d.Hkv = ctypes.cast(wide, ctypes.POINTER(arc.Seq)), 1, 32, 8
     assert L.arc_attn_decode_q8(ctypes.byref(d), None, 0, None) == arc.ARC_ERR_UNSUPPORTED
+
+
+def test_merge_validation_before_any_launch(arc):
+    L = arc.lib()
+    m = arc.MergeArgs()
+    m.n_parts, m.rows, m.dv, m.dtype = 2, 10, 128, arc.ARC_DTYPE_F32
+    assert L.arc_attn_merge(ctypes.byref(m), None) == arc.ARC_ERR_INVALID_ARG     # NULL pointers
+    fake = 1 << 20                                                                # never dereferenced
+    for i in range(2):
+        m.o_parts[i], m.lse_parts[i] = fake, fake
+    m.o, m.lse = fake, fake
+    for field, value, want in (("n_parts", 0, arc.ARC_ERR_INVALID_ARG), ("n_parts", 17, arc.ARC_ERR_INVALID_ARG),
+                               ("dv", 127, arc.ARC_ERR_INVALID_ARG), ("dv", 2048, arc.ARC_ERR_UNSUPPORTED),
+                               ("dtype", 7, arc.ARC_ERR_INVALID_ARG), ("rows", -1, arc.ARC_ERR_INVALID_ARG)):
+        old = getattr(m, field)
+        setattr(m, field, value)
+        assert L.arc_attn_merge(ctypes.byref(m), None) == want, (field, value)
+        setattr(m, field, old)
+    m.o_parts[1] = fake + 4                                                       # misaligned part
+    assert L.arc_attn_merge(ctypes.byref(m), None) == arc.ARC_ERR_INVALID_ARG
+    m.o_parts[1] = fake
+    m.sinks, m.sink_heads, m.sink_rows = fake, 0, 5                               # sinks without a head count
+    assert L.arc_attn_merge(ctypes.byref(m), None) == arc.ARC_ERR_INVALID_ARG
+    m.sinks, m.rows = None, 0                                                     # nothing to do
+    assert L.arc_attn_merge(ctypes.byref(m), None) == arc.ARC_OK
+    info = arc.PlanInfo()
+    m.rows = 100
+    assert L.arc_plan(arc.ARC_OP_MERGE, ctypes.byref(m), ctypes.byref(info)) == arc.ARC_OK
+    assert info.kernel.decode() == "merge_kernel" and info.launches == 1 and info.n_ctas == 13
 
 
 def test_plan_names_the_tensor_core_kernels(arc):

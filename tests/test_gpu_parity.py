@@ -350,3 +350,59 @@ def test_invalid_arguments_launch_nothing():
         arc.attn_fwd(q, k, k, out=out)
     assert e.value.status == arc.ARC_ERR_INVALID_ARG
     assert torch.all(out == 7.0)
+
+
+# ------------------------------------------------------------------ merge over disjoint key sets
+
+@pytest.mark.parametrize("n_parts,dv,dtype,sinks", [(1, 64, "f32", False), (3, 128, "f32", True),
+                                                     (5, 512, "bf16", True), (2, 256, "bf16", False)])
+def test_merge_matches_oracle(n_parts, dv, dtype, sinks):
+    rng = np.random.default_rng(50 + n_parts)
+    B, H, T = 2, 6, 97
+    o_np = [rng.standard_normal((B, H, T, dv)).astype(np.float32) for _ in range(n_parts)]
+    l_np = [(3.0 * rng.standard_normal((B, H, T))).astype(np.float32) for _ in range(n_parts)]
+    for i in range(n_parts):                      # scattered empty parts, and some rows empty in every part
+        l_np[i][rng.random((B, H, T)) < 0.2] = -np.inf
+    for i in range(n_parts):
+        l_np[i][0, 0, :5] = -np.inf
+    s_np = rng.standard_normal(H).astype(np.float32) if sinks else None
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    o_dev = [torch.from_numpy(x).cuda().to(tdt) for x in o_np]
+    l_dev = [torch.from_numpy(x).cuda() for x in l_np]
+    s_dev = torch.from_numpy(s_np).cuda() if sinks else None
+    o, lse = arc.attn_merge(o_dev, l_dev, sinks=s_dev, sink_rows=T if sinks else None)
+    torch.cuda.synchronize()
+    o_in = [x.float().cpu().numpy() for x in o_dev]          # the oracle merges the same (rounded) parts
+    rows = None if s_np is None else np.broadcast_to(s_np.astype(np.float64)[None, :, None], (B, H, T))
+    ro, rl = oracle.merge(o_in, l_np, sink_rows=rows)
+    compare(o, lse, ro, rl, TOL_O_F32 if dtype == "f32" else TOL_O_BF16)
+    info = arc.plan_merge(o_dev, l_dev, o, lse)
+    assert info["kernel"] == "merge_kernel" and info["launches"] == 1
+
+
+def test_merge_in_place_over_the_first_part():
+    rng = np.random.default_rng(57)
+    o_np = [rng.standard_normal((40, 128)).astype(np.float32) for _ in range(2)]
+    l_np = [rng.standard_normal(40).astype(np.float32) for _ in range(2)]
+    o_dev = [torch.from_numpy(x).cuda() for x in o_np]
+    l_dev = [torch.from_numpy(x).cuda() for x in l_np]
+    o, lse = arc.attn_merge(o_dev, l_dev, out=o_dev[0], lse=l_dev[0])
+    torch.cuda.synchronize()
+    ro, rl = oracle.merge(o_np, l_np)
+    compare(o, lse, ro, rl, TOL_O_F32)
+
+
+@pytest.mark.parametrize("world,B,H,Hkv,L,D,sinks", [(2, 1, 8, 2, 200, 128, True), (4, 2, 4, 4, 130, 64, False)])
+def test_context_parallel_chunks_merge_to_attention_over_the_whole_sequence(world, B, H, Hkv, L, D, sinks):
+    """Each emulated rank runs the ring schedule with the library's attention and merge
+    kernels on one GPU; its chunk of O / LSE matches the oracle over the whole sequence."""
+    from exact_attention_131_b200 import cp
+
+    c = W.dense_case(B, H, Hkv, world * L, world * L, D, dtype="bf16", std=0.5, causal=True, sinks=sinks, seed=58)
+    q, k, v = dev(c.q, torch.bfloat16), dev(c.k, torch.bfloat16), dev(c.v, torch.bfloat16)
+    s = dev(c.sinks) if sinks else None
+    outs = cp.context_parallel_forward_local(q, k, v, world, causal=True, scale=c.scale, sinks=s)
+    torch.cuda.synchronize()
+    ro, rl = oracle.attn(c.q, c.k, c.v, scale=c.scale, causal=True, sinks=c.sinks if sinks else None)
+    for r, (o, lse) in enumerate(outs):
+        compare(o, lse, ro[:, :, r * L:(r + 1) * L], rl[:, :, r * L:(r + 1) * L], TOL_O_BF16)

@@ -338,6 +338,71 @@ def test_decode_matches_torch_per_sequence(kv_type):
         assert np.abs(got - ref).max() < TOL
 
 
+# ------------------------------------------------------------------ merge over disjoint key sets
+
+def ref_lse_gqa(q, k, scale, causal_br):
+    """LSE over explicitly masked fp64 scores, K repeated kv-major to every query head."""
+    g = q.shape[1] // k.shape[1]
+    return logsumexp_scores(q, np.repeat(oracle.widen(k), g, axis=1), scale, causal_br)
+
+
+def test_merge_of_key_chunks_equals_attention_over_all_keys():
+    """Attention over random disjoint chunks of the keys (no mask), merged by
+    log-sum-exp, equals torch's fp64 SDPA over all keys.  With sinks the chunks are
+    computed without them and the merge adds the sink once; that equals attention
+    with the sink inside the softmax (pinned against torch elsewhere)."""
+    c = W.dense_case(2, 4, 2, 37, 101, 16, 24, dtype="bf16", causal=False, sinks=True, seed=40)
+    cuts = [0, 13, 14, 70, 101]                                   # one chunk of a single key
+    parts = [oracle.attn(c.q, c.k[:, :, a:b], c.v[:, :, a:b], scale=c.scale, causal=False)
+             for a, b in zip(cuts, cuts[1:])]
+    o, lse = oracle.merge([p[0] for p in parts], [p[1] for p in parts])
+    ref_o = sdpa(c.q, c.k, c.v, scale=c.scale, gqa=True)
+    ref_lse = ref_lse_gqa(c.q, c.k, c.scale, False)
+    assert np.abs(o - ref_o).max() < TOL and np.abs(lse - ref_lse).max() < TOL
+    sink_rows = np.broadcast_to(oracle.widen(c.sinks)[None, :, None], lse.shape)
+    os_, ls_ = oracle.merge([p[0] for p in parts], [p[1] for p in parts], sink_rows=sink_rows)
+    so, sl = oracle.attn(c.q, c.k, c.v, scale=c.scale, causal=False, sinks=c.sinks)
+    assert np.abs(os_ - so).max() < TOL and np.abs(ls_ - sl).max() < TOL
+
+
+def test_merge_reassembles_causal_attention_from_sequence_chunks():
+    """The context-parallel split: with Q and K/V cut into n equal sequence chunks,
+    query chunk r merges its own chunk under the causal mask with every earlier
+    chunk unmasked; later chunks are invisible.  Equals causal SDPA over the whole
+    sequence."""
+    n, L = 4, 23
+    c = W.dense_case(1, 6, 3, n * L, n * L, 16, dtype="bf16", causal=True, seed=41)
+    ref_o = sdpa(c.q, c.k, c.v, scale=c.scale, causal_br=True, gqa=True)
+    ref_lse = ref_lse_gqa(c.q, c.k, c.scale, True)
+    for r in range(n):
+        q = c.q[:, :, r * L:(r + 1) * L]
+        parts = []
+        for s_ in range(r + 1):
+            k, v = c.k[:, :, s_ * L:(s_ + 1) * L], c.v[:, :, s_ * L:(s_ + 1) * L]
+            parts.append(oracle.attn(q, k, v, scale=c.scale, causal=(s_ == r)))
+        o, lse = oracle.merge([p[0] for p in parts], [p[1] for p in parts])
+        assert np.abs(o - ref_o[:, :, r * L:(r + 1) * L]).max() < TOL
+        assert np.abs(lse - ref_lse[:, :, r * L:(r + 1) * L]).max() < TOL
+
+
+def test_merge_special_cases():
+    rng = np.random.default_rng(42)
+    o1 = rng.standard_normal((5, 8))
+    l1 = rng.standard_normal(5)
+    o, lse = oracle.merge([o1], [l1])                             # one part: identity
+    assert np.abs(o - o1).max() < TOL and np.abs(lse - l1).max() < TOL
+    empty = np.full(5, -np.inf)
+    o, lse = oracle.merge([o1, rng.standard_normal((5, 8))], [l1, empty])   # an empty part adds nothing
+    assert np.abs(o - o1).max() < TOL and np.abs(lse - l1).max() < TOL
+    o, lse = oracle.merge([o1, o1], [empty, empty])               # nothing visible
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+    sink = rng.standard_normal(5)
+    o, lse = oracle.merge([o1], [empty], sink_rows=sink)          # only the sink: LSE = sink, O = 0
+    assert np.all(o == 0) and np.abs(lse - sink).max() < TOL
+    o, lse = oracle.merge([o1, 3 * o1], [l1, l1])                 # equal weights: the mean, LSE + ln 2
+    assert np.abs(o - 2 * o1).max() < TOL and np.abs(lse - (l1 + math.log(2))).max() < TOL
+
+
 # ------------------------------------------------------------------ mutations are caught
 
 def test_mutation_rep_major_is_caught(mutation):
@@ -376,3 +441,12 @@ def test_mutation_swapped_nibbles_is_caught(mutation):
     deq = oracle.dequant_cache(W.KV_Q4_0, enc, 8, 1, 64)
     step = np.abs(x.reshape(8, 1, 2, 32)).max(-1, keepdims=True) / 8.0
     assert not np.all(np.abs(deq.reshape(8, 1, 2, 32) - x.reshape(8, 1, 2, 32)) <= 1.01 * step)
+
+
+def test_mutation_unweighted_merge_is_caught(mutation):
+    c = W.dense_case(1, 4, 4, 20, 60, 16, dtype="bf16", causal=False, seed=43)
+    parts = [oracle.attn(c.q, c.k[:, :, a:b], c.v[:, :, a:b], scale=c.scale, causal=False)
+             for a, b in ((0, 10), (10, 60))]
+    mutation(oracle.MUT_MERGE_UNWEIGHTED)
+    o, _ = oracle.merge([p[0] for p in parts], [p[1] for p in parts])
+    assert np.abs(o - sdpa(c.q, c.k, c.v, scale=c.scale, gqa=True)).max() > 1e-2
