@@ -47,7 +47,18 @@ CONFIGS = {
                  metric="decode GB/s", dtype="q8_0"),
     "c5q4": dict(cfg=5, kv_type=W.KV_Q4_0, name="multi-seq decode, 4 seq x 4 tok, H=32 Hkv=8 D=128, 8192 cells/seq, q4_0",
                  metric="decode GB/s", dtype="q4_0"),
+    # the context-parallel output merge (not a configuration of the method's own benchmark):
+    # two bf16 partial outputs shaped like c2's, with sinks
+    "merge": dict(cfg=6, merge=dict(n_parts=2, B=1, H=64, T=1400, Dv=512), name="LSE output merge, 2 parts of "
+                  "B=1 H=64 T=1400 Dv=512 bf16, sinks", metric="merge GB/s", dtype="bf16"),
 }
+
+
+def make_case(spec):
+    if "merge" in spec:
+        return W.merge_case(**spec["merge"], seed=spec["cfg"])
+    kw = {"kv_type": spec["kv_type"]} if "kv_type" in spec else {}
+    return W.config(spec["cfg"], **kw)
 
 
 # ------------------------------------------------------------------ algorithmic work
@@ -73,6 +84,9 @@ def work(case):
         kv = case.k_cache.nbytes + case.v_cache.nbytes
         qo = case.q.nbytes * 2 + case.n_tok * case.H * 4
         return kv + qo, "byte"
+    if isinstance(case, W.MergeCase):
+        # every part's O and LSE read once, the merged O and LSE written once
+        return (len(case.o_parts) + 1) * (case.o_parts[0].nbytes + case.lse_parts[0].nbytes), "byte"
     raise TypeError(type(case))
 
 
@@ -141,6 +155,19 @@ def build_call(case, torch, arc, status):
             arc.attn_decode_q8(q, kc, vc, kv_type=case.kv_type, scale=case.scale, workspace=ws, out=o, lse=lse,
                                status=status, **kw)
         return call, {"q": q, "k_cache": kc, "v_cache": vc}, [o, lse], info
+    if isinstance(case, W.MergeCase):
+        parts = [U.to_dev(x) for x in case.o_parts]
+        lses = [U.to_dev(x) for x in case.lse_parts]
+        sinks = U.to_dev(case.sinks) if case.sinks is not None else None
+        o = torch.empty_like(parts[0])
+        lse = torch.empty_like(lses[0])
+        info = arc.plan_merge(parts, lses, o, lse)
+
+        def call():
+            arc.attn_merge(parts, lses, sinks=sinks, sink_rows=case.T, out=o, lse=lse)
+        ins = {f"o{i}": x for i, x in enumerate(parts)}
+        ins.update({f"lse{i}": x for i, x in enumerate(lses)})
+        return call, ins, [o, lse], info
     raise TypeError(type(case))
 
 
@@ -209,7 +236,7 @@ def kernel_source_hash(kernel):
              "tc_attn_pair_kernel<mla>": "attn_pair.cu",
              "tc_attn2_kernel": "attn_tc.cu", "tc_attn2_kernel<mla>": "attn_tc.cu",
              "sparse_tc_kernel": "sparse_tc.cu", "simple_attn_kernel<sparse>": "simple_kernels.cu",
-             "simple_attn_kernel": "simple_kernels.cu"}
+             "simple_attn_kernel": "simple_kernels.cu", "merge_kernel": "merge.cu"}
     f = files.get(kernel)
     if kernel.startswith("decode_split_kernel") or kernel.startswith("decode_ws_kernel"):
         f = "decode.cu"
@@ -271,6 +298,20 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
                 break
         return {"value": done_units / spent / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                 "sample": f"{n_rows} random query tokens x 64 heads x all top-k slots", "seconds": round(spent, 2)}
+    if isinstance(case, W.MergeCase):
+        rows_done, T = 0, case.T
+        row_bytes = work(case)[0] / T
+        while spent < budget_s[0]:
+            rows = np.sort(rng.choice(T, size=16, replace=False))
+            t0 = time.perf_counter()
+            oracle.run_case(case, rows=rows)
+            spent += time.perf_counter() - t0
+            rows_done += len(rows)
+            if spent > budget_s[1]:
+                break
+        return {"value": row_bytes * rows_done / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                "sample": f"{rows_done} random positions x all {case.B * case.H} (batch, head) rows",
+                "seconds": round(spent, 2)}
     if isinstance(case, W.DecodeCase):
         reps = 0
         units, _ = work(case)
@@ -385,7 +426,8 @@ def run_ours(args, spec, case):
         achieved = units / (mean_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
-                "note": "whole call (split kernel + combine) timed"}
+                "note": ("whole call (split kernel + combine) timed" if info["kernel"].startswith("decode")
+                         else "one merge_kernel launch")}
         e2e_val = units / (e2e_mean * 1e-3) / 1e9
     roof["traffic"] = recorded_traffic(args.config, info["kernel"])
     roof["kernel"] = info["kernel"]
@@ -430,6 +472,11 @@ def run_reference(args, spec, case):
             u = case.B * case.H * vis * (2 * Dqk + 2 * case.Dv)
             t0 = time.perf_counter()
             oracle.run_case(case, rows=rows)
+        elif isinstance(case, W.MergeCase):
+            rows = np.sort(rng.choice(case.T, size=4, replace=False))
+            u = work(case)[0] / case.T * len(rows)
+            t0 = time.perf_counter()
+            oracle.run_case(case, rows=rows)
         elif isinstance(case, W.SparseCase):
             rows = np.array([rng.integers(case.Sq)])
             valid = int(((case.idx[rows] >= 0) & (case.idx[rows] < case.Skv)).sum())
@@ -449,6 +496,7 @@ def run_reference(args, spec, case):
     unit = "TFLOP/s" if scale == 1e12 else "GB/s"
     value = sum(per_step_units) / total / scale
     sample = ("2 random query positions x all heads per step" if isinstance(case, (W.DenseCase, W.MlaCase))
+              else "4 random positions x all heads per step" if isinstance(case, W.MergeCase)
               else "1 random query token x all heads x all slots per step" if isinstance(case, W.SparseCase)
               else "the whole decode step per step")
     line = {"impl": "reference", "metric": spec["metric"], "value": value, "unit": unit, "n_gpus": world,
@@ -474,8 +522,7 @@ def main():
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     spec = CONFIGS[args.config]
-    kw = {"kv_type": spec["kv_type"]} if "kv_type" in spec else {}
-    case = W.config(spec["cfg"], **kw)
+    case = make_case(spec)
     if args.impl == "reference":
         run_reference(args, spec, case)
     else:

@@ -240,7 +240,7 @@ def dequant_cache(kv_type, cache, n_cells, Hkv, D):
 # ------------------------------------------------------------------ whole cases
 
 def run_case(case, rows=None):
-    """Evaluate a workloads case (Dense/Mla/Sparse/Decode).  rows selects query rows."""
+    """Evaluate a workloads case (Dense/Mla/Sparse/Decode/Merge).  rows selects query rows."""
     import workloads as W
     if isinstance(case, W.DenseCase):
         return attn(case.q, case.k, case.v, scale=case.scale, causal=case.causal,
@@ -256,6 +256,13 @@ def run_case(case, rows=None):
                       v=case.v)
     if isinstance(case, W.DecodeCase):
         return decode_q(case)
+    if isinstance(case, W.MergeCase):
+        sl = slice(None) if rows is None else np.asarray(rows)
+        parts = [x[:, :, sl] for x in case.o_parts]
+        lses = [x[:, :, sl] for x in case.lse_parts]
+        sr = None if case.sinks is None else np.broadcast_to(case.sinks.astype(np.float64)[None, :, None],
+                                                              lses[0].shape)
+        return merge(parts, lses, sink_rows=sr)
     raise TypeError(type(case))
 
 

@@ -355,7 +355,8 @@ def test_invalid_arguments_launch_nothing():
 # ------------------------------------------------------------------ merge over disjoint key sets
 
 @pytest.mark.parametrize("n_parts,dv,dtype,sinks", [(1, 64, "f32", False), (3, 128, "f32", True),
-                                                     (5, 512, "bf16", True), (2, 256, "bf16", False)])
+                                                     (5, 512, "bf16", True), (2, 256, "bf16", False),
+                                                     (2, 94, "bf16", True)])   # dv % 8 != 0: 2-element path
 def test_merge_matches_oracle(n_parts, dv, dtype, sinks):
     rng = np.random.default_rng(50 + n_parts)
     B, H, T = 2, 6, 97

@@ -275,6 +275,33 @@ def decode_case(n_seq=4, n_q=4, n_kv=8192, H=32, Hkv=8, D=128, *, kv_type=KV_Q8_
                       enc(k), enc(v), qb, nq, kb, nkv, seed)
 
 
+@dataclass
+class MergeCase:
+    """Partial results over disjoint key sets, to be merged (context-parallel output merge)."""
+    B: int
+    H: int
+    T: int
+    Dv: int
+    o_parts: list           # n_parts x [B,H,T,Dv] bf16 bits
+    lse_parts: list         # n_parts x [B,H,T] fp32, natural log; -inf marks an empty part
+    sinks: np.ndarray | None = None   # [H] fp32
+    seed: int = 0
+
+
+def merge_case(n_parts=2, B=1, H=64, T=1400, Dv=512, *, sinks=True, empty_frac=0.02, seed=6) -> MergeCase:
+    """Seeded parts shaped like an attention output: O ~ 0.5*N(0,1) in bf16, LSE ~ 3 + N(0,1),
+    a few rows empty in each part."""
+    rng = make_rng(seed)
+    o = [bf16_bits(normal(rng, (B, H, T, Dv), 0.5)) for _ in range(n_parts)]
+    lse = []
+    for _ in range(n_parts):
+        l = (3.0 + normal(rng, (B, H, T), 1.0)).astype(np.float32)
+        l[rng.random((B, H, T)) < empty_frac] = -np.inf
+        lse.append(l)
+    s = normal(rng, (H,), 1.0).astype(np.float32) if sinks else None
+    return MergeCase(B, H, T, Dv, o, lse, s, seed)
+
+
 # The five workload configurations, by number, with seed = number.
 def config(i: int, **over):
     if i == 1:
