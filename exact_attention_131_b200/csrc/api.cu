@@ -18,6 +18,7 @@ using namespace arc;
 
 namespace arc {
 int decode_smem_bytes(int kv_type, int D, bool tma);
+int decode_blocks_per_sm(int kv_type, int D, bool tma);
 int decode_box_bytes(int kv_type, int D);
 }
 
@@ -399,8 +400,13 @@ DecodePlan plan_decode(const arc_decode_args *a)
     const int pairs = a->n_seq * a->Hkv;
     const int64_t cell_bytes = (int64_t)a->Hkv * (a->D / 32) * (a->kv_type == ARC_KV_Q8_0 ? 34 : 18);
     pl.tma = cell_bytes % 16 == 0;
+    // One wave: as many CTAs as the SMs hold at once.  The occupancy API counts
+    // registers as well as shared memory (the warp-specialised kernel is register-
+    // limited to 3 CTAs per SM even where its stages would leave room for a fourth);
+    // without a device, the shared-memory estimate.
     const int smem = decode_smem_bytes(a->kv_type, a->D, pl.tma);
-    const int per_sm = std::max(1, std::min(4, (228 * 1024) / (smem + 1024)));
+    const int occ = decode_blocks_per_sm(a->kv_type, a->D, pl.tma);
+    const int per_sm = occ > 0 ? std::min(4, occ) : std::max(1, std::min(4, (228 * 1024) / (smem + 1024)));
     const int target = sm_count() * per_sm;
     int splits = std::min(256, std::max(1, target / std::max(1, pairs)));
     int chunk = (pl.max_kv + splits - 1) / splits;

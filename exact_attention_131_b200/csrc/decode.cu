@@ -950,6 +950,36 @@ cudaError_t launch_k(const DecodeParams &p, cudaStream_t s)
 
 int decode_smem_bytes(int kv_type, int D, bool tma) { return tma ? smem_t<true>(kv_type, D) : smem_t<false>(kv_type, D); }
 
+// CTAs of the split kernel that fit on one SM at once (registers, threads and
+// shared memory together), from the occupancy API; 0 if it cannot be asked (no device).
+int decode_blocks_per_sm(int kv_type, int D, bool tma)
+{
+    int n = 0;
+    const int smem = decode_smem_bytes(kv_type, D, tma);
+    auto ask = [&](auto kern, int threads) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+    };
+    const bool q8 = kv_type == ARC_KV_Q8_0;
+    if (tma) {
+        if (q8)
+            D == 64 ? ask(decode_ws_kernel<ARC_KV_Q8_0, 64>, WS_WARPS * 32) : ask(decode_ws_kernel<ARC_KV_Q8_0, 128>, WS_WARPS * 32);
+        else
+            D == 64 ? ask(decode_ws_kernel<ARC_KV_Q4_0, 64>, WS_WARPS * 32) : ask(decode_ws_kernel<ARC_KV_Q4_0, 128>, WS_WARPS * 32);
+    } else {
+        if (q8)
+            D == 64 ? ask(decode_split_kernel<ARC_KV_Q8_0, 64, false>, WARPS * 32)
+                    : ask(decode_split_kernel<ARC_KV_Q8_0, 128, false>, WARPS * 32);
+        else
+            D == 64 ? ask(decode_split_kernel<ARC_KV_Q4_0, 64, false>, WARPS * 32)
+                    : ask(decode_split_kernel<ARC_KV_Q4_0, 128, false>, WARPS * 32);
+    }
+    return n;
+}
+
 // Box width in bytes of the TMA path (covers a head row from the 16-byte boundary below it).
 int decode_box_bytes(int kv_type, int D)
 {
