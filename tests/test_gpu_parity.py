@@ -407,3 +407,32 @@ def test_context_parallel_chunks_merge_to_attention_over_the_whole_sequence(worl
     ro, rl = oracle.attn(c.q, c.k, c.v, scale=c.scale, causal=True, sinks=c.sinks if sinks else None)
     for r, (o, lse) in enumerate(outs):
         compare(o, lse, ro[:, :, r * L:(r + 1) * L], rl[:, :, r * L:(r + 1) * L], TOL_O_BF16)
+
+
+@pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
+def test_single_stream_decode_one_token_long_context(kv_type):
+    """One sequence, one new token (t_q = 1), a long cache: few (sequence, kv head)
+    pairs, so many splits and the two-kernel merge."""
+    c = W.decode_case(1, 1, 40000, 32, 4, 128, kv_type=kv_type, seed=59)
+    st = status_word()
+    o, lse, (q, kc, vc) = run_decode(c, status=st)
+    info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                           n_kv=c.n_kv)
+    assert info["kernel"].startswith("decode_ws_kernel") and info["splits"] > 16 and info["launches"] == 2
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
+def test_merge_sixteen_parts_and_empty_call():
+    rng = np.random.default_rng(61)
+    o_np = [rng.standard_normal((33, 64)).astype(np.float32) for _ in range(16)]
+    l_np = [rng.standard_normal(33).astype(np.float32) for _ in range(16)]
+    o, lse = arc.attn_merge([torch.from_numpy(x).cuda() for x in o_np], [torch.from_numpy(x).cuda() for x in l_np])
+    torch.cuda.synchronize()
+    ro, rl = oracle.merge(o_np, l_np)
+    compare(o, lse, ro, rl, TOL_O_F32)
+    e = [torch.empty(0, 64, device="cuda")] * 2
+    el = [torch.empty(0, device="cuda")] * 2
+    o0, l0 = arc.attn_merge(e, el)                      # zero rows: nothing launched, nothing written
+    assert o0.shape == (0, 64) and l0.shape == (0,)
