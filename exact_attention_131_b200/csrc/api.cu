@@ -697,7 +697,7 @@ arc_status arc_attn_decode_q8_noalloc(const arc_decode_args *a, void *stream)
     return arc_attn_decode_q8(a, scratch, ARC_DECODE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-arc_status arc_attn_merge(const arc_merge_args *a, void *stream)
+static arc_status check_merge(const arc_merge_args *a)
 {
     if (!a) return ARC_ERR_INVALID_ARG;
     if (a->n_parts < 1 || a->n_parts > ARC_MERGE_MAX_PARTS || a->rows < 0 || a->dv <= 0 || (a->dv & 1))
@@ -711,6 +711,13 @@ arc_status arc_attn_merge(const arc_merge_args *a, void *stream)
     for (int i = 0; i < a->n_parts; ++i)
         if (bad(a->o_parts[i]) || !a->lse_parts[i] || (reinterpret_cast<uintptr_t>(a->lse_parts[i]) & 3u))
             return ARC_ERR_INVALID_ARG;
+    return ARC_OK;
+}
+
+arc_status arc_attn_merge(const arc_merge_args *a, void *stream)
+{
+    const arc_status st = check_merge(a);
+    if (st != ARC_OK || a->rows == 0) return st;
     MergeParams p{};
     p.n_parts = a->n_parts, p.rows = a->rows, p.dv = a->dv, p.dtype = a->dtype;
     for (int i = 0; i < a->n_parts; ++i) p.o_parts[i] = a->o_parts[i], p.lse_parts[i] = a->lse_parts[i];
@@ -777,8 +784,8 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
     }
     if (op == ARC_OP_MERGE) {
         const arc_merge_args *a = static_cast<const arc_merge_args *>(args);
-        if (a->n_parts < 1 || a->n_parts > ARC_MERGE_MAX_PARTS || a->rows < 0 || a->dv <= 0 || (a->dv & 1))
-            return ARC_ERR_INVALID_ARG;
+        arc_status st = check_merge(a);
+        if (st != ARC_OK) return st;
         set_name(out, "merge_kernel");
         out->n_ctas = (a->rows + 7) / 8;
         out->launches = a->rows > 0 ? 1 : 0;

@@ -121,7 +121,13 @@ arc_status arc_attn_fwd(const arc_attn_args *args, void *stream);
  *   v      [B,H,Tk,Dv]  bf16, device
  *   o      [B,H,Tq,Dv]  bf16, device, written
  *   lse    [B,H,Tq]     fp32, device, contiguous, written
- * Dn, Dr multiples of 64 with Dn + Dr <= 256; Dv in {64,128,256}.
+ * Dn, Dr multiples of 64 with Dn + Dr <= 256; Dv in {64,128,256}; 16-byte
+ * aligned base pointers and strides, and each head's query rows evenly spaced
+ * (head stride == Tq * token stride).  Other shapes or layouts return
+ * ARC_ERR_UNSUPPORTED unless ARC_FLAG_FORCE_SIMPLE is set, which runs the
+ * CUDA-core kernel for any Dn + Dr <= 512, Dv <= 512.  Dn + Dr or Dv above 512
+ * is ARC_ERR_UNSUPPORTED; negative sizes or a NULL tensor that the call reads
+ * are ARC_ERR_INVALID_ARG.  B == 0 or Tq == 0 launches nothing.
  * ------------------------------------------------------------------------ */
 typedef struct {
     int32_t B, H, Tq, Tk, Dn, Dr, Dv;
@@ -157,7 +163,13 @@ arc_status arc_mla_fwd(const arc_mla_args *args, void *stream);
  *   o    [Sq,H,Dv]    bf16, device, strides o_strides = {token, head}, written
  *   lse  [Sq,H]       fp32, device, contiguous, written
  *   sinks [H]         fp32, device, or NULL
- * Dqk in {64,128,256,512}, Dv <= Dqk a multiple of 64.
+ * Dqk in {64,128,256,512}, Dv <= Dqk a multiple of 64.  The tensor-core
+ * kernel takes (Dqk, Dv) = (512, 512), (512, 256), (256, 256), (128, 128) with
+ * V inside the kv row, and (128, 64), (128, 128), (256, 256) with a separate v,
+ * on 16-byte aligned base pointers and strides; every other supported call runs
+ * the CUDA-core kernel (arc_plan names which).  Dqk or Dv above 512 is
+ * ARC_ERR_UNSUPPORTED; negative sizes, Dv > Dqk without v, or a NULL tensor
+ * that the call reads are ARC_ERR_INVALID_ARG.  Sq == 0 launches nothing.
  * ------------------------------------------------------------------------ */
 typedef struct {
     int32_t Sq, H, Skv, Dqk, Dv, topk;
@@ -204,6 +216,12 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *args, void *stream);
  * aligned; used for the split-KV partial results and overwritten.  Its
  * contents need no initialisation (every byte read is first written by the
  * same call).  Two calls in flight at once need two workspaces.
+ * Errors, all returned before anything is launched: D outside {64,128}, n_seq
+ * above ARC_DECODE_MAX_SEQ or (H/Hkv) * n_q above 16 is ARC_ERR_UNSUPPORTED; an
+ * unknown kv_type, negative sizes, H % Hkv != 0, n_kv < n_q, a sequence whose
+ * tokens or cells run past n_tok / n_cells, a NULL tensor, or q, o or a cache
+ * not 8-byte aligned is ARC_ERR_INVALID_ARG; a missing, short or unaligned
+ * workspace is ARC_ERR_WORKSPACE.  n_seq == 0 or n_tok == 0 launches nothing.
  * ------------------------------------------------------------------------ */
 #define ARC_DECODE_MAX_SEQ 64
 
