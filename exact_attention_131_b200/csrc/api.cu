@@ -372,7 +372,7 @@ arc_status check_decode(const arc_decode_args *a, bool need_ptrs = true)
     if (a->n_tok < 0 || a->H <= 0 || a->Hkv <= 0 || a->H % a->Hkv || a->n_cells < 0 || a->n_seq < 0)
         return ARC_ERR_INVALID_ARG;
     if (a->n_seq > ARC_DECODE_MAX_SEQ) return ARC_ERR_UNSUPPORTED;
-    if (!in_set(a->D, {64, 128})) return ARC_ERR_UNSUPPORTED;
+    if (!in_set(a->D, {64, 128, 256, 512})) return ARC_ERR_UNSUPPORTED;
     if (a->n_seq > 0 && !a->seqs) return ARC_ERR_INVALID_ARG;
     const int G = a->H / a->Hkv;
     for (int s = 0; s < a->n_seq; ++s) {
@@ -394,7 +394,9 @@ arc_status check_decode(const arc_decode_args *a, bool need_ptrs = true)
 DecodePlan plan_decode(const arc_decode_args *a)
 {
     DecodePlan pl;
-    pl.simple = (a->flags & ARC_FLAG_FORCE_SIMPLE) != 0;
+    // head dims 256 / 512 run on the CUDA-core kernel: the register-direct split
+    // kernel holds a 16-row x D fp32 accumulator and one head row per TMA box only up to D = 128
+    pl.simple = (a->flags & ARC_FLAG_FORCE_SIMPLE) != 0 || a->D > 128;
     for (int s = 0; s < a->n_seq; ++s) pl.max_kv = std::max(pl.max_kv, a->seqs[s].n_kv);
     if (pl.simple || pl.max_kv == 0) return pl;
     const int pairs = a->n_seq * a->Hkv;

@@ -210,18 +210,22 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *args, void *stream);
  *   o        [n_tok,H,D]            fp32, device, written (rows of tokens that no
  *            sequence owns are left untouched)
  *   lse      [n_tok,H]              fp32, device, written likewise
- * D in {64,128}; H % Hkv == 0; (H/Hkv) * n_q <= 16 for every sequence;
- * n_seq <= ARC_DECODE_MAX_SEQ.
+ * D in {64,128,256,512}; H % Hkv == 0; (H/Hkv) * n_q <= 16 for every
+ * sequence; n_seq <= ARC_DECODE_MAX_SEQ.  D 64 and 128 run the split-KV tensor-
+ * core kernel and its combine (two launches); D 256 and 512 run the CUDA-core
+ * kernel (one warp per query row over all its cells, one launch, no workspace:
+ * arc_decode_workspace_size() returns 0), as does ARC_FLAG_FORCE_SIMPLE.
  * workspace: device, at least arc_decode_workspace_size(args) bytes, 256-byte
  * aligned; used for the split-KV partial results and overwritten.  Its
  * contents need no initialisation (every byte read is first written by the
  * same call).  Two calls in flight at once need two workspaces.
- * Errors, all returned before anything is launched: D outside {64,128}, n_seq
- * above ARC_DECODE_MAX_SEQ or (H/Hkv) * n_q above 16 is ARC_ERR_UNSUPPORTED; an
- * unknown kv_type, negative sizes, H % Hkv != 0, n_kv < n_q, a sequence whose
- * tokens or cells run past n_tok / n_cells, a NULL tensor, or q, o or a cache
- * not 8-byte aligned is ARC_ERR_INVALID_ARG; a missing, short or unaligned
- * workspace is ARC_ERR_WORKSPACE.  n_seq == 0 or n_tok == 0 launches nothing.
+ * Errors, all returned before anything is launched: D outside {64,128,256,512},
+ * n_seq above ARC_DECODE_MAX_SEQ or (H/Hkv) * n_q above 16 is
+ * ARC_ERR_UNSUPPORTED; an unknown kv_type, negative sizes, H % Hkv != 0,
+ * n_kv < n_q, a sequence whose tokens or cells run past n_tok / n_cells, a NULL
+ * tensor, or q, o or a cache not 8-byte aligned is ARC_ERR_INVALID_ARG; a
+ * missing, short or unaligned workspace (where one is needed) is
+ * ARC_ERR_WORKSPACE.  n_seq == 0 or n_tok == 0 launches nothing.
  * ------------------------------------------------------------------------ */
 #define ARC_DECODE_MAX_SEQ 64
 

@@ -318,6 +318,21 @@ def test_decode_head_dim_64_and_control_arm():
     compare(o2, lse2, ro, rl, TOL_O_BF16)
 
 
+@pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
+@pytest.mark.parametrize("D", [256, 512])
+def test_decode_wide_head_dims(kv_type, D):
+    """Head dims 256 / 512 (the CUDA-core decode kernel): ragged sequences, GQA 4."""
+    c = W.decode_case(3, 0, 0, 8, 2, D, kv_type=kv_type, seed=62, n_q_list=[2, 1, 4], n_kv_list=[700, 1, 130])
+    st = status_word()
+    o, lse, (q, kc, vc) = run_decode(c, status=st)
+    info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                           n_kv=c.n_kv)
+    assert info["kernel"] == "simple_decode_kernel"
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
 # ------------------------------------------------------------------ edge cases and failure reporting
 
 def test_empty_and_degenerate_shapes():

@@ -323,8 +323,9 @@ def test_quant_roundtrip_within_half_step(kv_type):
 
 
 @pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
-def test_decode_matches_torch_per_sequence(kv_type):
-    c = W.decode_case(3, 4, 0, 8, 2, 64, kv_type=kv_type, seed=22, n_q_list=[4, 1, 3],
+@pytest.mark.parametrize("D", [64, 512])
+def test_decode_matches_torch_per_sequence(kv_type, D):
+    c = W.decode_case(3, 4, 0, 8, 2, D, kv_type=kv_type, seed=22, n_q_list=[4, 1, 3],
                       n_kv_list=[40, 17, 3])
     o, lse = oracle.decode_q(c)
     K = oracle.dequant_cache(kv_type, c.k_cache, c.n_cells, c.Hkv, c.D)

@@ -185,6 +185,14 @@ def test_decode_single_stream_and_empty_caches(arc):
     assert arc.plan(arc.ARC_OP_DECODE, d)["kernel"] == "simple_decode_kernel"
 
 
+@pytest.mark.parametrize("D", [256, 512])
+def test_decode_wide_heads_run_the_cuda_core_kernel_without_workspace(arc, D):
+    d = decode_args(arc, arc.ARC_KV_Q4_0, D=D)
+    info = arc.plan(arc.ARC_OP_DECODE, d)
+    assert info["kernel"] == "simple_decode_kernel" and info["launches"] == 1 and info["tensor_cores"] == 0
+    assert arc.lib().arc_decode_workspace_size(ctypes.byref(d)) == 0
+
+
 def test_decode_workspace_errors_come_before_any_launch(arc):
     L = arc.lib()
     d = decode_args(arc, arc.ARC_KV_Q8_0)
@@ -195,15 +203,15 @@ def test_decode_workspace_errors_come_before_any_launch(arc):
 
 
 @pytest.mark.parametrize("change,want", [
-    ("D=256", "ARC_ERR_UNSUPPORTED"), ("H%Hkv", "ARC_ERR_INVALID_ARG"), ("q misaligned", "ARC_ERR_INVALID_ARG"),
+    ("D=384", "ARC_ERR_UNSUPPORTED"), ("H%Hkv", "ARC_ERR_INVALID_ARG"), ("q misaligned", "ARC_ERR_INVALID_ARG"),
     ("cache misaligned", "ARC_ERR_INVALID_ARG"), ("tokens past n_tok", "ARC_ERR_INVALID_ARG"),
     ("cells past n_cells", "ARC_ERR_INVALID_ARG"), ("lse NULL", "ARC_ERR_INVALID_ARG"),
     ("negative kv_begin", "ARC_ERR_INVALID_ARG"),
 ])
 def test_decode_validation(arc, change, want):
     d = decode_args(arc, arc.ARC_KV_Q4_0, n_seq=2, n_q=2, n_kv=256)
-    if change == "D=256":
-        d.D = 256
+    if change == "D=384":
+        d.D = 384
     elif change == "H%Hkv":
         d.Hkv = 6
     elif change == "q misaligned":
