@@ -5,10 +5,11 @@ Only tests/, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 shares no code with it; the only thing both sides read is the seeded inputs
 from ``workloads``.
 
-The arithmetic lives in ``arc_oracle.c`` (plain loops, double precision,
-OpenMP over independent rows).  This module builds it with gcc, widens the
+The forward arithmetic lives in ``arc_oracle.c`` (plain loops, double precision,
+OpenMP over independent rows); the backward (``backward.py``) is numpy fp64, the
+derivative of the same definition.  This module builds it with gcc, widens the
 stored inputs exactly to float64 (bf16 bits -> fp32 -> fp64, fp32 -> fp64) and
-marshals arguments.  Every function returns ``(o, lse)`` as float64 arrays.
+marshals arguments.  Every forward function returns ``(o, lse)`` as float64 arrays.
 
 Pins: see tests/test_oracle_pins.py.  Every function here is pinned there
 against something other than itself (torch's fp64 SDPA, closed forms,
@@ -284,3 +285,6 @@ def merge(o_parts, lse_parts, *, sink_rows=None):
                               _ptr(o, _dp), _ptr(lse, _dp))
     _check(rc, "merge")
     return o.reshape(shape), lse.reshape(shape[:-1])
+
+
+from .backward import MUT_BWD_DROP_DELTA, attn_bwd, mla_bwd, sparse_bwd  # noqa: E402
