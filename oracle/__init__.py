@@ -11,8 +11,9 @@ derivative of the same definition.  This module builds it with gcc, widens the
 stored inputs exactly to float64 (bf16 bits -> fp32 -> fp64, fp32 -> fp64) and
 marshals arguments.  Every forward function returns ``(o, lse)`` as float64 arrays.
 
-Pins: see tests/test_oracle_pins.py.  Every function here is pinned there
-against something other than itself (torch's fp64 SDPA, closed forms,
+Pins: tests/test_oracle_pins.py (forward) and tests/test_oracle_backward_pins.py
+(backward).  Every function here is pinned there against something other than
+itself (torch's fp64 SDPA or autograd, finite differences, closed forms,
 invariants the pages state); none is "parity unpinned".
 """
 from __future__ import annotations
