@@ -196,15 +196,18 @@ def sparse_indices(rng, Sq, Skv, topk, pad_frac=0.05, pad_mode="random") -> np.n
     idx = np.empty((Sq, topk), dtype=np.int32)
     draw = min(Skv, max(topk + 64, int(topk * 1.25)))
     for i in range(Sq):
-        while True:
-            if topk > Skv // 2:
-                row = rng.permutation(Skv)[:topk]
-                break
-            cand = rng.integers(0, Skv, size=draw)
-            _, first = np.unique(cand, return_index=True)
-            if first.size >= topk:
-                row = cand[np.sort(first)][:topk]
-                break
+        row = None
+        if topk <= Skv // 2:
+            # rejection draws; when topk is near Skv / 2 a draw can keep falling short
+            # of topk distinct values, so after a bounded number of tries take a permutation
+            for _ in range(64):
+                cand = rng.integers(0, Skv, size=draw)
+                _, first = np.unique(cand, return_index=True)
+                if first.size >= topk:
+                    row = cand[np.sort(first)][:topk]
+                    break
+        if row is None:
+            row = rng.permutation(Skv)[:topk]
         idx[i] = row
     n_pad = int(round(pad_frac * topk))
     if n_pad > 0:
