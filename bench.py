@@ -429,6 +429,8 @@ def run_ours(args, spec, case):
                 "note": ("whole call (split kernel + combine) timed" if info["kernel"].startswith("decode")
                          else "one merge_kernel launch")}
         e2e_val = units / (e2e_mean * 1e-3) / 1e9
+    if not e2e_ms:                      # --no-e2e: no host-buffer leg; JSON null rather than NaN
+        e2e_val = e2e_mean = None
     roof["traffic"] = recorded_traffic(args.config, info["kernel"])
     roof["kernel"] = info["kernel"]
 
