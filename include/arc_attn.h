@@ -85,7 +85,7 @@ typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE
  * each (b, kv) group of g*Tq query rows evenly spaced (head stride ==
  * Tq * token stride), 16-byte aligned rows and base pointers; otherwise the
  * call returns ARC_ERR_UNSUPPORTED unless ARC_FLAG_FORCE_SIMPLE is set.
- * dtype F32 ("reference mode"): any D, Dv <= 512, a multiple of 32 up to 512;
+ * dtype F32 ("reference mode"): any D and Dv from 1 to 512, any strides;
  * CUDA-core fp32 arithmetic, no TF32.
  * ------------------------------------------------------------------------ */
 typedef struct {
