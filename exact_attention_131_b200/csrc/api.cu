@@ -28,6 +28,11 @@ constexpr int kTcBM = 128, kTcBN = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A zero stride over an extent above one: a broadcast view of an input (legal for the
+// CUDA-core kernels, which index it as given; a TMA tensor map cannot describe it), or
+// output rows that would alias one another (refused everywhere).
+bool broadcast(int64_t stride, int64_t extent) { return stride == 0 && extent > 1; }
 bool in_set(int x, std::initializer_list<int> s) { return std::find(s.begin(), s.end(), x) != s.end(); }
 
 int sm_count()
@@ -187,6 +192,8 @@ arc_status check_attn(const arc_attn_args *a)
     for (int i = 0; i < 3; ++i)
         if (a->q_strides[i] < 0 || a->k_strides[i] < 0 || a->v_strides[i] < 0 || a->o_strides[i] < 0)
             return ARC_ERR_INVALID_ARG;
+    if (broadcast(a->o_strides[0], a->B) || broadcast(a->o_strides[1], a->H) || broadcast(a->o_strides[2], a->Tq))
+        return ARC_ERR_INVALID_ARG;
     return ARC_OK;
 }
 
@@ -238,6 +245,9 @@ AttnPlan plan_attn(const arc_attn_args *a)
     if (a->Dv % pl.dvs || !tc_pair_supported(a->D, pl.dvs, false)) return pl;
     // the fold view needs the g*Tq rows of a kv group evenly spaced
     if (a->q_strides[1] != (int64_t)a->Tq * a->q_strides[2] && a->H > 1) return pl;
+    if (broadcast(a->q_strides[0], a->B) || broadcast(a->k_strides[0], a->B) || broadcast(a->v_strides[0], a->B) ||
+        broadcast(a->k_strides[1], a->Hkv) || broadcast(a->v_strides[1], a->Hkv))
+        return pl;
     if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o)) return pl;
     if (!tma_strides_ok({a->q_strides[2], a->q_strides[0] ? a->q_strides[0] : 8, a->k_strides[2],
                          a->k_strides[1] ? a->k_strides[1] : 8, a->k_strides[0] ? a->k_strides[0] : 8,
@@ -285,6 +295,8 @@ arc_status check_mla(const arc_mla_args *a)
     if (a->B == 0 || a->Tq == 0) return ARC_OK;
     if (!a->q_nope || (a->Dr > 0 && !a->q_rope) || !a->o || !a->lse) return ARC_ERR_INVALID_ARG;
     if (a->Tk > 0 && (!a->k_nope || (a->Dr > 0 && !a->k_rope) || !a->v)) return ARC_ERR_INVALID_ARG;
+    if (broadcast(a->o_strides[0], a->B) || broadcast(a->o_strides[1], a->H) || broadcast(a->o_strides[2], a->Tq))
+        return ARC_ERR_INVALID_ARG;
     return ARC_OK;
 }
 
@@ -300,6 +312,10 @@ AttnPlan plan_mla(const arc_mla_args *a)
     if (a->Dn % 64 || a->Dr % 64 || a->Dr == 0 || a->Dv > 256 || !tc_pair_supported(dqk, a->Dv, true)) return pl;
     if (a->q_nope_strides[1] != (int64_t)a->Tq * a->q_nope_strides[2] && a->H > 1) return pl;
     if (a->q_rope_strides[1] != (int64_t)a->Tq * a->q_rope_strides[2] && a->H > 1) return pl;
+    if (broadcast(a->q_nope_strides[0], a->B) || broadcast(a->q_rope_strides[0], a->B) ||
+        broadcast(a->k_nope_strides[0], a->B) || broadcast(a->k_nope_strides[1], a->H) ||
+        broadcast(a->k_rope_strides[0], a->B) || broadcast(a->v_strides[0], a->B) || broadcast(a->v_strides[1], a->H))
+        return pl;
     if (!aligned16(a->q_nope) || !aligned16(a->q_rope) || !aligned16(a->k_nope) || !aligned16(a->k_rope) ||
         !aligned16(a->v) || !aligned16(a->o))
         return pl;
@@ -339,6 +355,7 @@ arc_status check_sparse(const arc_sparse_args *a)
     if (!a->v && a->Dv > a->Dqk) return ARC_ERR_INVALID_ARG;
     if (a->Sq == 0) return ARC_OK;
     if (!a->q || !a->o || !a->lse || (a->topk > 0 && (!a->idx || !a->kv))) return ARC_ERR_INVALID_ARG;
+    if (broadcast(a->o_strides[0], a->Sq) || broadcast(a->o_strides[1], a->H)) return ARC_ERR_INVALID_ARG;
     return ARC_OK;
 }
 

@@ -18,7 +18,12 @@
  *     state; a call only reads its inputs and writes its outputs (and, for
  *     decode, the caller's workspace).
  *   - Strides are in ELEMENTS, int64.  The last dimension of every tensor is
- *     contiguous (stride 1).
+ *     contiguous (stride 1).  A zero stride over a dimension of extent above 1
+ *     (a broadcast view) is accepted for inputs by the CUDA-core kernels, which
+ *     index it as given: the tensor-core attn / MLA paths cannot describe it in
+ *     a TMA map and return ARC_ERR_UNSUPPORTED for it unless
+ *     ARC_FLAG_FORCE_SIMPLE is set (the sparse gather reads it as given).  An
+ *     output with such a stride (rows that alias) is ARC_ERR_INVALID_ARG.
  *   - `stream` is a cudaStream_t passed as void*.  NULL is the legacy default
  *     stream and is a valid stream.  Launches are asynchronous on it.
  *   - Arguments are validated on the host before anything is launched.  On

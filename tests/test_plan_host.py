@@ -243,3 +243,56 @@ def test_dense_simple_fallback_and_unsupported_layouts(arc):
     a.flags = arc.ARC_FLAG_FORCE_SIMPLE
     info = arc.plan(arc.ARC_OP_ATTN, a)
     assert info["kernel"] == "simple_attn_kernel" and info["n_ctas"] == (4 * 64 + 3) // 4
+
+
+# ----------------------------------------------------------------------- broadcast strides
+def dense_args(arc, B=2, H=4, Hkv=2, T=64, D=64):
+    a = arc.AttnArgs()
+    a.dtype, a.B, a.H, a.Hkv, a.Tq, a.Tk, a.D, a.Dv = arc.ARC_DTYPE_BF16, B, H, Hkv, T, T, D, D
+    a.q, a.k, a.v, a.o, a.lse = (FAKE,) * 5
+    for name, shape in (("q", (B, H, T, D)), ("k", (B, Hkv, T, D)), ("v", (B, Hkv, T, D)), ("o", (B, H, T, D))):
+        setattr(a, name + "_strides", (arc._i64 * 3)(*contiguous(*shape)))
+    return a
+
+
+@pytest.mark.parametrize("name,dim", [("k", 0), ("v", 0), ("q", 0), ("k", 1), ("v", 1)])
+def test_broadcast_inputs_are_refused_by_the_tma_path(arc, name, dim):
+    """A zero stride over an extent above one cannot be a TMA map stride; it must not be
+    replaced by the contiguous default (that map would run past the allocation)."""
+    a = dense_args(arc)
+    assert arc.plan(arc.ARC_OP_ATTN, a)["tensor_cores"] == 1
+    getattr(a, name + "_strides")[dim] = 0
+    assert arc.lib().arc_attn_fwd(ctypes.byref(a), None) == arc.ARC_ERR_UNSUPPORTED
+    a.flags = arc.ARC_FLAG_FORCE_SIMPLE
+    assert arc.plan(arc.ARC_OP_ATTN, a)["kernel"] == "simple_attn_kernel"
+
+
+def test_zero_strides_over_extent_one_still_take_the_tma_path(arc):
+    a = dense_args(arc, B=1, Hkv=1)
+    a.q_strides[0] = a.k_strides[0] = a.v_strides[0] = a.k_strides[1] = a.v_strides[1] = 0
+    assert arc.plan(arc.ARC_OP_ATTN, a)["tensor_cores"] == 1
+
+
+@pytest.mark.parametrize("dim", [0, 1, 2])
+def test_aliasing_output_rows_are_invalid(arc, dim):
+    a = dense_args(arc)
+    a.o_strides[dim] = 0
+    assert arc.lib().arc_attn_fwd(ctypes.byref(a), None) == arc.ARC_ERR_INVALID_ARG
+    m = mla_args(arc, Tq=256, Tk=256)
+    m.o_strides[dim] = 0
+    assert arc.lib().arc_mla_fwd(ctypes.byref(m), None) == arc.ARC_ERR_INVALID_ARG
+    if dim < 2:
+        s = sparse_args(arc, Sq=4, topk=64)
+        s.o_strides[dim] = 0
+        assert arc.lib().arc_sparse_mla_fwd(ctypes.byref(s), None) == arc.ARC_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field,dim", [("k_rope_strides", 0), ("k_nope_strides", 1), ("v_strides", 0),
+                                       ("q_rope_strides", 0)])
+def test_mla_broadcast_inputs_are_refused_by_the_tma_path(arc, field, dim):
+    m = mla_args(arc, Tq=256, Tk=256)
+    getattr(m, field)[dim] = 0
+    assert arc.lib().arc_mla_fwd(ctypes.byref(m), None) == arc.ARC_ERR_UNSUPPORTED
+    m.flags = arc.ARC_FLAG_FORCE_SIMPLE
+    assert arc.plan(arc.ARC_OP_MLA, m)["kernel"] == "simple_attn_kernel"
+
