@@ -295,6 +295,10 @@ arc_status check_mla(const arc_mla_args *a)
     if (a->B == 0 || a->Tq == 0) return ARC_OK;
     if (!a->q_nope || (a->Dr > 0 && !a->q_rope) || !a->o || !a->lse) return ARC_ERR_INVALID_ARG;
     if (a->Tk > 0 && (!a->k_nope || (a->Dr > 0 && !a->k_rope) || !a->v)) return ARC_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (a->q_nope_strides[i] < 0 || a->q_rope_strides[i] < 0 || a->k_nope_strides[i] < 0 || a->v_strides[i] < 0 ||
+            a->o_strides[i] < 0 || (i < 2 && a->k_rope_strides[i] < 0))
+            return ARC_ERR_INVALID_ARG;
     if (broadcast(a->o_strides[0], a->B) || broadcast(a->o_strides[1], a->H) || broadcast(a->o_strides[2], a->Tq))
         return ARC_ERR_INVALID_ARG;
     return ARC_OK;
@@ -355,6 +359,9 @@ arc_status check_sparse(const arc_sparse_args *a)
     if (!a->v && a->Dv > a->Dqk) return ARC_ERR_INVALID_ARG;
     if (a->Sq == 0) return ARC_OK;
     if (!a->q || !a->o || !a->lse || (a->topk > 0 && (!a->idx || !a->kv))) return ARC_ERR_INVALID_ARG;
+    if (a->q_strides[0] < 0 || a->q_strides[1] < 0 || a->o_strides[0] < 0 || a->o_strides[1] < 0 || a->kv_stride < 0 ||
+        a->v_stride < 0 || a->idx_stride < 0)
+        return ARC_ERR_INVALID_ARG;
     if (broadcast(a->o_strides[0], a->Sq) || broadcast(a->o_strides[1], a->H)) return ARC_ERR_INVALID_ARG;
     return ARC_OK;
 }

@@ -131,8 +131,8 @@ arc_status arc_attn_fwd(const arc_attn_args *args, void *stream);
  * (head stride == Tq * token stride).  Other shapes or layouts return
  * ARC_ERR_UNSUPPORTED unless ARC_FLAG_FORCE_SIMPLE is set, which runs the
  * CUDA-core kernel for any Dn + Dr <= 512, Dv <= 512.  Dn + Dr or Dv above 512
- * is ARC_ERR_UNSUPPORTED; negative sizes or a NULL tensor that the call reads
- * are ARC_ERR_INVALID_ARG.  B == 0 or Tq == 0 launches nothing.
+ * is ARC_ERR_UNSUPPORTED; negative sizes or strides, or a NULL tensor that the
+ * call reads, are ARC_ERR_INVALID_ARG.  B == 0 or Tq == 0 launches nothing.
  * ------------------------------------------------------------------------ */
 typedef struct {
     int32_t B, H, Tq, Tk, Dn, Dr, Dv;
@@ -173,8 +173,9 @@ arc_status arc_mla_fwd(const arc_mla_args *args, void *stream);
  * V inside the kv row, and (128, 64), (128, 128), (256, 256) with a separate v,
  * on 16-byte aligned base pointers and strides; every other supported call runs
  * the CUDA-core kernel (arc_plan names which).  Dqk or Dv above 512 is
- * ARC_ERR_UNSUPPORTED; negative sizes, Dv > Dqk without v, or a NULL tensor
- * that the call reads are ARC_ERR_INVALID_ARG.  Sq == 0 launches nothing.
+ * ARC_ERR_UNSUPPORTED; negative sizes or strides, Dv > Dqk without v, or a
+ * NULL tensor that the call reads are ARC_ERR_INVALID_ARG.  Sq == 0 launches
+ * nothing.
  * ------------------------------------------------------------------------ */
 typedef struct {
     int32_t Sq, H, Skv, Dqk, Dv, topk;

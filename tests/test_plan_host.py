@@ -296,3 +296,16 @@ def test_mla_broadcast_inputs_are_refused_by_the_tma_path(arc, field, dim):
     m.flags = arc.ARC_FLAG_FORCE_SIMPLE
     assert arc.plan(arc.ARC_OP_MLA, m)["kernel"] == "simple_attn_kernel"
 
+
+@pytest.mark.parametrize("call,field,dim", [("mla", "q_nope_strides", 2), ("mla", "k_rope_strides", 1),
+                                            ("mla", "o_strides", 0), ("sparse", "kv_stride", None),
+                                            ("sparse", "idx_stride", None), ("sparse", "q_strides", 1)])
+def test_negative_strides_are_invalid(arc, call, field, dim):
+    x = mla_args(arc, Tq=256, Tk=256) if call == "mla" else sparse_args(arc, Sq=4, topk=64)
+    if dim is None:
+        setattr(x, field, -8)
+    else:
+        getattr(x, field)[dim] = -8
+    fn = arc.lib().arc_mla_fwd if call == "mla" else arc.lib().arc_sparse_mla_fwd
+    assert fn(ctypes.byref(x), None) == arc.ARC_ERR_INVALID_ARG
+
