@@ -85,8 +85,9 @@ typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE
  *   lse [B,H,Tq]      fp32, device, contiguous, written
  *   sinks [H]         fp32, device, or NULL for no sink; a raw logit (not scaled)
  *
- * dtype BF16: D in {64,128,192,256,512}, Dv in {64,128,256,512}; fp32
- * accumulation; P is rounded to bf16 before P*V.  The tensor-core path needs
+ * dtype BF16: (D, Dv) in {(64,64), (128,64), (128,128), (192,128), (256,128),
+ * (256,256), (256,512), (512,128), (512,256), (512,512)}; fp32 accumulation;
+ * P is rounded to bf16 before P*V.  The tensor-core path needs
  * each (b, kv) group of g*Tq query rows evenly spaced (head stride ==
  * Tq * token stride), 16-byte aligned rows and base pointers; otherwise the
  * call returns ARC_ERR_UNSUPPORTED unless ARC_FLAG_FORCE_SIMPLE is set.
@@ -126,7 +127,8 @@ arc_status arc_attn_fwd(const arc_attn_args *args, void *stream);
  *   v      [B,H,Tk,Dv]  bf16, device
  *   o      [B,H,Tq,Dv]  bf16, device, written
  *   lse    [B,H,Tq]     fp32, device, contiguous, written
- * Dn, Dr multiples of 64 with Dn + Dr <= 256; Dv in {64,128,256}; 16-byte
+ * Dn, Dr multiples of 64 (Dr > 0) with (Dn + Dr, Dv) in {(128,128), (192,64),
+ * (192,128), (256,128), (256,256)}; 16-byte
  * aligned base pointers and strides, and each head's query rows evenly spaced
  * (head stride == Tq * token stride).  Other shapes or layouts return
  * ARC_ERR_UNSUPPORTED unless ARC_FLAG_FORCE_SIMPLE is set, which runs the
