@@ -309,3 +309,38 @@ def test_negative_strides_are_invalid(arc, call, field, dim):
     fn = arc.lib().arc_mla_fwd if call == "mla" else arc.lib().arc_sparse_mla_fwd
     assert fn(ctypes.byref(x), None) == arc.ARC_ERR_INVALID_ARG
 
+
+
+def test_tensor_core_shape_sets_match_the_header(arc):
+    """The (D, Dv) pairs arc_plan sends to tensor-core kernels are exactly those the header lists."""
+    import re
+    text = open(os.path.join(ROOT, "include", "arc_attn.h")).read()
+
+    def pairs_after(marker):
+        seg = text[text.index(marker):]
+        seg = seg[:seg.index("}") + 1]
+        return {tuple(int(x) for x in m) for m in re.findall(r"\((\d+),\s*(\d+)\)", seg)}
+
+    dense_doc = pairs_after("dtype BF16: (D, Dv) in {")
+    mla_doc = pairs_after("with (Dn + Dr, Dv) in {")
+    dense, mla = set(), set()
+    for D in (64, 128, 192, 256, 320, 384, 512):
+        for Dv in (64, 128, 192, 256, 384, 512):
+            a = arc.AttnArgs()
+            B, H, Hkv, T = 1, 4, 2, 64
+            a.dtype, a.B, a.H, a.Hkv, a.Tq, a.Tk, a.D, a.Dv = arc.ARC_DTYPE_BF16, B, H, Hkv, T, T, D, Dv
+            a.q, a.k, a.v, a.o, a.lse = (FAKE,) * 5
+            for name, shape in (("q", (B, H, T, D)), ("k", (B, Hkv, T, D)), ("v", (B, Hkv, T, Dv)), ("o", (B, H, T, Dv))):
+                setattr(a, name + "_strides", (arc._i64 * 3)(*contiguous(*shape)))
+            info = arc.PlanInfo()
+            if arc.lib().arc_plan(arc.ARC_OP_ATTN, ctypes.byref(a), ctypes.byref(info)) == arc.ARC_OK:
+                assert info.tensor_cores == 1
+                dense.add((D, Dv))
+    for Dn in (64, 128, 192):
+        for Dr in (64, 128):
+            for Dv in (64, 128, 256):
+                m = mla_args(arc, B=1, H=2, Tq=64, Tk=64, Dn=Dn, Dr=Dr, Dv=Dv)
+                if arc.lib().arc_plan(arc.ARC_OP_MLA, ctypes.byref(m), ctypes.byref(arc.PlanInfo())) == arc.ARC_OK:
+                    mla.add((Dn + Dr, Dv))
+    assert dense == dense_doc and len(dense) == 10
+    assert mla == mla_doc and len(mla) == 5
