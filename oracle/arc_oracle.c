@@ -54,6 +54,7 @@ enum {
     MUT_TOP_LEFT_CAUSAL = 4,  /* causal mask aligned top-left instead of bottom-right */
     MUT_SWAP_NIBBLES = 5,     /* q4_0: low/high nibble roles swapped */
     MUT_MERGE_UNWEIGHTED = 6, /* merge: plain mean of the parts, no log-sum-exp weights */
+    MUT_BWD_DROP_DELTA = 7,   /* read by the numpy backward (backward.py): D_i dropped from dS */
 };
 
 static int g_mutation = MUT_NONE;
