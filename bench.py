@@ -8,7 +8,11 @@ the headline metric is quoted on.  Other workloads: --config c1 c3 c4 c5q8 c5q4.
 
 Timing: W untimed warm-up steps, then K steps; before each timed step a
 256 MiB buffer is written to flush L2 (outside the timed interval), and the
-step is bracketed by CUDA events on the launching stream.  Multi-GPU (torchrun):
+step is bracketed by CUDA events on the launching stream.  A single-GPU run
+also times every other graded workload (c2, c3, c4, c5q8, c5q4) in the same
+way, each on a loop of at least --per-config-wall seconds so the clock sampler
+sees it, and adds them under "per_config"; the decode workloads are timed a
+second time replaying the call from a CUDA graph.  Multi-GPU (torchrun):
 every rank runs the same per-GPU work (weak scaling, no data-path collective);
 the time is the max over ranks.  --impl reference times the CPU oracle on the
 host cores on a bounded sample of the same workload.
@@ -342,6 +346,109 @@ def job_throughput(units_per_step, world, steps, total_ms, unit_kind):
     return units_per_step * world * steps / (total_ms * 1e-3) / scale
 
 
+def time_steps(call, steps, stream, flush, local, graph=None):
+    """Device time of `steps` calls: a 256 MiB write flushes L2 before each, CUDA events on
+    the launching stream bracket the call only.  With `graph`, each step replays it instead
+    of calling.  Returns (per-step ms list, wall seconds of the loop, clock record)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    sampler = ClockSampler(local)
+    torch.cuda.synchronize()
+    with sampler:
+        wall0 = time.perf_counter()
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            if graph is None:
+                call()
+            else:
+                graph.replay()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    return [a.elapsed_time(b) for a, b in ev], wall, sampler.result()
+
+
+def capture(call, stream):
+    """One call captured into a CUDA graph (the serving form of a decode step)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        call()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            call()
+    torch.cuda.synchronize()
+    return g
+
+
+def steps_for(call, stream, flush, local, min_wall_s):
+    """Enough steps that the timed loop lasts min_wall_s (so the clock sampler sees it)."""
+    _, wall, _ = time_steps(call, 20, stream, flush, local)
+    return max(20, int(math.ceil(min_wall_s / max(wall / 20, 1e-6))))
+
+
+def roofline(units, unit_kind, mean_ms, peaks, config_key, kernel):
+    if unit_kind == "flop":
+        achieved = units / (mean_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst bf16",
+                "frac_of_sustained": (achieved / peaks["bf16_tflops_sustained"]
+                                      if peaks.get("bf16_tflops_sustained") else None)}
+    else:
+        achieved = units / (mean_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
+                "note": ("whole call (split kernel + combine) timed" if kernel.startswith("decode")
+                         else "one launch")}
+    roof["traffic"] = recorded_traffic(config_key, kernel)
+    roof["kernel"] = kernel
+    return roof
+
+
+def measure_config(key, status, stream, flush, local, peaks, min_wall_s):
+    """One graded workload on this GPU, for the per-workload record beside the headline:
+    device time over a loop long enough for the clock sampler, and for the decode
+    workloads the same call replayed from a CUDA graph as well."""
+    import torch
+    import exact_attention_131_b200 as arc
+    spec = CONFIGS[key]
+    case = make_case(spec)
+    call, ins, outs, info = build_call(case, torch, arc, status)
+    units, unit_kind = work(case)
+    for _ in range(5):
+        call()
+    steps = steps_for(call, stream, flush, local, min_wall_s)
+    times, wall, clocks = time_steps(call, steps, stream, flush, local)
+    mean_ms = sum(times) / len(times)
+    scale = 1e12 if unit_kind == "flop" else 1e9
+    rec = {"workload": spec["name"], "metric": spec["metric"], "value": units / (mean_ms * 1e-3) / scale,
+           "unit": "TFLOP/s" if unit_kind == "flop" else "GB/s", "ms_per_step": mean_ms, "steps": steps,
+           "dtype": spec["dtype"], "roofline": roofline(units, unit_kind, mean_ms, peaks, key, info["kernel"]),
+           "clocks": clocks, "wall_s_timed_region": wall, "gpu_launches": int(info["launches"]) * steps}
+    if isinstance(case, W.DecodeCase):
+        g = capture(call, stream)
+        for _ in range(5):
+            g.replay()
+        gsteps = max(steps, 20)
+        gt, gwall, gclocks = time_steps(call, gsteps, stream, flush, local, graph=g)
+        gmean = sum(gt) / len(gt)
+        rec["graph_replay"] = {"value": units / (gmean * 1e-3) / scale, "ms_per_step": gmean, "steps": gsteps,
+                               "frac": units / (gmean * 1e-3) / scale / peaks["hbm_gbs"], "clocks": gclocks,
+                               "note": "the same call captured once into a CUDA graph and replayed"}
+        del g
+    del call, ins, outs, case
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
+
+
+# The graded workloads: the headline (--config) plus these, each measured in the same run.
+GRADED = ["c2", "c3", "c4", "c5q8", "c5q4"]
+
+
 def run_ours(args, spec, case):
     import torch
     import torch.distributed as dist
@@ -369,21 +476,9 @@ def run_ours(args, spec, case):
         call()
     torch.cuda.synchronize()
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    sampler = ClockSampler(local)
     barrier()
-    torch.cuda.synchronize()
-    with sampler:
-        wall0 = time.perf_counter()
-        for i in range(args.steps):
-            flush.fill_(i & 0xFF)
-            ev[i][0].record(stream)
-            call()
-            ev[i][1].record(stream)
-        torch.cuda.synchronize()
-        wall = time.perf_counter() - wall0
+    times_ms, wall, clocks = time_steps(call, args.steps, stream, flush, local)
     barrier()
-    times_ms = [a.elapsed_time(b) for a, b in ev]
     mean_ms = sum(times_ms) / len(times_ms)
     total_ms = sum(times_ms)
     total_ms = max_over_ranks(total_ms, world, "cuda")
@@ -412,27 +507,13 @@ def run_ours(args, spec, case):
     e2e_mean = sum(e2e_ms) / len(e2e_ms) if e2e_ms else float("nan")
 
     peaks = load_peaks()
-    if unit_kind == "flop":
-        value = job_throughput(units, world, args.steps, total_ms, unit_kind)
-        unit = "TFLOP/s"
-        achieved = units / (mean_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "peak_source": peaks["source"] + " burst bf16",
-                "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"] if peaks.get("bf16_tflops_sustained") else None}
-        e2e_val = units / (e2e_mean * 1e-3) / 1e12
-    else:
-        value = job_throughput(units, world, args.steps, total_ms, unit_kind)
-        unit = "GB/s"
-        achieved = units / (mean_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
-                "note": ("whole call (split kernel + combine) timed" if info["kernel"].startswith("decode")
-                         else "one merge_kernel launch")}
-        e2e_val = units / (e2e_mean * 1e-3) / 1e9
+    scale = 1e12 if unit_kind == "flop" else 1e9
+    unit = "TFLOP/s" if unit_kind == "flop" else "GB/s"
+    value = job_throughput(units, world, args.steps, total_ms, unit_kind)
+    roof = roofline(units, unit_kind, mean_ms, peaks, args.config, info["kernel"])
+    e2e_val = units / (e2e_mean * 1e-3) / scale
     if not e2e_ms:                      # --no-e2e: no host-buffer leg; JSON null rather than NaN
         e2e_val = e2e_mean = None
-    roof["traffic"] = recorded_traffic(args.config, info["kernel"])
-    roof["kernel"] = info["kernel"]
 
     line = {
         "metric": spec["metric"], "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
@@ -445,9 +526,17 @@ def run_ours(args, spec, case):
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_mean},
         "gpu_launches": int(info["launches"]) * args.steps,
-        "clocks": sampler.result(),
+        "clocks": clocks,
         "wall_s_timed_region": wall,
     }
+    del call, ins, outs, host_ins, host_outs
+    torch.cuda.empty_cache()
+    # Every graded workload, each on its own long-enough loop, in the same run (rank 0 of a
+    # single-GPU run only: under torchrun each rank would time its own replicas again).
+    if world == 1 and not args.no_per_config:
+        line["per_config"] = {k: measure_config(k, status, stream, flush, local, peaks, args.per_config_wall)
+                              for k in GRADED if k != args.config}
+        assert arc.check_device_error(status) == arc.ARC_OK, "a device-side wait timed out"
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case, args.config)
     if rank == 0:
@@ -514,12 +603,15 @@ def run_reference(args, spec, case):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(CONFIGS), default="c2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (for profiler runs)")
+    ap.add_argument("--no-per-config", action="store_true", help="time the --config workload only")
+    ap.add_argument("--per-config-wall", type=float, default=1.5,
+                    help="seconds each extra graded workload's timed loop lasts at least")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")

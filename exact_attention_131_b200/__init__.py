@@ -15,7 +15,6 @@ Names follow the C ABI:
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,6 +28,7 @@ ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE, ARC_OP_MERGE = 1, 2, 3, 4
 ARC_MERGE_MAX_PARTS = 16
 ARC_FLAG_FORCE_SIMPLE = 1
 ARC_FLAG_SINGLE_CTA = 2
+ARC_FLAG_DEFAULT_SCALE = 4
 ARC_DECODE_MAX_SEQ = 64
 
 _i32, _i64, _u32, _f32, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float, ctypes.c_void_p
@@ -169,6 +169,13 @@ def _s3(t):
     return (_i64 * 3)(*t.stride()[:3])
 
 
+def _scale_flags(scale, flags):
+    """scale=None asks the library for its default 1/sqrt(d_qk) (ARC_FLAG_DEFAULT_SCALE)."""
+    if scale is None:
+        return 0.0, int(flags) | ARC_FLAG_DEFAULT_SCALE
+    return float(scale), int(flags)
+
+
 # ------------------------------------------------------------------ entry points
 
 def _attn_args(q, k, v, o, lse, sinks, scale, causal, flags, status):
@@ -185,9 +192,8 @@ def _attn_args(q, k, v, o, lse, sinks, scale, causal, flags, status):
     a.v, a.v_strides = _p(v), _s3(v)
     a.o, a.o_strides = _p(o), _s3(o)
     a.lse, a.sinks = _p(lse), _p(sinks)
-    a.scale = float(scale)
+    a.scale, a.flags = _scale_flags(scale, flags)
     a.causal = int(bool(causal))
-    a.flags = int(flags)
     a.status = _p(status)
     return a
 
@@ -205,7 +211,6 @@ def attn_fwd(q, k, v, *, scale=None, causal=True, sinks=None, out=None, lse=None
         out = torch.empty(B, H, Tq, Dv, dtype=q.dtype, device=q.device)
     if lse is None:
         lse = torch.empty(B, H, Tq, dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(D) if scale is None else scale
     a = _attn_args(q, k, v, out, lse, sinks, scale, causal, flags, status)
     _check(lib().arc_attn_fwd(ctypes.byref(a), _stream(stream)), "arc_attn_fwd")
     return out, lse
@@ -224,9 +229,8 @@ def _mla_args(q_nope, q_rope, k_nope, k_rope, v, o, lse, scale, causal, flags, s
     a.v, a.v_strides = _p(v), _s3(v)
     a.o, a.o_strides = _p(o), _s3(o)
     a.lse = _p(lse)
-    a.scale = float(scale)
+    a.scale, a.flags = _scale_flags(scale, flags)
     a.causal = int(bool(causal))
-    a.flags = int(flags)
     a.status = _p(status)
     return a
 
@@ -244,7 +248,6 @@ def mla_fwd(q_nope, q_rope, k_nope, k_rope, v, *, scale=None, causal=True, out=N
         out = torch.empty(B, H, Tq, Dv, dtype=bf, device=q_nope.device)
     if lse is None:
         lse = torch.empty(B, H, Tq, dtype=torch.float32, device=q_nope.device)
-    scale = 1.0 / math.sqrt(Dn + q_rope.shape[-1]) if scale is None else scale
     a = _mla_args(q_nope, q_rope, k_nope, k_rope, v, out, lse, scale, causal, flags, status)
     _check(lib().arc_mla_fwd(ctypes.byref(a), _stream(stream)), "arc_mla_fwd")
     return out, lse
@@ -260,8 +263,7 @@ def _sparse_args(q, kv, idx, v, o, lse, sinks, Dv, scale, flags, status):
     a.idx, a.idx_stride = _p(idx), idx.stride(0)
     a.o, a.o_strides = _p(o), (_i64 * 2)(*o.stride()[:2])
     a.lse, a.sinks = _p(lse), _p(sinks)
-    a.scale = float(scale)
-    a.flags = int(flags)
+    a.scale, a.flags = _scale_flags(scale, flags)
     a.status = _p(status)
     return a
 
@@ -280,7 +282,6 @@ def sparse_mla_fwd(q, kv, idx, *, Dv=None, v=None, scale=None, sinks=None, out=N
         out = torch.empty(Sq, H, Dv, dtype=bf, device=q.device)
     if lse is None:
         lse = torch.empty(Sq, H, dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(Dqk) if scale is None else scale
     a = _sparse_args(q, kv, idx, v, out, lse, sinks, Dv, scale, flags, status)
     _check(lib().arc_sparse_mla_fwd(ctypes.byref(a), _stream(stream)), "arc_sparse_mla_fwd")
     return out, lse
@@ -301,8 +302,7 @@ def _decode_args(kv_type, q, k_cache, v_cache, seqs, n_seq, Hkv, n_cells, o, lse
     a.q, a.k_cache, a.v_cache = _p(q), _p(k_cache), _p(v_cache)
     a.seqs = ctypes.cast(seqs, ctypes.POINTER(Seq))
     a.o, a.lse = _p(o), _p(lse)
-    a.scale = float(scale)
-    a.flags = int(flags)
+    a.scale, a.flags = _scale_flags(scale, flags)
     a.status = _p(status)
     return a
 
@@ -313,19 +313,46 @@ def decode_workspace_size(kv_type, q, Hkv, n_cells, q_begin, n_q, kv_begin, n_kv
     return int(lib().arc_decode_workspace_size(ctypes.byref(a)))
 
 
-def attn_decode_q8(q, k_cache, v_cache, *, kv_type, Hkv, q_begin, n_q, kv_begin, n_kv, scale=None,
-                   workspace=None, out=None, lse=None, flags=0, status=None, stream=None):
-    """O, LSE = arc_attn_decode_q8(q [n_tok,H,D] fp32, caches [n_cells,Hkv,D/32 blocks] uint8)."""
+def _decode_tensors(kv_type, q, k_cache, v_cache, Hkv, out, lse):
+    """The decode ABI takes no strides: every tensor must be contiguous and of the shape
+    the call implies, or the kernels would read or write past it.  Returns (out, lse),
+    created when not given."""
     torch = _torch()
     _dev(q, "q", torch.float32), _dev(k_cache, "k_cache", torch.uint8), _dev(v_cache, "v_cache", torch.uint8)
+    if q.dim() != 3 or not q.is_contiguous():
+        raise ValueError("q must be a contiguous [n_tok, H, D] tensor")
     n_tok, H, D = q.shape
-    n_cells = k_cache.shape[0]
-    seqs = make_seqs(q_begin, n_q, kv_begin, n_kv)
+    if Hkv <= 0 or H % Hkv or D % 32:
+        raise ValueError("H must be a multiple of Hkv and D a multiple of 32")
+    block = {ARC_KV_Q8_0: 34, ARC_KV_Q4_0: 18}.get(kv_type)
+    if block is None:
+        raise ValueError(f"unknown kv_type {kv_type}")
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if not t.is_contiguous() or t.dim() < 1 or t.device != q.device:
+            raise ValueError(f"{n} must be contiguous and on q's device")
+        if t.numel() != t.shape[0] * Hkv * (D // 32) * block:
+            raise ValueError(f"{n} rows must hold Hkv * D/32 blocks of {block} bytes")
+    if k_cache.shape != v_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape")
+    for n, t, shape in (("out", out, (n_tok, H, D)), ("lse", lse, (n_tok, H))):
+        if t is None:
+            continue
+        if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() or t.device != q.device:
+            raise ValueError(f"{n} must be a contiguous fp32 {list(shape)} tensor on q's device")
     if out is None:
         out = torch.empty(n_tok, H, D, dtype=torch.float32, device=q.device)
     if lse is None:
         lse = torch.empty(n_tok, H, dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    return out, lse
+
+
+def attn_decode_q8(q, k_cache, v_cache, *, kv_type, Hkv, q_begin, n_q, kv_begin, n_kv, scale=None,
+                   workspace=None, out=None, lse=None, flags=0, status=None, stream=None):
+    """O, LSE = arc_attn_decode_q8(q [n_tok,H,D] fp32, caches [n_cells,Hkv,D/32 blocks] uint8)."""
+    torch = _torch()
+    out, lse = _decode_tensors(kv_type, q, k_cache, v_cache, Hkv, out, lse)
+    n_cells = k_cache.shape[0]
+    seqs = make_seqs(q_begin, n_q, kv_begin, n_kv)
     a = _decode_args(kv_type, q, k_cache, v_cache, seqs, len(q_begin), Hkv, n_cells, out, lse, scale, flags,
                      status)
     need = int(lib().arc_decode_workspace_size(ctypes.byref(a)))
@@ -349,15 +376,8 @@ def attn_decode_q8_noalloc(q, k_cache, v_cache, *, kv_type, Hkv, q_begin, n_q, k
     with torch when they are not given; pass them to keep the call allocation-free.)
     Calls on unordered streams race on the shared scratch.
     """
-    torch = _torch()
-    _dev(q, "q", torch.float32), _dev(k_cache, "k_cache", torch.uint8), _dev(v_cache, "v_cache", torch.uint8)
-    n_tok, H, D = q.shape
+    out, lse = _decode_tensors(kv_type, q, k_cache, v_cache, Hkv, out, lse)
     seqs = make_seqs(q_begin, n_q, kv_begin, n_kv)
-    if out is None:
-        out = torch.empty(n_tok, H, D, dtype=torch.float32, device=q.device)
-    if lse is None:
-        lse = torch.empty(n_tok, H, dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(D) if scale is None else scale
     a = _decode_args(kv_type, q, k_cache, v_cache, seqs, len(q_begin), Hkv, k_cache.shape[0], out, lse, scale,
                      flags, status)
     _check(lib().arc_attn_decode_q8_noalloc(ctypes.byref(a), _stream(stream)), "arc_attn_decode_q8_noalloc")

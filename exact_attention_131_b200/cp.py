@@ -16,7 +16,6 @@ runs.  All ranks take the same steps in the same order.
 """
 from __future__ import annotations
 
-import math
 
 from . import attn_fwd, attn_merge
 
@@ -62,7 +61,6 @@ def ring_attention_forward(q, k, v, *, group=None, causal=True, scale=None, sink
     attn = attn or _default_attn
     merge = merge or _default_merge
     world, rank = dist.get_world_size(group), dist.get_rank(group)
-    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
     nxt, prv = (rank + 1) % world, (rank - 1) % world
     if group is not None:
         nxt, prv = dist.get_global_rank(group, nxt), dist.get_global_rank(group, prv)
@@ -98,7 +96,6 @@ def context_parallel_forward_local(q, k, v, world, *, causal=True, scale=None, s
     if T % world:
         raise ValueError("the sequence length must divide into world equal chunks")
     L = T // world
-    scale = 1.0 / math.sqrt(q.shape[-1]) if scale is None else scale
     chunk = lambda x, r: x[:, :, r * L:(r + 1) * L].contiguous()
     out = []
     for rank in range(world):

@@ -3,6 +3,7 @@
 // Nothing here allocates device memory; nothing is launched when validation
 // fails.
 #include <cudaTypedefs.h>
+#include <math.h>
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -34,6 +35,16 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // output rows that would alias one another (refused everywhere).
 bool broadcast(int64_t stride, int64_t extent) { return stride == 0 && extent > 1; }
 bool in_set(int x, std::initializer_list<int> s) { return std::find(s.begin(), s.end(), x) != s.end(); }
+
+// The softmax scale a call computes with: 1/sqrt(d_qk) under ARC_FLAG_DEFAULT_SCALE
+// (evaluated in double, then rounded once to fp32), otherwise the caller's value.
+float call_scale(uint32_t flags, float scale, int dqk)
+{
+    return (flags & ARC_FLAG_DEFAULT_SCALE) ? (float)(1.0 / sqrt((double)dqk)) : scale;
+}
+
+// A NaN scale is refused unless the flag replaces it.
+bool scale_ok(uint32_t flags, float scale) { return (flags & ARC_FLAG_DEFAULT_SCALE) || scale == scale; }
 
 int sm_count()
 {
@@ -136,6 +147,39 @@ bool make_map_bytes(CUtensorMap *m, const void *base, uint64_t width, uint64_t r
     return r == CUDA_SUCCESS;
 }
 
+// The decode caches are the same few buffers call after call, so their byte-tensor maps
+// are kept: a map is a pure function of (base, width, rows, box), which is the key.
+bool make_map_bytes_cached(CUtensorMap *m, const void *base, uint64_t width, uint64_t rows, uint32_t box_w,
+                           uint32_t box_rows)
+{
+    struct Entry {
+        const void *base;
+        uint64_t width, rows;
+        uint32_t box_w, box_rows;
+        CUtensorMap map;
+    };
+    static std::mutex mu;
+    static Entry cache[16];
+    static int used = 0, next = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i) {
+            const Entry &e = cache[i];
+            if (e.base == base && e.width == width && e.rows == rows && e.box_w == box_w && e.box_rows == box_rows) {
+                *m = e.map;
+                return true;
+            }
+        }
+    }
+    if (!make_map_bytes(m, base, width, rows, box_w, box_rows)) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    Entry &e = cache[next];
+    e.base = base, e.width = width, e.rows = rows, e.box_w = box_w, e.box_rows = box_rows, e.map = *m;
+    next = (next + 1) % 16;
+    used = std::max(used, next == 0 ? 16 : next);
+    return true;
+}
+
 bool tma_strides_ok(std::initializer_list<int64_t> strides_el)
 {
     for (int64_t s : strides_el)
@@ -188,7 +232,7 @@ arc_status check_attn(const arc_attn_args *a)
     if (a->D <= 0 || a->Dv <= 0 || a->D > 512 || a->Dv > 512) return ARC_ERR_UNSUPPORTED;
     if (a->B == 0 || a->Tq == 0) return ARC_OK;
     if (!a->q || !a->o || !a->lse || (a->Tk > 0 && (!a->k || !a->v))) return ARC_ERR_INVALID_ARG;
-    if (!(a->scale == a->scale)) return ARC_ERR_INVALID_ARG;
+    if (!scale_ok(a->flags, a->scale)) return ARC_ERR_INVALID_ARG;
     for (int i = 0; i < 3; ++i)
         if (a->q_strides[i] < 0 || a->k_strides[i] < 0 || a->v_strides[i] < 0 || a->o_strides[i] < 0)
             return ARC_ERR_INVALID_ARG;
@@ -280,7 +324,8 @@ SimpleParams simple_from_attn(const arc_attn_args *a)
     p.q = a->q, p.k = a->k, p.v = a->v, p.o = a->o;
     for (int i = 0; i < 3; ++i) p.qs[i] = a->q_strides[i], p.ks[i] = a->k_strides[i], p.vs[i] = a->v_strides[i],
                                 p.os[i] = a->o_strides[i];
-    p.lse = a->lse, p.sinks = a->sinks, p.scale = a->scale, p.causal = a->causal, p.status = a->status;
+    p.lse = a->lse, p.sinks = a->sinks, p.scale = call_scale(a->flags, a->scale, a->D), p.causal = a->causal;
+    p.status = a->status;
     return p;
 }
 
@@ -293,6 +338,7 @@ arc_status check_mla(const arc_mla_args *a)
         return ARC_ERR_INVALID_ARG;
     if (a->Dn + a->Dr > 512 || a->Dv > 512) return ARC_ERR_UNSUPPORTED;
     if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    if (!scale_ok(a->flags, a->scale)) return ARC_ERR_INVALID_ARG;
     if (!a->q_nope || (a->Dr > 0 && !a->q_rope) || !a->o || !a->lse) return ARC_ERR_INVALID_ARG;
     if (a->Tk > 0 && (!a->k_nope || (a->Dr > 0 && !a->k_rope) || !a->v)) return ARC_ERR_INVALID_ARG;
     for (int i = 0; i < 3; ++i)
@@ -358,6 +404,7 @@ arc_status check_sparse(const arc_sparse_args *a)
     if (a->Dqk > 512 || a->Dv > 512) return ARC_ERR_UNSUPPORTED;
     if (!a->v && a->Dv > a->Dqk) return ARC_ERR_INVALID_ARG;
     if (a->Sq == 0) return ARC_OK;
+    if (!scale_ok(a->flags, a->scale)) return ARC_ERR_INVALID_ARG;
     if (!a->q || !a->o || !a->lse || (a->topk > 0 && (!a->idx || !a->kv))) return ARC_ERR_INVALID_ARG;
     if (a->q_strides[0] < 0 || a->q_strides[1] < 0 || a->o_strides[0] < 0 || a->o_strides[1] < 0 || a->kv_stride < 0 ||
         a->v_stride < 0 || a->idx_stride < 0)
@@ -407,6 +454,7 @@ arc_status check_decode(const arc_decode_args *a, bool need_ptrs = true)
         if (G * q.n_q > 16) return ARC_ERR_UNSUPPORTED;
     }
     if (need_ptrs && a->n_seq > 0 && a->n_tok > 0) {
+        if (!scale_ok(a->flags, a->scale)) return ARC_ERR_INVALID_ARG;
         if (!a->q || !a->o || !a->lse || !a->k_cache || !a->v_cache) return ARC_ERR_INVALID_ARG;
         if ((reinterpret_cast<uintptr_t>(a->k_cache) | reinterpret_cast<uintptr_t>(a->v_cache)) & 7u)
             return ARC_ERR_INVALID_ARG;
@@ -512,7 +560,8 @@ arc_status arc_attn_fwd(const arc_attn_args *a, void *stream)
         p.n_tiles = pl.n_tiles, p.n_slices = pl.n_slices, p.kc_first = a->D / 64, p.stages = pl.stages;
         p.o = a->o;
         for (int i = 0; i < 3; ++i) p.os[i] = a->o_strides[i];
-        p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = a->scale * kLog2e, p.causal = a->causal;
+        p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = call_scale(a->flags, a->scale, a->D) * kLog2e;
+        p.causal = a->causal;
         p.status = a->status;
         if (pl.two) {
             order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
@@ -552,7 +601,8 @@ arc_status arc_mla_fwd(const arc_mla_args *a, void *stream)
             p.vs[i] = a->v_strides[i], p.os[i] = a->o_strides[i];
         }
         p.k2s[0] = a->k_rope_strides[0], p.k2s[1] = a->k_rope_strides[1];
-        p.lse = a->lse, p.scale = a->scale, p.causal = a->causal, p.status = a->status;
+        p.lse = a->lse, p.scale = call_scale(a->flags, a->scale, a->Dn + a->Dr), p.causal = a->causal;
+        p.status = a->status;
         note_dispatch("simple_attn_kernel");
         e = launch_simple_attn(p, s);
     } else {
@@ -580,7 +630,8 @@ arc_status arc_mla_fwd(const arc_mla_args *a, void *stream)
         p.n_tiles = pl.n_tiles, p.n_slices = 1, p.kc_first = a->Dn / 64, p.stages = pl.stages;
         p.o = a->o;
         for (int i = 0; i < 3; ++i) p.os[i] = a->o_strides[i];
-        p.lse = a->lse, p.sinks = nullptr, p.scale_log2 = a->scale * kLog2e, p.causal = a->causal;
+        p.lse = a->lse, p.sinks = nullptr, p.scale_log2 = call_scale(a->flags, a->scale, a->Dn + a->Dr) * kLog2e;
+        p.causal = a->causal;
         p.status = a->status;
         if (pl.pair) {
             order_tiles(p, (pl.n_tiles + 1) / 2, 2 * kTcBM);
@@ -614,7 +665,8 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *a, void *stream)
         p.v = static_cast<const __nv_bfloat16 *>(a->v), p.v_stride = a->v_stride;
         p.idx = a->idx, p.idx_stride = a->idx_stride;
         p.o = static_cast<__nv_bfloat16 *>(a->o), p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
-        p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = a->scale * kLog2e, p.status = a->status;
+        p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = call_scale(a->flags, a->scale, a->Dqk) * kLog2e;
+        p.status = a->status;
         note_dispatch("sparse_tc_kernel");
         e = launch_sparse_tc(p, s);
     } else {
@@ -626,7 +678,7 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *a, void *stream)
         p.qs[0] = a->q_strides[0], p.qs[1] = a->q_strides[1];
         p.ks[0] = a->kv_stride, p.vs[0] = a->v_stride;
         p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
-        p.lse = a->lse, p.sinks = a->sinks, p.scale = a->scale, p.causal = 0;
+        p.lse = a->lse, p.sinks = a->sinks, p.scale = call_scale(a->flags, a->scale, a->Dqk), p.causal = 0;
         p.idx = a->idx, p.idx_stride = a->idx_stride, p.topk = a->topk, p.Skv = a->Skv, p.status = a->status;
         note_dispatch("simple_attn_kernel<sparse>");
         e = launch_simple_attn(p, s);
@@ -655,7 +707,7 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
         p.q = a->q, p.k_cache = static_cast<const uint8_t *>(a->k_cache);
         p.v_cache = static_cast<const uint8_t *>(a->v_cache);
         memcpy(p.seqs, a->seqs, sizeof(arc_seq) * a->n_seq);
-        p.o = a->o, p.lse = a->lse, p.scale = a->scale;
+        p.o = a->o, p.lse = a->lse, p.scale = call_scale(a->flags, a->scale, a->D);
         note_dispatch("simple_decode_kernel");
         e = launch_simple_decode(p, s);
     } else {
@@ -670,7 +722,7 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
         const size_t parts = (size_t)a->n_seq * a->Hkv * pl.splits;
         p.ws_o = static_cast<float *>(workspace);
         p.ws_ml = p.ws_o + parts * 16 * a->D;
-        p.scale_log2 = a->scale * kLog2e;
+        p.scale_log2 = call_scale(a->flags, a->scale, a->D) * kLog2e;
         p.status = a->status;
         // K/V tiles by TMA when the cache rows allow it: a byte tensor {cell bytes, n_cells} per cache.
         p.tma = pl.tma && (reinterpret_cast<uintptr_t>(a->k_cache) & 15) == 0 &&
@@ -678,8 +730,8 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
         if (p.tma) {
             const int64_t cell_bytes = (int64_t)a->Hkv * (a->D / 32) * (a->kv_type == ARC_KV_Q8_0 ? 34 : 18);
             const uint32_t box_w = (uint32_t)decode_box_bytes(a->kv_type, a->D);
-            if (!make_map_bytes(&p.tm_kc, a->k_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64) ||
-                !make_map_bytes(&p.tm_vc, a->v_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64))
+            if (!make_map_bytes_cached(&p.tm_kc, a->k_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64) ||
+                !make_map_bytes_cached(&p.tm_vc, a->v_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64))
                 return ARC_ERR_CUDA;
         }
         if (p.tma)
@@ -693,22 +745,68 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
 
 // Library-owned scratch for arc_attn_decode_q8_noalloc.  In host code the
 // symbol is only a stand-in; its device address comes from
-// cudaGetSymbolAddress, looked up once per device with that device current.
+// cudaGetSymbolAddress, looked up with the caller's context current.
 static __device__ __align__(256) unsigned char g_decode_noalloc_scratch[ARC_DECODE_NOALLOC_SCRATCH_BYTES];
 
+// Identity of the calling thread's current CUDA context, unique for the life of the
+// process (a context re-created after cudaDeviceReset gets a new one), or 0 when
+// there is no current context or the driver cannot say.
+static unsigned long long current_context_id()
+{
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+// The scratch array's device address in the current context.  The symbol can sit at a
+// different address in every context that loads the library (another device, a context
+// made current through the driver API, the primary context re-created after a reset), so
+// the address is cached per context id, never per device ordinal.  Without an id the
+// lookup runs on every call.
 static arc_status noalloc_scratch_address(void **out)
 {
+    struct Entry {
+        unsigned long long ctx;
+        void *addr;
+    };
     static std::mutex mu;
-    static void *addr[256] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) return ARC_ERR_CUDA;
+    static Entry cache[64];
+    static int used = 0, next = 0;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || !p) return ARC_ERR_CUDA;
-        addr[dev] = p;
+    unsigned long long id = current_context_id();
+    for (int i = 0; id && i < used; ++i)
+        if (cache[i].ctx == id) {
+            *out = cache[i].addr;
+            return ARC_OK;
+        }
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return ARC_ERR_CUDA;
     }
-    *out = addr[dev];
+    if (!id) id = current_context_id();   // the lookup may have made the primary context current
+    if (id) {
+        cache[next] = {id, p};
+        next = (next + 1) % 64;
+        used = std::max(used, next == 0 ? 64 : next);
+    }
+    *out = p;
     return ARC_OK;
 }
 

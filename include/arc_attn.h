@@ -14,9 +14,14 @@
  *
  * Conventions shared by all calls
  *   - Pointers marked "device" are CUDA device (or managed) memory owned by the
- *     caller.  The library allocates no memory and keeps no mutable global
- *     state; a call only reads its inputs and writes its outputs (and, for
- *     decode, the caller's workspace).
+ *     caller.  The library allocates no memory.  A call reads its inputs and
+ *     writes its outputs (and, for decode, the caller's workspace), with two
+ *     exceptions, both library-wide state: arc_attn_decode_q8_noalloc keeps its
+ *     split-KV partials in one static device buffer that every call shares (see
+ *     that call for its race and first-call-before-capture rules), and with
+ *     ARC_LOG=1 in the environment the first launch of each kernel is noted on
+ *     stderr (host-side bookkeeping that never changes a result).  Tensor maps
+ *     for the decode caches are cached on the host, keyed by pointer and shape.
  *   - Strides are in ELEMENTS, int64.  The last dimension of every tensor is
  *     contiguous (stride 1).  A zero stride over a dimension of extent above 1
  *     (a broadcast view) is accepted for inputs by the CUDA-core kernels, which
@@ -68,6 +73,11 @@ typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE
 /* flags (all calls) */
 #define ARC_FLAG_FORCE_SIMPLE 1u   /* run the CUDA-core kernel instead of the tensor-core one */
 #define ARC_FLAG_SINGLE_CTA 2u     /* do not use the CTA-pair (cta_group::2) kernel */
+/* Use the standard softmax scale 1/sqrt(d_qk) and ignore the `scale` field:
+ * d_qk is D (arc_attn_fwd, arc_attn_decode_q8), Dn + Dr (arc_mla_fwd) or Dqk
+ * (arc_sparse_mla_fwd).  Without the flag, `scale` is used as given (any
+ * finite value; NaN is ARC_ERR_INVALID_ARG). */
+#define ARC_FLAG_DEFAULT_SCALE 4u
 
 /* --------------------------------------------------------------------------
  * arc_attn_fwd: dense attention with GQA / MQA and optional per-head sinks.
@@ -277,8 +287,12 @@ arc_status arc_attn_decode_q8(const arc_decode_args *args, void *workspace, size
  *   - A call whose partial results would need more than that buffer returns
  *     ARC_ERR_WORKSPACE and launches nothing (arc_decode_workspace_size()
  *     gives the bytes a call needs).
- *   - The first call on a device (that device current) looks up the buffer's
- *     device address once; make that first call before any stream capture.
+ *   - The buffer's device address differs from context to context.  The first
+ *     call in each CUDA context (the context current on the calling thread)
+ *     looks it up with cudaGetSymbolAddress and keeps it, keyed by the
+ *     context's unique id, so a context made current through the driver API or
+ *     re-created after cudaDeviceReset gets its own lookup.  Make that first
+ *     call before any stream capture.
  *   - All calls share the one buffer and it keeps the last call's contents
  *     (nothing in it needs to start at zero).  Calls that may overlap on the
  *     GPU -- on different streams without ordering between them -- race on it;

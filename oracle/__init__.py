@@ -252,10 +252,11 @@ def run_case(case, rows=None):
                    causal=case.causal, rows=rows)
     if isinstance(case, W.SparseCase):
         if rows is None:
-            return sparse(case.q, case.kv, case.idx, scale=case.scale, Dv=case.Dv, v=case.v)
+            return sparse(case.q, case.kv, case.idx, scale=case.scale, Dv=case.Dv, v=case.v,
+                          sinks=case.sinks)
         rows = np.asarray(rows)
         return sparse(case.q[rows], case.kv, case.idx[rows], scale=case.scale, Dv=case.Dv,
-                      v=case.v)
+                      v=case.v, sinks=case.sinks)
     if isinstance(case, W.DecodeCase):
         return decode_q(case)
     if isinstance(case, W.MergeCase):

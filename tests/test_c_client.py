@@ -1,7 +1,7 @@
 """The boundary is a C ABI: a plain C program, compiled against include/arc_attn.h
 and linked to the built library with no Python or torch in between, plans the
-GQA prefill and the quantised decode, sizes a decode workspace, and gets the
-documented validation errors back (host logic only: nothing is launched)."""
+GQA prefill and the quantised decode, sizes a decode workspace, asks for the
+library's default softmax scale by flag, and gets the documented validation errors back (host logic only: nothing is launched)."""
 import os
 import subprocess
 import tempfile
@@ -11,6 +11,7 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 CLIENT = r"""
+#include <math.h>
 #include <stdio.h>
 #include <string.h>
 #include "arc_attn.h"
@@ -34,6 +35,15 @@ int main(void)
     memset(&info, 0, sizeof info);
     if (arc_plan(ARC_OP_ATTN, &a, &info) != ARC_OK) return 2;
     printf("attn %s tensor_cores=%d tile_m=%d d_slice=%d\n", info.kernel, info.tensor_cores, info.tile_m, info.d_slice);
+
+    /* ARC_FLAG_DEFAULT_SCALE: the library takes 1/sqrt(D) and ignores the field, so
+       even a NaN there is accepted; without the flag a NaN scale is refused */
+    a.scale = NAN;
+    if (arc_plan(ARC_OP_ATTN, &a, &info) != ARC_ERR_INVALID_ARG) return 6;
+    a.flags = ARC_FLAG_DEFAULT_SCALE;
+    if (arc_plan(ARC_OP_ATTN, &a, &info) != ARC_OK) return 7;
+    a.flags = 0;
+    a.scale = 0.044194173f;
 
     a.Hkv = 7;                                   /* 64 heads do not divide over 7 kv heads */
     if (arc_attn_fwd(&a, NULL) != ARC_ERR_INVALID_ARG) return 3;
@@ -66,7 +76,7 @@ def test_plain_c_client_plans_and_validates():
         src, exe = os.path.join(d, "client.c"), os.path.join(d, "client")
         open(src, "w").write(CLIENT)
         subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src,
-                               "-o", exe, "-L", libdir, "-larc_attn", "-Wl,-rpath," + libdir])
+                               "-o", exe, "-L", libdir, "-larc_attn", "-lm", "-Wl,-rpath," + libdir])
         r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, (r.returncode, r.stdout, r.stderr)
     lines = r.stdout.splitlines()

@@ -1,16 +1,19 @@
-"""The allocation-free decode entry point, against the workspace entry point.
+"""The allocation-free decode entry point, against the oracle and the workspace entry point.
 
 arc_attn_decode_q8_noalloc serves callers that cannot call cudaMalloc (an
 engine whose planner owns all device memory, a fixed memory budget): it keeps
 its split-KV partials in the library's own static 8 MiB device buffer.  These
-checks call it through the C ABI and compare it with arc_attn_decode_q8 fed a
-caller workspace, over consecutive calls that reuse the shared buffer.  The
-file name sorts last so a stop-at-first-failure run has run everything else.
+checks call it through the C ABI, twice in a row on the shared buffer, and
+compare each result element by element with the fp64 oracle and with
+arc_attn_decode_q8 fed a caller workspace.  The cases reach every decode
+kernel: the TMA split kernel, the cp.async split kernel (a cell stride that is
+not a multiple of 16 bytes) and the CUDA-core kernel (head dim 256).  The file
+name sorts last so a stop-at-first-failure run has run everything else.
 """
-import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads as W
 import exact_attention_131_b200 as arc
 from tests._util import TOL_LSE, TOL_O_BF16, compare, dev, host
@@ -27,21 +30,55 @@ def _kw(c):
                 n_kv=c.n_kv, scale=c.scale)
 
 
-def test_noalloc_decode_matches_workspace_entry_on_consecutive_calls():
-    cases = [W.config(5, kv_type=W.KV_Q8_0), W.config(5, kv_type=W.KV_Q4_0),
-             W.decode_case(3, 2, 0, 16, 4, 64, kv_type=W.KV_Q8_0, seed=41, n_q_list=[2, 4, 1],
-                           n_kv_list=[900, 33, 5])]
-    for c in cases:
-        q, kc, vc = _inputs(c)
-        o_ref, l_ref = arc.attn_decode_q8(q, kc, vc, **_kw(c))
+CASES = {
+    "c5-q8_0": lambda: W.config(5, kv_type=W.KV_Q8_0),
+    "c5-q4_0": lambda: W.config(5, kv_type=W.KV_Q4_0),
+    "d64-ragged": lambda: W.decode_case(3, 2, 0, 16, 4, 64, kv_type=W.KV_Q8_0, seed=41, n_q_list=[2, 4, 1],
+                                        n_kv_list=[900, 33, 5]),
+    "cp_async-path": lambda: W.decode_case(3, 2, 700, 6, 3, 128, kv_type=W.KV_Q4_0, seed=44),
+    "d256-cuda-cores": lambda: W.decode_case(2, 0, 0, 8, 2, 256, kv_type=W.KV_Q8_0, seed=45, n_q_list=[2, 1],
+                                             n_kv_list=[300, 77]),
+}
+KERNELS = {"c5-q8_0": "decode_ws_kernel", "c5-q4_0": "decode_ws_kernel", "d64-ragged": "decode_ws_kernel",
+           "cp_async-path": "decode_split_kernel", "d256-cuda-cores": "simple_decode_kernel"}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_noalloc_decode_matches_oracle_and_workspace_entry_on_consecutive_calls(name):
+    c = CASES[name]()
+    q, kc, vc = _inputs(c)
+    info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                           n_kv=c.n_kv)
+    assert info["kernel"].startswith(KERNELS[name])
+    ro, rl = oracle.run_case(c)
+    o_ws, l_ws = arc.attn_decode_q8(q, kc, vc, **_kw(c))
+    torch.cuda.synchronize()
+    compare(o_ws, l_ws, ro, rl, TOL_O_BF16, TOL_LSE)
+    for _ in range(2):                      # two calls in a row on the shared buffer
+        o = torch.full_like(o_ws, float("nan"))
+        lse = torch.full_like(l_ws, float("nan"))
+        arc.attn_decode_q8_noalloc(q, kc, vc, out=o, lse=lse, **_kw(c))
         torch.cuda.synchronize()
-        ro, rl = host(o_ref), host(l_ref)
-        for _ in range(2):                      # two calls in a row on the shared buffer
-            o = torch.full_like(o_ref, float("nan"))
-            lse = torch.full_like(l_ref, float("nan"))
-            arc.attn_decode_q8_noalloc(q, kc, vc, out=o, lse=lse, **_kw(c))
-            torch.cuda.synchronize()
-            compare(o, lse, ro, rl, TOL_O_BF16, TOL_LSE)
+        compare(o, lse, ro, rl, TOL_O_BF16, TOL_LSE)
+        compare(o, lse, host(o_ws), host(l_ws), TOL_O_BF16, TOL_LSE)
+
+
+def test_noalloc_decode_takes_no_device_memory():
+    """With out / lse passed in, a call changes the device's free memory by nothing:
+    no allocation happens on either side of the C ABI."""
+    c = W.config(5, kv_type=W.KV_Q8_0)
+    q, kc, vc = _inputs(c)
+    o = torch.empty(c.n_tok, c.H, c.D, device="cuda")
+    lse = torch.empty(c.n_tok, c.H, device="cuda")
+    arc.attn_decode_q8_noalloc(q, kc, vc, out=o, lse=lse, **_kw(c))      # first call: address lookup
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        arc.attn_decode_q8_noalloc(q, kc, vc, out=o, lse=lse, **_kw(c))
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16, TOL_LSE)
 
 
 def test_noalloc_decode_rejects_calls_beyond_its_buffer():

@@ -189,6 +189,7 @@ class SparseCase:
     idx: np.ndarray         # [Sq,topk] int32, -1 = padding
     v: np.ndarray | None = None
     seed: int = 0
+    sinks: np.ndarray | None = None   # [H] fp32
 
 
 def sparse_indices(rng, Sq, Skv, topk, pad_frac=0.05, pad_mode="random") -> np.ndarray:
@@ -222,13 +223,15 @@ def sparse_indices(rng, Sq, Skv, topk, pad_frac=0.05, pad_mode="random") -> np.n
 
 
 def sparse_case(Sq, H, Skv, Dqk=512, Dv=512, topk=2176, *, std=0.3, pad_frac=0.05,
-                pad_mode="random", separate_v=False, seed=0) -> SparseCase:
+                pad_mode="random", separate_v=False, sinks=False, seed=0) -> SparseCase:
     rng = make_rng(seed)
     q = bf16_bits(normal(rng, (Sq, H, Dqk), std))
     kv = bf16_bits(normal(rng, (Skv, Dqk), std))
     v = bf16_bits(normal(rng, (Skv, Dv), std)) if separate_v else None
     idx = sparse_indices(rng, Sq, Skv, topk, pad_frac, pad_mode)
-    return SparseCase(Sq, H, Skv, Dqk, Dv, topk, float(1.0 / math.sqrt(Dqk)), q, kv, idx, v, seed)
+    # drawn last, so a case without sinks is unchanged by the option
+    s = normal(rng, (H,), 1.0).astype(np.float32) if sinks else None
+    return SparseCase(Sq, H, Skv, Dqk, Dv, topk, float(1.0 / math.sqrt(Dqk)), q, kv, idx, v, seed, s)
 
 
 @dataclass
