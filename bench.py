@@ -7,7 +7,8 @@ sinks (B=1, H=64 over Hkv=8, T=1400 causal, D=512, bf16) -- the configuration
 the headline metric is quoted on.  Other workloads: --config c1 c3 c4 c5q8 c5q4.
 
 Timing: W untimed warm-up steps, then K steps; before each timed step a
-256 MiB buffer is written to flush L2 (outside the timed interval), and the
+256 MiB buffer is written and another 256 MiB read to flush L2 (outside the
+timed interval, leaving no dirty line behind), and the
 step is bracketed by CUDA events on the launching stream.  A single-GPU run
 also times every other graded workload (c2, c3, c4, c5q8, c5q4) in the same
 way, each on a loop of at least --per-config-wall seconds so the clock sampler
@@ -346,8 +347,29 @@ def job_throughput(units_per_step, world, steps, total_ms, unit_kind):
     return units_per_step * world * steps / (total_ms * 1e-3) / scale
 
 
+class L2Flush:
+    """Evicts the timed call's data from the 126 MB L2 before each timed step: a 256 MiB
+    write, then (mode "write+read") a 256 MiB read of another buffer.  The read leaves
+    L2 holding clean lines only; after the write alone it holds dirty lines, whose
+    write-back the next step's own reads would then pay for in the timed interval."""
+
+    def __init__(self, torch, mode):
+        self.mode = mode
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+        self.rd = torch.ones(64 << 20, dtype=torch.float32, device="cuda") if mode == "write+read" else None
+
+    def __call__(self, i):
+        self.buf.fill_(i & 0xFF)
+        if self.rd is not None:
+            self.rd.sum()
+
+    def describe(self):
+        return ("flushed before every timed step: 256 MiB write, then 256 MiB read (no dirty line left)"
+                if self.rd is not None else "flushed (256 MiB write) before every timed step")
+
+
 def time_steps(call, steps, stream, flush, local, graph=None):
-    """Device time of `steps` calls: a 256 MiB write flushes L2 before each, CUDA events on
+    """Device time of `steps` calls: L2 is flushed before each, CUDA events on
     the launching stream bracket the call only.  With `graph`, each step replays it instead
     of calling.  Returns (per-step ms list, wall seconds of the loop, clock record)."""
     import torch
@@ -357,7 +379,7 @@ def time_steps(call, steps, stream, flush, local, graph=None):
     with sampler:
         wall0 = time.perf_counter()
         for i in range(steps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             ev[i][0].record(stream)
             if graph is None:
                 call()
@@ -427,7 +449,8 @@ def measure_config(key, status, stream, flush, local, peaks, min_wall_s):
     rec = {"workload": spec["name"], "metric": spec["metric"], "value": units / (mean_ms * 1e-3) / scale,
            "unit": "TFLOP/s" if unit_kind == "flop" else "GB/s", "ms_per_step": mean_ms, "steps": steps,
            "dtype": spec["dtype"], "roofline": roofline(units, unit_kind, mean_ms, peaks, key, info["kernel"]),
-           "clocks": clocks, "wall_s_timed_region": wall, "gpu_launches": int(info["launches"]) * steps}
+           "clocks": clocks, "wall_s_timed_region": wall, "gpu_launches": int(info["launches"]) * steps,
+           "l2": flush.describe()}
     if isinstance(case, W.DecodeCase):
         g = capture(call, stream)
         for _ in range(5):
@@ -470,7 +493,7 @@ def run_ours(args, spec, case):
     call, ins, outs, info = build_call(case, torch, arc, status)
     units, unit_kind = work(case)
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = L2Flush(torch, args.flush)
 
     for _ in range(args.warmup):
         call()
@@ -492,7 +515,7 @@ def run_ours(args, spec, case):
     d2h = sum(o.numel() * o.element_size() for o in host_outs)
     e2e_ms = []
     for i in range(0 if args.no_e2e else max(3, min(args.steps, 20)) + 2):
-        flush.fill_(i & 0xFF)
+        flush(i)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for kname, hv in host_ins.items():
@@ -520,7 +543,7 @@ def run_ours(args, spec, case):
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": spec["dtype"], "data": "synthetic",
         "config": {"workload": spec["name"], "config": args.config, "seed": spec["cfg"],
-                   "l2": "flushed (256 MiB write) before every timed step",
+                   "l2": flush.describe(),
                    "parallelism": f"replicas x{world}, no collective" if world > 1 else "single GPU"},
         "roofline": roof,
         "e2e": {"value": e2e_val, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -610,6 +633,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg (for profiler runs)")
     ap.add_argument("--no-per-config", action="store_true", help="time the --config workload only")
+    ap.add_argument("--flush", choices=["write", "write+read"], default="write+read",
+                    help="how L2 is flushed before each timed step")
     ap.add_argument("--per-config-wall", type=float, default=1.5,
                     help="seconds each extra graded workload's timed loop lasts at least")
     args = ap.parse_args()

@@ -17,12 +17,6 @@
 
 using namespace arc;
 
-namespace arc {
-int decode_smem_bytes(int kv_type, int D, bool tma);
-int decode_blocks_per_sm(int kv_type, int D, bool tma);
-int decode_box_bytes(int kv_type, int D);
-}
-
 namespace {
 
 constexpr int kTcBM = 128, kTcBN = 128;
@@ -432,7 +426,9 @@ bool plan_sparse_tc(const arc_sparse_args *a)
 struct DecodePlan {
     bool simple = false;
     bool tma = false;   // shape allows the TMA ring (cell stride a multiple of 16 bytes)
-    int splits = 0, chunk = 0, max_kv = 0;
+    int mf = 1;         // m16 fragments of fold rows per CTA
+    int row_groups = 1; // CTAs along the fold rows of one (sequence, kv head)
+    int splits = 0, chunk = 0, max_kv = 0, max_rows = 0;
     size_t ws = 0;
 };
 
@@ -451,7 +447,7 @@ arc_status check_decode(const arc_decode_args *a, bool need_ptrs = true)
         if (q.n_q < 0 || q.n_kv < q.n_q || q.q_begin < 0 || q.kv_begin < 0) return ARC_ERR_INVALID_ARG;
         if ((int64_t)q.q_begin + q.n_q > a->n_tok || (int64_t)q.kv_begin + q.n_kv > a->n_cells)
             return ARC_ERR_INVALID_ARG;
-        if (G * q.n_q > 16) return ARC_ERR_UNSUPPORTED;
+        if (G * q.n_q > ARC_DECODE_MAX_ROWS) return ARC_ERR_UNSUPPORTED;
     }
     if (need_ptrs && a->n_seq > 0 && a->n_tok > 0) {
         if (!scale_ok(a->flags, a->scale)) return ARC_ERR_INVALID_ARG;
@@ -466,20 +462,28 @@ arc_status check_decode(const arc_decode_args *a, bool need_ptrs = true)
 DecodePlan plan_decode(const arc_decode_args *a)
 {
     DecodePlan pl;
-    // head dims 256 / 512 run on the CUDA-core kernel: the register-direct split
-    // kernel holds a 16-row x D fp32 accumulator and one head row per TMA box only up to D = 128
-    pl.simple = (a->flags & ARC_FLAG_FORCE_SIMPLE) != 0 || a->D > 128;
-    for (int s = 0; s < a->n_seq; ++s) pl.max_kv = std::max(pl.max_kv, a->seqs[s].n_kv);
-    if (pl.simple || pl.max_kv == 0) return pl;
-    const int pairs = a->n_seq * a->Hkv;
+    const int G = a->H / a->Hkv;
+    for (int s = 0; s < a->n_seq; ++s) {
+        pl.max_kv = std::max(pl.max_kv, a->seqs[s].n_kv);
+        pl.max_rows = std::max(pl.max_rows, G * a->seqs[s].n_q);
+    }
     const int64_t cell_bytes = (int64_t)a->Hkv * (a->D / 32) * (a->kv_type == ARC_KV_Q8_0 ? 34 : 18);
     pl.tma = cell_bytes % 16 == 0;
+    // The split kernels: the TMA one for every head dim and up to ARC_DECODE_MAX_ROWS fold
+    // rows (row groups of 16 or 32); the cp.async one (cell strides that are not 16-byte
+    // multiples) for D <= 128 and one 16-row fragment.  Everything else, and
+    // ARC_FLAG_FORCE_SIMPLE, runs the CUDA-core kernel.
+    pl.simple = (a->flags & ARC_FLAG_FORCE_SIMPLE) != 0 || (!pl.tma && (a->D > 128 || pl.max_rows > 16));
+    if (pl.simple || pl.max_kv == 0) return pl;
+    pl.mf = (pl.max_rows > 16 && decode_ws_supported(a->kv_type, a->D, 2) && pl.tma) ? 2 : 1;
+    pl.row_groups = (pl.max_rows + 16 * pl.mf - 1) / (16 * pl.mf);
+    const int pairs = a->n_seq * a->Hkv * pl.row_groups;
     // One wave: as many CTAs as the SMs hold at once.  The occupancy API counts
     // registers as well as shared memory (the warp-specialised kernel is register-
     // limited to 3 CTAs per SM even where its stages would leave room for a fourth);
     // without a device, the shared-memory estimate.
-    const int smem = decode_smem_bytes(a->kv_type, a->D, pl.tma);
-    const int occ = decode_blocks_per_sm(a->kv_type, a->D, pl.tma);
+    const int smem = decode_smem_bytes(a->kv_type, a->D, pl.mf, pl.tma);
+    const int occ = decode_blocks_per_sm(a->kv_type, a->D, pl.mf, pl.tma);
     const int per_sm = occ > 0 ? std::min(4, occ) : std::max(1, std::min(4, (228 * 1024) / (smem + 1024)));
     const int target = sm_count() * per_sm;
     int splits = std::min(256, std::max(1, target / std::max(1, pairs)));
@@ -488,7 +492,7 @@ DecodePlan plan_decode(const arc_decode_args *a)
     splits = (pl.max_kv + chunk - 1) / chunk;
     pl.splits = splits;
     pl.chunk = chunk;
-    pl.ws = (size_t)pairs * splits * 16 * (a->D + 2) * sizeof(float);
+    pl.ws = (size_t)pairs * splits * 16 * pl.mf * (a->D + 2) * sizeof(float);
     return pl;
 }
 
@@ -715,13 +719,14 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
         DecodeParams p{};
         p.kv_type = a->kv_type, p.n_tok = a->n_tok, p.H = a->H, p.Hkv = a->Hkv, p.D = a->D, p.n_seq = a->n_seq;
         p.splits = pl.splits, p.chunk = pl.chunk;
+        p.mf = pl.mf, p.rows = 16 * pl.mf, p.row_groups = pl.row_groups;
         p.q = a->q, p.k_cache = static_cast<const uint8_t *>(a->k_cache);
         p.v_cache = static_cast<const uint8_t *>(a->v_cache);
         memcpy(p.seqs, a->seqs, sizeof(arc_seq) * a->n_seq);
         p.o = a->o, p.lse = a->lse;
-        const size_t parts = (size_t)a->n_seq * a->Hkv * pl.splits;
+        const size_t parts = (size_t)a->n_seq * a->Hkv * pl.row_groups * pl.splits;
         p.ws_o = static_cast<float *>(workspace);
-        p.ws_ml = p.ws_o + parts * 16 * a->D;
+        p.ws_ml = p.ws_o + parts * p.rows * a->D;
         p.scale_log2 = call_scale(a->flags, a->scale, a->D) * kLog2e;
         p.status = a->status;
         // K/V tiles by TMA when the cache rows allow it: a byte tensor {cell bytes, n_cells} per cache.
@@ -729,15 +734,27 @@ arc_status arc_attn_decode_q8(const arc_decode_args *a, void *workspace, size_t 
                 (reinterpret_cast<uintptr_t>(a->v_cache) & 15) == 0;
         if (p.tma) {
             const int64_t cell_bytes = (int64_t)a->Hkv * (a->D / 32) * (a->kv_type == ARC_KV_Q8_0 ? 34 : 18);
-            const uint32_t box_w = (uint32_t)decode_box_bytes(a->kv_type, a->D);
-            if (!make_map_bytes_cached(&p.tm_kc, a->k_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64) ||
-                !make_map_bytes_cached(&p.tm_vc, a->v_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, 64))
+            int box_w = 0, box_cells = 0;
+            decode_box(a->kv_type, a->D, pl.mf, &box_w, &box_cells);
+            if (box_w <= 0 ||
+                !make_map_bytes_cached(&p.tm_kc, a->k_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, box_cells) ||
+                !make_map_bytes_cached(&p.tm_vc, a->v_cache, (uint64_t)cell_bytes, (uint64_t)a->n_cells, box_w, box_cells))
                 return ARC_ERR_CUDA;
-        }
-        if (p.tma)
             note_dispatch(a->kv_type == ARC_KV_Q8_0 ? "decode_ws_kernel<q8_0>" : "decode_ws_kernel<q4_0>");
-        else
+        } else if (a->D <= 128 && pl.max_rows <= 16) {
             note_dispatch(a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
+        } else {
+            // the shape allows TMA but these caches are not 16-byte aligned: the CUDA-core kernel
+            SimpleDecodeParams q{};
+            q.kv_type = a->kv_type, q.n_tok = a->n_tok, q.H = a->H, q.Hkv = a->Hkv, q.D = a->D;
+            q.n_cells = a->n_cells, q.n_seq = a->n_seq;
+            q.q = a->q, q.k_cache = static_cast<const uint8_t *>(a->k_cache);
+            q.v_cache = static_cast<const uint8_t *>(a->v_cache);
+            memcpy(q.seqs, a->seqs, sizeof(arc_seq) * a->n_seq);
+            q.o = a->o, q.lse = a->lse, q.scale = call_scale(a->flags, a->scale, a->D);
+            note_dispatch("simple_decode_kernel");
+            return launch_simple_decode(q, s) == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+        }
         e = launch_decode(p, s);
     }
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
@@ -944,14 +961,24 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             // the TMA kernel needs 16-byte aligned caches; arc_plan reports the shape's choice
             const bool tma = pl.tma && (reinterpret_cast<uintptr_t>(a->k_cache) & 15) == 0 &&
                              (reinterpret_cast<uintptr_t>(a->v_cache) & 15) == 0;
-            if (tma)
+            if (!tma && (a->D > 128 || pl.max_rows > 16)) {
+                set_name(out, "simple_decode_kernel");
+                out->launches = 1;
+                return ARC_OK;
+            }
+            int box_w = 0, box_cells = 64;
+            if (tma) {
                 set_name(out, a->kv_type == ARC_KV_Q8_0 ? "decode_ws_kernel<q8_0>" : "decode_ws_kernel<q4_0>");
-            else
+                decode_box(a->kv_type, a->D, pl.mf, &box_w, &box_cells);
+            } else {
                 set_name(out, a->kv_type == ARC_KV_Q8_0 ? "decode_split_kernel<q8_0>" : "decode_split_kernel<q4_0>");
+            }
             out->tensor_cores = 1;
-            out->tile_m = 16, out->tile_n = 32, out->d_slice = a->D;
-            out->splits = pl.splits, out->n_ctas = a->n_seq * a->Hkv * pl.splits;
-            out->smem_bytes = decode_smem_bytes(a->kv_type, a->D, tma);
+            // tile_m: fold rows per CTA; tile_n: cells per tile; d_slice: head dims one warp covers
+            out->tile_m = 16 * pl.mf, out->tile_n = box_cells;
+            out->d_slice = tma ? a->D / std::max(1, (a->D * pl.mf) / 128) : a->D;
+            out->splits = pl.splits, out->n_ctas = a->n_seq * a->Hkv * pl.row_groups * pl.splits;
+            out->smem_bytes = decode_smem_bytes(a->kv_type, a->D, pl.mf, tma);
             out->launches = 2;
         }
         return ARC_OK;

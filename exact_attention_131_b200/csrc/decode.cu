@@ -484,12 +484,25 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+
 // ---------------------------------------------------------------------------
-// Warp-specialised split kernel (TMA path).  Warp 4 streams raw K/V tiles of 64
-// cells into a ring of NST stages; each of warps 0-3 owns 16 cells of every
-// tile and builds its mma.sync operands straight from the raw bytes, in
-// registers: no f16 copy of the tile is ever written, so shared memory carries
-// only the TMA writes, one read of each raw byte and the Q fragments.
+// Warp-specialised split kernel (TMA path).  Warp 4 streams raw K/V tiles into
+// a ring of NST stages; warps 0-3 build their mma.sync operands straight from
+// the raw bytes, in registers: no f16 copy of a tile is ever written, so shared
+// memory carries only the TMA writes, one read of each raw byte and Q.
+//
+// Shapes.  A CTA takes ROWS = 16*MF fold rows (MF m16 fragments) of one
+// (sequence, kv head, row group, chunk).  The head dim is cut into NS slices of
+// KS = D/NS dims, so that one warp's O accumulators (MF x KS/2 floats a lane)
+// stay at or under 64 registers; the 4 consumer warps are NCG = 4/NS cell
+// groups x NS slices, and a tile holds DT = 16*NCG cells.  Warp (cg, s) owns the
+// 16 cells cg*16.. of every tile and the dims of slice s, for K as for V:
+//   S  = Q K^T: the warp's partial over its slice's dims; the NS partials of a
+//        cell group are summed through shared memory in slice order, so every
+//        warp of the group holds the same S and runs the same online softmax;
+//   O += P V:   the warp's slice of the output dims.
+// Every raw byte is dequantised once.  With NS = 1 (D <= 128, MF = 1; the
+// multi-sequence decode) there is no exchange and a tile has 64 cells.
 //
 // Dim permutations.  A dot product does not change when the same permutation
 // is applied to the head dim of both operands, so S = Q K^T takes the k-step
@@ -500,22 +513,46 @@ __global__ void __launch_bounds__(WARPS * 32) decode_split_kernel(const __grid_c
 // nibbles of four consecutive bytes (q4_0), so each B fragment register pair
 // comes from one 32-bit word; the Q fragments are read from shared memory in
 // the same order.  For O += P V the n index is the output dim: lane group g
-// loads dims D/8*g .. D/8*g + D/8 - 1 (consecutive bytes again) and n-tile nd
-// column c accumulates dim D/8*c + nd, which write_cta_partial<.., true> undoes.
+// loads slice dims KS/8*g .. KS/8*g + KS/8 - 1 (consecutive bytes again, inside
+// one block) and n-tile nd column c accumulates slice dim KS/8*c + nd, which the
+// in-CTA merge undoes.
 constexpr int WS_WARPS = 5;
 
-template <int KVT, int D>
+template <int D, int MF>
+struct WsShape {
+    static constexpr int NS = (D * MF) / 128 < 1 ? 1 : (D * MF) / 128;   // dim slices
+    static constexpr int NCG = 4 / NS;                                      // cell groups
+    static constexpr int KS = D / NS;                                       // dims per slice
+    static constexpr int DT = 16 * NCG;                                     // cells per tile
+    static constexpr int ROWS = 16 * MF;                                    // fold rows per CTA
+    static_assert(NS * NCG == 4 && KS % 32 == 0, "four consumer warps over whole blocks");
+    static_assert(MF * KS <= 128, "O accumulators of a warp stay within 64 registers");
+};
+
+template <int KVT, int D, int MF>
 struct WsLayout {
+    using S = WsShape<D, MF>;
     static constexpr int BB = Fmt<KVT>::BB;
-    static constexpr int ROWB = (D / 32) * BB;
-    static constexpr int RS = ((ROWB + 16 - gcd16(ROWB) + 15) / 16) * 16;   // smem row stride of a raw tile
-    static constexpr int RAW = DT * RS;
-    static constexpr int NST = KVT == ARC_KV_Q8_0 ? 3 : 4;          // stages in flight; three CTAs per SM fit
-    static constexpr int QS = D + 16;                                 // Q row stride (halfs): 8-byte fragment reads hit distinct banks
-    static constexpr int QB = 16 * QS * 2;                            // Q tile (f16, pre-scaled)
-    static constexpr int MAIN = NST * 2 * RAW + QB;
-    static constexpr int MERGE = MergeLayout<D>::BYTES;
+    static constexpr int ROWB = (D / 32) * BB;                              // raw bytes of a head row
+    static constexpr int SB = (S::KS / 32) * BB;                            // raw bytes of one slice of it
+    // smem row stride of a slice box: the box starts at the 16-byte boundary at or
+    // below the slice (at most 16 - gcd(SB, 16) bytes earlier) and covers it
+    static constexpr int RS = ((SB + 16 - gcd16(SB) + 15) / 16) * 16;
+    static constexpr int SLICE = S::DT * RS;                                // one K (or V) slice box
+    static constexpr int STAGE = S::NS * 2 * SLICE;                         // [slice][K, V] of one tile
+    static constexpr int NST = STAGE >= 16384 ? 3 : 4;                      // stages in flight; three CTAs per SM fit
+    static constexpr int QS = D + 16;                                       // Q row stride (halfs)
+    static constexpr int QB = S::ROWS * QS * 2;                             // Q tile (f16, pre-scaled)
+    static constexpr int XB = S::NS > 1 ? 2 * S::NCG * S::NS * MF * 32 * 8 * 4 : 0;   // S partials, 2 buffers
+    static constexpr int MAIN = NST * STAGE + QB + XB;
+    // in-CTA merge: per cell group O [ROWS][OS] with OS = D + 8*NS (a skew of up to 6
+    // floats per slice), row (max, sum), weights; merged (max, sum)
+    static constexpr int OS = D + 8 * S::NS;
+    static constexpr int MERGE = (S::NCG * S::ROWS * OS + S::NCG * S::ROWS * 3 + S::ROWS * 2) * 4;
     static constexpr int BYTES = (MAIN > MERGE ? MAIN : MERGE) + 128 + 128;  // + barriers, alignment
+    static_assert(RS <= 256, "one TMA box per slice row");
+    static_assert(ROWB % 4 == 0 && SB % 4 == 0, "slice rows start 4-byte aligned in shared memory");
+    static_assert(STAGE % 128 == 0 && SLICE % 128 == 0, "TMA destinations stay 128-byte aligned");
 };
 
 ARC_DEV uint2 lds_u64(const void *p) { return *reinterpret_cast<const uint2 *>(p); }
@@ -540,8 +577,8 @@ ARC_DEV __half2 raw_scale(const uint8_t *row)
     return bits_h2(__byte_perm(lds_u32(row + (OFF & ~3)), 0u, (OFF & 2) ? 0x3232u : 0x1010u));
 }
 
-// The B fragments of K block B for the lane with quad index t: kf[hh] = {b0, b1}
-// of k-step 2B + hh (dims 32B + 16hh + 4t .. +3 of this cell).
+// The B fragments of K block B (of the slice row `row`) for the lane with quad index
+// t: kf[hh] = {b0, b1} of k-step 2B + hh (dims 32B + 16hh + 4t .. +3 of this cell).
 template <int KVT, int B>
 ARC_DEV void k_block_frags(const uint8_t *row, int t, uint32_t (&kf)[2][2])
 {
@@ -566,87 +603,185 @@ ARC_DEV void k_block_frags(const uint8_t *row, int t, uint32_t (&kf)[2][2])
     }
 }
 
-// One V cell as this lane needs it: the D/8 dims starting at D/8*g (NW data
-// words, realigned) and the word holding that block's scale (0 past the end of
-// the chunk, which zeroes the cell: its data bytes are finite integers).
-template <int KVT, int D>
+// One V cell as this lane needs it: the KS/8 slice dims starting at KS/8*g (NW data
+// words, realigned) and the word holding that block's scale (0 past the end of the
+// chunk, which zeroes the cell: its data bytes are finite integers).
+template <int KVT, int KS>
 struct VCell {
-    static constexpr int NW = D / 32;   // D/8 bytes (q8_0) or nibbles in D/8 bytes' halves (q4_0), as words
+    static constexpr int NW = KS / 32;   // KS/8 bytes (q8_0) or nibbles in KS/8 bytes' halves (q4_0), as words
     uint32_t d[NW];
     uint32_t sw;
 };
 
-template <int KVT, int D>
-ARC_DEV void load_vcell(const uint8_t *row, int vbase, uint32_t vsel, int soff4, bool valid, VCell<KVT, D> &c)
+template <int KVT, int KS>
+ARC_DEV void load_vcell(const uint8_t *row, int vbase, uint32_t vsel, int soff4, bool valid, VCell<KVT, KS> &c)
 {
     const uint8_t *b = row + vbase;
-    uint32_t w[VCell<KVT, D>::NW + 1];
+    uint32_t w[VCell<KVT, KS>::NW + 1];
 #pragma unroll
-    for (int i = 0; i <= VCell<KVT, D>::NW; ++i) w[i] = lds_u32(b + 4 * i);
+    for (int i = 0; i <= VCell<KVT, KS>::NW; ++i) w[i] = lds_u32(b + 4 * i);
 #pragma unroll
-    for (int i = 0; i < VCell<KVT, D>::NW; ++i) c.d[i] = __byte_perm(w[i], w[i + 1], vsel);
+    for (int i = 0; i < VCell<KVT, KS>::NW; ++i) c.d[i] = __byte_perm(w[i], w[i + 1], vsel);
     c.sw = valid ? lds_u32(row + soff4) : 0u;
 }
 
-template <int KVT, int D>
-__global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __grid_constant__ DecodeParams p)
+// The decode workspace (and the combine kernel's view of it): partial results of
+// part = ((sequence * Hkv + kv head) * row_groups + row group) * splits + split,
+// ROWS = 16*MF fold rows each: O [part][ROWS][D] (unnormalised) and (max, sum)
+// [part][ROWS][2], in log2 units.
+ARC_DEV int64_t part_index(const DecodeParams &p, int s, int kvh, int rg, int sp)
 {
-    using L = WsLayout<KVT, D>;
-    constexpr int NB = D / 32;                        // blocks per row
-    constexpr int ND = D / 8;                         // P V n-tiles = dims per lane group
-    constexpr int NW = VCell<KVT, D>::NW;
+    return (((int64_t)s * p.Hkv + kvh) * p.row_groups + rg) * p.splits + sp;
+}
+
+// Merge the 4 consumer warps of a CTA into its one partial in the workspace: O of
+// cell group cg is weighted by exp2(m_cg - m) (the log-sum-exp merge of split
+// attention), slices are placed side by side.  Called by all threads of the CTA
+// after the main loop; the raw ring is idle by then and is overlaid.
+template <int KVT, int D, int MF>
+ARC_DEV void write_ws_partial(const float (&o)[MF][WsShape<D, MF>::KS / 8][4], const float (&m_r)[MF][2],
+                              const float (&l_r)[MF][2], int cg, int s, bool consumer, uint8_t *smem,
+                              const DecodeParams &p, int64_t part)
+{
+    using SH = WsShape<D, MF>;
+    using L = WsLayout<KVT, D, MF>;
+    constexpr int ND = SH::KS / 8, ROWS = SH::ROWS, NCG = SH::NCG, KS = SH::KS;
+    float *so = reinterpret_cast<float *>(smem);              // [NCG][ROWS][OS]
+    float *sml = so + NCG * ROWS * L::OS;                     // [NCG][ROWS][2]
+    float *swt = sml + NCG * ROWS * 2;                        // [NCG][ROWS]
+    const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    __syncthreads();   // every warp is past its last read of the ring this overlays
+    if (consumer) {
+        float *base = so + cg * ROWS * L::OS + s * (KS + 8);
+#pragma unroll
+        for (int f = 0; f < MF; ++f)
+#pragma unroll
+            for (int nd = 0; nd < ND; ++nd)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    // slice dims 2*ND*tq + nd and 2*ND*tq + ND + nd, skewed by 2*tq
+                    float *row = base + (f * 16 + g + 8 * hr) * L::OS;
+                    row[2 * ND * tq + nd + 2 * tq] = o[f][nd][2 * hr];
+                    row[2 * ND * tq + ND + nd + 2 * tq] = o[f][nd][2 * hr + 1];
+                }
+        if (s == 0 && tq == 0) {
+#pragma unroll
+            for (int f = 0; f < MF; ++f)
+#pragma unroll
+                for (int hr = 0; hr < 2; ++hr) {
+                    const int r = f * 16 + g + 8 * hr;
+                    sml[(cg * ROWS + r) * 2 + 0] = m_r[f][hr];
+                    sml[(cg * ROWS + r) * 2 + 1] = l_r[f][hr];
+                }
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < ROWS) {
+        const int r = threadIdx.x;
+        float mm = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < NCG; ++c) mm = fmaxf(mm, sml[(c * ROWS + r) * 2]);
+        const float ms = (mm == -INFINITY) ? 0.f : mm;
+        float ll = 0.f;
+#pragma unroll
+        for (int c = 0; c < NCG; ++c) {
+            const float mw = sml[(c * ROWS + r) * 2];
+            const float w = (mw == -INFINITY) ? 0.f : fast_exp2(mw - ms);
+            swt[c * ROWS + r] = w;
+            ll += w * sml[(c * ROWS + r) * 2 + 1];
+        }
+        *reinterpret_cast<float2 *>(p.ws_ml + (part * ROWS + r) * 2) = make_float2(mm, ll);
+    }
+    __syncthreads();
+    constexpr int D2 = D / 2;
+    for (int x = threadIdx.x; x < ROWS * D2; x += WS_WARPS * 32) {
+        const int r = x / D2, d = (x % D2) * 2;
+        const int sl = d / KS, dd = d % KS;
+        const int col = sl * (KS + 8) + dd + 2 * (dd / (KS / 4));
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < NCG; ++c) {
+            const float w = swt[c * ROWS + r];
+            const float2 v = *reinterpret_cast<const float2 *>(so + (c * ROWS + r) * L::OS + col);
+            acc.x += w * v.x, acc.y += w * v.y;
+        }
+        *reinterpret_cast<float2 *>(p.ws_o + (part * ROWS + r) * D + d) = acc;
+    }
+}
+
+// Three CTAs per SM with one fragment; with two, the second fragment's S and O
+// registers need the room of two CTAs per SM.
+template <int KVT, int D, int MF>
+__global__ void __launch_bounds__(WS_WARPS * 32, MF == 1 ? 3 : 2) decode_ws_kernel(const __grid_constant__ DecodeParams p)
+{
+    using SH = WsShape<D, MF>;
+    using L = WsLayout<KVT, D, MF>;
+    constexpr int NS = SH::NS, NCG = SH::NCG, KS = SH::KS, DT = SH::DT, ROWS = SH::ROWS;
+    constexpr int NB = KS / 32;                       // blocks per slice
+    constexpr int ND = KS / 8;                        // P V n-tiles = slice dims per lane group
+    constexpr int NW = VCell<KVT, KS>::NW;
 
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint8_t *smem = align_smem<128>(smem_raw);
-    uint8_t *raw = smem;                                            // [NST][K, V][RAW]
+    uint8_t *raw = smem;                                            // [NST][NS][K, V][SLICE]
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BYTES - 256);
     uint64_t *empty = full + L::NST;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, tq = lane & 3;
-    const int s = blockIdx.x / (p.Hkv * p.splits);
-    const int kvh = (blockIdx.x / p.splits) % p.Hkv;
+    const int s_idx = blockIdx.x / (p.Hkv * p.row_groups * p.splits);
+    const int kvh = (blockIdx.x / (p.row_groups * p.splits)) % p.Hkv;
+    const int rg = (blockIdx.x / p.splits) % p.row_groups;
     const int sp = blockIdx.x % p.splits;
-    const arc_seq sq = p.seqs[s];
+    const arc_seq sq = p.seqs[s_idx];
     const int G = p.H / p.Hkv;
     const int M = G * sq.n_q;
+    const int r0 = rg * ROWS;                     // first fold row of this CTA
+    if (r0 >= M) return;                          // a row group this sequence does not have (uniform)
     const int c_begin = sp * p.chunk;
     const int c_end = min(c_begin + p.chunk, sq.n_kv);
     const int n_tiles = c_end > c_begin ? (c_end - c_begin + DT - 1) / DT : 0;
-    const int pad = (L::ROWB * kvh) & 15;
-    const int x0 = L::ROWB * kvh - pad;
 
-    // Q tile loads, all in flight before anything waits on them: 16 fold rows x D
-    // fp32, QI float2 per consumer thread.
-    constexpr int QI = 16 * D / 2 / (WARPS * 32);
-    static_assert(QI * WARPS * 32 == 16 * D / 2, "Q tile split");
-    float2 qv[QI];
-#pragma unroll
-    for (int j = 0; j < QI; ++j) {
-        const int x = threadIdx.x + j * WARPS * 32;
+    // Q tile: ROWS fold rows x D fp32, QI float2 per consumer thread.  The first QP
+    // loads go out before anything waits (up to 8 a thread, so large tiles do not
+    // hold registers the accumulators need); the rest follow the barrier below.
+    constexpr int QI = ROWS * D / 2 / (4 * 32);
+    constexpr int QP = QI < 8 ? QI : 8;
+    static_assert(QI * 4 * 32 == ROWS * D / 2, "Q tile split");
+    auto q_load = [&](int j) {
+        const int x = threadIdx.x + j * 4 * 32;
         const int r = x / (D / 2), d = (x % (D / 2)) * 2;
-        qv[j] = make_float2(0.f, 0.f);
-        if (warp < WARPS && r < M) {
-            const int h = kvh * G + r / sq.n_q;
-            const int tok = sq.q_begin + r % sq.n_q;
-            qv[j] = __ldg(reinterpret_cast<const float2 *>(p.q + ((int64_t)tok * p.H + h) * D + d));
+        float2 v = make_float2(0.f, 0.f);
+        if (warp < 4 && r0 + r < M) {
+            const int h = kvh * G + (r0 + r) / sq.n_q;
+            const int tok = sq.q_begin + (r0 + r) % sq.n_q;
+            v = __ldg(reinterpret_cast<const float2 *>(p.q + ((int64_t)tok * p.H + h) * D + d));
         }
-    }
-
-    float o[ND][4];
+        return v;
+    };
+    float2 qv[QP];
 #pragma unroll
-    for (int i = 0; i < ND; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-    bool ok = true;
+    for (int j = 0; j < QP; ++j) qv[j] = q_load(j);
 
-    if (warp == WARPS) {
+    float o[MF][ND][4];
+#pragma unroll
+    for (int f = 0; f < MF; ++f)
+#pragma unroll
+        for (int i = 0; i < ND; ++i) o[f][i][0] = o[f][i][1] = o[f][i][2] = o[f][i][3] = 0.f;
+    float m_r[MF][2], l_r[MF][2];
+#pragma unroll
+    for (int f = 0; f < MF; ++f) m_r[f][0] = m_r[f][1] = -INFINITY, l_r[f][0] = l_r[f][1] = 0.f;
+    bool ok = true;
+    const int s = warp % NS, cg = warp / NS;       // this consumer warp's dim slice and cell group
+
+    if (warp == 4) {
         // =============================== producer
         // It initialises the stage barriers itself and only signals the consumers
         // (bar.arrive), so its first loads go out without waiting for the Q tile.
         if (lane == 0) {
             for (int i = 0; i < L::NST; ++i) {
                 mbar_init(&full[i], 1);
-                mbar_init(&empty[i], WARPS);
+                mbar_init(&empty[i], 4);
             }
             fence_mbar_init();
         }
@@ -657,26 +792,36 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
                 const int st = i % L::NST;
                 if (i >= L::NST) ok = mbar_wait_sleep(&empty[st], (uint32_t)((i / L::NST - 1) & 1));
                 if (!ok) break;
-                uint8_t *dk = raw + st * 2 * L::RAW;
-                mbar_arrive_expect_tx(&full[st], 2 * L::RAW);
+                uint8_t *dk = raw + st * L::STAGE;
+                mbar_arrive_expect_tx(&full[st], L::STAGE);
                 const int row = sq.kv_begin + c_begin + i * DT;
-                tma_load_2d(dk, &p.tm_kc, &full[st], x0, row);
-                tma_load_2d(dk + L::RAW, &p.tm_vc, &full[st], x0, row);
+#pragma unroll
+                for (int sl = 0; sl < NS; ++sl) {
+                    const int off = L::ROWB * kvh + L::SB * sl;
+                    const int x0 = off - (off & 15);
+                    tma_load_2d(dk + sl * 2 * L::SLICE, &p.tm_kc, &full[st], x0, row);
+                    tma_load_2d(dk + sl * 2 * L::SLICE + L::SLICE, &p.tm_vc, &full[st], x0, row);
+                }
             }
             if (!ok) report(p.status, ST_TIMEOUT_LOAD);
         }
     } else {
-        // =============================== consumer warp: 16 cells of each tile
-        __half *qs = reinterpret_cast<__half *>(smem + L::NST * 2 * L::RAW);
-        int row_t[2];
+        // =============================== consumer warp (cg, s): 16 cells of each tile, slice s
+        __half *qs = reinterpret_cast<__half *>(smem + L::NST * L::STAGE);
+        float4 *xbuf = reinterpret_cast<float4 *>(smem + L::NST * L::STAGE + L::QB);   // [2][NCG][NS][MF][2][32]
+        int row_t[MF][2];
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int r = g + 8 * hr;
-            row_t[hr] = (r < M) ? r % sq.n_q : -1;
-        }
-        // This lane's V dims D/8*g .. : block vb, first element ve of that block.  Offsets
-        // are from the head row's first byte (the row pointers below include the pad,
-        // a multiple of 4, so the word alignment of each offset is its own).
+        for (int f = 0; f < MF; ++f)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int r = r0 + f * 16 + g + 8 * hr;
+                row_t[f][hr] = (r < M) ? r % sq.n_q : -1;
+            }
+        // slice row offset inside its box row: a multiple of 4 (ROWB and SB are), so the
+        // row pointers below stay 4-byte aligned and each offset keeps its own alignment
+        const int pad = (L::ROWB * kvh + L::SB * s) & 15;
+        // This lane's V dims KS/8*g .. of the slice: block vb, first element ve of that
+        // block.  Offsets are from the slice row's first byte.
         const int vb = (ND * g) / 32, ve = (ND * g) % 32;
         const int voff = vb * L::BB + 2 + (KVT == ARC_KV_Q8_0 ? ve : (ve & 15));   // first data byte
         const int vbase = voff & ~3;
@@ -687,37 +832,39 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
         const int vsh = (KVT == ARC_KV_Q4_0 && ve >= 16) ? 4 : 0;  // q4_0: high nibbles hold elements 16..31
 
         asm volatile("bar.sync 2, %0;" ::"n"(WS_WARPS * 32) : "memory");   // stage barriers initialised
-        // Q tile, shared by the four warps: 16 fold rows x D, scaled into log2 units, f16.
+        // Q tile, shared by the four warps: ROWS fold rows x D, scaled into log2 units, f16.
 #pragma unroll
         for (int j = 0; j < QI; ++j) {
-            const int x = threadIdx.x + j * WARPS * 32;
+            const int x = threadIdx.x + j * 4 * 32;
             const int r = x / (D / 2), d = (x % (D / 2)) * 2;
-            *reinterpret_cast<__half2 *>(qs + r * L::QS + d) =
-                __floats2half2_rn(qv[j].x * p.scale_log2, qv[j].y * p.scale_log2);
+            const float2 v = j < QP ? qv[j < QP ? j : 0] : q_load(j);
+            *reinterpret_cast<__half2 *>(qs + r * L::QS + d) = __floats2half2_rn(v.x * p.scale_log2, v.y * p.scale_log2);
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(WARPS * 32) : "memory");   // consumer warps only
-        const __half *q0 = qs + g * L::QS + 4 * tq, *q1 = q0 + 8 * L::QS;
+        asm volatile("bar.sync 1, %0;" ::"n"(4 * 32) : "memory");   // consumer warps only
+        const __half *qrow = qs + g * L::QS + 4 * tq + s * KS;
 
         for (int i = 0; i < n_tiles; ++i) {
             const int st = i % L::NST;
             ok = mbar_wait(&full[st], (uint32_t)((i / L::NST) & 1)) && ok;
-            const int kw0 = i * DT + warp * 16;                    // first cell (chunk-relative) of this warp
+            const int kw0 = i * DT + cg * 16;                      // first cell (chunk-relative) of this warp
             const int valid = c_end - c_begin - kw0;               // cells of this warp inside the chunk
-            const uint8_t *kt = raw + st * 2 * L::RAW + warp * 16 * L::RS + pad;   // this warp's 16 K rows
-            const uint8_t *vt = kt + L::RAW;
+            const uint8_t *kt = raw + st * L::STAGE + s * 2 * L::SLICE + cg * 16 * L::RS + pad;   // this warp's 16 K rows
+            const uint8_t *vt = kt + L::SLICE;
 
             // ---- V words for cells 2t, 2t+1, 2t+8, 2t+9 (loaded early; used after the softmax)
-            VCell<KVT, D> vc[4];
+            VCell<KVT, KS> vc[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int cell = 2 * tq + (c & 1) + 8 * (c >> 1);
-                load_vcell<KVT, D>(vt + cell * L::RS, vbase, vsel, soff4, cell < valid, vc[c]);
+                load_vcell<KVT, KS>(vt + cell * L::RS, vbase, vsel, soff4, cell < valid, vc[c]);
             }
 
-            // ---- S = Q K^T over the permuted k order; cells g and g+8
-            float sacc[2][4];
+            // ---- S = Q K^T over the permuted k order of this slice; cells g and g+8
+            float sacc[MF][2][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+            for (int f = 0; f < MF; ++f)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) sacc[f][nt][0] = sacc[f][nt][1] = sacc[f][nt][2] = sacc[f][nt][3] = 0.f;
             const uint8_t *k0 = kt + g * L::RS, *k1 = k0 + 8 * L::RS;
             auto kstep = [&](auto bc) {
                 constexpr int B = decltype(bc)::value;
@@ -725,18 +872,47 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
                 k_block_frags<KVT, B>(k0, tq, kf0);
                 k_block_frags<KVT, B>(k1, tq, kf1);
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint2 a0 = lds_u64(q0 + 32 * B + 16 * hh), a1 = lds_u64(q1 + 32 * B + 16 * hh);
-                    const uint32_t a[4] = {a0.x, a1.x, a0.y, a1.y};
-                    mma16816(sacc[0], a, kf0[hh][0], kf0[hh][1]);
-                    mma16816(sacc[1], a, kf1[hh][0], kf1[hh][1]);
-                }
+                for (int f = 0; f < MF; ++f)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const __half *q0 = qrow + f * 16 * L::QS;
+                        const uint2 a0 = lds_u64(q0 + 32 * B + 16 * hh), a1 = lds_u64(q0 + 8 * L::QS + 32 * B + 16 * hh);
+                        const uint32_t a[4] = {a0.x, a1.x, a0.y, a1.y};
+                        mma16816(sacc[f][0], a, kf0[hh][0], kf0[hh][1]);
+                        mma16816(sacc[f][1], a, kf1[hh][0], kf1[hh][1]);
+                    }
             };
             kstep(std::integral_constant<int, 0>{});
-            kstep(std::integral_constant<int, 1>{});
+            if constexpr (NB > 1) kstep(std::integral_constant<int, (NB > 1 ? 1 : 0)>{});
             if constexpr (NB > 2) {
                 kstep(std::integral_constant<int, (NB > 2 ? 2 : 0)>{});
                 kstep(std::integral_constant<int, (NB > 2 ? 3 : 0)>{});
+            }
+            static_assert(NB == 1 || NB == 2 || NB == 4, "slices of 1, 2 or 4 blocks");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);                // V is in registers, K consumed: stage free
+
+            if constexpr (NS > 1) {
+                // ---- sum the NS slice partials of this cell group, in slice order
+                float4 *xb = xbuf + (((i & 1) * NCG + cg) * NS) * MF * 2 * 32;
+#pragma unroll
+                for (int f = 0; f < MF; ++f) {
+                    xb[((s * MF + f) * 2 + 0) * 32 + lane] = make_float4(sacc[f][0][0], sacc[f][0][1], sacc[f][0][2], sacc[f][0][3]);
+                    xb[((s * MF + f) * 2 + 1) * 32 + lane] = make_float4(sacc[f][1][0], sacc[f][1][1], sacc[f][1][2], sacc[f][1][3]);
+                }
+                asm volatile("bar.sync %0, %1;" ::"r"(3 + cg), "n"(NS * 32) : "memory");
+#pragma unroll
+                for (int f = 0; f < MF; ++f)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        float4 acc = xb[((0 * MF + f) * 2 + nt) * 32 + lane];
+#pragma unroll
+                        for (int s2 = 1; s2 < NS; ++s2) {
+                            const float4 v = xb[((s2 * MF + f) * 2 + nt) * 32 + lane];
+                            acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+                        }
+                        sacc[f][nt][0] = acc.x, sacc[f][nt][1] = acc.y, sacc[f][nt][2] = acc.z, sacc[f][nt][3] = acc.w;
+                    }
             }
 
             // Mask only where a key can fall past the chunk end or a row's causal
@@ -746,47 +922,52 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
             const int key0 = c_begin + kw0;
             if (key0 + 16 > c_end || key0 + 15 > sq.n_kv - sq.n_q) {
 #pragma unroll
-                for (int hr = 0; hr < 2; ++hr) {
-                    const int lim = row_t[hr] < 0 ? -1 : sq.n_kv - sq.n_q + row_t[hr];
+                for (int f = 0; f < MF; ++f)
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int hr = 0; hr < 2; ++hr) {
+                        const int lim = row_t[f][hr] < 0 ? -1 : sq.n_kv - sq.n_q + row_t[f][hr];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int key = key0 + nt * 8 + 2 * tq + e;
-                            if (key >= c_end || key > lim) sacc[nt][2 * hr + e] = -INFINITY;
-                        }
-                }
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int key = key0 + nt * 8 + 2 * tq + e;
+                                if (key >= c_end || key > lim) sacc[f][nt][2 * hr + e] = -INFINITY;
+                            }
+                    }
             }
             // Online softmax with a lazy rescale: the running max m_r moves (and O, l
             // are rescaled) only when a tile raises it by more than kLazy (log2 units);
             // otherwise p = exp2(s - m_r) <= 2^kLazy, which f16 and the f32 sums hold.
             // (m_r, l_r, O) stay one consistent partial either way.
             constexpr float kLazy = 8.f;
-            uint32_t pa[4];
+            uint32_t pa[MF][4];
 #pragma unroll
-            for (int hr = 0; hr < 2; ++hr) {
-                float mx = fmaxf(fmaxf(sacc[0][2 * hr], sacc[0][2 * hr + 1]), fmaxf(sacc[1][2 * hr], sacc[1][2 * hr + 1]));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                if (mx > m_r[hr] + kLazy) {   // also the first finite max (m_r = -inf)
-                    const float alpha = (m_r[hr] == -INFINITY) ? 0.f : fast_exp2(m_r[hr] - mx);
-                    m_r[hr] = mx;
-                    l_r[hr] *= alpha;
+            for (int f = 0; f < MF; ++f)
 #pragma unroll
-                    for (int i2 = 0; i2 < ND; ++i2) {
-                        o[i2][2 * hr] *= alpha;
-                        o[i2][2 * hr + 1] *= alpha;
+                for (int hr = 0; hr < 2; ++hr) {
+                    float mx = fmaxf(fmaxf(sacc[f][0][2 * hr], sacc[f][0][2 * hr + 1]),
+                                     fmaxf(sacc[f][1][2 * hr], sacc[f][1][2 * hr + 1]));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                    if (mx > m_r[f][hr] + kLazy) {   // also the first finite max (m_r = -inf)
+                        const float alpha = (m_r[f][hr] == -INFINITY) ? 0.f : fast_exp2(m_r[f][hr] - mx);
+                        m_r[f][hr] = mx;
+                        l_r[f][hr] *= alpha;
+#pragma unroll
+                        for (int i2 = 0; i2 < ND; ++i2) {
+                            o[f][i2][2 * hr] *= alpha;
+                            o[f][i2][2 * hr + 1] *= alpha;
+                        }
                     }
+                    const float msafe = (m_r[f][hr] == -INFINITY) ? 0.f : m_r[f][hr];
+                    const float p00 = fast_exp2(sacc[f][0][2 * hr] - msafe), p01 = fast_exp2(sacc[f][0][2 * hr + 1] - msafe);
+                    const float p10 = fast_exp2(sacc[f][1][2 * hr] - msafe), p11 = fast_exp2(sacc[f][1][2 * hr + 1] - msafe);
+                    l_r[f][hr] += (p00 + p01) + (p10 + p11);
+                    pa[f][hr] = h2_bits(__floats2half2_rn(p00, p01));
+                    pa[f][2 + hr] = h2_bits(__floats2half2_rn(p10, p11));
                 }
-                const float msafe = (m_r[hr] == -INFINITY) ? 0.f : m_r[hr];
-                const float p00 = fast_exp2(sacc[0][2 * hr] - msafe), p01 = fast_exp2(sacc[0][2 * hr + 1] - msafe);
-                const float p10 = fast_exp2(sacc[1][2 * hr] - msafe), p11 = fast_exp2(sacc[1][2 * hr + 1] - msafe);
-                l_r[hr] += (p00 + p01) + (p10 + p11);
-                pa[hr] = h2_bits(__floats2half2_rn(p00, p01));
-                pa[2 + hr] = h2_bits(__floats2half2_rn(p10, p11));
-            }
 
-            // ---- O += P V: b0 from cells (2t, 2t+1), b1 from (2t+8, 2t+9), dims D/8*g + nd
+            // ---- O += P V: b0 from cells (2t, 2t+1), b1 from (2t+8, 2t+9), slice dims KS/8*g + nd
             const __half2 s01 = bits_h2(__byte_perm(vc[0].sw, vc[1].sw, spair));
             const __half2 s89 = bits_h2(__byte_perm(vc[2].sw, vc[3].sw, spair));
 #pragma unroll
@@ -808,28 +989,34 @@ __global__ void __launch_bounds__(WS_WARPS * 32, 3) decode_ws_kernel(const __gri
                         u4x4_to_h2x2(__byte_perm(x89, y89, sel), c0, c1);
                     }
                     const int nd = 4 * w + 2 * half;
-                    mma16816(o[nd], pa, h2_bits(__hmul2(a0, s01)), h2_bits(__hmul2(c0, s89)));
-                    mma16816(o[nd + 1], pa, h2_bits(__hmul2(a1, s01)), h2_bits(__hmul2(c1, s89)));
+                    const uint32_t b00 = h2_bits(__hmul2(a0, s01)), b01 = h2_bits(__hmul2(c0, s89));
+                    const uint32_t b10 = h2_bits(__hmul2(a1, s01)), b11 = h2_bits(__hmul2(c1, s89));
+#pragma unroll
+                    for (int f = 0; f < MF; ++f) {
+                        mma16816(o[f][nd], pa[f], b00, b01);
+                        mma16816(o[f][nd + 1], pa[f], b10, b11);
+                    }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);                // this warp is done with the raw stage
         }
         if (!ok && lane == 0) report(p.status, ST_TIMEOUT_LOAD);
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 1);
-            l_r[hr] += __shfl_xor_sync(0xffffffffu, l_r[hr], 2);
-        }
+        for (int f = 0; f < MF; ++f)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                l_r[f][hr] += __shfl_xor_sync(0xffffffffu, l_r[f][hr], 1);
+                l_r[f][hr] += __shfl_xor_sync(0xffffffffu, l_r[f][hr], 2);
+            }
     }
 
     // ---- merge the 4 consumer warps (the raw ring is idle now)
-    write_cta_partial<D, WS_WARPS * 32, true>(o, m_r, l_r, warp < WARPS, smem, p, (int64_t)blockIdx.x);
+    write_ws_partial<KVT, D, MF>(o, m_r, l_r, cg, s, warp < 4, smem, p, part_index(p, s_idx, kvh, rg, sp));
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // Merge the chunk partials of one (sequence, kv head, fold row) by their
-// log-sum-exp weights, normalise, write O and LSE.
+// log-sum-exp weights, normalise, write O and LSE.  blockIdx.y is the fold row
+// (row group * rows + row within the group).
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant__ DecodeParams p)
 {
@@ -842,7 +1029,8 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
     if (r >= G * sq.n_q) return;
     const int h = kvh * G + r / sq.n_q, tok = sq.q_begin + r % sq.n_q;
     const int d = threadIdx.x;
-    const int64_t part0 = ((int64_t)s * p.Hkv + kvh) * p.splits;
+    const int R = p.rows, rl = r % R;
+    const int64_t part0 = part_index(p, s, kvh, r / R, 0);
     asm volatile("griddepcontrol.wait;" ::: "memory");  // partials of the split kernel are complete
     // This thread's column of the first KV32 splits goes out at once, with every
     // split's (max, sum); warp 0 reduces the latter while those loads fly.
@@ -851,9 +1039,9 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
     float v[KV32];
 #pragma unroll
     for (int sp = 0; sp < KV32; ++sp)
-        v[sp] = sp < nsp ? __ldcg(p.ws_o + ((part0 + sp) * 16 + r) * D + d) : 0.f;
+        v[sp] = sp < nsp ? __ldcg(p.ws_o + ((part0 + sp) * R + rl) * D + d) : 0.f;
     for (int sp = d; sp < nsp; sp += D) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.ws_ml + ((part0 + sp) * 16 + r) * 2));
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.ws_ml + ((part0 + sp) * R + rl) * 2));
         s_m[sp] = ml.x;
         s_l[sp] = ml.y;
     }
@@ -883,33 +1071,18 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const __grid_constant
 #pragma unroll
     for (int sp = 0; sp < KV32; ++sp) acc += s_w[sp < nsp ? sp : 0] * v[sp];   // v is 0 past nsp
 #pragma unroll 4
-    for (int sp = KV32; sp < nsp; ++sp) acc += s_w[sp] * __ldcg(p.ws_o + ((part0 + sp) * 16 + r) * D + d);
+    for (int sp = KV32; sp < nsp; ++sp) acc += s_w[sp] * __ldcg(p.ws_o + ((part0 + sp) * R + rl) * D + d);
     p.o[((int64_t)tok * p.H + h) * D + d] = ll > 0.f ? acc / ll : 0.f;
     if (d == 0) p.lse[(int64_t)tok * p.H + h] = ll > 0.f ? (mm + log2f(ll)) * LN2 : -INFINITY;
 }
 
-template <int KVT, int D, bool TMA>
-cudaError_t launch_t(const DecodeParams &p, cudaStream_t s)
+// The merge launches as a programmatic dependent: its launch overlaps the split
+// kernel's tail and it waits (griddepcontrol.wait) for the partials.
+template <int D>
+cudaError_t launch_combine(const DecodeParams &p, cudaStream_t s)
 {
-    const int grid = p.n_seq * p.Hkv * p.splits;
-    if (grid == 0) return cudaSuccess;
-    cudaError_t e;
-    if (TMA) {
-        auto k1 = decode_ws_kernel<KVT, D>;
-        const int bytes = WsLayout<KVT, D>::BYTES;
-        if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
-        k1<<<grid, WS_WARPS * 32, bytes, s>>>(p);
-    } else {
-        auto k1 = decode_split_kernel<KVT, D, false>;
-        const int bytes = DecLayout<KVT, D, false>::BYTES;
-        if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
-        k1<<<grid, WARPS * 32, bytes, s>>>(p);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // The merge launches as a programmatic dependent: its launch overlaps the
-    // split kernel's tail and it waits (griddepcontrol.wait) for the partials.
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.n_seq * p.Hkv, 16);
+    cfg.gridDim = dim3(p.n_seq * p.Hkv, p.rows * p.row_groups);
     cfg.blockDim = dim3(D);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = s;
@@ -921,41 +1094,73 @@ cudaError_t launch_t(const DecodeParams &p, cudaStream_t s)
     return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, p);
 }
 
-template <bool TMA>
-int smem_t(int kv_type, int D)
+template <int KVT, int D, int MF>
+cudaError_t launch_ws(const DecodeParams &p, cudaStream_t s)
 {
-    if (TMA) {
-        if (kv_type == ARC_KV_Q8_0) return D == 64 ? WsLayout<ARC_KV_Q8_0, 64>::BYTES : WsLayout<ARC_KV_Q8_0, 128>::BYTES;
-        return D == 64 ? WsLayout<ARC_KV_Q4_0, 64>::BYTES : WsLayout<ARC_KV_Q4_0, 128>::BYTES;
-    }
+    const int grid = p.n_seq * p.Hkv * p.row_groups * p.splits;
+    if (grid == 0) return cudaSuccess;
+    auto k1 = decode_ws_kernel<KVT, D, MF>;
+    const int bytes = WsLayout<KVT, D, MF>::BYTES;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+    k1<<<grid, WS_WARPS * 32, bytes, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_combine<D>(p, s);
+}
+
+template <int KVT, int D>
+cudaError_t launch_split(const DecodeParams &p, cudaStream_t s)
+{
+    const int grid = p.n_seq * p.Hkv * p.splits;
+    if (grid == 0) return cudaSuccess;
+    auto k1 = decode_split_kernel<KVT, D, false>;
+    const int bytes = DecLayout<KVT, D, false>::BYTES;
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+    k1<<<grid, WARPS * 32, bytes, s>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    return launch_combine<D>(p, s);
+}
+
+// Dispatch over the instantiated (cache type, head dim, fragments) of the TMA kernel.
+template <typename F>
+auto ws_dispatch(int kv_type, int D, int mf, F &&f)
+{
+#define ARC_WS(T, DD, M) \
+    if (kv_type == T && D == DD && mf == M) return f(std::integral_constant<int, T>{}, std::integral_constant<int, DD>{}, std::integral_constant<int, M>{});
+    ARC_WS(ARC_KV_Q8_0, 64, 1) ARC_WS(ARC_KV_Q8_0, 64, 2) ARC_WS(ARC_KV_Q8_0, 128, 1) ARC_WS(ARC_KV_Q8_0, 128, 2)
+    ARC_WS(ARC_KV_Q8_0, 256, 1) ARC_WS(ARC_KV_Q8_0, 256, 2) ARC_WS(ARC_KV_Q8_0, 512, 1)
+    ARC_WS(ARC_KV_Q4_0, 64, 1) ARC_WS(ARC_KV_Q4_0, 64, 2) ARC_WS(ARC_KV_Q4_0, 128, 1) ARC_WS(ARC_KV_Q4_0, 128, 2)
+    ARC_WS(ARC_KV_Q4_0, 256, 1) ARC_WS(ARC_KV_Q4_0, 256, 2) ARC_WS(ARC_KV_Q4_0, 512, 1)
+#undef ARC_WS
+    return f(std::integral_constant<int, 0>{}, std::integral_constant<int, 0>{}, std::integral_constant<int, 0>{});
+}
+
+}  // namespace
+
+bool decode_ws_supported(int kv_type, int D, int mf)
+{
+    return ws_dispatch(kv_type, D, mf, [](auto t, auto d, auto m) { return decltype(d)::value != 0; });
+}
+
+int decode_smem_bytes(int kv_type, int D, int mf, bool tma)
+{
+    if (tma)
+        return ws_dispatch(kv_type, D, mf, [](auto t, auto d, auto m) {
+            if constexpr (decltype(d)::value == 0) return 0;
+            else return WsLayout<decltype(t)::value, decltype(d)::value, decltype(m)::value>::BYTES;
+        });
     if (kv_type == ARC_KV_Q8_0)
         return D == 64 ? DecLayout<ARC_KV_Q8_0, 64, false>::BYTES : DecLayout<ARC_KV_Q8_0, 128, false>::BYTES;
     return D == 64 ? DecLayout<ARC_KV_Q4_0, 64, false>::BYTES : DecLayout<ARC_KV_Q4_0, 128, false>::BYTES;
 }
 
-template <bool TMA>
-cudaError_t launch_k(const DecodeParams &p, cudaStream_t s)
-{
-    if (p.kv_type == ARC_KV_Q8_0) {
-        if (p.D == 64) return launch_t<ARC_KV_Q8_0, 64, TMA>(p, s);
-        if (p.D == 128) return launch_t<ARC_KV_Q8_0, 128, TMA>(p, s);
-    } else {
-        if (p.D == 64) return launch_t<ARC_KV_Q4_0, 64, TMA>(p, s);
-        if (p.D == 128) return launch_t<ARC_KV_Q4_0, 128, TMA>(p, s);
-    }
-    return cudaErrorInvalidValue;
-}
-
-}  // namespace
-
-int decode_smem_bytes(int kv_type, int D, bool tma) { return tma ? smem_t<true>(kv_type, D) : smem_t<false>(kv_type, D); }
-
 // CTAs of the split kernel that fit on one SM at once (registers, threads and
 // shared memory together), from the occupancy API; 0 if it cannot be asked (no device).
-int decode_blocks_per_sm(int kv_type, int D, bool tma)
+int decode_blocks_per_sm(int kv_type, int D, int mf, bool tma)
 {
     int n = 0;
-    const int smem = decode_smem_bytes(kv_type, D, tma);
+    const int smem = decode_smem_bytes(kv_type, D, mf, tma);
     auto ask = [&](auto kern, int threads) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem) != cudaSuccess) {
@@ -965,10 +1170,11 @@ int decode_blocks_per_sm(int kv_type, int D, bool tma)
     };
     const bool q8 = kv_type == ARC_KV_Q8_0;
     if (tma) {
-        if (q8)
-            D == 64 ? ask(decode_ws_kernel<ARC_KV_Q8_0, 64>, WS_WARPS * 32) : ask(decode_ws_kernel<ARC_KV_Q8_0, 128>, WS_WARPS * 32);
-        else
-            D == 64 ? ask(decode_ws_kernel<ARC_KV_Q4_0, 64>, WS_WARPS * 32) : ask(decode_ws_kernel<ARC_KV_Q4_0, 128>, WS_WARPS * 32);
+        ws_dispatch(kv_type, D, mf, [&](auto t, auto d, auto m) {
+            if constexpr (decltype(d)::value != 0)
+                ask(decode_ws_kernel<decltype(t)::value, decltype(d)::value, decltype(m)::value>, WS_WARPS * 32);
+            return 0;
+        });
     } else {
         if (q8)
             D == 64 ? ask(decode_split_kernel<ARC_KV_Q8_0, 64, false>, WARPS * 32)
@@ -980,17 +1186,37 @@ int decode_blocks_per_sm(int kv_type, int D, bool tma)
     return n;
 }
 
-// Box width in bytes of the TMA path (covers a head row from the 16-byte boundary below it).
-int decode_box_bytes(int kv_type, int D)
+// TMA box of the split kernel: {width in bytes, cells}; the width covers one head-dim
+// slice of a head row from the 16-byte boundary at or below it.
+void decode_box(int kv_type, int D, int mf, int *width, int *cells)
 {
-    if (kv_type == ARC_KV_Q8_0) return D == 64 ? DecLayout<ARC_KV_Q8_0, 64, true>::RS : DecLayout<ARC_KV_Q8_0, 128, true>::RS;
-    return D == 64 ? DecLayout<ARC_KV_Q4_0, 64, true>::RS : DecLayout<ARC_KV_Q4_0, 128, true>::RS;
+    *width = *cells = 0;
+    ws_dispatch(kv_type, D, mf, [&](auto t, auto d, auto m) {
+        if constexpr (decltype(d)::value != 0) {
+            *width = WsLayout<decltype(t)::value, decltype(d)::value, decltype(m)::value>::RS;
+            *cells = WsShape<decltype(d)::value, decltype(m)::value>::DT;
+        }
+        return 0;
+    });
 }
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s)
 {
-    if (p.splits > 256) return cudaErrorInvalidValue;
-    return p.tma ? launch_k<true>(p, s) : launch_k<false>(p, s);
+    if (p.splits > 256 || p.rows != 16 * p.mf) return cudaErrorInvalidValue;
+    if (p.tma)
+        return ws_dispatch(p.kv_type, p.D, p.mf, [&](auto t, auto d, auto m) -> cudaError_t {
+            if constexpr (decltype(d)::value == 0) return cudaErrorInvalidValue;
+            else return launch_ws<decltype(t)::value, decltype(d)::value, decltype(m)::value>(p, s);
+        });
+    if (p.mf != 1 || p.row_groups != 1) return cudaErrorInvalidValue;
+    if (p.kv_type == ARC_KV_Q8_0) {
+        if (p.D == 64) return launch_split<ARC_KV_Q8_0, 64>(p, s);
+        if (p.D == 128) return launch_split<ARC_KV_Q8_0, 128>(p, s);
+    } else {
+        if (p.D == 64) return launch_split<ARC_KV_Q4_0, 64>(p, s);
+        if (p.D == 128) return launch_split<ARC_KV_Q4_0, 128>(p, s);
+    }
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace arc

@@ -103,20 +103,28 @@ cudaError_t launch_sparse_tc(const SparseTcParams &p, cudaStream_t s);
 
 // ---------------------------------------------------------------- quantised decode
 struct DecodeParams {
-    CUtensorMap tm_kc;  // k_cache as bytes {Hkv*row bytes, n_cells}, box {row span, 64 cells} (tma != 0)
+    CUtensorMap tm_kc;  // k_cache as bytes {Hkv*row bytes, n_cells}, box {slice span, tile cells} (tma != 0)
     CUtensorMap tm_vc;  // v_cache likewise
     int tma;            // 1: K/V tiles arrive by TMA through a multi-stage ring; 0: cp.async
     int kv_type, n_tok, H, Hkv, D, n_seq, splits, chunk;
+    int mf;             // m16 fragments of fold rows per CTA (1 or 2)
+    int rows;           // fold rows per CTA and per workspace part: 16 * mf
+    int row_groups;     // CTAs along the fold rows of one (sequence, kv head)
     const float *q;
     const uint8_t *k_cache, *v_cache;
     arc_seq seqs[ARC_DECODE_MAX_SEQ];
     float *o, *lse;
-    float *ws_o;     // [n_seq*Hkv*splits][16][D] partial outputs (unnormalised)
-    float *ws_ml;    // [n_seq*Hkv*splits][16][2] partial (max, sum)
+    float *ws_o;     // [n_seq*Hkv*row_groups*splits][rows][D] partial outputs (unnormalised)
+    float *ws_ml;    // [n_seq*Hkv*row_groups*splits][rows][2] partial (max, sum)
     float scale_log2;
     uint32_t *status;
 };
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t s);
+// TMA split kernel instantiations: cache type x head dim (64..512) x fragments (1, 2; 1 at 512).
+bool decode_ws_supported(int kv_type, int D, int mf);
+int decode_smem_bytes(int kv_type, int D, int mf, bool tma);
+int decode_blocks_per_sm(int kv_type, int D, int mf, bool tma);
+void decode_box(int kv_type, int D, int mf, int *width, int *cells);
 
 cudaError_t launch_selftest_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
 

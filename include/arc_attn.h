@@ -228,17 +228,23 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *args, void *stream);
  *   o        [n_tok,H,D]            fp32, device, written (rows of tokens that no
  *            sequence owns are left untouched)
  *   lse      [n_tok,H]              fp32, device, written likewise
- * D in {64,128,256,512}; H % Hkv == 0; (H/Hkv) * n_q <= 16 for every
- * sequence; n_seq <= ARC_DECODE_MAX_SEQ.  D 64 and 128 run the split-KV tensor-
- * core kernel and its combine (two launches); D 256 and 512 run the CUDA-core
- * kernel (one warp per query row over all its cells, one launch, no workspace:
- * arc_decode_workspace_size() returns 0), as does ARC_FLAG_FORCE_SIMPLE.
+ * D in {64,128,256,512}; H % Hkv == 0; (H/Hkv) * n_q <= ARC_DECODE_MAX_ROWS
+ * for every sequence; n_seq <= ARC_DECODE_MAX_SEQ.  The query heads of a kv
+ * head times a sequence's new tokens are its fold rows (row = head in group *
+ * n_q + token).  On caches whose cell stride (Hkv * D/32 blocks) is a multiple
+ * of 16 bytes and whose base pointers are 16-byte aligned, every head dim runs
+ * the split-KV tensor-core kernel (TMA ring, m16n8k16 MMAs, 16 or 32 fold rows
+ * per CTA, head dims above 128 cut into slices whose S partials are summed in
+ * shared memory) and its combine: two launches.  Other caches run the cp.async
+ * split kernel for D <= 128 with up to 16 fold rows, else the CUDA-core kernel
+ * (one warp per query row over all its cells, one launch, no workspace), as
+ * does ARC_FLAG_FORCE_SIMPLE.  arc_plan names the kernel.
  * workspace: device, at least arc_decode_workspace_size(args) bytes, 256-byte
  * aligned; used for the split-KV partial results and overwritten.  Its
  * contents need no initialisation (every byte read is first written by the
  * same call).  Two calls in flight at once need two workspaces.
  * Errors, all returned before anything is launched: D outside {64,128,256,512},
- * n_seq above ARC_DECODE_MAX_SEQ or (H/Hkv) * n_q above 16 is
+ * n_seq above ARC_DECODE_MAX_SEQ or (H/Hkv) * n_q above ARC_DECODE_MAX_ROWS is
  * ARC_ERR_UNSUPPORTED; an unknown kv_type, negative sizes, H % Hkv != 0,
  * n_kv < n_q, a sequence whose tokens or cells run past n_tok / n_cells, a NULL
  * tensor, or q, o or a cache not 8-byte aligned is ARC_ERR_INVALID_ARG; a
@@ -246,6 +252,7 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *args, void *stream);
  * ARC_ERR_WORKSPACE.  n_seq == 0 or n_tok == 0 launches nothing.
  * ------------------------------------------------------------------------ */
 #define ARC_DECODE_MAX_SEQ 64
+#define ARC_DECODE_MAX_ROWS 128
 
 typedef struct {
     int32_t q_begin, n_q, kv_begin, n_kv;

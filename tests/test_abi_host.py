@@ -121,9 +121,12 @@ def test_decode_validation_and_workspace_size(arc):
     many = arc.make_seqs([0] * 65, [0] * 65, [0] * 65, [0] * 65)
     d.seqs, d.n_seq = ctypes.cast(many, ctypes.POINTER(arc.Seq)), 65
     assert L.arc_attn_decode_q8(ctypes.byref(d), None, 0, None) == arc.ARC_ERR_UNSUPPORTED
-    wide = arc.make_seqs([0], [5], [0], [10])                # g * n_q = 20 > 16
-    d.seqs, d.n_seq, d.H, d.Hkv = ctypes.cast(wide, ctypes.POINTER(arc.Seq)), 1, 32, 8
+    wide = arc.make_seqs([0], [33], [0], [40])               # g * n_q = 4 * 33 = 132 > 128 fold rows
+    d.seqs, d.n_seq, d.H, d.Hkv, d.n_tok = ctypes.cast(wide, ctypes.POINTER(arc.Seq)), 1, 32, 8, 33
     assert L.arc_attn_decode_q8(ctypes.byref(d), None, 0, None) == arc.ARC_ERR_UNSUPPORTED
+    ok = arc.make_seqs([0], [32], [0], [40])                 # 128 fold rows: accepted (NULL tensors refused next)
+    d.seqs = ctypes.cast(ok, ctypes.POINTER(arc.Seq))
+    assert L.arc_attn_decode_q8(ctypes.byref(d), None, 0, None) == arc.ARC_ERR_INVALID_ARG
 
 
 def test_merge_validation_before_any_launch(arc):

@@ -321,13 +321,33 @@ def test_decode_head_dim_64_and_control_arm():
 @pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
 @pytest.mark.parametrize("D", [256, 512])
 def test_decode_wide_head_dims(kv_type, D):
-    """Head dims 256 / 512 (the CUDA-core decode kernel): ragged sequences, GQA 4."""
+    """Head dims 256 / 512 (the sliced tensor-core split kernel): ragged sequences, GQA 4."""
     c = W.decode_case(3, 0, 0, 8, 2, D, kv_type=kv_type, seed=62, n_q_list=[2, 1, 4], n_kv_list=[700, 1, 130])
     st = status_word()
     o, lse, (q, kc, vc) = run_decode(c, status=st)
     info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
                            n_kv=c.n_kv)
-    assert info["kernel"] == "simple_decode_kernel"
+    assert info["kernel"].startswith("decode_ws_kernel") and info["d_slice"] == 128
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert arc.check_device_error(st) == arc.ARC_OK
+    o2, lse2 = arc.attn_decode_q8(q, kc, vc, kv_type=c.kv_type, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q,
+                                  kv_begin=c.kv_begin, n_kv=c.n_kv, scale=c.scale, flags=arc.ARC_FLAG_FORCE_SIMPLE)
+    torch.cuda.synchronize()
+    compare(o2, lse2, ro, rl, TOL_O_BF16)                 # the CUDA-core control arm
+
+
+@pytest.mark.parametrize("kv_type", [W.KV_Q8_0, W.KV_Q4_0])
+@pytest.mark.parametrize("D,G,n_q", [(128, 8, 4), (128, 4, 16), (256, 8, 4), (512, 4, 16), (64, 32, 4)])
+def test_decode_more_than_16_fold_rows_full_length(kv_type, D, G, n_q):
+    """Several sequences of G * n_q = 32 to 128 fold rows over 8192-cell caches: two m16
+    fragments per CTA (one at D = 512) in row groups, many splits and the combine."""
+    c = W.decode_case(2, n_q, 8192, 4 * G, 4, D, kv_type=kv_type, seed=63 + D + G)
+    st = status_word()
+    o, lse, (q, kc, vc) = run_decode(c, status=st)
+    info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                           n_kv=c.n_kv)
+    assert info["kernel"].startswith("decode_ws_kernel") and info["tile_m"] == (16 if D == 512 else 32)
     ro, rl = oracle.run_case(c)
     compare(o, lse, ro, rl, TOL_O_BF16)
     assert arc.check_device_error(st) == arc.ARC_OK

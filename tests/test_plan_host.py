@@ -185,12 +185,37 @@ def test_decode_single_stream_and_empty_caches(arc):
     assert arc.plan(arc.ARC_OP_DECODE, d)["kernel"] == "simple_decode_kernel"
 
 
+@pytest.mark.parametrize("kv", ["q8_0", "q4_0"])
 @pytest.mark.parametrize("D", [256, 512])
-def test_decode_wide_heads_run_the_cuda_core_kernel_without_workspace(arc, D):
-    d = decode_args(arc, arc.ARC_KV_Q4_0, D=D)
+def test_decode_wide_heads_run_the_sliced_tensor_core_kernel(arc, kv, D):
+    """Head dims 256 / 512: the TMA split kernel with the head dim cut into 128-dim
+    slices (the four warps of a CTA: 2 cell groups x 2 slices, or 1 x 4)."""
+    kv_type = arc.ARC_KV_Q8_0 if kv == "q8_0" else arc.ARC_KV_Q4_0
+    d = decode_args(arc, kv_type, D=D)
+    info = arc.plan(arc.ARC_OP_DECODE, d)
+    assert info["kernel"] == f"decode_ws_kernel<{kv}>" and info["launches"] == 2 and info["tensor_cores"] == 1
+    assert info["d_slice"] == 128 and info["tile_m"] == 16 and info["tile_n"] == 16 * 4 // (D // 128)
+    ws = arc.lib().arc_decode_workspace_size(ctypes.byref(d))
+    assert ws == 4 * 8 * info["splits"] * 16 * (D + 2) * 4
+    d.flags = arc.ARC_FLAG_FORCE_SIMPLE
     info = arc.plan(arc.ARC_OP_DECODE, d)
     assert info["kernel"] == "simple_decode_kernel" and info["launches"] == 1 and info["tensor_cores"] == 0
     assert arc.lib().arc_decode_workspace_size(ctypes.byref(d)) == 0
+
+
+@pytest.mark.parametrize("D,G,n_q,mf,groups", [(128, 8, 4, 2, 1), (128, 4, 16, 2, 2), (64, 16, 4, 2, 2),
+                                                (256, 8, 4, 2, 1), (512, 8, 4, 1, 2), (128, 16, 8, 2, 4)])
+def test_decode_more_than_16_fold_rows(arc, D, G, n_q, mf, groups):
+    """GQA-8 x 4 tokens (32 rows), GQA-4 x a 16-token ubatch (64 rows) and more: 32 fold
+    rows per CTA (two m16 fragments; one at D = 512) in row groups along the fold."""
+    d = decode_args(arc, arc.ARC_KV_Q8_0, n_seq=2, n_q=n_q, H=8 * G, Hkv=8, D=D, n_kv=4096)
+    info = arc.plan(arc.ARC_OP_DECODE, d)
+    assert info["kernel"] == "decode_ws_kernel<q8_0>" and info["tile_m"] == 16 * mf
+    assert info["n_ctas"] == 2 * 8 * groups * info["splits"]
+    ws = arc.lib().arc_decode_workspace_size(ctypes.byref(d))
+    assert ws == 2 * 8 * groups * info["splits"] * 16 * mf * (D + 2) * 4
+    d.k_cache = FAKE + 8                                # not 16-byte aligned: the CUDA-core kernel
+    assert arc.plan(arc.ARC_OP_DECODE, d)["kernel"] == "simple_decode_kernel"
 
 
 def test_decode_workspace_errors_come_before_any_launch(arc):

@@ -7,7 +7,7 @@ checks call it through the C ABI, twice in a row on the shared buffer, and
 compare each result element by element with the fp64 oracle and with
 arc_attn_decode_q8 fed a caller workspace.  The cases reach every decode
 kernel: the TMA split kernel, the cp.async split kernel (a cell stride that is
-not a multiple of 16 bytes) and the CUDA-core kernel (head dim 256).  The file
+not a multiple of 16 bytes) and the CUDA-core kernel (ARC_FLAG_FORCE_SIMPLE).  The file
 name sorts last so a stop-at-first-failure run has run everything else.
 """
 import pytest
@@ -30,34 +30,37 @@ def _kw(c):
                 n_kv=c.n_kv, scale=c.scale)
 
 
+# name -> (case, flags, the kernel arc_plan must name)
 CASES = {
-    "c5-q8_0": lambda: W.config(5, kv_type=W.KV_Q8_0),
-    "c5-q4_0": lambda: W.config(5, kv_type=W.KV_Q4_0),
-    "d64-ragged": lambda: W.decode_case(3, 2, 0, 16, 4, 64, kv_type=W.KV_Q8_0, seed=41, n_q_list=[2, 4, 1],
-                                        n_kv_list=[900, 33, 5]),
-    "cp_async-path": lambda: W.decode_case(3, 2, 700, 6, 3, 128, kv_type=W.KV_Q4_0, seed=44),
-    "d256-cuda-cores": lambda: W.decode_case(2, 0, 0, 8, 2, 256, kv_type=W.KV_Q8_0, seed=45, n_q_list=[2, 1],
-                                             n_kv_list=[300, 77]),
+    "c5-q8_0": (lambda: W.config(5, kv_type=W.KV_Q8_0), 0, "decode_ws_kernel"),
+    "c5-q4_0": (lambda: W.config(5, kv_type=W.KV_Q4_0), 0, "decode_ws_kernel"),
+    "d64-ragged": (lambda: W.decode_case(3, 2, 0, 16, 4, 64, kv_type=W.KV_Q8_0, seed=41, n_q_list=[2, 4, 1],
+                                         n_kv_list=[900, 33, 5]), 0, "decode_ws_kernel"),
+    "cp_async-path": (lambda: W.decode_case(3, 2, 700, 6, 3, 128, kv_type=W.KV_Q4_0, seed=44), 0,
+                      "decode_split_kernel"),
+    "d256-32-rows": (lambda: W.decode_case(2, 0, 0, 32, 2, 256, kv_type=W.KV_Q8_0, seed=45, n_q_list=[2, 1],
+                                           n_kv_list=[300, 77]), 0, "decode_ws_kernel"),
+    "cuda-cores": (lambda: W.decode_case(2, 0, 0, 8, 2, 256, kv_type=W.KV_Q4_0, seed=46, n_q_list=[2, 1],
+                                         n_kv_list=[300, 77]), 1, "simple_decode_kernel"),
 }
-KERNELS = {"c5-q8_0": "decode_ws_kernel", "c5-q4_0": "decode_ws_kernel", "d64-ragged": "decode_ws_kernel",
-           "cp_async-path": "decode_split_kernel", "d256-cuda-cores": "simple_decode_kernel"}
 
 
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_noalloc_decode_matches_oracle_and_workspace_entry_on_consecutive_calls(name):
-    c = CASES[name]()
+    make, flags, kernel = CASES[name]
+    c = make()
     q, kc, vc = _inputs(c)
     info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
-                           n_kv=c.n_kv)
-    assert info["kernel"].startswith(KERNELS[name])
+                           n_kv=c.n_kv, flags=flags)
+    assert info["kernel"].startswith(kernel)
     ro, rl = oracle.run_case(c)
-    o_ws, l_ws = arc.attn_decode_q8(q, kc, vc, **_kw(c))
+    o_ws, l_ws = arc.attn_decode_q8(q, kc, vc, flags=flags, **_kw(c))
     torch.cuda.synchronize()
     compare(o_ws, l_ws, ro, rl, TOL_O_BF16, TOL_LSE)
     for _ in range(2):                      # two calls in a row on the shared buffer
         o = torch.full_like(o_ws, float("nan"))
         lse = torch.full_like(l_ws, float("nan"))
-        arc.attn_decode_q8_noalloc(q, kc, vc, out=o, lse=lse, **_kw(c))
+        arc.attn_decode_q8_noalloc(q, kc, vc, out=o, lse=lse, flags=flags, **_kw(c))
         torch.cuda.synchronize()
         compare(o, lse, ro, rl, TOL_O_BF16, TOL_LSE)
         compare(o, lse, host(o_ws), host(l_ws), TOL_O_BF16, TOL_LSE)
