@@ -52,6 +52,17 @@ CONFIGS = {
                  metric="decode GB/s", dtype="q8_0"),
     "c5q4": dict(cfg=5, kv_type=W.KV_Q4_0, name="multi-seq decode, 4 seq x 4 tok, H=32 Hkv=8 D=128, 8192 cells/seq, q4_0",
                  metric="decode GB/s", dtype="q4_0"),
+    # quantised decode at head dim 256 and with 32 fold rows per (sequence, kv head)
+    "c5d256": dict(cfg=8, decode=dict(n_seq=4, n_q=4, n_kv=8192, H=32, Hkv=8, D=256, kv_type=W.KV_Q8_0),
+                   name="multi-seq decode, 4 seq x 4 tok, H=32 Hkv=8 D=256, 8192 cells/seq, q8_0",
+                   metric="decode GB/s", dtype="q8_0"),
+    "c5g8": dict(cfg=9, decode=dict(n_seq=4, n_q=4, n_kv=8192, H=64, Hkv=8, D=128, kv_type=W.KV_Q8_0),
+                 name="multi-seq decode, 4 seq x 4 tok, H=64 Hkv=8 (32 fold rows) D=128, 8192 cells/seq, q8_0",
+                 metric="decode GB/s", dtype="q8_0"),
+    # decode-shaped sparse MLA: c4's per-token shape at a decode batch of 32 tokens
+    "c4d": dict(cfg=7, sparse_decode=dict(Sq=32, H=64, Skv=65536, Dqk=512, Dv=512, topk=2176),
+                name="sparse MLA decode, 32 tokens x 64 h x 2176 top-k, d_qk=d_v=512, pool 65536",
+                metric="sparse decode GB/s", dtype="bf16"),
     # the context-parallel output merge (not a configuration of the method's own benchmark):
     # two bf16 partial outputs shaped like c2's, with sinks
     "merge": dict(cfg=6, merge=dict(n_parts=2, B=1, H=64, T=1400, Dv=512), name="LSE output merge, 2 parts of "
@@ -62,11 +73,21 @@ CONFIGS = {
 def make_case(spec):
     if "merge" in spec:
         return W.merge_case(**spec["merge"], seed=spec["cfg"])
+    if "sparse_decode" in spec:
+        return SparseDecode(W.sparse_case(**spec["sparse_decode"], seed=spec["cfg"]))
+    if "decode" in spec:
+        return W.decode_case(**spec["decode"], seed=spec["cfg"])
     kw = {"kv_type": spec["kv_type"]} if "kv_type" in spec else {}
     return W.config(spec["cfg"], **kw)
 
 
 # ------------------------------------------------------------------ algorithmic work
+
+class SparseDecode:
+    """A sparse case run through arc_sparse_mla_decode (few tokens, top-k split over CTAs)."""
+
+    def __init__(self, case):
+        self.case = case
 
 def dense_pairs(Tq, Tk, causal):
     if not causal:
@@ -76,6 +97,13 @@ def dense_pairs(Tq, Tk, causal):
 
 def work(case):
     """(algorithmic units, unit name) of one call: FLOPs over visible pairs, or bytes for decode."""
+    if isinstance(case, SparseDecode):
+        # memory-bound: every distinct pool row a call gathers crosses HBM once, plus Q, O,
+        # LSE and the index lists
+        c = case.case
+        valid = c.idx[(c.idx >= 0) & (c.idx < c.Skv)]
+        rows = int(np.unique(valid).size)
+        return rows * c.Dqk * 2 + c.q.nbytes + c.Sq * c.H * (c.Dv * 2 + 4) + c.idx.nbytes, "byte"
     if isinstance(case, W.DenseCase):
         pairs = case.B * case.H * dense_pairs(case.Tq, case.Tk, case.causal)
         return pairs * (2 * case.D + 2 * case.Dv), "flop"
@@ -115,6 +143,18 @@ class Uploaded:
 def build_call(case, torch, arc, status):
     """Returns (call(), inputs dict of device tensors, outputs list, n_launches, kernel name)."""
     U = Uploaded(case, torch, arc)
+    if isinstance(case, SparseDecode):
+        c = case.case
+        q, kv, idx = U.to_dev(c.q), U.to_dev(c.kv), U.to_dev(c.idx)
+        o = torch.empty(c.Sq, c.H, c.Dv, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty(c.Sq, c.H, dtype=torch.float32, device="cuda")
+        info = arc.plan_sparse_decode(q, kv, idx, o, lse, Dv=c.Dv)
+        ws = torch.empty(max(256, arc.sparse_decode_workspace_size(q, kv, idx, o, lse, Dv=c.Dv)), dtype=torch.uint8,
+                         device="cuda")
+
+        def call():
+            arc.sparse_mla_decode(q, kv, idx, Dv=c.Dv, scale=c.scale, out=o, lse=lse, workspace=ws, status=status)
+        return call, {"q": q, "kv": kv, "idx": idx}, [o, lse], info
     if isinstance(case, W.DenseCase):
         q, k, v = U.to_dev(case.q), U.to_dev(case.k), U.to_dev(case.v)
         s = U.to_dev(case.sinks) if case.sinks is not None else None
@@ -269,6 +309,16 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
     import oracle
     oracle.build()
     cores = oracle.num_threads()
+    if isinstance(case, SparseDecode):
+        units, _ = work(case)
+        reps, spent = 0, 0.0
+        while spent < budget_s[0] and reps < 50:
+            t0 = time.perf_counter()
+            oracle.run_case(case.case)
+            spent += time.perf_counter() - t0
+            reps += 1
+        return {"value": units * reps / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                "sample": f"the whole decode batch, {reps} repetitions", "seconds": round(spent, 2)}
     rng = np.random.default_rng(0)
     done_units, spent, n_rows = 0, 0.0, 0
     if isinstance(case, (W.DenseCase, W.MlaCase)):
@@ -412,7 +462,7 @@ def steps_for(call, stream, flush, local, min_wall_s):
     return max(20, int(math.ceil(min_wall_s / max(wall / 20, 1e-6))))
 
 
-def roofline(units, unit_kind, mean_ms, peaks, config_key, kernel):
+def roofline(units, unit_kind, mean_ms, peaks, config_key, kernel, launches=1):
     if unit_kind == "flop":
         achieved = units / (mean_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -423,8 +473,7 @@ def roofline(units, unit_kind, mean_ms, peaks, config_key, kernel):
         achieved = units / (mean_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"] + " copy bandwidth",
-                "note": ("whole call (split kernel + combine) timed" if kernel.startswith("decode")
-                         else "one launch")}
+                "note": f"whole call timed ({launches} launch{'es' if launches > 1 else ''})"}
     roof["traffic"] = recorded_traffic(config_key, kernel)
     roof["kernel"] = kernel
     return roof
@@ -448,10 +497,10 @@ def measure_config(key, status, stream, flush, local, peaks, min_wall_s):
     scale = 1e12 if unit_kind == "flop" else 1e9
     rec = {"workload": spec["name"], "metric": spec["metric"], "value": units / (mean_ms * 1e-3) / scale,
            "unit": "TFLOP/s" if unit_kind == "flop" else "GB/s", "ms_per_step": mean_ms, "steps": steps,
-           "dtype": spec["dtype"], "roofline": roofline(units, unit_kind, mean_ms, peaks, key, info["kernel"]),
+           "dtype": spec["dtype"], "roofline": roofline(units, unit_kind, mean_ms, peaks, key, info["kernel"], info["launches"]),
            "clocks": clocks, "wall_s_timed_region": wall, "gpu_launches": int(info["launches"]) * steps,
            "l2": flush.describe()}
-    if isinstance(case, W.DecodeCase):
+    if isinstance(case, (W.DecodeCase, SparseDecode)):
         g = capture(call, stream)
         for _ in range(5):
             g.replay()
@@ -469,7 +518,8 @@ def measure_config(key, status, stream, flush, local, peaks, min_wall_s):
 
 
 # The graded workloads: the headline (--config) plus these, each measured in the same run.
-GRADED = ["c2", "c3", "c4", "c5q8", "c5q4"]
+GRADED = ["c2", "c3", "c4", "c5q8", "c5q4",
+          "c5d256", "c5g8", "c4d"]          # and the decode variants beyond the five workloads
 
 
 def run_ours(args, spec, case):
@@ -533,7 +583,7 @@ def run_ours(args, spec, case):
     scale = 1e12 if unit_kind == "flop" else 1e9
     unit = "TFLOP/s" if unit_kind == "flop" else "GB/s"
     value = job_throughput(units, world, args.steps, total_ms, unit_kind)
-    roof = roofline(units, unit_kind, mean_ms, peaks, args.config, info["kernel"])
+    roof = roofline(units, unit_kind, mean_ms, peaks, args.config, info["kernel"], info["launches"])
     e2e_val = units / (e2e_mean * 1e-3) / scale
     if not e2e_ms:                      # --no-e2e: no host-buffer leg; JSON null rather than NaN
         e2e_val = e2e_mean = None
@@ -600,7 +650,7 @@ def run_reference(args, spec, case):
         else:
             u, _ = work(case)
             t0 = time.perf_counter()
-            oracle.run_case(case)
+            oracle.run_case(case.case if isinstance(case, SparseDecode) else case)
         dt = time.perf_counter() - t0
         if i >= args.warmup:
             times.append(dt)

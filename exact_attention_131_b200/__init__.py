@@ -8,6 +8,7 @@ Names follow the C ABI:
     attn_fwd            -> arc_attn_fwd         dense / GQA / MQA (+ sinks)
     mla_fwd             -> arc_mla_fwd          q_nope||q_rope, d_qk != d_v
     sparse_mla_fwd      -> arc_sparse_mla_fwd   per-query top-k index lists
+    sparse_mla_decode   -> arc_sparse_mla_decode   the same, top-k split over CTAs for few tokens
     attn_decode_q8      -> arc_attn_decode_q8   q8_0 / q4_0 cache, multi-sequence
     attn_merge          -> arc_attn_merge       results over disjoint key sets -> the whole
     plan                -> arc_plan             engagement record, no launch
@@ -24,7 +25,7 @@ _lib = None
 ARC_OK, ARC_ERR_INVALID_ARG, ARC_ERR_UNSUPPORTED, ARC_ERR_CUDA, ARC_ERR_DEVICE_TIMEOUT, ARC_ERR_WORKSPACE = range(6)
 ARC_DTYPE_BF16, ARC_DTYPE_F32 = 0, 1
 ARC_KV_Q4_0, ARC_KV_Q8_0 = 2, 8
-ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE, ARC_OP_MERGE = 1, 2, 3, 4, 5
+ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE, ARC_OP_MERGE, ARC_OP_SPARSE_DECODE, ARC_OP_ATTN_BWD = range(1, 8)
 ARC_MERGE_MAX_PARTS = 16
 ARC_FLAG_FORCE_SIMPLE = 1
 ARC_FLAG_SINGLE_CTA = 2
@@ -84,7 +85,8 @@ class PlanInfo(ctypes.Structure):
 
 EXPORTS = ["arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
            "arc_decode_workspace_size", "arc_plan", "arc_abi_version", "arc_status_string",
-           "arc_check_device_error", "arc_selftest_timeout", "arc_attn_decode_q8_noalloc", "arc_attn_merge"]
+           "arc_check_device_error", "arc_selftest_timeout", "arc_attn_decode_q8_noalloc", "arc_attn_merge",
+           "arc_sparse_mla_decode", "arc_sparse_decode_workspace_size"]
 
 
 class ArcError(RuntimeError):
@@ -104,6 +106,9 @@ def lib():
         L.arc_attn_fwd.argtypes = [ctypes.POINTER(AttnArgs), _vp]
         L.arc_mla_fwd.argtypes = [ctypes.POINTER(MlaArgs), _vp]
         L.arc_sparse_mla_fwd.argtypes = [ctypes.POINTER(SparseArgs), _vp]
+        L.arc_sparse_mla_decode.argtypes = [ctypes.POINTER(SparseArgs), _vp, ctypes.c_size_t, _vp]
+        L.arc_sparse_decode_workspace_size.argtypes = [ctypes.POINTER(SparseArgs)]
+        L.arc_sparse_decode_workspace_size.restype = ctypes.c_size_t
         L.arc_attn_decode_q8.argtypes = [ctypes.POINTER(DecodeArgs), _vp, ctypes.c_size_t, _vp]
         L.arc_attn_decode_q8_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         L.arc_attn_merge.argtypes = [ctypes.POINTER(MergeArgs), _vp]
@@ -114,7 +119,7 @@ def lib():
         L.arc_status_string.restype = ctypes.c_char_p
         L.arc_check_device_error.argtypes = [_vp, _vp]
         L.arc_selftest_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
-        for f in ("arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
+        for f in ("arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_sparse_mla_decode", "arc_attn_decode_q8",
                   "arc_attn_decode_q8_noalloc", "arc_attn_merge", "arc_plan",
                   "arc_check_device_error", "arc_selftest_timeout", "arc_abi_version"):
             getattr(L, f).restype = _i32
@@ -287,6 +292,37 @@ def sparse_mla_fwd(q, kv, idx, *, Dv=None, v=None, scale=None, sinks=None, out=N
     return out, lse
 
 
+def sparse_mla_decode(q, kv, idx, *, Dv=None, v=None, scale=None, sinks=None, out=None, lse=None, workspace=None,
+                      flags=0, status=None, stream=None):
+    """O, LSE = arc_sparse_mla_decode: arc_sparse_mla_fwd with each token's top-k list split
+    over several CTAs when the tokens do not fill the GPU (a workspace holds the partials)."""
+    torch = _torch()
+    bf = torch.bfloat16
+    _dev(q, "q", bf), _dev(kv, "kv", bf), _dev(idx, "idx", torch.int32), _dev(v, "v", bf)
+    _dev(sinks, "sinks", torch.float32)
+    Sq, H, Dqk = q.shape
+    if Dv is None:
+        Dv = v.shape[1] if v is not None else Dqk
+    if out is None:
+        out = torch.empty(Sq, H, Dv, dtype=bf, device=q.device)
+    if lse is None:
+        lse = torch.empty(Sq, H, dtype=torch.float32, device=q.device)
+    a = _sparse_args(q, kv, idx, v, out, lse, sinks, Dv, scale, flags, status)
+    need = int(lib().arc_sparse_decode_workspace_size(ctypes.byref(a)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _p(workspace) if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().arc_sparse_mla_decode(ctypes.byref(a), ws_ptr, ws_len, _stream(stream)), "arc_sparse_mla_decode")
+    return out, lse
+
+
+def sparse_decode_workspace_size(q, kv, idx, out, lse, *, Dv=None, v=None, sinks=None, flags=0) -> int:
+    Dv = Dv if Dv is not None else (v.shape[1] if v is not None else q.shape[-1])
+    a = _sparse_args(q, kv, idx, v, out, lse, sinks, Dv, 1.0, flags, None)
+    return int(lib().arc_sparse_decode_workspace_size(ctypes.byref(a)))
+
+
 def make_seqs(q_begin, n_q, kv_begin, n_kv):
     n = len(q_begin)
     arr = (Seq * max(n, 1))()
@@ -453,6 +489,11 @@ def plan_mla(q_nope, q_rope, k_nope, k_rope, v, out, lse, *, causal=True, flags=
 def plan_sparse(q, kv, idx, out, lse, *, Dv=None, v=None, sinks=None, flags=0):
     Dv = Dv if Dv is not None else (v.shape[1] if v is not None else q.shape[-1])
     return plan(ARC_OP_SPARSE, _sparse_args(q, kv, idx, v, out, lse, sinks, Dv, 1.0, flags, None))
+
+
+def plan_sparse_decode(q, kv, idx, out, lse, *, Dv=None, v=None, sinks=None, flags=0):
+    Dv = Dv if Dv is not None else (v.shape[1] if v is not None else q.shape[-1])
+    return plan(ARC_OP_SPARSE_DECODE, _sparse_args(q, kv, idx, v, out, lse, sinks, Dv, 1.0, flags, None))
 
 
 def plan_decode(kv_type, q, k_cache, v_cache, *, Hkv, q_begin, n_q, kv_begin, n_kv, flags=0):

@@ -421,6 +421,36 @@ bool plan_sparse_tc(const arc_sparse_args *a)
     return true;
 }
 
+// Decode-shaped sparse calls: when the tokens' (token, head group) CTAs leave SMs idle,
+// each token's slots are cut into `splits` chunks of whole 64-slot tiles (at least two
+// tiles each, at most ARC_MERGE_MAX_PARTS chunks), merged afterwards by the LSE merge.
+struct SparseDecodePlan {
+    bool tc = false;    // the tensor-core kernel takes the call
+    int splits = 1, chunk = 0;
+    size_t ws = 0;      // fp32 partials: O [splits][Sq][H][Dv] then LSE [splits][Sq][H]
+};
+
+SparseDecodePlan plan_sparse_decode(const arc_sparse_args *a)
+{
+    SparseDecodePlan pl;
+    pl.chunk = std::max(1, a->topk);
+    if (a->Sq == 0 || !plan_sparse_tc(a)) return pl;
+    pl.tc = true;
+    // the merge writes rows r = token * H + head at r * Dv: O must be [Sq, H, Dv] contiguous
+    if (a->o_strides[1] != a->Dv || a->o_strides[0] != (int64_t)a->H * a->Dv) return pl;
+    const int base = a->Sq * ((a->H + 63) / 64);
+    const int tiles = (a->topk + 63) / 64;
+    int splits = std::min({ARC_MERGE_MAX_PARTS, sm_count() / std::max(1, base), tiles / 2});
+    if (splits < 2) return pl;
+    const int chunk = ((tiles + splits - 1) / splits) * 64;
+    splits = (a->topk + chunk - 1) / chunk;
+    if (splits < 2) return pl;
+    pl.splits = splits;
+    pl.chunk = chunk;
+    pl.ws = (size_t)splits * a->Sq * a->H * (a->Dv + 1) * sizeof(float);
+    return pl;
+}
+
 // ------------------------------------------------------------------ decode
 
 struct DecodePlan {
@@ -671,6 +701,7 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *a, void *stream)
         p.o = static_cast<__nv_bfloat16 *>(a->o), p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
         p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = call_scale(a->flags, a->scale, a->Dqk) * kLog2e;
         p.status = a->status;
+        p.splits = 1, p.chunk = std::max(1, a->topk);
         note_dispatch("sparse_tc_kernel");
         e = launch_sparse_tc(p, s);
     } else {
@@ -688,6 +719,48 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *a, void *stream)
         e = launch_simple_attn(p, s);
     }
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+size_t arc_sparse_decode_workspace_size(const arc_sparse_args *a)
+{
+    if (check_sparse(a) != ARC_OK) return 0;
+    return plan_sparse_decode(a).ws;
+}
+
+arc_status arc_sparse_mla_decode(const arc_sparse_args *a, void *workspace, size_t ws_bytes, void *stream)
+{
+    arc_status st = check_sparse(a);
+    if (st != ARC_OK) return st;
+    if (a->Sq == 0) return ARC_OK;
+    const SparseDecodePlan pl = plan_sparse_decode(a);
+    if (pl.splits == 1) return arc_sparse_mla_fwd(a, stream);
+    if (!workspace || ws_bytes < pl.ws || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return ARC_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    SparseTcParams p{};
+    p.Sq = a->Sq, p.H = a->H, p.Skv = a->Skv, p.Dqk = a->Dqk, p.Dv = a->Dv, p.topk = a->topk;
+    p.q = static_cast<const __nv_bfloat16 *>(a->q), p.qs[0] = a->q_strides[0], p.qs[1] = a->q_strides[1];
+    p.kv = static_cast<const __nv_bfloat16 *>(a->kv), p.kv_stride = a->kv_stride;
+    p.v = static_cast<const __nv_bfloat16 *>(a->v), p.v_stride = a->v_stride;
+    p.idx = a->idx, p.idx_stride = a->idx_stride;
+    p.o = static_cast<__nv_bfloat16 *>(a->o), p.os[0] = a->o_strides[0], p.os[1] = a->o_strides[1];
+    p.lse = a->lse, p.sinks = a->sinks, p.scale_log2 = call_scale(a->flags, a->scale, a->Dqk) * kLog2e;
+    p.status = a->status;
+    p.splits = pl.splits, p.chunk = pl.chunk;
+    const size_t rows = (size_t)a->Sq * a->H;
+    p.part_o = static_cast<float *>(workspace);
+    p.part_lse = p.part_o + (size_t)pl.splits * rows * a->Dv;
+    note_dispatch("sparse_tc_kernel<split>");
+    if (launch_sparse_tc(p, s) != cudaSuccess) return ARC_ERR_CUDA;
+    // LSE merge of the splits (and the sink, once), fp32 partials into the bf16 output
+    MergeParams m{};
+    m.n_parts = pl.splits, m.rows = (int)rows, m.dv = a->Dv, m.dtype = ARC_DTYPE_F32, m.out_dtype = ARC_DTYPE_BF16;
+    for (int i = 0; i < pl.splits; ++i) {
+        m.o_parts[i] = p.part_o + (size_t)i * rows * a->Dv;
+        m.lse_parts[i] = p.part_lse + (size_t)i * rows;
+    }
+    m.sinks = a->sinks, m.sink_heads = a->H, m.sink_rows = 1;
+    m.o = a->o, m.lse = a->lse;
+    return launch_merge(m, s) == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
 
 size_t arc_decode_workspace_size(const arc_decode_args *a)
@@ -860,7 +933,7 @@ arc_status arc_attn_merge(const arc_merge_args *a, void *stream)
     const arc_status st = check_merge(a);
     if (st != ARC_OK || a->rows == 0) return st;
     MergeParams p{};
-    p.n_parts = a->n_parts, p.rows = a->rows, p.dv = a->dv, p.dtype = a->dtype;
+    p.n_parts = a->n_parts, p.rows = a->rows, p.dv = a->dv, p.dtype = a->dtype, p.out_dtype = a->dtype;
     for (int i = 0; i < a->n_parts; ++i) p.o_parts[i] = a->o_parts[i], p.lse_parts[i] = a->lse_parts[i];
     p.sinks = a->sinks, p.sink_heads = a->sink_heads, p.sink_rows = a->sink_rows;
     p.o = a->o, p.lse = a->lse;
@@ -947,6 +1020,30 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             out->tile_m = 4;
         }
         out->launches = 1;
+        return ARC_OK;
+    }
+    if (op == ARC_OP_SPARSE_DECODE) {
+        const arc_sparse_args *a = static_cast<const arc_sparse_args *>(args);
+        arc_status st = check_sparse(a);
+        if (st != ARC_OK) return st;
+        const SparseDecodePlan pl = plan_sparse_decode(a);
+        if (a->Sq == 0) {
+            set_name(out, "none");
+            return ARC_OK;
+        }
+        if (!pl.tc) {
+            set_name(out, "simple_attn_kernel<sparse>");
+            out->tile_m = 4;
+            out->launches = 1;
+            return ARC_OK;
+        }
+        set_name(out, pl.splits > 1 ? "sparse_tc_kernel<split>" : "sparse_tc_kernel");
+        out->tensor_cores = 1;
+        out->tile_m = 64, out->tile_n = 64, out->d_slice = a->Dv;
+        out->splits = pl.splits;
+        out->n_ctas = a->Sq * ((a->H + 63) / 64) * pl.splits;
+        out->smem_bytes = sparse_smem_bytes(a->Dqk, a->Dv, a->v != nullptr), out->tmem_cols = 512;
+        out->launches = pl.splits > 1 ? 2 : 1;
         return ARC_OK;
     }
     if (op == ARC_OP_DECODE) {

@@ -96,6 +96,12 @@ struct SparseTcParams {
     const float *sinks;
     float scale_log2;
     uint32_t *status;
+    // Split top-k (decode-shaped calls): CTA (token, head group, split) takes slots
+    // [split*chunk, min(topk, split*chunk + chunk)) and writes its normalised fp32 partial
+    // O [splits][Sq][H][Dv] and LSE [splits][Sq][H] (no sink: the merge adds it).
+    // splits == 1 and part_o == NULL: the whole list per CTA, bf16 O written directly.
+    int splits, chunk;
+    float *part_o, *part_lse;
 };
 int sparse_smem_bytes(int dqk, int dv, bool sepv);
 bool sparse_tc_supported(int dqk, int dv, bool sepv);
@@ -131,6 +137,7 @@ cudaError_t launch_selftest_timeout(uint32_t *status, uint64_t timeout_ns, cudaS
 // Merge of partial results over disjoint key sets (arc_attn_merge), one warp per row.
 struct MergeParams {
     int n_parts, rows, dv, dtype;
+    int out_dtype;      // dtype of o (the parts' dtype for arc_attn_merge; fp32 parts -> bf16 o for sparse decode)
     const void *o_parts[ARC_MERGE_MAX_PARTS];
     const float *lse_parts[ARC_MERGE_MAX_PARTS];
     const float *sinks;

@@ -89,7 +89,8 @@ struct Pair<__nv_bfloat16> {
 constexpr int MERGE_ROWS_PER_CTA = 8;   // one warp per row
 
 // NP: a compile-time bound on the number of parts (the loops over parts unroll to it).
-template <typename T, bool VEC, int NP>
+// T: the parts' element type; TO: the output's (the same, or bf16 from fp32 partials).
+template <typename T, typename TO, bool VEC, int NP>
 __global__ void __launch_bounds__(32 * MERGE_ROWS_PER_CTA) merge_kernel(const __grid_constant__ MergeParams p)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(32 * MERGE_ROWS_PER_CTA) merge_kernel(const __
             }
 #pragma unroll
             for (int u = 0; u < U; ++u)
-                if (c0 + 32 * u < nch) Oct<T>::store(p.o, base + 8 * (c0 + 32 * u), acc[u]);
+                if (c0 + 32 * u < nch) Oct<TO>::store(p.o, base + 8 * (c0 + 32 * u), acc[u]);
         }
     } else {
         for (int d = 2 * lane; d < p.dv; d += 64) {
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(32 * MERGE_ROWS_PER_CTA) merge_kernel(const __
                     acc.x += w[i] * v.x, acc.y += w[i] * v.y;
                 }
             }
-            Pair<T>::store(p.o, base + d, acc);
+            Pair<TO>::store(p.o, base + d, acc);
         }
     }
 }
@@ -177,16 +178,21 @@ cudaError_t launch_merge(const MergeParams &p, cudaStream_t s)
     const dim3 block(32 * MERGE_ROWS_PER_CTA);
     auto go = [&](auto np) {
         constexpr int NP = decltype(np)::value;
-        if (p.dtype == ARC_DTYPE_F32) {
+        if (p.dtype == ARC_DTYPE_F32 && p.out_dtype == ARC_DTYPE_F32) {
             if (vec)
-                merge_kernel<float, true, NP><<<grid, block, 0, s>>>(p);
+                merge_kernel<float, float, true, NP><<<grid, block, 0, s>>>(p);
             else
-                merge_kernel<float, false, NP><<<grid, block, 0, s>>>(p);
+                merge_kernel<float, float, false, NP><<<grid, block, 0, s>>>(p);
+        } else if (p.dtype == ARC_DTYPE_F32) {
+            if (vec)
+                merge_kernel<float, __nv_bfloat16, true, NP><<<grid, block, 0, s>>>(p);
+            else
+                merge_kernel<float, __nv_bfloat16, false, NP><<<grid, block, 0, s>>>(p);
         } else {
             if (vec)
-                merge_kernel<__nv_bfloat16, true, NP><<<grid, block, 0, s>>>(p);
+                merge_kernel<__nv_bfloat16, __nv_bfloat16, true, NP><<<grid, block, 0, s>>>(p);
             else
-                merge_kernel<__nv_bfloat16, false, NP><<<grid, block, 0, s>>>(p);
+                merge_kernel<__nv_bfloat16, __nv_bfloat16, false, NP><<<grid, block, 0, s>>>(p);
         }
     };
     if (p.n_parts <= 2)

@@ -81,9 +81,12 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_hgroups = (p.H + SM_ROWS - 1) / SM_ROWS;
-    const int tok = blockIdx.x / n_hgroups;
-    const int h0 = (blockIdx.x % n_hgroups) * SM_ROWS;
-    const int nt = (p.topk + SBN - 1) / SBN;
+    const int sp = blockIdx.x % p.splits;                      // top-k split (decode-shaped calls)
+    const int tok = blockIdx.x / (n_hgroups * p.splits);
+    const int h0 = ((blockIdx.x / p.splits) % n_hgroups) * SM_ROWS;
+    const int s_begin = sp * p.chunk;                          // this CTA's slots: [s_begin, s_begin + cnt)
+    const int cnt = max(0, min(p.topk - s_begin, p.chunk));
+    const int nt = (cnt + SBN - 1) / SBN;
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 128);
@@ -121,16 +124,16 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
         fence_proxy_async_smem();
         mbar_arrive(&bars->q_full);
 
-        const int32_t *idx_row = p.idx + (int64_t)tok * p.idx_stride;
+        const int32_t *idx_row = p.idx + (int64_t)tok * p.idx_stride + s_begin;
         // Lane i < 16 of warp w holds the index of tile row w + 4i; warp 0 also holds
         // one index per lane for each half of the tile, for the validity mask.
         auto fetch = [&](int j, int32_t &mine, int32_t &m0, int32_t &m1) {
             const int slot = j * SBN + warp + 4 * (lane & 15);
-            mine = (lane < 16 && slot < p.topk) ? idx_row[slot] : -1;
+            mine = (lane < 16 && slot < cnt) ? idx_row[slot] : -1;
             if (warp == 0) {
                 const int s0 = j * SBN + lane, s1 = s0 + 32;
-                m0 = s0 < p.topk ? idx_row[s0] : -1;
-                m1 = s1 < p.topk ? idx_row[s1] : -1;
+                m0 = s0 < cnt ? idx_row[s0] : -1;
+                m1 = s1 < cnt ? idx_row[s1] : -1;
             }
         };
         int32_t mine = -1, m0 = -1, m1 = -1;
@@ -323,7 +326,7 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
         if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
         l += __shfl_xor_sync(0xffffffffu, l, 16);
         float fac, lse;
-        if (p.sinks) {
+        if (p.sinks && !p.part_o) {   // a split's partial leaves the sink to the merge
             const float sg = row_ok ? p.sinks[h] * S_LOG2E : 0.f;
             const float mf = fmaxf(m_use, sg);
             const float a = (m_use == -INFINITY) ? 0.f : exp2f(m_use - mf);
@@ -335,6 +338,7 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
             lse = l > 0.f ? (m_use + log2f(l)) * S_LN2 : -INFINITY;
         }
         __nv_bfloat16 *orow = p.o + (int64_t)tok * p.os[0] + (int64_t)h * p.os[1];
+        const int64_t prow = ((int64_t)sp * p.Sq + tok) * p.H + h;   // partial row (split calls)
 #pragma unroll 1
         for (int c = 0; c < VC; ++c) {
             uint32_t ov[32];
@@ -345,7 +349,13 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
 #pragma unroll
                 for (int i = 0; i < 32; ++i) ov[i] = 0u;
             }
-            if (row_ok) {
+            if (row_ok && p.part_o) {
+                float4 *dst = reinterpret_cast<float4 *>(p.part_o + prow * p.Dv + c * 64 + half * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(__uint_as_float(ov[4 * i]) * fac, __uint_as_float(ov[4 * i + 1]) * fac,
+                                         __uint_as_float(ov[4 * i + 2]) * fac, __uint_as_float(ov[4 * i + 3]) * fac);
+            } else if (row_ok) {
                 uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
@@ -355,7 +365,12 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                 for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
             }
         }
-        if (row_ok && half == 0) p.lse[(int64_t)tok * p.H + h] = lse;
+        if (row_ok && half == 0) {
+            if (p.part_o)
+                p.part_lse[prow] = lse;
+            else
+                p.lse[(int64_t)tok * p.H + h] = lse;
+        }
     }
 
     tc_fence_before();
@@ -373,7 +388,8 @@ cudaError_t launch_sp(const SparseTcParams &p, cudaStream_t s)
     auto kern = sparse_tc_kernel<KC, VC, SEPV>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::BYTES);
     if (e != cudaSuccess) return e;
-    const int grid = p.Sq * ((p.H + SM_ROWS - 1) / SM_ROWS);
+    if (p.splits < 1 || (p.splits > 1 && (!p.part_o || !p.part_lse)) || p.chunk < 1) return cudaErrorInvalidValue;
+    const int grid = p.Sq * ((p.H + SM_ROWS - 1) / SM_ROWS) * p.splits;
     kern<<<grid, S_THREADS, L::BYTES, s>>>(p);
     return cudaGetLastError();
 }

@@ -68,7 +68,10 @@ typedef enum { ARC_DTYPE_BF16 = 0, ARC_DTYPE_F32 = 1 } arc_dtype;
 /* Quantised KV block types; the values are the ggml type ids. */
 typedef enum { ARC_KV_Q4_0 = 2, ARC_KV_Q8_0 = 8 } arc_kv_type;
 
-typedef enum { ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE = 4, ARC_OP_MERGE = 5 } arc_op;
+typedef enum {
+    ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE = 4, ARC_OP_MERGE = 5,
+    ARC_OP_SPARSE_DECODE = 6, ARC_OP_ATTN_BWD = 7
+} arc_op;
 
 /* flags (all calls) */
 #define ARC_FLAG_FORCE_SIMPLE 1u   /* run the CUDA-core kernel instead of the tensor-core one */
@@ -204,6 +207,35 @@ typedef struct {
 } arc_sparse_args;
 
 arc_status arc_sparse_mla_fwd(const arc_sparse_args *args, void *stream);
+
+/* --------------------------------------------------------------------------
+ * arc_sparse_mla_decode: the same sparse attention, shaped for decode batches.
+ *
+ * Source: "TensorRT-LLM: FlashMLA without -rdc", its ptxas list: next to the
+ * sparse prefill, FlashMLA builds a sparse decode kernel for 64 heads ("sm100
+ * sparse decode (h64)").  A decode batch has few query tokens, and
+ * arc_sparse_mla_fwd runs one CTA per (token, 64-head group), which leaves most
+ * SMs idle below ~148 tokens.  This call takes the same arguments and computes
+ * the same O and LSE, but when the tokens do not fill the GPU it cuts each
+ * token's top-k list into `splits` chunks of whole 64-slot tiles (one CTA each,
+ * at most ARC_MERGE_MAX_PARTS), writes every chunk's normalised fp32 partial O
+ * and LSE to the workspace, and merges them with the LSE-weighted output merge
+ * of arc_attn_merge (the sink, if any, enters once, there): two launches.
+ * When the tokens fill the GPU, or the call does not take the tensor-core
+ * kernel, or o is not a contiguous [Sq,H,Dv] tensor, it is exactly
+ * arc_sparse_mla_fwd (one launch, no workspace).
+ *   workspace  device, at least arc_sparse_decode_workspace_size(args) bytes
+ *              (0: none needed), 256-byte aligned, overwritten; its contents
+ *              need no initialisation.  Two calls in flight need two.
+ * Errors: those of arc_sparse_mla_fwd; a missing, short or unaligned workspace
+ * where one is needed is ARC_ERR_WORKSPACE.  arc_plan(ARC_OP_SPARSE_DECODE)
+ * names the kernel ("sparse_tc_kernel<split>" with the split count).
+ * The fp8 KV variant the page also lists is an sm90 kernel; it is not built here
+ * (the page gives no cache format for it).
+ * ------------------------------------------------------------------------ */
+size_t arc_sparse_decode_workspace_size(const arc_sparse_args *args);
+
+arc_status arc_sparse_mla_decode(const arc_sparse_args *args, void *workspace, size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
  * arc_attn_decode_q8: multi-sequence decode over one unified q8_0 / q4_0 cache,

@@ -369,3 +369,25 @@ def test_tensor_core_shape_sets_match_the_header(arc):
                     mla.add((Dn + Dr, Dv))
     assert dense == dense_doc and len(dense) == 10
     assert mla == mla_doc and len(mla) == 5
+
+
+# -------------------------------------------------------------------------- sparse decode
+@pytest.mark.parametrize("Sq,want_splits", [(1, 12), (4, 12), (37, 4), (74, 2), (148, 1), (400, 1)])
+def test_sparse_decode_splits_the_top_k_when_tokens_leave_sms_idle(arc, Sq, want_splits):
+    """64 heads, 2176 slots (34 tiles of 64): few tokens cut their lists into chunks of whole
+    tiles, at least two tiles each and at most 16 chunks; enough tokens run one CTA each."""
+    s = sparse_args(arc, Sq=Sq, topk=2176, D=512, Dv=512)
+    info = arc.plan(arc.ARC_OP_SPARSE_DECODE, s)
+    assert info["splits"] == want_splits and info["tensor_cores"] == 1
+    ws = arc.lib().arc_sparse_decode_workspace_size(ctypes.byref(s))
+    if want_splits == 1:
+        assert info["kernel"] == "sparse_tc_kernel" and info["launches"] == 1 and ws == 0
+    else:
+        assert info["kernel"] == "sparse_tc_kernel<split>" and info["launches"] == 2
+        tiles = -(-34 // min(16, SMS // Sq, 17))
+        assert want_splits == -(-2176 // (tiles * 64))
+        assert ws == want_splits * Sq * 64 * (512 + 1) * 4
+        assert info["n_ctas"] == Sq * want_splits
+        # a missing or short workspace is refused before anything launches
+        assert arc.lib().arc_sparse_mla_decode(ctypes.byref(s), None, ws, None) == arc.ARC_ERR_WORKSPACE
+        assert arc.lib().arc_sparse_mla_decode(ctypes.byref(s), FAKE, ws - 4, None) == arc.ARC_ERR_WORKSPACE
