@@ -6,6 +6,7 @@ no fallback: if the library is missing, importing a function raises.
 
 Names follow the C ABI:
     attn_fwd            -> arc_attn_fwd         dense / GQA / MQA (+ sinks)
+    attn_bwd            -> arc_attn_bwd         its gradients: dq, dk, dv, d sinks
     mla_fwd             -> arc_mla_fwd          q_nope||q_rope, d_qk != d_v
     sparse_mla_fwd      -> arc_sparse_mla_fwd   per-query top-k index lists
     sparse_mla_decode   -> arc_sparse_mla_decode   the same, top-k split over CTAs for few tokens
@@ -60,6 +61,16 @@ class SparseArgs(ctypes.Structure):
                 ("flags", _u32), ("status", _vp)]
 
 
+class BwdArgs(ctypes.Structure):
+    _fields_ = [("B", _i32), ("H", _i32), ("Hkv", _i32), ("Tq", _i32), ("Tk", _i32), ("D", _i32), ("Dv", _i32),
+                ("q", _vp), ("q_strides", _i64 * 3), ("k", _vp), ("k_strides", _i64 * 3),
+                ("v", _vp), ("v_strides", _i64 * 3), ("o", _vp), ("o_strides", _i64 * 3),
+                ("dout", _vp), ("do_strides", _i64 * 3), ("lse", _vp), ("dlse", _vp), ("sinks", _vp),
+                ("dq", _vp), ("dq_strides", _i64 * 3), ("dk", _vp), ("dk_strides", _i64 * 3),
+                ("dv", _vp), ("dv_strides", _i64 * 3), ("dsinks", _vp), ("scale", _f32), ("causal", _i32),
+                ("flags", _u32), ("status", _vp)]
+
+
 class Seq(ctypes.Structure):
     _fields_ = [("q_begin", _i32), ("n_q", _i32), ("kv_begin", _i32), ("n_kv", _i32)]
 
@@ -86,7 +97,7 @@ class PlanInfo(ctypes.Structure):
 EXPORTS = ["arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
            "arc_decode_workspace_size", "arc_plan", "arc_abi_version", "arc_status_string",
            "arc_check_device_error", "arc_selftest_timeout", "arc_attn_decode_q8_noalloc", "arc_attn_merge",
-           "arc_sparse_mla_decode", "arc_sparse_decode_workspace_size"]
+           "arc_sparse_mla_decode", "arc_sparse_decode_workspace_size", "arc_attn_bwd", "arc_attn_bwd_workspace_size"]
 
 
 class ArcError(RuntimeError):
@@ -109,6 +120,9 @@ def lib():
         L.arc_sparse_mla_decode.argtypes = [ctypes.POINTER(SparseArgs), _vp, ctypes.c_size_t, _vp]
         L.arc_sparse_decode_workspace_size.argtypes = [ctypes.POINTER(SparseArgs)]
         L.arc_sparse_decode_workspace_size.restype = ctypes.c_size_t
+        L.arc_attn_bwd.argtypes = [ctypes.POINTER(BwdArgs), _vp, ctypes.c_size_t, _vp]
+        L.arc_attn_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
+        L.arc_attn_bwd_workspace_size.restype = ctypes.c_size_t
         L.arc_attn_decode_q8.argtypes = [ctypes.POINTER(DecodeArgs), _vp, ctypes.c_size_t, _vp]
         L.arc_attn_decode_q8_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         L.arc_attn_merge.argtypes = [ctypes.POINTER(MergeArgs), _vp]
@@ -119,7 +133,8 @@ def lib():
         L.arc_status_string.restype = ctypes.c_char_p
         L.arc_check_device_error.argtypes = [_vp, _vp]
         L.arc_selftest_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
-        for f in ("arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_sparse_mla_decode", "arc_attn_decode_q8",
+        for f in ("arc_attn_fwd", "arc_attn_bwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_sparse_mla_decode",
+                  "arc_attn_decode_q8",
                   "arc_attn_decode_q8_noalloc", "arc_attn_merge", "arc_plan",
                   "arc_check_device_error", "arc_selftest_timeout", "arc_abi_version"):
             getattr(L, f).restype = _i32
@@ -219,6 +234,63 @@ def attn_fwd(q, k, v, *, scale=None, causal=True, sinks=None, out=None, lse=None
     a = _attn_args(q, k, v, out, lse, sinks, scale, causal, flags, status)
     _check(lib().arc_attn_fwd(ctypes.byref(a), _stream(stream)), "arc_attn_fwd")
     return out, lse
+
+
+def _bwd_args(q, k, v, o, lse, dout, dlse, sinks, dq, dk, dv, dsinks, scale, causal, flags, status):
+    B, H, Tq, D = q.shape
+    _, Hkv, Tk, Dv = v.shape
+    a = BwdArgs()
+    a.B, a.H, a.Hkv, a.Tq, a.Tk, a.D, a.Dv = B, H, Hkv, Tq, Tk, D, Dv
+    a.q, a.q_strides = _p(q), _s3(q)
+    a.k, a.k_strides = _p(k), _s3(k)
+    a.v, a.v_strides = _p(v), _s3(v)
+    a.o, a.o_strides = _p(o), _s3(o)
+    a.dout, a.do_strides = _p(dout), _s3(dout)
+    a.lse, a.dlse, a.sinks = _p(lse), _p(dlse), _p(sinks)
+    a.dq, a.dq_strides = _p(dq), _s3(dq)
+    a.dk, a.dk_strides = _p(dk), _s3(dk)
+    a.dv, a.dv_strides = _p(dv), _s3(dv)
+    a.dsinks = _p(dsinks)
+    a.scale, a.flags = _scale_flags(scale, flags)
+    a.causal = int(bool(causal))
+    a.status = _p(status)
+    return a
+
+
+def attn_bwd(q, k, v, o, lse, dout, *, scale=None, causal=True, sinks=None, dlse=None, dq=None, dk=None, dv=None,
+             dsinks=None, workspace=None, flags=0, status=None, stream=None):
+    """dq, dk, dv, dsinks = arc_attn_bwd: gradients of attn_fwd(q, k, v) given its o, lse and
+    the upstream dout (and optionally dlse).  dsinks is None without sinks."""
+    torch = _torch()
+    bf = torch.bfloat16
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _dev(t, n, bf)
+    for n, t in (("lse", lse), ("dlse", dlse), ("sinks", sinks)):
+        _dev(t, n, torch.float32)
+    for n, t in (("lse", lse), ("dlse", dlse)):
+        if t is not None and (tuple(t.shape) != tuple(q.shape[:3]) or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous [B, H, Tq] fp32 tensor")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if sinks is not None and dsinks is None:
+        dsinks = torch.empty_like(sinks)
+    a = _bwd_args(q, k, v, o, lse, dout, dlse, sinks, dq, dk, dv, dsinks, scale, causal, flags, status)
+    need = int(lib().arc_attn_bwd_workspace_size(ctypes.byref(a)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _p(workspace) if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().arc_attn_bwd(ctypes.byref(a), ws_ptr, ws_len, _stream(stream)), "arc_attn_bwd")
+    return dq, dk, dv, dsinks
+
+
+def plan_attn_bwd(q, k, v, o, lse, dout, *, causal=True, sinks=None, flags=0):
+    torch = _torch()
+    dq, dk, dv = q, k, v            # shapes and strides only: nothing is launched
+    ds = sinks if sinks is not None else None
+    return plan(ARC_OP_ATTN_BWD, _bwd_args(q, k, v, o, lse, dout, None, sinks, dq, dk, dv, ds, 1.0, causal, flags,
+                                           None))
 
 
 def _mla_args(q_nope, q_rope, k_nope, k_rope, v, o, lse, scale, causal, flags, status):

@@ -19,7 +19,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libarc_attn.so")
 PTXAS_LOG = os.path.join(HERE, "_ptxas_report.txt")
-SOURCES = ["api.cu", "simple_kernels.cu", "attn_tc.cu", "attn_pair.cu", "sparse_tc.cu", "decode.cu", "merge.cu"]
+SOURCES = ["api.cu", "simple_kernels.cu", "attn_tc.cu", "attn_pair.cu", "sparse_tc.cu", "decode.cu", "merge.cu",
+           "attn_bwd.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xptxas", "-v", "--expt-relaxed-constexpr"]

@@ -451,6 +451,72 @@ SparseDecodePlan plan_sparse_decode(const arc_sparse_args *a)
     return pl;
 }
 
+// ------------------------------------------------------------------ backward
+
+arc_status check_bwd(const arc_attn_bwd_args *a)
+{
+    if (!a) return ARC_ERR_INVALID_ARG;
+    if (a->B < 0 || a->H <= 0 || a->Hkv <= 0 || a->H % a->Hkv || a->Tq < 0 || a->Tk < 0 || a->D <= 0 || a->Dv <= 0)
+        return ARC_ERR_INVALID_ARG;
+    if (!bwd_supported(a->D, a->Dv)) return ARC_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    if (!scale_ok(a->flags, a->scale)) return ARC_ERR_INVALID_ARG;
+    if (!a->q || !a->o || !a->dout || !a->lse || !a->dq || (a->Tk > 0 && (!a->k || !a->v || !a->dk || !a->dv)))
+        return ARC_ERR_INVALID_ARG;
+    if (a->sinks && !a->dsinks) return ARC_ERR_INVALID_ARG;
+    const int64_t *all[] = {a->q_strides, a->k_strides, a->v_strides, a->o_strides, a->do_strides,
+                            a->dq_strides, a->dk_strides, a->dv_strides};
+    for (const int64_t *st : all)
+        for (int i = 0; i < 3; ++i)
+            if (st[i] < 0) return ARC_ERR_INVALID_ARG;
+    // outputs whose rows would alias one another
+    if (broadcast(a->dq_strides[0], a->B) || broadcast(a->dq_strides[1], a->H) || broadcast(a->dq_strides[2], a->Tq) ||
+        broadcast(a->dk_strides[0], a->B) || broadcast(a->dk_strides[1], a->Hkv) || broadcast(a->dk_strides[2], a->Tk) ||
+        broadcast(a->dv_strides[0], a->B) || broadcast(a->dv_strides[1], a->Hkv) || broadcast(a->dv_strides[2], a->Tk))
+        return ARC_ERR_INVALID_ARG;
+    // the tensor-core layout: fold rows evenly spaced, 16-byte rows and bases
+    if (a->H > 1 && (a->q_strides[1] != (int64_t)a->Tq * a->q_strides[2] ||
+                     a->do_strides[1] != (int64_t)a->Tq * a->do_strides[2]))
+        return ARC_ERR_UNSUPPORTED;
+    const void *ptrs[] = {a->q, a->k, a->v, a->o, a->dout, a->dq, a->dk, a->dv};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return ARC_ERR_UNSUPPORTED;
+    for (const int64_t *st : all)
+        for (int i = 0; i < 3; ++i)
+            if ((st[i] * 2) % 16) return ARC_ERR_UNSUPPORTED;
+    if (broadcast(a->q_strides[0], a->B) || broadcast(a->k_strides[0], a->B) || broadcast(a->v_strides[0], a->B) ||
+        broadcast(a->k_strides[1], a->Hkv) || broadcast(a->v_strides[1], a->Hkv) || broadcast(a->do_strides[0], a->B))
+        return ARC_ERR_UNSUPPORTED;
+    return ARC_OK;
+}
+
+struct BwdPlan {
+    int rsplit = 1, tiles_per_split = 0, n_kt = 0, n_qt = 0;
+    size_t delta_bytes = 0, ws = 0;
+};
+
+// dK/dV: one CTA per (batch, kv head, key tile); when those leave SMs idle, each key
+// tile's fold rows are split over several CTAs (at least 4 fold tiles each) whose
+// fp32 partials a reduction sums.
+BwdPlan plan_bwd(const arc_attn_bwd_args *a)
+{
+    BwdPlan pl;
+    pl.delta_bytes = (((size_t)a->B * a->H * a->Tq * sizeof(float)) + 255) / 256 * 256;
+    pl.ws = pl.delta_bytes;
+    if (a->B == 0 || a->Tq == 0 || a->Tk == 0) return pl;
+    const int BR = bwd_tile_rows(a->D, a->Dv);
+    pl.n_kt = (a->Tk + 127) / 128;
+    pl.n_qt = (a->H / a->Hkv * a->Tq + BR - 1) / BR;
+    const int base = a->B * a->Hkv * pl.n_kt;
+    int rsplit = std::min(sm_count() / std::max(1, base), pl.n_qt / 4);
+    rsplit = std::max(1, std::min(rsplit, 64));
+    pl.tiles_per_split = (pl.n_qt + rsplit - 1) / rsplit;
+    pl.rsplit = (pl.n_qt + pl.tiles_per_split - 1) / pl.tiles_per_split;
+    if (pl.rsplit > 1)
+        pl.ws += (size_t)pl.rsplit * a->B * a->Hkv * a->Tk * (a->D + a->Dv) * sizeof(float);
+    return pl;
+}
+
 // ------------------------------------------------------------------ decode
 
 struct DecodePlan {
@@ -719,6 +785,69 @@ arc_status arc_sparse_mla_fwd(const arc_sparse_args *a, void *stream)
         e = launch_simple_attn(p, s);
     }
     return e == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+size_t arc_attn_bwd_workspace_size(const arc_attn_bwd_args *a)
+{
+    if (check_bwd(a) != ARC_OK) return 0;
+    return plan_bwd(a).ws;
+}
+
+arc_status arc_attn_bwd(const arc_attn_bwd_args *a, void *workspace, size_t ws_bytes, void *stream)
+{
+    arc_status st = check_bwd(a);
+    if (st != ARC_OK) return st;
+    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    const BwdPlan pl = plan_bwd(a);
+    if (!workspace || ws_bytes < pl.ws || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return ARC_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const float scale = call_scale(a->flags, a->scale, a->D);
+    float *delta = static_cast<float *>(workspace);
+    BwdPrepParams pp{};
+    pp.B = a->B, pp.H = a->H, pp.Tq = a->Tq, pp.Dv = a->Dv;
+    pp.o = static_cast<const __nv_bfloat16 *>(a->o), pp.dout = static_cast<const __nv_bfloat16 *>(a->dout);
+    for (int i = 0; i < 3; ++i) pp.os[i] = a->o_strides[i], pp.dos[i] = a->do_strides[i];
+    pp.lse = a->lse, pp.dlse = a->dlse, pp.sinks = a->sinks, pp.delta = delta, pp.dsinks = a->dsinks;
+    note_dispatch("bwd_prep_kernel");
+    if (launch_bwd_prep(pp, s) != cudaSuccess) return ARC_ERR_CUDA;
+
+    BwdParams p;
+    memset(&p, 0, sizeof(p));
+    const int G = a->H / a->Hkv;
+    const int BR = bwd_tile_rows(a->D, a->Dv);
+    auto qmap = [&](CUtensorMap *m, const void *base, const int64_t *st3, int width, uint32_t rows) {
+        const uint64_t d[3] = {(uint64_t)width, (uint64_t)a->H * a->Tq, (uint64_t)a->B};
+        const int64_t sv[2] = {st3[2], st3[0] ? st3[0] : (int64_t)a->H * a->Tq * st3[2]};
+        return make_map(m, base, 3, d, sv, rows);
+    };
+    auto kmap = [&](CUtensorMap *m, const void *base, const int64_t *st3, int width) {
+        const uint64_t d[4] = {(uint64_t)width, (uint64_t)a->Tk, (uint64_t)a->Hkv, (uint64_t)a->B};
+        const int64_t sv[3] = {st3[2], st3[1] ? st3[1] : (int64_t)a->Tk * st3[2],
+                               st3[0] ? st3[0] : (int64_t)a->Hkv * a->Tk * st3[2]};
+        return make_map(m, base, 4, d, sv, 128);
+    };
+    if (a->Tk > 0 &&
+        (!qmap(&p.tm_q, a->q, a->q_strides, a->D, 128) || !qmap(&p.tm_do, a->dout, a->do_strides, a->Dv, 128) ||
+         !qmap(&p.tm_qr, a->q, a->q_strides, a->D, BR) || !qmap(&p.tm_dor, a->dout, a->do_strides, a->Dv, BR) ||
+         !kmap(&p.tm_k, a->k, a->k_strides, a->D) || !kmap(&p.tm_v, a->v, a->v_strides, a->Dv)))
+        return ARC_ERR_CUDA;
+    p.B = a->B, p.H = a->H, p.Hkv = a->Hkv, p.G = G, p.Tq = a->Tq, p.Tk = a->Tk, p.D = a->D, p.Dv = a->Dv;
+    p.causal = a->causal;
+    p.lse = a->lse, p.delta = delta;
+    p.scale = scale, p.scale_log2 = scale * kLog2e;
+    p.dq = static_cast<__nv_bfloat16 *>(a->dq), p.dk = static_cast<__nv_bfloat16 *>(a->dk);
+    p.dv = static_cast<__nv_bfloat16 *>(a->dv);
+    for (int i = 0; i < 3; ++i) p.dqs[i] = a->dq_strides[i], p.dks[i] = a->dk_strides[i], p.dvs[i] = a->dv_strides[i];
+    p.rsplit = pl.rsplit, p.tiles_per_split = pl.tiles_per_split;
+    p.dkv_part = pl.rsplit > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + pl.delta_bytes) : nullptr;
+    p.status = a->status;
+    if (a->Tk == 0) {
+        // no key: every gradient is zero; the dQ kernel writes them (no key tile to visit)
+        p.rsplit = 1;
+    }
+    note_dispatch("bwd_dkdv_kernel");
+    note_dispatch("bwd_dq_kernel");
+    return launch_bwd(p, s) == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
 }
 
 size_t arc_sparse_decode_workspace_size(const arc_sparse_args *a)
@@ -1020,6 +1149,24 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
             out->tile_m = 4;
         }
         out->launches = 1;
+        return ARC_OK;
+    }
+    if (op == ARC_OP_ATTN_BWD) {
+        const arc_attn_bwd_args *a = static_cast<const arc_attn_bwd_args *>(args);
+        arc_status st = check_bwd(a);
+        if (st != ARC_OK) return st;
+        if (a->B == 0 || a->Tq == 0) {
+            set_name(out, "none");
+            return ARC_OK;
+        }
+        const BwdPlan pl = plan_bwd(a);
+        set_name(out, "bwd_dkdv_kernel+bwd_dq_kernel");
+        out->tensor_cores = 1;
+        out->tile_m = 128, out->tile_n = bwd_tile_rows(a->D, a->Dv), out->d_slice = a->D;
+        out->splits = pl.rsplit;
+        out->n_ctas = a->B * a->Hkv * pl.n_kt * pl.rsplit;
+        out->smem_bytes = bwd_dkdv_smem_bytes(a->D, a->Dv), out->tmem_cols = 512;
+        out->launches = 3 + (a->sinks ? 1 : 0) + (pl.rsplit > 1 ? 1 : 0);
         return ARC_OK;
     }
     if (op == ARC_OP_SPARSE_DECODE) {

@@ -1,0 +1,721 @@
+// attn_bwd.cu -- backward of the fused attention forward (dense / GQA fold, sinks)
+// on tcgen05 tensor cores: dQ, dK, dV and the sink gradient from Q, K, V, O, dO
+// and the forward's LSE.
+//
+// The gradients are the derivative of the forward definition.  With
+// S = scale * Q K^T (masked entries -inf), P = exp(S - LSE) (the LSE includes the
+// sink, so P is the forward's softmax), D_i = sum_d dO_id O_id and an optional
+// upstream dLSE:
+//     dV = P^T dO        dP = dO V^T        dS = P * (dP - (D_i - dLSE_i))
+//     dQ = scale dS K    dK = scale dS^T Q  d sink_h = -sum_i exp(sink_h - LSE_i) (D_i - dLSE_i)
+// "TransformerEngine: FA4 in context-parallel attention" (flowchart) runs FA4's
+// raw backward per chunk in this form: P and D are rebuilt from the saved O and
+// LSE.  GQA sums dK, dV over the g query heads of a kv head; here that sum is a
+// loop over the kv group's g*Tq fold rows (the fold of "ArcFlash ... rung 0"),
+// inside one accumulator, with no atomics.
+//
+// Kernels (every wait bounded; a wait that runs out reports through p.status):
+//   bwd_prep_kernel   one warp per row: delta_i = D_i - dLSE_i (HBM-bound)
+//   bwd_dsink_kernel  one CTA per head: the sink gradient, a fixed-order sum
+//   bwd_dkdv_kernel   one CTA per (batch, kv head, 128-key tile[, row split]):
+//                       S^T  = K Q^T       M=128 keys, N=BR fold rows
+//                       dP^T = V dO^T
+//                       P^T, dS^T from S^T, dP^T, LSE, delta (softmax warps),
+//                       written back over S^T / dP^T as bf16 (TMEM A operands)
+//                       dV  += P^T dO      dK += dS^T Q   (dO, Q read MN-major)
+//                     TMEM: dV [0, DV), dK [DV, DV+D), S^T and dP^T (BR each)
+//   bwd_dq_kernel     one CTA per (batch, kv head, 128-row fold tile):
+//                       S = Q K^T, dP = dO V^T, dS (softmax warps, over S),
+//                       dQ += dS K         (K read MN-major)
+//                     TMEM: dQ [0, D), S [256, 384), dP [384, 512)
+//   bwd_reduce_kernel the fp32 partials of row-split dK/dV CTAs, summed in order
+// S and dP are computed in both main kernels (5 + 2 products per tile pair for
+// 5 algorithmic): the price of needing no atomics and no dS round trip
+// through memory.
+#include <math.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace arc {
+namespace {
+
+constexpr int BK = 128;                 // keys per tile (dK/dV: the CTA's keys; dQ: the streamed tile)
+constexpr int BQ = 128;                 // fold rows per dQ tile
+constexpr int KCH = 128 * 128;          // bytes of a [128 rows x 64 bf16] swizzled chunk
+constexpr int BW_THREADS = 256;         // producer, MMA issuer, 2 idle, 4 softmax / epilogue warps
+constexpr int BW_SMEM_LIMIT = 232448;
+constexpr float BW_LOG2E = 1.4426950408889634f;
+
+struct BwdBars {
+    uint64_t fixed_full;        // the CTA's resident operands (dK/dV: K, V; dQ: Q, dO)
+    uint64_t full[2], empty[2]; // two-stage ring of the streamed operand tiles
+    uint64_t s_full;            // S and dP are in TMEM
+    uint64_t p_full;            // the softmax warps wrote P / dS (128 arrivals)
+    uint64_t done;              // every MMA of the CTA finished
+    uint64_t cols;              // dK/dV: a fold tile's row quantities are in shared memory (128 arrivals)
+    uint32_t tmem_base;
+};
+
+// Where a bounded wait of the backward ran out (OR-ed into the status word beside
+// the role's ST_TIMEOUT_* code).
+enum : uint32_t {
+    BW_AT_FIXED = 1u << 8,
+    BW_AT_RING_EMPTY = 1u << 9,
+    BW_AT_RING_FULL = 1u << 10,
+    BW_AT_S_FULL = 1u << 11,
+    BW_AT_P_FULL = 1u << 12,
+    BW_AT_COLS = 1u << 13,
+    BW_AT_DONE = 1u << 14,
+    BW_IN_DQ = 1u << 15,        // the wait was in the dQ kernel (else dK / dV)
+};
+
+__device__ __forceinline__ bool bw_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// Does fold tile qt (rows qt*BR .. of the kv group) see any key at or after k0?
+__device__ __forceinline__ bool q_tile_live(const BwdParams &p, int qt, int BR, int k0)
+{
+    if (!p.causal) return true;
+    const int rows = p.G * p.Tq;
+    const int r0 = qt * BR, r_last = min(r0 + BR, rows) - 1;
+    const int t_max = (r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
+    return t_max + p.Tk - p.Tq >= k0;
+}
+
+// The per-row quantities of fold row r of kv head kvh: LSE in log2 units (+inf for a
+// row that sees nothing, so its P is 0), delta, and the last key it may see.
+struct RowInfo {
+    float lse2, delta;
+    int lim;
+};
+
+__device__ __forceinline__ RowInfo row_info(const BwdParams &p, int b, int kvh, int r)
+{
+    RowInfo ri{INFINITY, 0.f, -1};
+    if (r >= p.G * p.Tq) return ri;
+    const int h = kvh * p.G + r / p.Tq, t = r % p.Tq;
+    const int64_t i = ((int64_t)b * p.H + h) * p.Tq + t;
+    const float l = p.lse[i];
+    ri.lse2 = (l == -INFINITY) ? INFINITY : l * BW_LOG2E;
+    ri.delta = p.delta[i];
+    ri.lim = p.causal ? min(p.Tk - 1, t + p.Tk - p.Tq) : p.Tk - 1;
+    return ri;
+}
+
+template <int D, int DV, int BR>
+struct DkdvLayout {
+    static constexpr int KC = D / 64, VC = DV / 64;
+    static constexpr int QCH = BR * 128;                      // one 64-column chunk of a fold tile
+    static constexpr int STAGE = (KC + VC) * QCH;             // Q and dO of one fold tile
+    static constexpr int FIXED = (KC + VC) * KCH;             // K and V of the CTA's key tile
+    static constexpr int BYTES = 1024 + FIXED + 2 * STAGE + 3 * 2 * 128 * 4 + (int)sizeof(BwdBars);
+    static constexpr int DV_COL = 0, DK_COL = DV, S_COL = DV + D, DP_COL = DV + D + BR;
+    static_assert(DP_COL + BR <= 512, "TMEM: dV, dK, S^T and dP^T side by side");
+    static_assert(BYTES <= BW_SMEM_LIMIT, "shared memory");
+};
+
+template <int D, int DV, int BR>
+__global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
+{
+    using L = DkdvLayout<D, DV, BR>;
+    constexpr int KC = L::KC, VC = L::VC;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align_smem<1024>(smem_raw);
+    uint8_t *sK = smem, *sV = sK + KC * KCH;
+    uint8_t *sRing = sK + L::FIXED;                             // [2][Q chunks, dO chunks]
+    float *col_lse2 = reinterpret_cast<float *>(sRing + 2 * L::STAGE);   // [2][128]
+    float *col_delta = col_lse2 + 2 * 128;
+    int *col_lim = reinterpret_cast<int *>(col_delta + 2 * 128);
+    BwdBars *bars = reinterpret_cast<BwdBars *>(col_lim + 2 * 128);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_kt = (p.Tk + BK - 1) / BK;
+    const int rs = blockIdx.x % p.rsplit;
+    const int kt = (blockIdx.x / p.rsplit) % n_kt;
+    const int kvh = (blockIdx.x / (p.rsplit * n_kt)) % p.Hkv;
+    const int b = blockIdx.x / (p.rsplit * n_kt * p.Hkv);
+    const int k0 = kt * BK;
+    const int n_qt = (p.G * p.Tq + BR - 1) / BR;
+    const int qt_begin = rs * p.tiles_per_split, qt_end = min(n_qt, qt_begin + p.tiles_per_split);
+    const int row_base = kvh * p.G * p.Tq;                      // fold row 0 in the [H*Tq] view
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->fixed_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->full[i], 1);
+            mbar_init(&bars->empty[i], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->done, 1);
+        mbar_init(&bars->cols, 128);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // =============================== TMA producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(&bars->fixed_full, L::FIXED);
+            for (int c = 0; c < KC; ++c) tma_load_4d(sK + c * KCH, &p.tm_k, &bars->fixed_full, c * 64, k0, kvh, b);
+            for (int c = 0; c < VC; ++c) tma_load_4d(sV + c * KCH, &p.tm_v, &bars->fixed_full, c * 64, k0, kvh, b);
+            int it = 0;
+            bool ok = true;
+            for (int qt = qt_begin; qt < qt_end && ok; ++qt) {
+                if (!q_tile_live(p, qt, BR, k0)) continue;
+                const int st = it & 1;
+                if (it >= 2) ok = mbar_wait(&bars->empty[st], (uint32_t)(((it >> 1) - 1) & 1));
+                if (!ok) {
+                    report(p.status, BW_AT_RING_EMPTY);
+                    break;
+                }
+                uint8_t *dst = sRing + st * L::STAGE;
+                mbar_arrive_expect_tx(&bars->full[st], L::STAGE);
+                for (int c = 0; c < KC; ++c)
+                    tma_load_3d(dst + c * L::QCH, &p.tm_qr, &bars->full[st], c * 64, row_base + qt * BR, b);
+                for (int c = 0; c < VC; ++c)
+                    tma_load_3d(dst + (KC + c) * L::QCH, &p.tm_dor, &bars->full[st], c * 64, row_base + qt * BR, b);
+                ++it;
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_LOAD);
+            // every copy issued has landed before the CTA may exit
+            for (int i = (it > 2 ? it - 2 : 0); i < it; ++i) mbar_wait(&bars->full[i & 1], (uint32_t)((i >> 1) & 1));
+            mbar_wait(&bars->fixed_full, 0);
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16(128, BR, false, false);
+            const uint32_t idesc_dv = idesc_bf16(128, DV, false, true);
+            const uint32_t idesc_dk = idesc_bf16(128, D, false, true);
+            const uint64_t kd0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t vd0 = sdesc_sw128(smem_u32(sV), 16, 1024);
+            bool ok = mbar_wait(&bars->fixed_full, 0);
+            if (!ok) report(p.status, BW_AT_FIXED);
+            tc_fence_after();
+            int it = 0;
+            for (int qt = qt_begin; qt < qt_end && ok; ++qt) {
+                if (!q_tile_live(p, qt, BR, k0)) continue;
+                const int st = it & 1;
+                if (!(ok = mbar_wait(&bars->full[st], (uint32_t)((it >> 1) & 1)))) {
+                    report(p.status, BW_AT_RING_FULL);
+                    break;
+                }
+                tc_fence_after();
+                uint8_t *sq = sRing + st * L::STAGE, *sdo = sq + KC * L::QCH;
+                const uint64_t qd = sdesc_sw128(smem_u32(sq), 16, 1024);
+                const uint64_t dod = sdesc_sw128(smem_u32(sdo), 16, 1024);
+                // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+#pragma unroll
+                for (int c = 0; c < KC; ++c)
+                    umma_ss_k64(tmem + L::S_COL, kd0 + (uint64_t)(c * (KCH >> 4)), qd + (uint64_t)(c * (L::QCH >> 4)),
+                                idesc_s, c > 0);
+#pragma unroll
+                for (int c = 0; c < VC; ++c)
+                    umma_ss_k64(tmem + L::DP_COL, vd0 + (uint64_t)(c * (KCH >> 4)), dod + (uint64_t)(c * (L::QCH >> 4)),
+                                idesc_s, c > 0);
+                umma_commit(&bars->s_full);
+                if (!(ok = mbar_wait(&bars->p_full, (uint32_t)(it & 1)))) {
+                    report(p.status, BW_AT_P_FULL);
+                    break;
+                }
+                tc_fence_after();
+                // dV += P^T dO, dK += dS^T Q: A from TMEM, B read MN-major (16 fold rows = 2048 B per K step)
+                const uint64_t dob = sdesc_sw128(smem_u32(sdo), L::QCH, 1024);
+                const uint64_t qb = sdesc_sw128(smem_u32(sq), L::QCH, 1024);
+                const uint32_t acc = it > 0;
+#pragma unroll
+                for (int k4 = 0; k4 < BR / 64; ++k4)
+                    umma_ts_k64(tmem + L::DV_COL, tmem + L::S_COL + k4 * 32, dob + (uint64_t)(k4 * 512), 128, idesc_dv,
+                                acc | k4);
+#pragma unroll
+                for (int k4 = 0; k4 < BR / 64; ++k4)
+                    umma_ts_k64(tmem + L::DK_COL, tmem + L::DP_COL + k4 * 32, qb + (uint64_t)(k4 * 512), 128, idesc_dk,
+                                acc | k4);
+                umma_commit(&bars->empty[st]);   // the stage is free once these have read it
+                ++it;
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_MMA);
+            umma_commit(&bars->done);
+            mbar_wait(&bars->done, 0);
+        }
+    } else if (warp >= 4) {
+        // =============================== P^T, dS^T (one thread per key) and the epilogue
+        const int tid = threadIdx.x - 128;                      // key lane 0..127
+        const int kj = k0 + tid;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const float sl2 = p.scale_log2;
+        int it = 0;
+        bool ok = true;
+        for (int qt = qt_begin; qt < qt_end; ++qt) {
+            if (!q_tile_live(p, qt, BR, k0)) continue;
+            const int cb = (it & 1) * 128;
+            if (tid < BR) {
+                const RowInfo ri = row_info(p, b, kvh, qt * BR + tid);
+                col_lse2[cb + tid] = ri.lse2;
+                col_delta[cb + tid] = ri.delta;
+                col_lim[cb + tid] = ri.lim;
+            }
+            // every softmax thread has written its column (a bounded wait, unlike a named
+            // barrier, so a thread that stopped early cannot hold the others forever)
+            mbar_arrive(&bars->cols);
+            ok = bw_all(mbar_wait(&bars->cols, (uint32_t)(it & 1)));
+            if (!ok) {
+                report(p.status, BW_AT_COLS);
+                break;
+            }
+            ok = bw_all(mbar_wait(&bars->s_full, (uint32_t)(it & 1)));
+            if (!ok) {
+                report(p.status, BW_AT_S_FULL);
+                break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int ch = 0; ch < BR / 32; ++ch) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(tmem + lane_off + L::S_COL + 32 * ch, sv);
+                tmem_ld32(tmem + lane_off + L::DP_COL + 32 * ch, dv);
+                tmem_wait_ld();
+                uint32_t pk[16], dk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float pp[2], dd[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int c = cb + 32 * ch + 2 * i + e;
+                        const float pe = kj <= col_lim[c]
+                                             ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -col_lse2[c]))
+                                             : 0.f;
+                        pp[e] = pe;
+                        dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - col_delta[c]);
+                    }
+                    pk[i] = pack_bf16(pp[0], pp[1]);
+                    dk[i] = pack_bf16(dd[0], dd[1]);
+                }
+                // bf16 pairs over the first half of the columns just read
+                tmem_st16(tmem + lane_off + L::S_COL + 16 * ch, pk);
+                tmem_st16(tmem + lane_off + L::DP_COL + 16 * ch, dk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+            ++it;
+        }
+        if (ok && it > 0) ok = bw_all(mbar_wait(&bars->done, 0));
+        if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
+        tc_fence_after();
+        // ---- epilogue: dV and scale * dK of key kj (fp32 partials under a row split).
+        // The TMEM loads are warp-collective: every lane loads, only keys < Tk store.
+        const bool live = it > 0 && ok;
+        const bool key_ok = kj < p.Tk;
+        float *prow = p.dkv_part + ((((int64_t)rs * p.B + b) * p.Hkv + kvh) * p.Tk + kj) * (D + DV);
+        __nv_bfloat16 *dkrow = p.dk + (int64_t)b * p.dks[0] + (int64_t)kvh * p.dks[1] + (int64_t)kj * p.dks[2];
+        __nv_bfloat16 *dvrow = p.dv + (int64_t)b * p.dvs[0] + (int64_t)kvh * p.dvs[1] + (int64_t)kj * p.dvs[2];
+#pragma unroll 1
+        for (int c = 0; c < (D + DV) / 32; ++c) {
+            uint32_t v[32];
+            const bool is_k = c < D / 32;
+            const int col = is_k ? L::DK_COL + 32 * c : L::DV_COL + 32 * (c - D / 32);
+            if (live) {
+                tmem_ld32(tmem + lane_off + col, v);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0u;
+            }
+            if (!key_ok) continue;
+            if (p.rsplit > 1) {
+                float4 *dst = reinterpret_cast<float4 *>(prow + 32 * c);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            } else {
+                const float f = is_k ? p.scale : 1.f;
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    w[i] = pack_bf16(__uint_as_float(v[2 * i]) * f, __uint_as_float(v[2 * i + 1]) * f);
+                uint4 *dst = reinterpret_cast<uint4 *>(is_k ? dkrow + 32 * c : dvrow + 32 * (c - D / 32));
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D, int DV>
+struct DqLayout {
+    static constexpr int KC = D / 64, VC = DV / 64;
+    static constexpr int FIXED = (KC + VC) * KCH;             // Q and dO of the CTA's fold tile
+    static constexpr int STAGE = (KC + VC) * KCH;             // K and V of one key tile
+    // two ring stages where they fit beside Q and dO, else one (d 192: the next key
+    // tile then loads only once the last one is consumed)
+    static constexpr int NSTG = 1024 + FIXED + 2 * STAGE + (int)sizeof(BwdBars) <= BW_SMEM_LIMIT ? 2 : 1;
+    static constexpr int BYTES = 1024 + FIXED + NSTG * STAGE + (int)sizeof(BwdBars);
+    static constexpr int DQ_COL = 0, S_COL = 256, DP_COL = 384;
+    static_assert(D <= 256, "TMEM: dQ, S and dP side by side");
+    static_assert(BYTES <= BW_SMEM_LIMIT, "shared memory");
+};
+
+template <int D, int DV>
+__global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p)
+{
+    using L = DqLayout<D, DV>;
+    constexpr int KC = L::KC, VC = L::VC;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = align_smem<1024>(smem_raw);
+    uint8_t *sQ = smem, *sdO = sQ + KC * KCH;
+    uint8_t *sRing = smem + L::FIXED;                           // [NSTG][K chunks, V chunks]
+    BwdBars *bars = reinterpret_cast<BwdBars *>(sRing + L::NSTG * L::STAGE);
+    constexpr int NS = L::NSTG;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rows = p.G * p.Tq;
+    const int n_rt = (rows + BQ - 1) / BQ;
+    // heavier tiles (later positions see more keys) first
+    const int rt = n_rt - 1 - blockIdx.x % n_rt;
+    const int kvh = (blockIdx.x / n_rt) % p.Hkv;
+    const int b = blockIdx.x / (n_rt * p.Hkv);
+    const int r0 = rt * BQ;
+    int nt;
+    {
+        const int r_last = min(r0 + BQ, rows) - 1;
+        const int t_max = (r0 / p.Tq != r_last / p.Tq) ? p.Tq - 1 : r_last % p.Tq;
+        const int kv_last = p.causal ? min(p.Tk - 1, t_max + p.Tk - p.Tq) : p.Tk - 1;
+        nt = kv_last < 0 ? 0 : kv_last / BK + 1;
+    }
+    const int row_base = kvh * rows;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->fixed_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars->full[i], 1);
+            mbar_init(&bars->empty[i], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_full, 128);
+        mbar_init(&bars->done, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // =============================== TMA producer
+        if (lane == 0 && nt > 0) {
+            mbar_arrive_expect_tx(&bars->fixed_full, L::FIXED);
+            for (int c = 0; c < KC; ++c) tma_load_3d(sQ + c * KCH, &p.tm_q, &bars->fixed_full, c * 64, row_base + r0, b);
+            for (int c = 0; c < VC; ++c) tma_load_3d(sdO + c * KCH, &p.tm_do, &bars->fixed_full, c * 64, row_base + r0, b);
+            bool ok = true;
+            for (int j = 0; j < nt && ok; ++j) {
+                const int st = j % NS;
+                if (j >= NS) ok = mbar_wait(&bars->empty[st], (uint32_t)((j / NS - 1) & 1));
+                if (!ok) {
+                    report(p.status, BW_IN_DQ | BW_AT_RING_EMPTY);
+                    break;
+                }
+                uint8_t *dst = sRing + st * L::STAGE;
+                mbar_arrive_expect_tx(&bars->full[st], L::STAGE);
+                for (int c = 0; c < KC; ++c) tma_load_4d(dst + c * KCH, &p.tm_k, &bars->full[st], c * 64, j * BK, kvh, b);
+                for (int c = 0; c < VC; ++c)
+                    tma_load_4d(dst + (KC + c) * KCH, &p.tm_v, &bars->full[st], c * 64, j * BK, kvh, b);
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_LOAD);
+            for (int i = (nt > NS ? nt - NS : 0); i < nt; ++i) mbar_wait(&bars->full[i % NS], (uint32_t)((i / NS) & 1));
+            mbar_wait(&bars->fixed_full, 0);
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer
+        if (lane == 0 && nt > 0) {
+            const uint32_t idesc_s = idesc_bf16(128, BK, false, false);
+            const uint32_t idesc_dq = idesc_bf16(128, D, false, true);
+            const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dod0 = sdesc_sw128(smem_u32(sdO), 16, 1024);
+            bool ok = mbar_wait(&bars->fixed_full, 0);
+            if (!ok) report(p.status, BW_IN_DQ | BW_AT_FIXED);
+            tc_fence_after();
+            for (int j = 0; j < nt && ok; ++j) {
+                const int st = j % NS;
+                if (!(ok = mbar_wait(&bars->full[st], (uint32_t)((j / NS) & 1)))) {
+                    report(p.status, BW_IN_DQ | BW_AT_RING_FULL);
+                    break;
+                }
+                tc_fence_after();
+                uint8_t *sk = sRing + st * L::STAGE, *sv = sk + KC * KCH;
+                const uint64_t kd = sdesc_sw128(smem_u32(sk), 16, 1024);
+                const uint64_t vd = sdesc_sw128(smem_u32(sv), 16, 1024);
+#pragma unroll
+                for (int c = 0; c < KC; ++c)
+                    umma_ss_k64(tmem + L::S_COL, qd0 + (uint64_t)(c * (KCH >> 4)), kd + (uint64_t)(c * (KCH >> 4)), idesc_s,
+                                c > 0);
+#pragma unroll
+                for (int c = 0; c < VC; ++c)
+                    umma_ss_k64(tmem + L::DP_COL, dod0 + (uint64_t)(c * (KCH >> 4)), vd + (uint64_t)(c * (KCH >> 4)),
+                                idesc_s, c > 0);
+                umma_commit(&bars->s_full);
+                if (!(ok = mbar_wait(&bars->p_full, (uint32_t)(j & 1)))) {
+                    report(p.status, BW_IN_DQ | BW_AT_P_FULL);
+                    break;
+                }
+                tc_fence_after();
+                // dQ += dS K: dS from TMEM, K read MN-major (16 keys = 2048 B per K step)
+                const uint64_t kb = sdesc_sw128(smem_u32(sk), KCH, 1024);
+                const uint32_t acc = j > 0;
+#pragma unroll
+                for (int k4 = 0; k4 < BK / 64; ++k4)
+                    umma_ts_k64(tmem + L::DQ_COL, tmem + L::S_COL + k4 * 32, kb + (uint64_t)(k4 * 512), 128, idesc_dq,
+                                acc | k4);
+                umma_commit(&bars->empty[st]);
+            }
+            if (!ok) report(p.status, ST_TIMEOUT_MMA);
+            umma_commit(&bars->done);
+            mbar_wait(&bars->done, 0);
+        }
+    } else if (warp >= 4) {
+        // =============================== dS (one thread per fold row) and the epilogue
+        const int tid = threadIdx.x - 128;
+        const int r = r0 + tid;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const RowInfo ri = row_info(p, b, kvh, r);
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int j = 0; j < nt; ++j) {
+            ok = bw_all(mbar_wait(&bars->s_full, (uint32_t)(j & 1)));
+            if (!ok) {
+                report(p.status, BW_IN_DQ | BW_AT_S_FULL);
+                break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int ch = 0; ch < BK / 32; ++ch) {
+                uint32_t sv[32], dv[32];
+                tmem_ld32(tmem + lane_off + L::S_COL + 32 * ch, sv);
+                tmem_ld32(tmem + lane_off + L::DP_COL + 32 * ch, dv);
+                tmem_wait_ld();
+                const int key0 = j * BK + 32 * ch;
+                uint32_t dk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    float dd[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float pe = key0 + 2 * i + e <= ri.lim
+                                             ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ri.lse2))
+                                             : 0.f;
+                        dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - ri.delta);
+                    }
+                    dk[i] = pack_bf16(dd[0], dd[1]);
+                }
+                tmem_st16(tmem + lane_off + L::S_COL + 16 * ch, dk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->p_full);
+        }
+        if (ok && nt > 0) ok = bw_all(mbar_wait(&bars->done, 0));
+        if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
+        tc_fence_after();
+        // warp-collective TMEM loads by every lane; only rows of the group store
+        const bool row_ok = r < rows;
+        const int h = kvh * p.G + (row_ok ? r / p.Tq : 0), t = row_ok ? r % p.Tq : 0;
+        __nv_bfloat16 *dqrow = p.dq + (int64_t)b * p.dqs[0] + (int64_t)h * p.dqs[1] + (int64_t)t * p.dqs[2];
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            if (nt > 0 && ok) {
+                tmem_ld32(tmem + lane_off + L::DQ_COL + 32 * c, v);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0u;
+            }
+            if (!row_ok) continue;
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                w[i] = pack_bf16(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
+            uint4 *dst = reinterpret_cast<uint4 *>(dqrow + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// delta_i = sum_d dO_id O_id - dLSE_i, one warp per row (b, h, t); 8 elements per lane
+// and step (16-byte loads).
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ BwdPrepParams p)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+    if (row >= (int64_t)p.B * p.H * p.Tq) return;
+    const int t = (int)(row % p.Tq), h = (int)((row / p.Tq) % p.H), b = (int)(row / ((int64_t)p.Tq * p.H));
+    const __nv_bfloat16 *o = p.o + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)t * p.os[2];
+    const __nv_bfloat16 *g = p.dout + (int64_t)b * p.dos[0] + (int64_t)h * p.dos[1] + (int64_t)t * p.dos[2];
+    float acc = 0.f;
+    for (int d = lane * 8; d < p.Dv; d += 256) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(o + d), y = *reinterpret_cast<const uint4 *>(g + d);
+        const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw[k]));
+            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[k]));
+            acc = fmaf(a.x, c.x, acc);
+            acc = fmaf(a.y, c.y, acc);
+        }
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) p.delta[row] = acc - (p.dlse ? p.dlse[row] : 0.f);
+}
+
+// d sink_h = -sum_{b,t} exp(sink_h - LSE_bht) * delta_bht, one CTA per head, a fixed
+// summation order (strided per thread, then a tree), so the result is reproducible.
+__global__ void __launch_bounds__(256) bwd_dsink_kernel(const __grid_constant__ BwdPrepParams p)
+{
+    __shared__ float red[8];
+    const int h = blockIdx.x;
+    const float sink = p.sinks[h];
+    float acc = 0.f;
+    const int n = p.B * p.Tq;
+    for (int i = threadIdx.x; i < n; i += 256) {
+        const int b = i / p.Tq, t = i % p.Tq;
+        const int64_t row = ((int64_t)b * p.H + h) * p.Tq + t;
+        const float l = p.lse[row];
+        if (l != -INFINITY) acc += expf(sink - l) * p.delta[row];
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += red[w];
+        p.dsinks[h] = -s;
+    }
+}
+
+// Row-split dK / dV: sum the fp32 partials of the splits in split order, scale dK, write bf16.
+template <int D, int DV>
+__global__ void __launch_bounds__(256) bwd_reduce_kernel(const __grid_constant__ BwdParams p)
+{
+    constexpr int W = D + DV;
+    const int64_t x = (int64_t)blockIdx.x * 256 + threadIdx.x;      // one thread per 4 elements
+    const int64_t rows = (int64_t)p.B * p.Hkv * p.Tk;
+    if (x >= rows * (W / 4)) return;
+    const int64_t row = x / (W / 4);
+    const int e = (int)(x % (W / 4)) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < p.rsplit; ++s) {
+        const float4 v = *reinterpret_cast<const float4 *>(p.dkv_part + ((int64_t)s * rows + row) * W + e);
+        acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+    }
+    const int kj = (int)(row % p.Tk), kvh = (int)((row / p.Tk) % p.Hkv), b = (int)(row / ((int64_t)p.Tk * p.Hkv));
+    __nv_bfloat16 *dst;
+    float f = 1.f;
+    if (e < D) {
+        dst = p.dk + (int64_t)b * p.dks[0] + (int64_t)kvh * p.dks[1] + (int64_t)kj * p.dks[2] + e;
+        f = p.scale;
+    } else {
+        dst = p.dv + (int64_t)b * p.dvs[0] + (int64_t)kvh * p.dvs[1] + (int64_t)kj * p.dvs[2] + (e - D);
+    }
+    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16(acc.x * f, acc.y * f), pack_bf16(acc.z * f, acc.w * f));
+}
+
+template <int D, int DV, int BR>
+cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
+{
+    cudaError_t e;
+    {
+        auto kern = bwd_dkdv_kernel<D, DV, BR>;
+        // at least 116 KB so one CTA holds an SM: each allocates all 512 TMEM columns
+        const int bytes = DkdvLayout<D, DV, BR>::BYTES > 118784 ? DkdvLayout<D, DV, BR>::BYTES : 118784;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+        const int grid = p.B * p.Hkv * ((p.Tk + BK - 1) / BK) * p.rsplit;
+        if (grid > 0) kern<<<grid, BW_THREADS, bytes, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (p.rsplit > 1 && p.Tk > 0) {
+        const int64_t n = (int64_t)p.B * p.Hkv * p.Tk * ((D + DV) / 4);
+        bwd_reduce_kernel<D, DV><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        auto kern = bwd_dq_kernel<D, DV>;
+        const int bytes = DqLayout<D, DV>::BYTES > 118784 ? DqLayout<D, DV>::BYTES : 118784;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
+        const int grid = p.B * p.Hkv * ((p.G * p.Tq + BQ - 1) / BQ);
+        kern<<<grid, BW_THREADS, bytes, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool bwd_supported(int d, int dv) { return (d == 64 && dv == 64) || (d == 128 && dv == 128) || (d == 192 && dv == 128); }
+
+// fold rows per dK/dV tile: 128, or 64 where TMEM needs the room (d 192)
+int bwd_tile_rows(int d, int dv) { return d + dv + 2 * 128 <= 512 ? 128 : 64; }
+
+cudaError_t launch_bwd_prep(const BwdPrepParams &p, cudaStream_t s)
+{
+    const int64_t rows = (int64_t)p.B * p.H * p.Tq;
+    if (rows == 0) return cudaSuccess;
+    bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || !p.sinks) return e;
+    bwd_dsink_kernel<<<p.H, 256, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd(const BwdParams &p, cudaStream_t s)
+{
+    if (p.D == 64 && p.Dv == 64) return launch_bwd_t<64, 64, 128>(p, s);
+    if (p.D == 128 && p.Dv == 128) return launch_bwd_t<128, 128, 128>(p, s);
+    if (p.D == 192 && p.Dv == 128) return launch_bwd_t<192, 128, 64>(p, s);
+    return cudaErrorInvalidValue;
+}
+
+int bwd_dkdv_smem_bytes(int d, int dv)
+{
+    if (d == 64) return DkdvLayout<64, 64, 128>::BYTES;
+    if (d == 128) return DkdvLayout<128, 128, 128>::BYTES;
+    return DkdvLayout<192, 128, 64>::BYTES;
+}
+
+int bwd_dq_smem_bytes(int d, int dv)
+{
+    if (d == 64) return DqLayout<64, 64>::BYTES;
+    if (d == 128) return DqLayout<128, 128>::BYTES;
+    return DqLayout<192, 128>::BYTES;
+}
+
+}  // namespace arc

@@ -132,6 +132,38 @@ int decode_smem_bytes(int kv_type, int D, int mf, bool tma);
 int decode_blocks_per_sm(int kv_type, int D, int mf, bool tma);
 void decode_box(int kv_type, int D, int mf, int *width, int *cells);
 
+// ---------------------------------------------------------------- backward (dense / GQA, sinks)
+// delta = rowsum(dO * O) - dLSE per row, and the sink gradient.
+struct BwdPrepParams {
+    int B, H, Tq, Dv;
+    const __nv_bfloat16 *o, *dout;
+    int64_t os[3], dos[3];
+    const float *lse, *dlse, *sinks;
+    float *delta;       // [B,H,Tq] (workspace)
+    float *dsinks;      // [H]
+};
+cudaError_t launch_bwd_prep(const BwdPrepParams &p, cudaStream_t s);
+
+struct BwdParams {
+    CUtensorMap tm_q, tm_do;    // q / dO {D, H*Tq, B}, box {64, 128}      (dQ kernel)
+    CUtensorMap tm_qr, tm_dor;  // the same, box {64, fold-tile rows}      (dK/dV kernel)
+    CUtensorMap tm_k, tm_v;     // k / v {D, Tk, Hkv, B}, box {64, 128}
+    int B, H, Hkv, G, Tq, Tk, D, Dv;
+    int causal;
+    const float *lse, *delta;   // [B,H,Tq]
+    float scale, scale_log2;
+    __nv_bfloat16 *dq, *dk, *dv;
+    int64_t dqs[3], dks[3], dvs[3];
+    int rsplit, tiles_per_split;// dK/dV CTAs per key tile along the fold rows, and fold tiles each
+    float *dkv_part;            // rsplit > 1: fp32 [rsplit][B][Hkv][Tk][D + Dv] (dK unscaled, then dV)
+    uint32_t *status;
+};
+bool bwd_supported(int d, int dv);
+int bwd_tile_rows(int d, int dv);
+int bwd_dkdv_smem_bytes(int d, int dv);
+int bwd_dq_smem_bytes(int d, int dv);
+cudaError_t launch_bwd(const BwdParams &p, cudaStream_t s);
+
 cudaError_t launch_selftest_timeout(uint32_t *status, uint64_t timeout_ns, cudaStream_t s);
 
 // Merge of partial results over disjoint key sets (arc_attn_merge), one warp per row.

@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define ARC_ABI_VERSION 1
+#define ARC_ABI_VERSION 2
 
 typedef enum {
     ARC_OK = 0,
@@ -384,6 +384,64 @@ typedef struct {
 } arc_merge_args;
 
 arc_status arc_attn_merge(const arc_merge_args *args, void *stream);
+
+/* --------------------------------------------------------------------------
+ * arc_attn_bwd: gradients of arc_attn_fwd (dense / GQA, causal or not, sinks).
+ *
+ * Source: "TransformerEngine: FA4 in context-parallel attention", flowchart:
+ * the backward of each chunk is FA4's raw backward, from the saved O and LSE;
+ * "pith-train: FA4 b19 return arity and MLA q/k concat" trains through the same
+ * kernel.  The pages give no formula, so the gradients are the derivative of
+ * the forward definition above (sink included):
+ *     P = exp(scale q.k_j - LSE),  D_i = sum_d dO_id O_id,  delta_i = D_i - dLSE_i
+ *     dV = P^T dO,   dS = P * (dO V^T - delta),   dQ = scale dS K,   dK = scale dS^T Q
+ *     d sink_h = -sum_i exp(sink_h - LSE_i) delta_i
+ * summed over the g query heads of each kv head for dK and dV.
+ *
+ *   q, k, v, o, lse   as the forward's arguments and outputs (o, lse: the
+ *                     forward's results for these q, k, v, sinks)
+ *   dout [B,H,Tq,Dv]  bf16, device, strides do_strides: the gradient of the loss wrt o
+ *   dlse [B,H,Tq]     fp32, device, contiguous, or NULL: the gradient wrt lse
+ *   dq [B,H,Tq,D], dk [B,Hkv,Tk,D], dv [B,Hkv,Tk,Dv]  bf16, device, written
+ *   dsinks [H]        fp32, device, written when sinks != NULL
+ * bf16 only, (D, Dv) in {(64,64), (128,128), (192,128)}; the tensor-core
+ * layout needs each (b, kv) group's g*Tq query rows evenly spaced (head stride
+ * == Tq * token stride) for q and dout, and 16-byte aligned rows and base
+ * pointers everywhere.  P and dS are rounded to bf16 for the tensor cores, as in
+ * the forward; accumulation is fp32.  Every sum runs in a fixed order (no
+ * atomics): the same call twice gives the same bits.
+ *   workspace  device, at least arc_attn_bwd_workspace_size(args) bytes, 256-byte
+ *              aligned, overwritten; holds delta and, when the dK/dV work of a
+ *              key tile is split over CTAs along the query rows, their fp32
+ *              partials.  Its contents need no initialisation.
+ * Launches: delta (and the sink gradient), dK/dV, the split reduction when
+ * there is one, dQ.  Errors, before any launch: as arc_attn_fwd for shapes,
+ * strides and pointers (ARC_ERR_UNSUPPORTED for another head-dim pair or
+ * layout); a missing, short or unaligned workspace is ARC_ERR_WORKSPACE.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t B, H, Hkv, Tq, Tk, D, Dv;
+    const void *q;    int64_t q_strides[3];
+    const void *k;    int64_t k_strides[3];
+    const void *v;    int64_t v_strides[3];
+    const void *o;    int64_t o_strides[3];
+    const void *dout; int64_t do_strides[3];
+    const float *lse;
+    const float *dlse;
+    const float *sinks;
+    void *dq;         int64_t dq_strides[3];
+    void *dk;         int64_t dk_strides[3];
+    void *dv;         int64_t dv_strides[3];
+    float *dsinks;
+    float scale;
+    int32_t causal;
+    uint32_t flags;
+    uint32_t *status;
+} arc_attn_bwd_args;
+
+size_t arc_attn_bwd_workspace_size(const arc_attn_bwd_args *args);
+
+arc_status arc_attn_bwd(const arc_attn_bwd_args *args, void *workspace, size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
  * Engagement record and helpers.

@@ -308,6 +308,20 @@ def merge_case(n_parts=2, B=1, H=64, T=1400, Dv=512, *, sinks=True, empty_frac=0
     return MergeCase(B, H, T, Dv, o, lse, s, seed)
 
 
+@dataclass
+class Upstream:
+    """Upstream gradients for a backward pass: dO (bf16 bits) and optionally dLSE (fp32)."""
+    do: np.ndarray                    # [B,H,Tq,Dv] bf16 bits
+    dlse: np.ndarray | None = None    # [B,H,Tq] fp32
+
+
+def upstream(B, H, Tq, Dv, *, dlse=False, std=1.0, seed=0) -> Upstream:
+    rng = make_rng(seed)
+    do = bf16_bits(normal(rng, (B, H, Tq, Dv), std))
+    dl = normal(rng, (B, H, Tq), 0.5) if dlse else None
+    return Upstream(do, dl)
+
+
 # The five workload configurations, by number, with seed = number.
 def config(i: int, **over):
     if i == 1:
