@@ -59,6 +59,14 @@ CONFIGS = {
     "c5g8": dict(cfg=9, decode=dict(n_seq=4, n_q=4, n_kv=8192, H=64, Hkv=8, D=128, kv_type=W.KV_Q8_0),
                  name="multi-seq decode, 4 seq x 4 tok, H=64 Hkv=8 (32 fold rows) D=128, 8192 cells/seq, q8_0",
                  metric="decode GB/s", dtype="q8_0"),
+    # the backward: the GQA prefill's structure (64 heads over 8, causal, sinks) at head
+    # dim 128, and the MLA prefill's head dims (192 / 128) on concatenated q/k
+    "bwd_gqa": dict(cfg=10, bwd=dict(B=1, H=64, Hkv=8, T=1400, D=128, Dv=128, sinks=True),
+                    name="attention bwd, B=1 H=64 Hkv=8 T=1400 D=128 causal, sinks",
+                    metric="attention bwd TFLOP/s", dtype="bf16"),
+    "bwd_mla": dict(cfg=11, bwd=dict(B=2, H=16, Hkv=16, T=4096, D=192, Dv=128, sinks=False),
+                    name="attention bwd, B=2 H=16 T=4096 d_qk=192 d_v=128 causal",
+                    metric="attention bwd TFLOP/s", dtype="bf16"),
     # decode-shaped sparse MLA: c4's per-token shape at a decode batch of 32 tokens
     "c4d": dict(cfg=7, sparse_decode=dict(Sq=32, H=64, Skv=65536, Dqk=512, Dv=512, topk=2176),
                 name="sparse MLA decode, 32 tokens x 64 h x 2176 top-k, d_qk=d_v=512, pool 65536",
@@ -77,11 +85,23 @@ def make_case(spec):
         return SparseDecode(W.sparse_case(**spec["sparse_decode"], seed=spec["cfg"]))
     if "decode" in spec:
         return W.decode_case(**spec["decode"], seed=spec["cfg"])
+    if "bwd" in spec:
+        b = spec["bwd"]
+        case = W.dense_case(b["B"], b["H"], b["Hkv"], b["T"], b["T"], b["D"], b["Dv"], dtype="bf16", std=0.5,
+                            causal=True, sinks=b["sinks"], seed=spec["cfg"])
+        return Backward(case, W.upstream(b["B"], b["H"], b["T"], b["Dv"], seed=spec["cfg"] + 1000))
     kw = {"kv_type": spec["kv_type"]} if "kv_type" in spec else {}
     return W.config(spec["cfg"], **kw)
 
 
 # ------------------------------------------------------------------ algorithmic work
+
+class Backward:
+    """A dense case run through arc_attn_bwd, with seeded upstream gradients."""
+
+    def __init__(self, case, up):
+        self.case, self.up = case, up
+
 
 class SparseDecode:
     """A sparse case run through arc_sparse_mla_decode (few tokens, top-k split over CTAs)."""
@@ -97,6 +117,12 @@ def dense_pairs(Tq, Tk, causal):
 
 def work(case):
     """(algorithmic units, unit name) of one call: FLOPs over visible pairs, or bytes for decode."""
+    if isinstance(case, Backward):
+        # per visible (row, key) pair: S and dP recomputed... counted once each, plus dV,
+        # dK and dQ: 2*D (S) + 2*Dv (dP) + 2*Dv (dV) + 2*D (dK) + 2*D (dQ)
+        c = case.case
+        pairs = c.B * c.H * dense_pairs(c.Tq, c.Tk, c.causal)
+        return pairs * (6 * c.D + 4 * c.Dv), "flop"
     if isinstance(case, SparseDecode):
         # memory-bound: every distinct pool row a call gathers crosses HBM once, plus Q, O,
         # LSE and the index lists
@@ -143,6 +169,26 @@ class Uploaded:
 def build_call(case, torch, arc, status):
     """Returns (call(), inputs dict of device tensors, outputs list, n_launches, kernel name)."""
     U = Uploaded(case, torch, arc)
+    if isinstance(case, Backward):
+        c = case.case
+        q, k, v = U.to_dev(c.q), U.to_dev(c.k), U.to_dev(c.v)
+        s = U.to_dev(c.sinks) if c.sinks is not None else None
+        o, lse = arc.attn_fwd(q, k, v, scale=c.scale, causal=c.causal, sinks=s)
+        do = U.to_dev(case.up.do)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        dsk = torch.empty_like(s) if s is not None else None
+        info = arc.plan_attn_bwd(q, k, v, o, lse, do, causal=c.causal, sinks=s)
+        ws = torch.empty(max(256, arc.attn_bwd_workspace_size(q, k, v, o, lse, do, causal=c.causal, sinks=s)),
+                         dtype=torch.uint8, device="cuda")
+
+        def call():
+            arc.attn_bwd(q, k, v, o, lse, do, scale=c.scale, causal=c.causal, sinks=s, dq=dq, dk=dk, dv=dv,
+                         dsinks=dsk, workspace=ws, status=status)
+        ins = {"q": q, "k": k, "v": v, "o": o, "lse": lse, "do": do}
+        if s is not None:
+            ins["sinks"] = s
+        outs = [dq, dk, dv] + ([dsk] if dsk is not None else [])
+        return call, ins, outs, info
     if isinstance(case, SparseDecode):
         c = case.case
         q, kv, idx = U.to_dev(c.q), U.to_dev(c.kv), U.to_dev(c.idx)
@@ -309,6 +355,17 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
     import oracle
     oracle.build()
     cores = oracle.num_threads()
+    if isinstance(case, Backward):
+        units, _ = work(case)
+        reps, spent = 0, 0.0
+        c = case.case
+        while spent < budget_s[0] and reps < 20:
+            t0 = time.perf_counter()
+            oracle.attn_bwd(c.q, c.k, c.v, case.up.do, scale=c.scale, causal=c.causal, sinks=c.sinks)
+            spent += time.perf_counter() - t0
+            reps += 1
+        return {"value": units * reps / spent / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                "sample": f"the whole backward, {reps} repetitions", "seconds": round(spent, 2)}
     if isinstance(case, SparseDecode):
         units, _ = work(case)
         reps, spent = 0, 0.0
@@ -378,6 +435,10 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
         return {"value": units * reps / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
                 "sample": f"the whole decode step, {reps} repetitions", "seconds": round(spent, 2)}
     raise TypeError(type(case))
+
+
+def unit_is_flop(spec):
+    return "TFLOP" in spec["metric"]
 
 
 def max_over_ranks(x, world, device):
@@ -519,7 +580,8 @@ def measure_config(key, status, stream, flush, local, peaks, min_wall_s):
 
 # The graded workloads: the headline (--config) plus these, each measured in the same run.
 GRADED = ["c2", "c3", "c4", "c5q8", "c5q4",
-          "c5d256", "c5g8", "c4d"]          # and the decode variants beyond the five workloads
+          "c5d256", "c5g8", "c4d",          # the decode variants beyond the five workloads
+          "bwd_gqa", "bwd_mla"]             # and the backward
 
 
 def run_ours(args, spec, case):
@@ -647,6 +709,11 @@ def run_reference(args, spec, case):
             u = valid * case.H * (2 * case.Dqk + 2 * case.Dv)
             t0 = time.perf_counter()
             oracle.run_case(case, rows=rows)
+        elif isinstance(case, Backward):
+            u, _ = work(case)
+            c = case.case
+            t0 = time.perf_counter()
+            oracle.attn_bwd(c.q, c.k, c.v, case.up.do, scale=c.scale, causal=c.causal, sinks=c.sinks)
         else:
             u, _ = work(case)
             t0 = time.perf_counter()
@@ -656,7 +723,7 @@ def run_reference(args, spec, case):
             times.append(dt)
             per_step_units.append(u)
     total = sum(times)
-    scale = 1e12 if spec["metric"].startswith("attention") else 1e9
+    scale = 1e12 if unit_is_flop(spec) else 1e9
     unit = "TFLOP/s" if scale == 1e12 else "GB/s"
     value = sum(per_step_units) / total / scale
     sample = ("2 random query positions x all heads per step" if isinstance(case, (W.DenseCase, W.MlaCase))

@@ -285,8 +285,12 @@ def attn_bwd(q, k, v, o, lse, dout, *, scale=None, causal=True, sinks=None, dlse
     return dq, dk, dv, dsinks
 
 
+def attn_bwd_workspace_size(q, k, v, o, lse, dout, *, causal=True, sinks=None, flags=0) -> int:
+    a = _bwd_args(q, k, v, o, lse, dout, None, sinks, q, k, v, sinks, 1.0, causal, flags, None)
+    return int(lib().arc_attn_bwd_workspace_size(ctypes.byref(a)))
+
+
 def plan_attn_bwd(q, k, v, o, lse, dout, *, causal=True, sinks=None, flags=0):
-    torch = _torch()
     dq, dk, dv = q, k, v            # shapes and strides only: nothing is launched
     ds = sinks if sinks is not None else None
     return plan(ARC_OP_ATTN_BWD, _bwd_args(q, k, v, o, lse, dout, None, sinks, dq, dk, dv, ds, 1.0, causal, flags,

@@ -391,3 +391,64 @@ def test_sparse_decode_splits_the_top_k_when_tokens_leave_sms_idle(arc, Sq, want
         # a missing or short workspace is refused before anything launches
         assert arc.lib().arc_sparse_mla_decode(ctypes.byref(s), None, ws, None) == arc.ARC_ERR_WORKSPACE
         assert arc.lib().arc_sparse_mla_decode(ctypes.byref(s), FAKE, ws - 4, None) == arc.ARC_ERR_WORKSPACE
+
+
+# ------------------------------------------------------------------------------- backward
+def bwd_args(arc, B=1, H=64, Hkv=8, T=1400, D=128, Dv=128, sinks=True):
+    a = arc.BwdArgs()
+    a.B, a.H, a.Hkv, a.Tq, a.Tk, a.D, a.Dv = B, H, Hkv, T, T, D, Dv
+    for f in ("q", "k", "v", "o", "dout", "lse", "dq", "dk", "dv"):
+        setattr(a, f, FAKE)
+    if sinks:
+        a.sinks, a.dsinks = FAKE, FAKE
+    a.q_strides = a.o_strides = a.do_strides = a.dq_strides = (arc._i64 * 3)(*contiguous(B, H, T, D))
+    a.o_strides = a.do_strides = (arc._i64 * 3)(*contiguous(B, H, T, Dv))
+    a.k_strides = a.dk_strides = (arc._i64 * 3)(*contiguous(B, Hkv, T, D))
+    a.v_strides = a.dv_strides = (arc._i64 * 3)(*contiguous(B, Hkv, T, Dv))
+    a.scale, a.causal = D ** -0.5, 1
+    return a
+
+
+def test_backward_plans_the_tensor_core_kernels_and_its_workspace(arc):
+    """GQA-8 at d 128, T 1400 with sinks: one dK/dV CTA per (kv head, 128-key tile) with no
+    row split (88 CTAs over 88 fold tiles each, fewer under the causal mask), delta in the
+    workspace; four launches with the sink gradient."""
+    a = bwd_args(arc)
+    info = arc.plan(arc.ARC_OP_ATTN_BWD, a)
+    assert info["kernel"] == "bwd_dkdv_kernel+bwd_dq_kernel" and info["tensor_cores"] == 1
+    assert info["n_ctas"] == 8 * 11 and info["splits"] == 1 and info["launches"] == 4
+    assert arc.lib().arc_attn_bwd_workspace_size(ctypes.byref(a)) == 64 * 1400 * 4
+    # few key tiles: the fold rows of each are split over CTAs, whose fp32 partials add up
+    a = bwd_args(arc, H=16, Hkv=2, T=260, sinks=False)
+    info = arc.plan(arc.ARC_OP_ATTN_BWD, a)
+    n_qt = -(-8 * 260 // 128)
+    rsplit = min(SMS // (2 * 3), n_qt // 4)
+    tps = -(-n_qt // rsplit)
+    assert info["splits"] == -(-n_qt // tps) and info["launches"] == 4
+    delta = -(-16 * 260 * 4 // 256) * 256
+    assert arc.lib().arc_attn_bwd_workspace_size(ctypes.byref(a)) == delta + info["splits"] * 2 * 260 * 256 * 4
+    # d_qk 192 / d_v 128: 64-row fold tiles for dK / dV (TMEM room)
+    info = arc.plan(arc.ARC_OP_ATTN_BWD, bwd_args(arc, H=16, Hkv=16, T=4096, D=192, Dv=128, sinks=False))
+    assert info["tile_n"] == 64 and info["d_slice"] == 192
+
+
+def test_backward_validation_before_any_launch(arc):
+    L = arc.lib()
+    a = bwd_args(arc, D=256, Dv=256)
+    assert L.arc_attn_bwd(ctypes.byref(a), FAKE, 1 << 30, None) == arc.ARC_ERR_UNSUPPORTED
+    a = bwd_args(arc)
+    a.dsinks = None                                     # sinks without a place for their gradient
+    assert L.arc_attn_bwd(ctypes.byref(a), FAKE, 1 << 30, None) == arc.ARC_ERR_INVALID_ARG
+    a = bwd_args(arc)
+    a.Hkv = 7
+    assert L.arc_attn_bwd(ctypes.byref(a), FAKE, 1 << 30, None) == arc.ARC_ERR_INVALID_ARG
+    a = bwd_args(arc)
+    a.q = FAKE + 8                                      # not 16-byte aligned
+    assert L.arc_attn_bwd(ctypes.byref(a), FAKE, 1 << 30, None) == arc.ARC_ERR_UNSUPPORTED
+    a = bwd_args(arc)
+    ws = L.arc_attn_bwd_workspace_size(ctypes.byref(a))
+    assert L.arc_attn_bwd(ctypes.byref(a), None, ws, None) == arc.ARC_ERR_WORKSPACE
+    assert L.arc_attn_bwd(ctypes.byref(a), FAKE, ws - 4, None) == arc.ARC_ERR_WORKSPACE
+    assert L.arc_attn_bwd(ctypes.byref(a), FAKE + 16, ws, None) == arc.ARC_ERR_WORKSPACE
+    a.scale = float("nan")
+    assert L.arc_attn_bwd(ctypes.byref(a), FAKE, ws, None) == arc.ARC_ERR_INVALID_ARG
