@@ -495,9 +495,10 @@ struct BwdPlan {
     size_t delta_bytes = 0, ws = 0;
 };
 
-// dK/dV: one CTA per (batch, kv head, key tile); when those leave SMs idle, each key
-// tile's fold rows are split over several CTAs (at least 4 fold tiles each) whose
-// fp32 partials a reduction sums.
+// dK/dV: one CTA per (batch, kv head, key tile); when those are fewer than two per SM,
+// each key tile's fold rows are split over several CTAs (at least 4 fold tiles each,
+// about two CTAs per SM in all) whose fp32 partials a reduction sums.  More, smaller
+// CTAs also even out the causal mask's uneven work per key tile.
 BwdPlan plan_bwd(const arc_attn_bwd_args *a)
 {
     BwdPlan pl;
@@ -508,7 +509,8 @@ BwdPlan plan_bwd(const arc_attn_bwd_args *a)
     pl.n_kt = (a->Tk + 127) / 128;
     pl.n_qt = (a->H / a->Hkv * a->Tq + BR - 1) / BR;
     const int base = a->B * a->Hkv * pl.n_kt;
-    int rsplit = std::min(sm_count() / std::max(1, base), pl.n_qt / 4);
+    const int want = 2 * sm_count();
+    int rsplit = base >= want ? 1 : std::min((want + base - 1) / base, pl.n_qt / 4);
     rsplit = std::max(1, std::min(rsplit, 64));
     pl.tiles_per_split = (pl.n_qt + rsplit - 1) / rsplit;
     pl.rsplit = (pl.n_qt + pl.tiles_per_split - 1) / pl.tiles_per_split;

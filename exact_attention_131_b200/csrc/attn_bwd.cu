@@ -18,16 +18,20 @@
 //   bwd_prep_kernel   one warp per row: delta_i = D_i - dLSE_i (HBM-bound)
 //   bwd_dsink_kernel  one CTA per head: the sink gradient, a fixed-order sum
 //   bwd_dkdv_kernel   one CTA per (batch, kv head, 128-key tile[, row split]):
-//                       S^T  = K Q^T       M=128 keys, N=BR fold rows
+//                       S^T  = K Q^T       M=128 keys, N=64 fold rows (a half tile)
 //                       dP^T = V dO^T
 //                       P^T, dS^T from S^T, dP^T, LSE, delta (softmax warps),
 //                       written back over S^T / dP^T as bf16 (TMEM A operands)
 //                       dV  += P^T dO      dK += dS^T Q   (dO, Q read MN-major)
-//                     TMEM: dV [0, DV), dK [DV, DV+D), S^T and dP^T (BR each)
+//                     TMEM: dV [0, DV), dK [DV, DV+D), then S^T / dP^T of each half;
+//                     the two halves of a 128-row fold tile alternate, so one half's
+//                     softmax overlaps the other half's products (one half of 64
+//                     rows per tile at d_qk 192, where TMEM has no room for two)
 //   bwd_dq_kernel     one CTA per (batch, kv head, 128-row fold tile):
 //                       S = Q K^T, dP = dO V^T, dS (softmax warps, over S),
 //                       dQ += dS K         (K read MN-major)
-//                     TMEM: dQ [0, D), S [256, 384), dP [384, 512)
+//                     TMEM: dQ [0, D), S / dP of two 64-key halves at 256 and 384,
+//                     alternating like the dK / dV halves
 //   bwd_reduce_kernel the fp32 partials of row-split dK/dV CTAs, summed in order
 // S and dP are computed in both main kernels (5 + 2 products per tile pair for
 // 5 algorithmic): the price of needing no atomics and no dS round trip
@@ -50,8 +54,8 @@ constexpr float BW_LOG2E = 1.4426950408889634f;
 struct BwdBars {
     uint64_t fixed_full;        // the CTA's resident operands (dK/dV: K, V; dQ: Q, dO)
     uint64_t full[2], empty[2]; // two-stage ring of the streamed operand tiles
-    uint64_t s_full;            // S and dP are in TMEM
-    uint64_t p_full;            // the softmax warps wrote P / dS (128 arrivals)
+    uint64_t s_full[2];         // S and dP of a half are in TMEM
+    uint64_t p_full[2];         // the softmax warps wrote P / dS of a half (128 arrivals)
     uint64_t done;              // every MMA of the CTA finished
     uint64_t cols;              // dK/dV: a fold tile's row quantities are in shared memory (128 arrivals)
     uint32_t tmem_base;
@@ -102,23 +106,31 @@ __device__ __forceinline__ RowInfo row_info(const BwdParams &p, int b, int kvh, 
     return ri;
 }
 
-template <int D, int DV, int BR>
+
+// dK / dV.  A fold tile of BR rows is processed as NH halves of HR = BR/NH rows, each
+// with its own S^T / dP^T buffers in TMEM: while the softmax warps rebuild P and dS of
+// one half, the tensor core runs the other half's products.
+template <int D, int DV, int BR, int NH>
 struct DkdvLayout {
     static constexpr int KC = D / 64, VC = DV / 64;
+    static constexpr int HR = BR / NH;                        // fold rows per half
     static constexpr int QCH = BR * 128;                      // one 64-column chunk of a fold tile
     static constexpr int STAGE = (KC + VC) * QCH;             // Q and dO of one fold tile
     static constexpr int FIXED = (KC + VC) * KCH;             // K and V of the CTA's key tile
     static constexpr int BYTES = 1024 + FIXED + 2 * STAGE + 3 * 2 * 128 * 4 + (int)sizeof(BwdBars);
-    static constexpr int DV_COL = 0, DK_COL = DV, S_COL = DV + D, DP_COL = DV + D + BR;
-    static_assert(DP_COL + BR <= 512, "TMEM: dV, dK, S^T and dP^T side by side");
+    static constexpr int DV_COL = 0, DK_COL = DV;
+    __host__ __device__ static constexpr int s_col(int h) { return DV + D + h * 2 * HR; }
+    __host__ __device__ static constexpr int dp_col(int h) { return DV + D + h * 2 * HR + HR; }
+    static_assert(HR % 64 == 0 && BR % HR == 0, "halves of whole 64-row K groups");
+    static_assert(DV + D + NH * 2 * HR <= 512, "TMEM: dV, dK and NH pairs of S^T / dP^T side by side");
     static_assert(BYTES <= BW_SMEM_LIMIT, "shared memory");
 };
 
-template <int D, int DV, int BR>
+template <int D, int DV, int BR, int NH>
 __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
 {
-    using L = DkdvLayout<D, DV, BR>;
-    constexpr int KC = L::KC, VC = L::VC;
+    using L = DkdvLayout<D, DV, BR, NH>;
+    constexpr int KC = L::KC, VC = L::VC, HR = L::HR;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem<1024>(smem_raw);
     uint8_t *sK = smem, *sV = sK + KC * KCH;
@@ -138,15 +150,20 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
     const int n_qt = (p.G * p.Tq + BR - 1) / BR;
     const int qt_begin = rs * p.tiles_per_split, qt_end = min(n_qt, qt_begin + p.tiles_per_split);
     const int row_base = kvh * p.G * p.Tq;                      // fold row 0 in the [H*Tq] view
+    // the next fold tile at or after qt that sees one of this CTA's keys (qt_end if none)
+    auto next_live = [&](int qt) {
+        while (qt < qt_end && !q_tile_live(p, qt, BR, k0)) ++qt;
+        return qt;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->fixed_full, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->full[i], 1);
             mbar_init(&bars->empty[i], 1);
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 128);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 128);
         mbar_init(&bars->done, 1);
         mbar_init(&bars->cols, 128);
         fence_mbar_init();
@@ -168,8 +185,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
             for (int c = 0; c < VC; ++c) tma_load_4d(sV + c * KCH, &p.tm_v, &bars->fixed_full, c * 64, k0, kvh, b);
             int it = 0;
             bool ok = true;
-            for (int qt = qt_begin; qt < qt_end && ok; ++qt) {
-                if (!q_tile_live(p, qt, BR, k0)) continue;
+            for (int qt = next_live(qt_begin); qt < qt_end && ok; qt = next_live(qt + 1)) {
                 const int st = it & 1;
                 if (it >= 2) ok = mbar_wait(&bars->empty[st], (uint32_t)(((it >> 1) - 1) & 1));
                 if (!ok) {
@@ -191,56 +207,80 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
         }
     } else if (warp == 1) {
         // =============================== MMA issuer
+        // Per fold tile and half h: S^T_h = K Q_h^T and dP^T_h = V dO_h^T (SS), then, once the
+        // softmax warps have posted P^T_h / dS^T_h, dV += P^T_h dO_h and dK += dS^T_h Q_h (TS).
+        // The next tile's S^T_h / dP^T_h go out right after this tile's dV / dK of the same
+        // half (the tensor core runs them in issue order, so they overwrite the half's
+        // columns only after those have been read), before waiting on the other half.
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16(128, BR, false, false);
+            const uint32_t idesc_s = idesc_bf16(128, HR, false, false);
             const uint32_t idesc_dv = idesc_bf16(128, DV, false, true);
             const uint32_t idesc_dk = idesc_bf16(128, D, false, true);
             const uint64_t kd0 = sdesc_sw128(smem_u32(sK), 16, 1024);
             const uint64_t vd0 = sdesc_sw128(smem_u32(sV), 16, 1024);
+            constexpr uint32_t kHalf = HR * 128 >> 4;              // descriptor units of HR rows
             bool ok = mbar_wait(&bars->fixed_full, 0);
             if (!ok) report(p.status, BW_AT_FIXED);
             tc_fence_after();
-            int it = 0;
-            for (int qt = qt_begin; qt < qt_end && ok; ++qt) {
-                if (!q_tile_live(p, qt, BR, k0)) continue;
-                const int st = it & 1;
-                if (!(ok = mbar_wait(&bars->full[st], (uint32_t)((it >> 1) & 1)))) {
-                    report(p.status, BW_AT_RING_FULL);
-                    break;
-                }
-                tc_fence_after();
+            auto issue_s = [&](int st, int h) {
                 uint8_t *sq = sRing + st * L::STAGE, *sdo = sq + KC * L::QCH;
-                const uint64_t qd = sdesc_sw128(smem_u32(sq), 16, 1024);
-                const uint64_t dod = sdesc_sw128(smem_u32(sdo), 16, 1024);
-                // S^T = K Q^T and dP^T = V dO^T (both operands K-major)
+                const uint64_t qd = sdesc_sw128(smem_u32(sq), 16, 1024) + h * kHalf;
+                const uint64_t dod = sdesc_sw128(smem_u32(sdo), 16, 1024) + h * kHalf;
 #pragma unroll
                 for (int c = 0; c < KC; ++c)
-                    umma_ss_k64(tmem + L::S_COL, kd0 + (uint64_t)(c * (KCH >> 4)), qd + (uint64_t)(c * (L::QCH >> 4)),
-                                idesc_s, c > 0);
+                    umma_ss_k64(tmem + L::s_col(h), kd0 + (uint64_t)(c * (KCH >> 4)),
+                                qd + (uint64_t)(c * (L::QCH >> 4)), idesc_s, c > 0);
 #pragma unroll
                 for (int c = 0; c < VC; ++c)
-                    umma_ss_k64(tmem + L::DP_COL, vd0 + (uint64_t)(c * (KCH >> 4)), dod + (uint64_t)(c * (L::QCH >> 4)),
-                                idesc_s, c > 0);
-                umma_commit(&bars->s_full);
-                if (!(ok = mbar_wait(&bars->p_full, (uint32_t)(it & 1)))) {
-                    report(p.status, BW_AT_P_FULL);
-                    break;
-                }
+                    umma_ss_k64(tmem + L::dp_col(h), vd0 + (uint64_t)(c * (KCH >> 4)),
+                                dod + (uint64_t)(c * (L::QCH >> 4)), idesc_s, c > 0);
+                umma_commit(&bars->s_full[h]);
+            };
+            int it = 0;
+            int qt = next_live(qt_begin);
+            if (qt < qt_end) {
+                if (!(ok = ok && mbar_wait(&bars->full[0], 0))) report(p.status, BW_AT_RING_FULL);
                 tc_fence_after();
-                // dV += P^T dO, dK += dS^T Q: A from TMEM, B read MN-major (16 fold rows = 2048 B per K step)
+                if (ok)
+                    for (int h = 0; h < NH; ++h) issue_s(0, h);
+            }
+            for (; qt < qt_end && ok; ++it) {
+                const int st = it & 1;
+                const int qn = next_live(qt + 1);
+                uint8_t *sq = sRing + st * L::STAGE, *sdo = sq + KC * L::QCH;
                 const uint64_t dob = sdesc_sw128(smem_u32(sdo), L::QCH, 1024);
                 const uint64_t qb = sdesc_sw128(smem_u32(sq), L::QCH, 1024);
-                const uint32_t acc = it > 0;
+#pragma unroll 1
+                for (int h = 0; h < NH && ok; ++h) {
+                    if (!(ok = mbar_wait(&bars->p_full[h], (uint32_t)(it & 1)))) {
+                        report(p.status, BW_AT_P_FULL);
+                        break;
+                    }
+                    tc_fence_after();
+                    // dV += P^T_h dO_h, dK += dS^T_h Q_h: B read MN-major from the half's rows
+                    // (16 fold rows = 2048 B per K step)
+                    const uint32_t acc = (it > 0 || h > 0) ? 1u : 0u;
 #pragma unroll
-                for (int k4 = 0; k4 < BR / 64; ++k4)
-                    umma_ts_k64(tmem + L::DV_COL, tmem + L::S_COL + k4 * 32, dob + (uint64_t)(k4 * 512), 128, idesc_dv,
-                                acc | k4);
+                    for (int k4 = 0; k4 < HR / 64; ++k4)
+                        umma_ts_k64(tmem + L::DV_COL, tmem + L::s_col(h) + k4 * 32,
+                                    dob + (uint64_t)(h * kHalf + k4 * 512), 128, idesc_dv, acc | k4);
 #pragma unroll
-                for (int k4 = 0; k4 < BR / 64; ++k4)
-                    umma_ts_k64(tmem + L::DK_COL, tmem + L::DP_COL + k4 * 32, qb + (uint64_t)(k4 * 512), 128, idesc_dk,
-                                acc | k4);
-                umma_commit(&bars->empty[st]);   // the stage is free once these have read it
-                ++it;
+                    for (int k4 = 0; k4 < HR / 64; ++k4)
+                        umma_ts_k64(tmem + L::DK_COL, tmem + L::dp_col(h) + k4 * 32,
+                                    qb + (uint64_t)(h * kHalf + k4 * 512), 128, idesc_dk, acc | k4);
+                    if (h == NH - 1) umma_commit(&bars->empty[st]);   // the stage is free once these have read it
+                    if (qn < qt_end) {
+                        if (h == 0) {
+                            if (!(ok = mbar_wait(&bars->full[(it + 1) & 1], (uint32_t)(((it + 1) >> 1) & 1)))) {
+                                report(p.status, BW_AT_RING_FULL);
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        issue_s((it + 1) & 1, h);
+                    }
+                }
+                qt = qn;
             }
             if (!ok) report(p.status, ST_TIMEOUT_MMA);
             umma_commit(&bars->done);
@@ -254,8 +294,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
         const float sl2 = p.scale_log2;
         int it = 0;
         bool ok = true;
-        for (int qt = qt_begin; qt < qt_end; ++qt) {
-            if (!q_tile_live(p, qt, BR, k0)) continue;
+        for (int qt = next_live(qt_begin); qt < qt_end; qt = next_live(qt + 1)) {
             const int cb = (it & 1) * 128;
             if (tid < BR) {
                 const RowInfo ri = row_info(p, b, kvh, qt * BR + tid);
@@ -271,41 +310,46 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                 report(p.status, BW_AT_COLS);
                 break;
             }
-            ok = bw_all(mbar_wait(&bars->s_full, (uint32_t)(it & 1)));
-            if (!ok) {
-                report(p.status, BW_AT_S_FULL);
-                break;
-            }
-            tc_fence_after();
 #pragma unroll 1
-            for (int ch = 0; ch < BR / 32; ++ch) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tmem + lane_off + L::S_COL + 32 * ch, sv);
-                tmem_ld32(tmem + lane_off + L::DP_COL + 32 * ch, dv);
-                tmem_wait_ld();
-                uint32_t pk[16], dk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float pp[2], dd[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int c = cb + 32 * ch + 2 * i + e;
-                        const float pe = kj <= col_lim[c]
-                                             ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -col_lse2[c]))
-                                             : 0.f;
-                        pp[e] = pe;
-                        dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - col_delta[c]);
-                    }
-                    pk[i] = pack_bf16(pp[0], pp[1]);
-                    dk[i] = pack_bf16(dd[0], dd[1]);
+            for (int h = 0; h < NH && ok; ++h) {
+                ok = bw_all(mbar_wait(&bars->s_full[h], (uint32_t)(it & 1)));
+                if (!ok) {
+                    report(p.status, BW_AT_S_FULL);
+                    break;
                 }
-                // bf16 pairs over the first half of the columns just read
-                tmem_st16(tmem + lane_off + L::S_COL + 16 * ch, pk);
-                tmem_st16(tmem + lane_off + L::DP_COL + 16 * ch, dk);
+                tc_fence_after();
+#pragma unroll 1
+                for (int ch = 0; ch < HR / 32; ++ch) {
+                    uint32_t sv[32], dv[32];
+                    tmem_ld32(tmem + lane_off + L::s_col(h) + 32 * ch, sv);
+                    tmem_ld32(tmem + lane_off + L::dp_col(h) + 32 * ch, dv);
+                    tmem_wait_ld();
+                    const int c0 = cb + h * HR + 32 * ch;
+                    uint32_t pk[16], dk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float pp[2], dd[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int c = c0 + 2 * i + e;
+                            const float pe = kj <= col_lim[c]
+                                                 ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -col_lse2[c]))
+                                                 : 0.f;
+                            pp[e] = pe;
+                            dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - col_delta[c]);
+                        }
+                        pk[i] = pack_bf16(pp[0], pp[1]);
+                        dk[i] = pack_bf16(dd[0], dd[1]);
+                    }
+                    // bf16 pairs over the first half of the columns just read
+                    tmem_st16(tmem + lane_off + L::s_col(h) + 16 * ch, pk);
+                    tmem_st16(tmem + lane_off + L::dp_col(h) + 16 * ch, dk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars->p_full[h]);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full);
+            if (!ok) break;
             ++it;
         }
         if (ok && it > 0) ok = bw_all(mbar_wait(&bars->done, 0));
@@ -358,6 +402,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
     }
 }
 
+// dQ.  A key tile of 128 keys is processed as two halves of 64 keys, each with its own
+// S / dP buffers in TMEM, pipelined like the dK / dV kernel's halves.
 template <int D, int DV>
 struct DqLayout {
     static constexpr int KC = D / 64, VC = DV / 64;
@@ -367,8 +413,10 @@ struct DqLayout {
     // tile then loads only once the last one is consumed)
     static constexpr int NSTG = 1024 + FIXED + 2 * STAGE + (int)sizeof(BwdBars) <= BW_SMEM_LIMIT ? 2 : 1;
     static constexpr int BYTES = 1024 + FIXED + NSTG * STAGE + (int)sizeof(BwdBars);
-    static constexpr int DQ_COL = 0, S_COL = 256, DP_COL = 384;
-    static_assert(D <= 256, "TMEM: dQ, S and dP side by side");
+    static constexpr int DQ_COL = 0;
+    __host__ __device__ static constexpr int s_col(int h) { return 256 + h * 128; }
+    __host__ __device__ static constexpr int dp_col(int h) { return 256 + h * 128 + 64; }
+    static_assert(D <= 256, "TMEM: dQ, then two pairs of S / dP halves");
     static_assert(BYTES <= BW_SMEM_LIMIT, "shared memory");
 };
 
@@ -376,7 +424,7 @@ template <int D, int DV>
 __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p)
 {
     using L = DqLayout<D, DV>;
-    constexpr int KC = L::KC, VC = L::VC;
+    constexpr int KC = L::KC, VC = L::VC, HK = BK / 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem<1024>(smem_raw);
     uint8_t *sQ = smem, *sdO = sQ + KC * KCH;
@@ -406,9 +454,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->full[i], 1);
             mbar_init(&bars->empty[i], 1);
+            mbar_init(&bars->s_full[i], 1);
+            mbar_init(&bars->p_full[i], 128);
         }
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 128);
         mbar_init(&bars->done, 1);
         fence_mbar_init();
     }
@@ -448,45 +496,67 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
     } else if (warp == 1) {
         // =============================== MMA issuer
         if (lane == 0 && nt > 0) {
-            const uint32_t idesc_s = idesc_bf16(128, BK, false, false);
+            const uint32_t idesc_s = idesc_bf16(128, HK, false, false);
             const uint32_t idesc_dq = idesc_bf16(128, D, false, true);
             const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t dod0 = sdesc_sw128(smem_u32(sdO), 16, 1024);
+            constexpr uint32_t kHalf = HK * 128 >> 4;              // descriptor units of 64 key rows
             bool ok = mbar_wait(&bars->fixed_full, 0);
             if (!ok) report(p.status, BW_IN_DQ | BW_AT_FIXED);
             tc_fence_after();
-            for (int j = 0; j < nt && ok; ++j) {
-                const int st = j % NS;
-                if (!(ok = mbar_wait(&bars->full[st], (uint32_t)((j / NS) & 1)))) {
-                    report(p.status, BW_IN_DQ | BW_AT_RING_FULL);
-                    break;
-                }
-                tc_fence_after();
+            // S_h = Q K_h^T and dP_h = dO V_h^T for key half h of key tile j (ring stage st)
+            auto issue_s = [&](int st, int h) {
                 uint8_t *sk = sRing + st * L::STAGE, *sv = sk + KC * KCH;
-                const uint64_t kd = sdesc_sw128(smem_u32(sk), 16, 1024);
-                const uint64_t vd = sdesc_sw128(smem_u32(sv), 16, 1024);
+                const uint64_t kd = sdesc_sw128(smem_u32(sk), 16, 1024) + h * kHalf;
+                const uint64_t vd = sdesc_sw128(smem_u32(sv), 16, 1024) + h * kHalf;
 #pragma unroll
                 for (int c = 0; c < KC; ++c)
-                    umma_ss_k64(tmem + L::S_COL, qd0 + (uint64_t)(c * (KCH >> 4)), kd + (uint64_t)(c * (KCH >> 4)), idesc_s,
-                                c > 0);
+                    umma_ss_k64(tmem + L::s_col(h), qd0 + (uint64_t)(c * (KCH >> 4)), kd + (uint64_t)(c * (KCH >> 4)),
+                                idesc_s, c > 0);
 #pragma unroll
                 for (int c = 0; c < VC; ++c)
-                    umma_ss_k64(tmem + L::DP_COL, dod0 + (uint64_t)(c * (KCH >> 4)), vd + (uint64_t)(c * (KCH >> 4)),
+                    umma_ss_k64(tmem + L::dp_col(h), dod0 + (uint64_t)(c * (KCH >> 4)), vd + (uint64_t)(c * (KCH >> 4)),
                                 idesc_s, c > 0);
-                umma_commit(&bars->s_full);
-                if (!(ok = mbar_wait(&bars->p_full, (uint32_t)(j & 1)))) {
-                    report(p.status, BW_IN_DQ | BW_AT_P_FULL);
-                    break;
-                }
-                tc_fence_after();
-                // dQ += dS K: dS from TMEM, K read MN-major (16 keys = 2048 B per K step)
+                umma_commit(&bars->s_full[h]);
+            };
+            if (!(ok = ok && mbar_wait(&bars->full[0], 0))) report(p.status, BW_IN_DQ | BW_AT_RING_FULL);
+            tc_fence_after();
+            if (ok)
+                for (int h = 0; h < 2; ++h) issue_s(0, h);
+            for (int j = 0; j < nt && ok; ++j) {
+                const int st = j % NS;
+                uint8_t *sk = sRing + st * L::STAGE;
                 const uint64_t kb = sdesc_sw128(smem_u32(sk), KCH, 1024);
-                const uint32_t acc = j > 0;
-#pragma unroll
-                for (int k4 = 0; k4 < BK / 64; ++k4)
-                    umma_ts_k64(tmem + L::DQ_COL, tmem + L::S_COL + k4 * 32, kb + (uint64_t)(k4 * 512), 128, idesc_dq,
-                                acc | k4);
-                umma_commit(&bars->empty[st]);
+#pragma unroll 1
+                for (int h = 0; h < 2 && ok; ++h) {
+                    if (!(ok = mbar_wait(&bars->p_full[h], (uint32_t)(j & 1)))) {
+                        report(p.status, BW_IN_DQ | BW_AT_P_FULL);
+                        break;
+                    }
+                    tc_fence_after();
+                    // dQ += dS_h K_h: dS from TMEM, K read MN-major (16 keys = 2048 B per K step)
+                    umma_ts_k64(tmem + L::DQ_COL, tmem + L::s_col(h), kb + (uint64_t)(h * kHalf), 128, idesc_dq,
+                                (j > 0 || h > 0) ? 1u : 0u);
+                    if (h == 1) umma_commit(&bars->empty[st]);
+                    // the next key tile's half h, right behind this half's dQ; with one ring
+                    // stage the next tile can only have landed once this tile is released,
+                    // so both of its halves follow the second half
+                    if (j + 1 < nt && (NS > 1 || h == 1)) {
+                        if (NS > 1 ? h == 0 : true) {
+                            if (!(ok = mbar_wait(&bars->full[(j + 1) % NS], (uint32_t)(((j + 1) / NS) & 1)))) {
+                                report(p.status, BW_IN_DQ | BW_AT_RING_FULL);
+                                break;
+                            }
+                            tc_fence_after();
+                        }
+                        if (NS > 1) {
+                            issue_s((j + 1) % NS, h);
+                        } else {
+                            issue_s(0, 0);
+                            issue_s(0, 1);
+                        }
+                    }
+                }
             }
             if (!ok) report(p.status, ST_TIMEOUT_MMA);
             umma_commit(&bars->done);
@@ -500,38 +570,41 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
         const RowInfo ri = row_info(p, b, kvh, r);
         const float sl2 = p.scale_log2;
         bool ok = true;
-        for (int j = 0; j < nt; ++j) {
-            ok = bw_all(mbar_wait(&bars->s_full, (uint32_t)(j & 1)));
-            if (!ok) {
-                report(p.status, BW_IN_DQ | BW_AT_S_FULL);
-                break;
-            }
-            tc_fence_after();
+        for (int j = 0; j < nt && ok; ++j) {
 #pragma unroll 1
-            for (int ch = 0; ch < BK / 32; ++ch) {
-                uint32_t sv[32], dv[32];
-                tmem_ld32(tmem + lane_off + L::S_COL + 32 * ch, sv);
-                tmem_ld32(tmem + lane_off + L::DP_COL + 32 * ch, dv);
-                tmem_wait_ld();
-                const int key0 = j * BK + 32 * ch;
-                uint32_t dk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float dd[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const float pe = key0 + 2 * i + e <= ri.lim
-                                             ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ri.lse2))
-                                             : 0.f;
-                        dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - ri.delta);
-                    }
-                    dk[i] = pack_bf16(dd[0], dd[1]);
+            for (int h = 0; h < 2 && ok; ++h) {
+                ok = bw_all(mbar_wait(&bars->s_full[h], (uint32_t)(j & 1)));
+                if (!ok) {
+                    report(p.status, BW_IN_DQ | BW_AT_S_FULL);
+                    break;
                 }
-                tmem_st16(tmem + lane_off + L::S_COL + 16 * ch, dk);
+                tc_fence_after();
+#pragma unroll 1
+                for (int ch = 0; ch < HK / 32; ++ch) {
+                    uint32_t sv[32], dv[32];
+                    tmem_ld32(tmem + lane_off + L::s_col(h) + 32 * ch, sv);
+                    tmem_ld32(tmem + lane_off + L::dp_col(h) + 32 * ch, dv);
+                    tmem_wait_ld();
+                    const int key0 = j * BK + h * HK + 32 * ch;
+                    uint32_t dk[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float dd[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float pe = key0 + 2 * i + e <= ri.lim
+                                                 ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ri.lse2))
+                                                 : 0.f;
+                            dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - ri.delta);
+                        }
+                        dk[i] = pack_bf16(dd[0], dd[1]);
+                    }
+                    tmem_st16(tmem + lane_off + L::s_col(h) + 16 * ch, dk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars->p_full[h]);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars->p_full);
         }
         if (ok && nt > 0) ok = bw_all(mbar_wait(&bars->done, 0));
         if (!ok) report(p.status, ST_TIMEOUT_SOFTMAX);
@@ -569,31 +642,36 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
     }
 }
 
-// delta_i = sum_d dO_id O_id - dLSE_i, one warp per row (b, h, t); 8 elements per lane
-// and step (16-byte loads).
+// delta_i = sum_d dO_id O_id - dLSE_i.  A warp takes RPW = 256 / Dv rows (at least one):
+// each lane moves 8 elements (16 bytes) of one row per step, so a warp keeps 32 16-byte
+// loads of each tensor in flight; the lanes of a row reduce with shuffles.
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ BwdPrepParams p)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
-    if (row >= (int64_t)p.B * p.H * p.Tq) return;
-    const int t = (int)(row % p.Tq), h = (int)((row / p.Tq) % p.H), b = (int)(row / ((int64_t)p.Tq * p.H));
-    const __nv_bfloat16 *o = p.o + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)t * p.os[2];
-    const __nv_bfloat16 *g = p.dout + (int64_t)b * p.dos[0] + (int64_t)h * p.dos[1] + (int64_t)t * p.dos[2];
+    const int rpw = p.Dv >= 256 ? 1 : 256 / p.Dv;               // rows per warp (a power of two)
+    const int lpr = 32 / rpw;                                   // lanes per row
+    const int64_t rows = (int64_t)p.B * p.H * p.Tq;
+    const int64_t row = ((int64_t)blockIdx.x * 8 + warp) * rpw + lane / lpr;
+    const bool live = row < rows;
     float acc = 0.f;
-    for (int d = lane * 8; d < p.Dv; d += 256) {
-        const uint4 x = *reinterpret_cast<const uint4 *>(o + d), y = *reinterpret_cast<const uint4 *>(g + d);
-        const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
+    if (live) {
+        const int t = (int)(row % p.Tq), h = (int)((row / p.Tq) % p.H), b = (int)(row / ((int64_t)p.Tq * p.H));
+        const __nv_bfloat16 *o = p.o + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)t * p.os[2];
+        const __nv_bfloat16 *g = p.dout + (int64_t)b * p.dos[0] + (int64_t)h * p.dos[1] + (int64_t)t * p.dos[2];
+        for (int d = (lane % lpr) * 8; d < p.Dv; d += lpr * 8) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(o + d), y = *reinterpret_cast<const uint4 *>(g + d);
+            const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw[k]));
-            const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[k]));
-            acc = fmaf(a.x, c.x, acc);
-            acc = fmaf(a.y, c.y, acc);
+            for (int k = 0; k < 4; ++k) {
+                const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw[k]));
+                const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[k]));
+                acc = fmaf(a.x, c.x, acc);
+                acc = fmaf(a.y, c.y, acc);
+            }
         }
     }
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-    if (lane == 0) p.delta[row] = acc - (p.dlse ? p.dlse[row] : 0.f);
+    for (int s = lpr / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (live && lane % lpr == 0) p.delta[row] = acc - (p.dlse ? p.dlse[row] : 0.f);
 }
 
 // d sink_h = -sum_{b,t} exp(sink_h - LSE_bht) * delta_bht, one CTA per head, a fixed
@@ -649,14 +727,15 @@ __global__ void __launch_bounds__(256) bwd_reduce_kernel(const __grid_constant__
     *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16(acc.x * f, acc.y * f), pack_bf16(acc.z * f, acc.w * f));
 }
 
-template <int D, int DV, int BR>
+template <int D, int DV, int BR, int NH>
 cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
 {
     cudaError_t e;
     {
-        auto kern = bwd_dkdv_kernel<D, DV, BR>;
+        using L = DkdvLayout<D, DV, BR, NH>;
+        auto kern = bwd_dkdv_kernel<D, DV, BR, NH>;
         // at least 116 KB so one CTA holds an SM: each allocates all 512 TMEM columns
-        const int bytes = DkdvLayout<D, DV, BR>::BYTES > 118784 ? DkdvLayout<D, DV, BR>::BYTES : 118784;
+        const int bytes = L::BYTES > 118784 ? L::BYTES : 118784;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
         const int grid = p.B * p.Hkv * ((p.Tk + BK - 1) / BK) * p.rsplit;
         if (grid > 0) kern<<<grid, BW_THREADS, bytes, s>>>(p);
@@ -689,7 +768,8 @@ cudaError_t launch_bwd_prep(const BwdPrepParams &p, cudaStream_t s)
 {
     const int64_t rows = (int64_t)p.B * p.H * p.Tq;
     if (rows == 0) return cudaSuccess;
-    bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(p);
+    const int rpw = p.Dv >= 256 ? 1 : 256 / p.Dv;             // rows per warp, as in the kernel
+    bwd_prep_kernel<<<(unsigned)((rows + 8 * rpw - 1) / (8 * rpw)), 256, 0, s>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !p.sinks) return e;
     bwd_dsink_kernel<<<p.H, 256, 0, s>>>(p);
@@ -698,17 +778,17 @@ cudaError_t launch_bwd_prep(const BwdPrepParams &p, cudaStream_t s)
 
 cudaError_t launch_bwd(const BwdParams &p, cudaStream_t s)
 {
-    if (p.D == 64 && p.Dv == 64) return launch_bwd_t<64, 64, 128>(p, s);
-    if (p.D == 128 && p.Dv == 128) return launch_bwd_t<128, 128, 128>(p, s);
-    if (p.D == 192 && p.Dv == 128) return launch_bwd_t<192, 128, 64>(p, s);
+    if (p.D == 64 && p.Dv == 64) return launch_bwd_t<64, 64, 128, 2>(p, s);
+    if (p.D == 128 && p.Dv == 128) return launch_bwd_t<128, 128, 128, 2>(p, s);
+    if (p.D == 192 && p.Dv == 128) return launch_bwd_t<192, 128, 64, 1>(p, s);
     return cudaErrorInvalidValue;
 }
 
 int bwd_dkdv_smem_bytes(int d, int dv)
 {
-    if (d == 64) return DkdvLayout<64, 64, 128>::BYTES;
-    if (d == 128) return DkdvLayout<128, 128, 128>::BYTES;
-    return DkdvLayout<192, 128, 64>::BYTES;
+    if (d == 64) return DkdvLayout<64, 64, 128, 2>::BYTES;
+    if (d == 128) return DkdvLayout<128, 128, 128, 2>::BYTES;
+    return DkdvLayout<192, 128, 64, 1>::BYTES;
 }
 
 int bwd_dq_smem_bytes(int d, int dv)

@@ -410,23 +410,33 @@ def bwd_args(arc, B=1, H=64, Hkv=8, T=1400, D=128, Dv=128, sinks=True):
 
 
 def test_backward_plans_the_tensor_core_kernels_and_its_workspace(arc):
-    """GQA-8 at d 128, T 1400 with sinks: one dK/dV CTA per (kv head, 128-key tile) with no
-    row split (88 CTAs over 88 fold tiles each, fewer under the causal mask), delta in the
-    workspace; four launches with the sink gradient."""
+    """GQA-8 at d 128, T 1400 with sinks: 8 kv heads x 11 key tiles = 88 dK/dV CTAs, fewer
+    than two per SM, so each key tile's 88 fold tiles are split over 4 CTAs (22 each) whose
+    fp32 partials a fifth launch adds up; delta and the partials in the workspace."""
+    def expect_split(base, n_qt):
+        want = 2 * SMS
+        r = 1 if base >= want else min(-(-want // base), n_qt // 4)
+        r = max(1, min(r, 64))
+        tps = -(-n_qt // r)
+        return -(-n_qt // tps)
+
     a = bwd_args(arc)
     info = arc.plan(arc.ARC_OP_ATTN_BWD, a)
     assert info["kernel"] == "bwd_dkdv_kernel+bwd_dq_kernel" and info["tensor_cores"] == 1
-    assert info["n_ctas"] == 8 * 11 and info["splits"] == 1 and info["launches"] == 4
-    assert arc.lib().arc_attn_bwd_workspace_size(ctypes.byref(a)) == 64 * 1400 * 4
-    # few key tiles: the fold rows of each are split over CTAs, whose fp32 partials add up
+    assert info["splits"] == expect_split(8 * 11, 88) == 4
+    assert info["n_ctas"] == 8 * 11 * 4 and info["launches"] == 5
+    delta = 64 * 1400 * 4
+    assert arc.lib().arc_attn_bwd_workspace_size(ctypes.byref(a)) == delta + 4 * 8 * 1400 * 256 * 4
+    # few key tiles, no sinks
     a = bwd_args(arc, H=16, Hkv=2, T=260, sinks=False)
     info = arc.plan(arc.ARC_OP_ATTN_BWD, a)
     n_qt = -(-8 * 260 // 128)
-    rsplit = min(SMS // (2 * 3), n_qt // 4)
-    tps = -(-n_qt // rsplit)
-    assert info["splits"] == -(-n_qt // tps) and info["launches"] == 4
+    assert info["splits"] == expect_split(2 * 3, n_qt) > 1 and info["launches"] == 4
     delta = -(-16 * 260 * 4 // 256) * 256
     assert arc.lib().arc_attn_bwd_workspace_size(ctypes.byref(a)) == delta + info["splits"] * 2 * 260 * 256 * 4
+    # enough key tiles: no split, no reduction
+    info = arc.plan(arc.ARC_OP_ATTN_BWD, bwd_args(arc, B=2, H=16, Hkv=16, T=4096, sinks=False))
+    assert info["splits"] == 1 and info["launches"] == 3
     # d_qk 192 / d_v 128: 64-row fold tiles for dK / dV (TMEM room)
     info = arc.plan(arc.ARC_OP_ATTN_BWD, bwd_args(arc, H=16, Hkv=16, T=4096, D=192, Dv=128, sinks=False))
     assert info["tile_n"] == 64 and info["d_slice"] == 192
