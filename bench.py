@@ -64,8 +64,8 @@ CONFIGS = {
     "bwd_gqa": dict(cfg=10, bwd=dict(B=1, H=64, Hkv=8, T=1400, D=128, Dv=128, sinks=True),
                     name="attention bwd, B=1 H=64 Hkv=8 T=1400 D=128 causal, sinks",
                     metric="attention bwd TFLOP/s", dtype="bf16"),
-    "bwd_mla": dict(cfg=11, bwd=dict(B=2, H=16, Hkv=16, T=4096, D=192, Dv=128, sinks=False),
-                    name="attention bwd, B=2 H=16 T=4096 d_qk=192 d_v=128 causal",
+    "bwd_mla": dict(cfg=11, bwd_mla=dict(B=2, H=16, T=4096, Dn=128, Dr=64, Dv=128),
+                    name="MLA bwd, B=2 H=16 T=4096 d_qk=192 (128+64) d_v=128 causal",
                     metric="attention bwd TFLOP/s", dtype="bf16"),
     # decode-shaped sparse MLA: c4's per-token shape at a decode batch of 32 tokens
     "c4d": dict(cfg=7, sparse_decode=dict(Sq=32, H=64, Skv=65536, Dqk=512, Dv=512, topk=2176),
@@ -85,6 +85,11 @@ def make_case(spec):
         return SparseDecode(W.sparse_case(**spec["sparse_decode"], seed=spec["cfg"]))
     if "decode" in spec:
         return W.decode_case(**spec["decode"], seed=spec["cfg"])
+    if "bwd_mla" in spec:
+        b = spec["bwd_mla"]
+        case = W.mla_case(b["B"], b["H"], b["T"], b["T"], b["Dn"], b["Dr"], b["Dv"], std=0.3, causal=True,
+                          seed=spec["cfg"])
+        return Backward(case, W.upstream(b["B"], b["H"], b["T"], b["Dv"], seed=spec["cfg"] + 1000))
     if "bwd" in spec:
         b = spec["bwd"]
         case = W.dense_case(b["B"], b["H"], b["Hkv"], b["T"], b["T"], b["D"], b["Dv"], dtype="bf16", std=0.5,
@@ -118,11 +123,12 @@ def dense_pairs(Tq, Tk, causal):
 def work(case):
     """(algorithmic units, unit name) of one call: FLOPs over visible pairs, or bytes for decode."""
     if isinstance(case, Backward):
-        # per visible (row, key) pair: S and dP recomputed... counted once each, plus dV,
-        # dK and dQ: 2*D (S) + 2*Dv (dP) + 2*Dv (dV) + 2*D (dK) + 2*D (dQ)
+        # per visible (row, key) pair, each product counted once: 2*d_qk (S) + 2*d_v (dP)
+        # + 2*d_v (dV) + 2*d_qk (dK) + 2*d_qk (dQ)
         c = case.case
+        dqk = c.D if isinstance(c, W.DenseCase) else c.Dn + c.Dr
         pairs = c.B * c.H * dense_pairs(c.Tq, c.Tk, c.causal)
-        return pairs * (6 * c.D + 4 * c.Dv), "flop"
+        return pairs * (6 * dqk + 4 * c.Dv), "flop"
     if isinstance(case, SparseDecode):
         # memory-bound: every distinct pool row a call gathers crosses HBM once, plus Q, O,
         # LSE and the index lists
@@ -169,6 +175,18 @@ class Uploaded:
 def build_call(case, torch, arc, status):
     """Returns (call(), inputs dict of device tensors, outputs list, n_launches, kernel name)."""
     U = Uploaded(case, torch, arc)
+    if isinstance(case, Backward) and isinstance(case.case, W.MlaCase):
+        c = case.case
+        t = [U.to_dev(x) for x in (c.q_nope, c.q_rope, c.k_nope, c.k_rope, c.v)]
+        o, lse = arc.mla_fwd(*t, scale=c.scale, causal=c.causal)
+        do = U.to_dev(case.up.do)
+        info = arc.plan_mla_bwd(*t, o, lse, do, causal=c.causal)
+
+        def call():
+            arc.mla_bwd(*t, o, lse, do, scale=c.scale, causal=c.causal, status=status)
+        ins = dict(zip(["q_nope", "q_rope", "k_nope", "k_rope", "v"], t))
+        ins.update({"o": o, "lse": lse, "do": do})
+        return call, ins, [o], info
     if isinstance(case, Backward):
         c = case.case
         q, k, v = U.to_dev(c.q), U.to_dev(c.k), U.to_dev(c.v)
@@ -358,10 +376,9 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
     if isinstance(case, Backward):
         units, _ = work(case)
         reps, spent = 0, 0.0
-        c = case.case
         while spent < budget_s[0] and reps < 20:
             t0 = time.perf_counter()
-            oracle.attn_bwd(c.q, c.k, c.v, case.up.do, scale=c.scale, causal=c.causal, sinks=c.sinks)
+            oracle_backward(oracle, case)
             spent += time.perf_counter() - t0
             reps += 1
         return {"value": units * reps / spent / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
@@ -435,6 +452,13 @@ def cpu_baseline(case, key, budget_s=(10.0, 30.0)):
         return {"value": units * reps / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
                 "sample": f"the whole decode step, {reps} repetitions", "seconds": round(spent, 2)}
     raise TypeError(type(case))
+
+
+def oracle_backward(oracle, case):
+    c = case.case
+    if isinstance(c, W.MlaCase):
+        return oracle.mla_bwd(c.q_nope, c.q_rope, c.k_nope, c.k_rope, c.v, case.up.do, scale=c.scale, causal=c.causal)
+    return oracle.attn_bwd(c.q, c.k, c.v, case.up.do, scale=c.scale, causal=c.causal, sinks=c.sinks)
 
 
 def unit_is_flop(spec):
@@ -711,9 +735,8 @@ def run_reference(args, spec, case):
             oracle.run_case(case, rows=rows)
         elif isinstance(case, Backward):
             u, _ = work(case)
-            c = case.case
             t0 = time.perf_counter()
-            oracle.attn_bwd(c.q, c.k, c.v, case.up.do, scale=c.scale, causal=c.causal, sinks=c.sinks)
+            oracle_backward(oracle, case)
         else:
             u, _ = work(case)
             t0 = time.perf_counter()

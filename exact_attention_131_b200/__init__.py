@@ -7,6 +7,7 @@ no fallback: if the library is missing, importing a function raises.
 Names follow the C ABI:
     attn_fwd            -> arc_attn_fwd         dense / GQA / MQA (+ sinks)
     attn_bwd            -> arc_attn_bwd         its gradients: dq, dk, dv, d sinks
+    mla_bwd             -> arc_mla_bwd          mla_fwd's gradients (dk_rope summed over heads)
     mla_fwd             -> arc_mla_fwd          q_nope||q_rope, d_qk != d_v
     sparse_mla_fwd      -> arc_sparse_mla_fwd   per-query top-k index lists
     sparse_mla_decode   -> arc_sparse_mla_decode   the same, top-k split over CTAs for few tokens
@@ -26,7 +27,8 @@ _lib = None
 ARC_OK, ARC_ERR_INVALID_ARG, ARC_ERR_UNSUPPORTED, ARC_ERR_CUDA, ARC_ERR_DEVICE_TIMEOUT, ARC_ERR_WORKSPACE = range(6)
 ARC_DTYPE_BF16, ARC_DTYPE_F32 = 0, 1
 ARC_KV_Q4_0, ARC_KV_Q8_0 = 2, 8
-ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE, ARC_OP_MERGE, ARC_OP_SPARSE_DECODE, ARC_OP_ATTN_BWD = range(1, 8)
+(ARC_OP_ATTN, ARC_OP_MLA, ARC_OP_SPARSE, ARC_OP_DECODE, ARC_OP_MERGE, ARC_OP_SPARSE_DECODE, ARC_OP_ATTN_BWD,
+ ARC_OP_MLA_BWD) = range(1, 9)
 ARC_MERGE_MAX_PARTS = 16
 ARC_FLAG_FORCE_SIMPLE = 1
 ARC_FLAG_SINGLE_CTA = 2
@@ -71,6 +73,18 @@ class BwdArgs(ctypes.Structure):
                 ("flags", _u32), ("status", _vp)]
 
 
+class MlaBwdArgs(ctypes.Structure):
+    _fields_ = [("B", _i32), ("H", _i32), ("Tq", _i32), ("Tk", _i32), ("Dn", _i32), ("Dr", _i32), ("Dv", _i32),
+                ("q_nope", _vp), ("q_nope_strides", _i64 * 3), ("q_rope", _vp), ("q_rope_strides", _i64 * 3),
+                ("k_nope", _vp), ("k_nope_strides", _i64 * 3), ("k_rope", _vp), ("k_rope_strides", _i64 * 2),
+                ("v", _vp), ("v_strides", _i64 * 3), ("o", _vp), ("o_strides", _i64 * 3),
+                ("dout", _vp), ("do_strides", _i64 * 3), ("lse", _vp), ("dlse", _vp),
+                ("dq_nope", _vp), ("dq_nope_strides", _i64 * 3), ("dq_rope", _vp), ("dq_rope_strides", _i64 * 3),
+                ("dk_nope", _vp), ("dk_nope_strides", _i64 * 3), ("dk_rope", _vp), ("dk_rope_strides", _i64 * 2),
+                ("dv", _vp), ("dv_strides", _i64 * 3), ("scale", _f32), ("causal", _i32), ("flags", _u32),
+                ("status", _vp)]
+
+
 class Seq(ctypes.Structure):
     _fields_ = [("q_begin", _i32), ("n_q", _i32), ("kv_begin", _i32), ("n_kv", _i32)]
 
@@ -97,7 +111,8 @@ class PlanInfo(ctypes.Structure):
 EXPORTS = ["arc_attn_fwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_attn_decode_q8",
            "arc_decode_workspace_size", "arc_plan", "arc_abi_version", "arc_status_string",
            "arc_check_device_error", "arc_selftest_timeout", "arc_attn_decode_q8_noalloc", "arc_attn_merge",
-           "arc_sparse_mla_decode", "arc_sparse_decode_workspace_size", "arc_attn_bwd", "arc_attn_bwd_workspace_size"]
+           "arc_sparse_mla_decode", "arc_sparse_decode_workspace_size", "arc_attn_bwd", "arc_attn_bwd_workspace_size",
+           "arc_mla_bwd", "arc_mla_bwd_workspace_size"]
 
 
 class ArcError(RuntimeError):
@@ -123,6 +138,9 @@ def lib():
         L.arc_attn_bwd.argtypes = [ctypes.POINTER(BwdArgs), _vp, ctypes.c_size_t, _vp]
         L.arc_attn_bwd_workspace_size.argtypes = [ctypes.POINTER(BwdArgs)]
         L.arc_attn_bwd_workspace_size.restype = ctypes.c_size_t
+        L.arc_mla_bwd.argtypes = [ctypes.POINTER(MlaBwdArgs), _vp, ctypes.c_size_t, _vp]
+        L.arc_mla_bwd_workspace_size.argtypes = [ctypes.POINTER(MlaBwdArgs)]
+        L.arc_mla_bwd_workspace_size.restype = ctypes.c_size_t
         L.arc_attn_decode_q8.argtypes = [ctypes.POINTER(DecodeArgs), _vp, ctypes.c_size_t, _vp]
         L.arc_attn_decode_q8_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         L.arc_attn_merge.argtypes = [ctypes.POINTER(MergeArgs), _vp]
@@ -133,7 +151,7 @@ def lib():
         L.arc_status_string.restype = ctypes.c_char_p
         L.arc_check_device_error.argtypes = [_vp, _vp]
         L.arc_selftest_timeout.argtypes = [_vp, ctypes.c_uint64, _vp]
-        for f in ("arc_attn_fwd", "arc_attn_bwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_sparse_mla_decode",
+        for f in ("arc_attn_fwd", "arc_attn_bwd", "arc_mla_bwd", "arc_mla_fwd", "arc_sparse_mla_fwd", "arc_sparse_mla_decode",
                   "arc_attn_decode_q8",
                   "arc_attn_decode_q8_noalloc", "arc_attn_merge", "arc_plan",
                   "arc_check_device_error", "arc_selftest_timeout", "arc_abi_version"):
@@ -295,6 +313,56 @@ def plan_attn_bwd(q, k, v, o, lse, dout, *, causal=True, sinks=None, flags=0):
     ds = sinks if sinks is not None else None
     return plan(ARC_OP_ATTN_BWD, _bwd_args(q, k, v, o, lse, dout, None, sinks, dq, dk, dv, ds, 1.0, causal, flags,
                                            None))
+
+
+def _mla_bwd_args(q_nope, q_rope, k_nope, k_rope, v, o, lse, dout, dlse, dq_nope, dq_rope, dk_nope, dk_rope, dv,
+                  scale, causal, flags, status):
+    B, H, Tq, Dn = q_nope.shape
+    a = MlaBwdArgs()
+    a.B, a.H, a.Tq, a.Tk, a.Dn, a.Dr, a.Dv = B, H, Tq, v.shape[2], Dn, q_rope.shape[-1], v.shape[3]
+    for f, t in (("q_nope", q_nope), ("q_rope", q_rope), ("k_nope", k_nope), ("v", v), ("o", o),
+                 ("dq_nope", dq_nope), ("dq_rope", dq_rope), ("dk_nope", dk_nope), ("dv", dv)):
+        setattr(a, f, _p(t))
+        setattr(a, f + "_strides", _s3(t))
+    a.dout, a.do_strides = _p(dout), _s3(dout)
+    a.k_rope, a.k_rope_strides = _p(k_rope), (_i64 * 2)(*k_rope.stride()[:2])
+    a.dk_rope, a.dk_rope_strides = _p(dk_rope), (_i64 * 2)(*dk_rope.stride()[:2])
+    a.lse, a.dlse = _p(lse), _p(dlse)
+    a.scale, a.flags = _scale_flags(scale, flags)
+    a.causal = int(bool(causal))
+    a.status = _p(status)
+    return a
+
+
+def mla_bwd(q_nope, q_rope, k_nope, k_rope, v, o, lse, dout, *, scale=None, causal=True, dlse=None, workspace=None,
+            flags=0, status=None, stream=None):
+    """dq_nope, dq_rope, dk_nope, dk_rope, dv = arc_mla_bwd: gradients of mla_fwd given its o,
+    lse and the upstream dout (and optionally dlse); dk_rope is summed over the heads."""
+    torch = _torch()
+    bf = torch.bfloat16
+    for n, t in (("q_nope", q_nope), ("q_rope", q_rope), ("k_nope", k_nope), ("k_rope", k_rope), ("v", v),
+                 ("o", o), ("dout", dout)):
+        _dev(t, n, bf)
+    for n, t in (("lse", lse), ("dlse", dlse)):
+        _dev(t, n, torch.float32)
+        if t is not None and (tuple(t.shape) != tuple(q_nope.shape[:3]) or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous [B, H, Tq] fp32 tensor")
+    dq_nope, dq_rope = torch.empty_like(q_nope), torch.empty_like(q_rope)
+    dk_nope, dk_rope, dv = torch.empty_like(k_nope), torch.empty_like(k_rope), torch.empty_like(v)
+    a = _mla_bwd_args(q_nope, q_rope, k_nope, k_rope, v, o, lse, dout, dlse, dq_nope, dq_rope, dk_nope, dk_rope, dv,
+                      scale, causal, flags, status)
+    need = int(lib().arc_mla_bwd_workspace_size(ctypes.byref(a)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_nope.device)
+    ws_ptr = _p(workspace) if workspace is not None else None
+    ws_len = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().arc_mla_bwd(ctypes.byref(a), ws_ptr, ws_len, _stream(stream)), "arc_mla_bwd")
+    return dq_nope, dq_rope, dk_nope, dk_rope, dv
+
+
+def plan_mla_bwd(q_nope, q_rope, k_nope, k_rope, v, o, lse, dout, *, causal=True, flags=0):
+    return plan(ARC_OP_MLA_BWD, _mla_bwd_args(q_nope, q_rope, k_nope, k_rope, v, o, lse, dout, None, q_nope, q_rope,
+                                              k_nope, k_rope, v, 1.0, causal, flags, None))
 
 
 def _mla_args(q_nope, q_rope, k_nope, k_rope, v, o, lse, scale, causal, flags, status):

@@ -795,14 +795,38 @@ size_t arc_attn_bwd_workspace_size(const arc_attn_bwd_args *a)
     return plan_bwd(a).ws;
 }
 
-arc_status arc_attn_bwd(const arc_attn_bwd_args *a, void *workspace, size_t ws_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// The MLA extras of a backward call: q = q_nope || q_rope and k = k_nope || k_rope, the
+// rope part of k one tensor shared by every head (its gradient is summed over them).
+struct MlaBwdExtra {
+    int Dn = 0, Dr = 0;
+    const void *q_rope = nullptr;
+    const int64_t *q_rope_strides = nullptr;
+    const void *k_rope = nullptr;
+    const int64_t *k_rope_strides = nullptr;
+    void *dq_rope = nullptr;
+    const int64_t *dq_rope_strides = nullptr;
+    void *dk_rope = nullptr;
+    const int64_t *dk_rope_strides = nullptr;
+};
+
+size_t mla_rope_part_bytes(const arc_attn_bwd_args *a, const BwdPlan &pl, int Dr)
 {
-    arc_status st = check_bwd(a);
-    if (st != ARC_OK) return st;
-    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    return (size_t)pl.rsplit * a->B * a->H * a->Tk * Dr * sizeof(float);
+}
+
+// Both backward calls after validation: delta (and the sink gradient), then dK / dV and
+// dQ.  `a` is the call seen as dense attention over the concatenated head dims (for MLA:
+// q and k are the nope tensors, D = Dn + Dr, Hkv = H); `mla` is non-null for MLA.
+arc_status run_bwd(const arc_attn_bwd_args *a, const MlaBwdExtra *mla, void *workspace, size_t ws_bytes,
+                   cudaStream_t s)
+{
     const BwdPlan pl = plan_bwd(a);
-    if (!workspace || ws_bytes < pl.ws || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return ARC_ERR_WORKSPACE;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t need = pl.ws + (mla ? mla_rope_part_bytes(a, pl, mla->Dr) : 0);
+    if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return ARC_ERR_WORKSPACE;
     const float scale = call_scale(a->flags, a->scale, a->D);
     float *delta = static_cast<float *>(workspace);
     BwdPrepParams pp{};
@@ -817,6 +841,7 @@ arc_status arc_attn_bwd(const arc_attn_bwd_args *a, void *workspace, size_t ws_b
     memset(&p, 0, sizeof(p));
     const int G = a->H / a->Hkv;
     const int BR = bwd_tile_rows(a->D, a->Dv);
+    const int dn = mla ? mla->Dn : a->D;                     // columns of q / k in the first tensor
     auto qmap = [&](CUtensorMap *m, const void *base, const int64_t *st3, int width, uint32_t rows) {
         const uint64_t d[3] = {(uint64_t)width, (uint64_t)a->H * a->Tq, (uint64_t)a->B};
         const int64_t sv[2] = {st3[2], st3[0] ? st3[0] : (int64_t)a->H * a->Tq * st3[2]};
@@ -829,10 +854,19 @@ arc_status arc_attn_bwd(const arc_attn_bwd_args *a, void *workspace, size_t ws_b
         return make_map(m, base, 4, d, sv, 128);
     };
     if (a->Tk > 0 &&
-        (!qmap(&p.tm_q, a->q, a->q_strides, a->D, 128) || !qmap(&p.tm_do, a->dout, a->do_strides, a->Dv, 128) ||
-         !qmap(&p.tm_qr, a->q, a->q_strides, a->D, BR) || !qmap(&p.tm_dor, a->dout, a->do_strides, a->Dv, BR) ||
-         !kmap(&p.tm_k, a->k, a->k_strides, a->D) || !kmap(&p.tm_v, a->v, a->v_strides, a->Dv)))
+        (!qmap(&p.tm_q, a->q, a->q_strides, dn, 128) || !qmap(&p.tm_do, a->dout, a->do_strides, a->Dv, 128) ||
+         !qmap(&p.tm_qr, a->q, a->q_strides, dn, BR) || !qmap(&p.tm_dor, a->dout, a->do_strides, a->Dv, BR) ||
+         !kmap(&p.tm_k, a->k, a->k_strides, dn) || !kmap(&p.tm_v, a->v, a->v_strides, a->Dv)))
         return ARC_ERR_CUDA;
+    if (mla && a->Tk > 0) {
+        const uint64_t kd[3] = {(uint64_t)mla->Dr, (uint64_t)a->Tk, (uint64_t)a->B};
+        const int64_t *kr = mla->k_rope_strides;
+        const int64_t ks[2] = {kr[1], kr[0] ? kr[0] : (int64_t)a->Tk * kr[1]};
+        if (!qmap(&p.tm_q2, mla->q_rope, mla->q_rope_strides, mla->Dr, 128) ||
+            !qmap(&p.tm_qr2, mla->q_rope, mla->q_rope_strides, mla->Dr, BR) || !make_map(&p.tm_k2, mla->k_rope, 3, kd, ks, 128))
+            return ARC_ERR_CUDA;
+    }
+    p.mla = mla != nullptr, p.kc_first = dn / 64;
     p.B = a->B, p.H = a->H, p.Hkv = a->Hkv, p.G = G, p.Tq = a->Tq, p.Tk = a->Tk, p.D = a->D, p.Dv = a->Dv;
     p.causal = a->causal;
     p.lse = a->lse, p.delta = delta;
@@ -840,16 +874,109 @@ arc_status arc_attn_bwd(const arc_attn_bwd_args *a, void *workspace, size_t ws_b
     p.dq = static_cast<__nv_bfloat16 *>(a->dq), p.dk = static_cast<__nv_bfloat16 *>(a->dk);
     p.dv = static_cast<__nv_bfloat16 *>(a->dv);
     for (int i = 0; i < 3; ++i) p.dqs[i] = a->dq_strides[i], p.dks[i] = a->dk_strides[i], p.dvs[i] = a->dv_strides[i];
+    p.dk_cols = dn;
+    if (mla) {
+        p.dq2 = static_cast<__nv_bfloat16 *>(mla->dq_rope);
+        for (int i = 0; i < 3; ++i) p.dq2s[i] = mla->dq_rope_strides[i];
+        p.dk2 = static_cast<__nv_bfloat16 *>(mla->dk_rope);
+        p.dk2s[0] = mla->dk_rope_strides[0], p.dk2s[1] = mla->dk_rope_strides[1];
+        p.dkr_part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + pl.ws);
+    }
     p.rsplit = pl.rsplit, p.tiles_per_split = pl.tiles_per_split;
     p.dkv_part = pl.rsplit > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + pl.delta_bytes) : nullptr;
     p.status = a->status;
-    if (a->Tk == 0) {
-        // no key: every gradient is zero; the dQ kernel writes them (no key tile to visit)
-        p.rsplit = 1;
-    }
-    note_dispatch("bwd_dkdv_kernel");
+    if (a->Tk == 0) p.rsplit = 1;   // no key: every gradient is zero; the dQ kernel writes dQ
+    note_dispatch(mla ? "bwd_dkdv_kernel<mla>" : "bwd_dkdv_kernel");
     note_dispatch("bwd_dq_kernel");
     return launch_bwd(p, s) == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;
+}
+
+// An MLA backward call as dense attention over the concatenated head dims (Hkv = H, the
+// nope tensors as q and k), for the shared checks, the plan and the launch.
+arc_attn_bwd_args mla_as_dense(const arc_mla_bwd_args *m)
+{
+    arc_attn_bwd_args a;
+    memset(&a, 0, sizeof(a));
+    a.B = m->B, a.H = m->H, a.Hkv = m->H, a.Tq = m->Tq, a.Tk = m->Tk, a.D = m->Dn + m->Dr, a.Dv = m->Dv;
+    a.q = m->q_nope, a.k = m->k_nope, a.v = m->v, a.o = m->o, a.dout = m->dout;
+    a.dq = m->dq_nope, a.dk = m->dk_nope, a.dv = m->dv;
+    for (int i = 0; i < 3; ++i) {
+        a.q_strides[i] = m->q_nope_strides[i], a.k_strides[i] = m->k_nope_strides[i], a.v_strides[i] = m->v_strides[i];
+        a.o_strides[i] = m->o_strides[i], a.do_strides[i] = m->do_strides[i];
+        a.dq_strides[i] = m->dq_nope_strides[i], a.dk_strides[i] = m->dk_nope_strides[i];
+        a.dv_strides[i] = m->dv_strides[i];
+    }
+    a.lse = m->lse, a.dlse = m->dlse;
+    a.scale = m->scale, a.causal = m->causal, a.flags = m->flags, a.status = m->status;
+    return a;
+}
+
+arc_status check_mla_bwd(const arc_mla_bwd_args *m)
+{
+    if (!m) return ARC_ERR_INVALID_ARG;
+    if (m->Dn <= 0 || m->Dr <= 0 || m->Dn % 64 || m->Dr % 64) return ARC_ERR_UNSUPPORTED;
+    const arc_attn_bwd_args a = mla_as_dense(m);
+    arc_status st = check_bwd(&a);
+    if (st != ARC_OK || m->B == 0 || m->Tq == 0) return st;
+    if (!m->q_rope || !m->dq_rope || (m->Tk > 0 && (!m->k_rope || !m->dk_rope))) return ARC_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i)
+        if (m->q_rope_strides[i] < 0 || m->dq_rope_strides[i] < 0 || (i < 2 && (m->k_rope_strides[i] < 0 || m->dk_rope_strides[i] < 0)))
+            return ARC_ERR_INVALID_ARG;
+    if (broadcast(m->dq_rope_strides[0], m->B) || broadcast(m->dq_rope_strides[1], m->H) ||
+        broadcast(m->dq_rope_strides[2], m->Tq) || broadcast(m->dk_rope_strides[0], m->B) ||
+        broadcast(m->dk_rope_strides[1], m->Tk))
+        return ARC_ERR_INVALID_ARG;
+    if (m->H > 1 && m->q_rope_strides[1] != (int64_t)m->Tq * m->q_rope_strides[2]) return ARC_ERR_UNSUPPORTED;
+    const void *ptrs[] = {m->q_rope, m->k_rope, m->dq_rope, m->dk_rope};
+    for (const void *ptr : ptrs)
+        if (!aligned16(ptr)) return ARC_ERR_UNSUPPORTED;
+    for (int i = 0; i < 3; ++i)
+        if ((m->q_rope_strides[i] * 2) % 16 || (m->dq_rope_strides[i] * 2) % 16 ||
+            (i < 2 && ((m->k_rope_strides[i] * 2) % 16 || (m->dk_rope_strides[i] * 2) % 16)))
+            return ARC_ERR_UNSUPPORTED;
+    if (broadcast(m->q_rope_strides[0], m->B) || broadcast(m->k_rope_strides[0], m->B)) return ARC_ERR_UNSUPPORTED;
+    return ARC_OK;
+}
+
+MlaBwdExtra mla_extra(const arc_mla_bwd_args *m)
+{
+    MlaBwdExtra x;
+    x.Dn = m->Dn, x.Dr = m->Dr;
+    x.q_rope = m->q_rope, x.q_rope_strides = m->q_rope_strides;
+    x.k_rope = m->k_rope, x.k_rope_strides = m->k_rope_strides;
+    x.dq_rope = m->dq_rope, x.dq_rope_strides = m->dq_rope_strides;
+    x.dk_rope = m->dk_rope, x.dk_rope_strides = m->dk_rope_strides;
+    return x;
+}
+
+}  // namespace
+
+extern "C" {
+
+arc_status arc_attn_bwd(const arc_attn_bwd_args *a, void *workspace, size_t ws_bytes, void *stream)
+{
+    arc_status st = check_bwd(a);
+    if (st != ARC_OK) return st;
+    if (a->B == 0 || a->Tq == 0) return ARC_OK;
+    return run_bwd(a, nullptr, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t arc_mla_bwd_workspace_size(const arc_mla_bwd_args *m)
+{
+    if (check_mla_bwd(m) != ARC_OK) return 0;
+    const arc_attn_bwd_args a = mla_as_dense(m);
+    const BwdPlan pl = plan_bwd(&a);
+    return pl.ws + mla_rope_part_bytes(&a, pl, m->Dr);
+}
+
+arc_status arc_mla_bwd(const arc_mla_bwd_args *m, void *workspace, size_t ws_bytes, void *stream)
+{
+    arc_status st = check_mla_bwd(m);
+    if (st != ARC_OK) return st;
+    if (m->B == 0 || m->Tq == 0) return ARC_OK;
+    const arc_attn_bwd_args a = mla_as_dense(m);
+    const MlaBwdExtra x = mla_extra(m);
+    return run_bwd(&a, &x, workspace, ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
 size_t arc_sparse_decode_workspace_size(const arc_sparse_args *a)
@@ -1169,6 +1296,25 @@ arc_status arc_plan(int32_t op, const void *args, arc_plan_info *out)
         out->n_ctas = a->B * a->Hkv * pl.n_kt * pl.rsplit;
         out->smem_bytes = bwd_dkdv_smem_bytes(a->D, a->Dv), out->tmem_cols = 512;
         out->launches = 3 + (a->sinks ? 1 : 0) + (pl.rsplit > 1 ? 1 : 0);
+        return ARC_OK;
+    }
+    if (op == ARC_OP_MLA_BWD) {
+        const arc_mla_bwd_args *m = static_cast<const arc_mla_bwd_args *>(args);
+        arc_status st = check_mla_bwd(m);
+        if (st != ARC_OK) return st;
+        if (m->B == 0 || m->Tq == 0) {
+            set_name(out, "none");
+            return ARC_OK;
+        }
+        const arc_attn_bwd_args a = mla_as_dense(m);
+        const BwdPlan pl = plan_bwd(&a);
+        set_name(out, "bwd_dkdv_kernel<mla>+bwd_dq_kernel");
+        out->tensor_cores = 1;
+        out->tile_m = 128, out->tile_n = bwd_tile_rows(a.D, a.Dv), out->d_slice = a.D;
+        out->splits = pl.rsplit;
+        out->n_ctas = a.B * a.Hkv * pl.n_kt * pl.rsplit;
+        out->smem_bytes = bwd_dkdv_smem_bytes(a.D, a.Dv), out->tmem_cols = 512;
+        out->launches = 4 + (pl.rsplit > 1 ? 1 : 0);
         return ARC_OK;
     }
     if (op == ARC_OP_SPARSE_DECODE) {

@@ -181,7 +181,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
         // =============================== TMA producer
         if (lane == 0) {
             mbar_arrive_expect_tx(&bars->fixed_full, L::FIXED);
-            for (int c = 0; c < KC; ++c) tma_load_4d(sK + c * KCH, &p.tm_k, &bars->fixed_full, c * 64, k0, kvh, b);
+            for (int c = 0; c < KC; ++c) {
+                if (!p.mla || c < p.kc_first)
+                    tma_load_4d(sK + c * KCH, &p.tm_k, &bars->fixed_full, c * 64, k0, kvh, b);
+                else   // MLA: the rope columns, one tensor shared by every head
+                    tma_load_3d(sK + c * KCH, &p.tm_k2, &bars->fixed_full, (c - p.kc_first) * 64, k0, b);
+            }
             for (int c = 0; c < VC; ++c) tma_load_4d(sV + c * KCH, &p.tm_v, &bars->fixed_full, c * 64, k0, kvh, b);
             int it = 0;
             bool ok = true;
@@ -194,8 +199,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                 }
                 uint8_t *dst = sRing + st * L::STAGE;
                 mbar_arrive_expect_tx(&bars->full[st], L::STAGE);
-                for (int c = 0; c < KC; ++c)
-                    tma_load_3d(dst + c * L::QCH, &p.tm_qr, &bars->full[st], c * 64, row_base + qt * BR, b);
+                for (int c = 0; c < KC; ++c) {
+                    if (!p.mla || c < p.kc_first)
+                        tma_load_3d(dst + c * L::QCH, &p.tm_qr, &bars->full[st], c * 64, row_base + qt * BR, b);
+                    else
+                        tma_load_3d(dst + c * L::QCH, &p.tm_qr2, &bars->full[st], (c - p.kc_first) * 64,
+                                    row_base + qt * BR, b);
+                }
                 for (int c = 0; c < VC; ++c)
                     tma_load_3d(dst + (KC + c) * L::QCH, &p.tm_dor, &bars->full[st], c * 64, row_base + qt * BR, b);
                 ++it;
@@ -362,6 +372,8 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
         float *prow = p.dkv_part + ((((int64_t)rs * p.B + b) * p.Hkv + kvh) * p.Tk + kj) * (D + DV);
         __nv_bfloat16 *dkrow = p.dk + (int64_t)b * p.dks[0] + (int64_t)kvh * p.dks[1] + (int64_t)kj * p.dks[2];
         __nv_bfloat16 *dvrow = p.dv + (int64_t)b * p.dvs[0] + (int64_t)kvh * p.dvs[1] + (int64_t)kj * p.dvs[2];
+        const int dr = D - p.dk_cols;                             // MLA: rope columns of dK (else 0)
+        float *rrow = p.dkr_part + ((((int64_t)rs * p.B + b) * p.Hkv + kvh) * p.Tk + kj) * dr;
 #pragma unroll 1
         for (int c = 0; c < (D + DV) / 32; ++c) {
             uint32_t v[32];
@@ -375,6 +387,16 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                 for (int i = 0; i < 32; ++i) v[i] = 0u;
             }
             if (!key_ok) continue;
+            if (is_k && 32 * c >= p.dk_cols) {
+                // MLA rope columns: this head's share of the shared k_rope's gradient (fp32,
+                // unscaled); a reduction sums the heads
+                float4 *dst = reinterpret_cast<float4 *>(rrow + 32 * c - p.dk_cols);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                         __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                continue;
+            }
             if (p.rsplit > 1) {
                 float4 *dst = reinterpret_cast<float4 *>(prow + 32 * c);
 #pragma unroll
@@ -473,7 +495,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
         // =============================== TMA producer
         if (lane == 0 && nt > 0) {
             mbar_arrive_expect_tx(&bars->fixed_full, L::FIXED);
-            for (int c = 0; c < KC; ++c) tma_load_3d(sQ + c * KCH, &p.tm_q, &bars->fixed_full, c * 64, row_base + r0, b);
+            for (int c = 0; c < KC; ++c) {
+                if (!p.mla || c < p.kc_first)
+                    tma_load_3d(sQ + c * KCH, &p.tm_q, &bars->fixed_full, c * 64, row_base + r0, b);
+                else
+                    tma_load_3d(sQ + c * KCH, &p.tm_q2, &bars->fixed_full, (c - p.kc_first) * 64, row_base + r0, b);
+            }
             for (int c = 0; c < VC; ++c) tma_load_3d(sdO + c * KCH, &p.tm_do, &bars->fixed_full, c * 64, row_base + r0, b);
             bool ok = true;
             for (int j = 0; j < nt && ok; ++j) {
@@ -485,7 +512,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
                 }
                 uint8_t *dst = sRing + st * L::STAGE;
                 mbar_arrive_expect_tx(&bars->full[st], L::STAGE);
-                for (int c = 0; c < KC; ++c) tma_load_4d(dst + c * KCH, &p.tm_k, &bars->full[st], c * 64, j * BK, kvh, b);
+                for (int c = 0; c < KC; ++c) {
+                    if (!p.mla || c < p.kc_first)
+                        tma_load_4d(dst + c * KCH, &p.tm_k, &bars->full[st], c * 64, j * BK, kvh, b);
+                    else
+                        tma_load_3d(dst + c * KCH, &p.tm_k2, &bars->full[st], (c - p.kc_first) * 64, j * BK, b);
+                }
                 for (int c = 0; c < VC; ++c)
                     tma_load_4d(dst + (KC + c) * KCH, &p.tm_v, &bars->full[st], c * 64, j * BK, kvh, b);
             }
@@ -613,6 +645,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
         const bool row_ok = r < rows;
         const int h = kvh * p.G + (row_ok ? r / p.Tq : 0), t = row_ok ? r % p.Tq : 0;
         __nv_bfloat16 *dqrow = p.dq + (int64_t)b * p.dqs[0] + (int64_t)h * p.dqs[1] + (int64_t)t * p.dqs[2];
+        // MLA: columns from kc_first * 64 on are dq_rope's
+        const int dn = p.mla ? p.kc_first * 64 : D;
+        __nv_bfloat16 *dq2row = p.mla ? p.dq2 + (int64_t)b * p.dq2s[0] + (int64_t)h * p.dq2s[1] + (int64_t)t * p.dq2s[2]
+                                      : nullptr;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             uint32_t v[32];
@@ -628,7 +664,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 w[i] = pack_bf16(__uint_as_float(v[2 * i]) * p.scale, __uint_as_float(v[2 * i + 1]) * p.scale);
-            uint4 *dst = reinterpret_cast<uint4 *>(dqrow + 32 * c);
+            uint4 *dst = reinterpret_cast<uint4 *>(32 * c < dn ? dqrow + 32 * c : dq2row + (32 * c - dn));
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
@@ -718,6 +754,7 @@ __global__ void __launch_bounds__(256) bwd_reduce_kernel(const __grid_constant__
     const int kj = (int)(row % p.Tk), kvh = (int)((row / p.Tk) % p.Hkv), b = (int)(row / ((int64_t)p.Tk * p.Hkv));
     __nv_bfloat16 *dst;
     float f = 1.f;
+    if (e >= p.dk_cols && e < D) return;      // MLA rope columns: summed over heads elsewhere
     if (e < D) {
         dst = p.dk + (int64_t)b * p.dks[0] + (int64_t)kvh * p.dks[1] + (int64_t)kj * p.dks[2] + e;
         f = p.scale;
@@ -725,6 +762,29 @@ __global__ void __launch_bounds__(256) bwd_reduce_kernel(const __grid_constant__
         dst = p.dv + (int64_t)b * p.dvs[0] + (int64_t)kvh * p.dvs[1] + (int64_t)kj * p.dvs[2] + (e - D);
     }
     *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16(acc.x * f, acc.y * f), pack_bf16(acc.z * f, acc.w * f));
+}
+
+// MLA: dk_rope[b, kj] = scale * sum over row splits and heads of the per-head rope columns
+// of dK, in a fixed order; one thread per 4 columns.
+__global__ void __launch_bounds__(256) bwd_rope_reduce_kernel(const __grid_constant__ BwdParams p)
+{
+    const int dr = p.D - p.dk_cols;
+    const int64_t x = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    const int64_t rows = (int64_t)p.B * p.Tk;
+    if (x >= rows * (dr / 4)) return;
+    const int64_t row = x / (dr / 4);
+    const int e = (int)(x % (dr / 4)) * 4;
+    const int kj = (int)(row % p.Tk), b = (int)(row / p.Tk);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < p.rsplit; ++s)
+        for (int h = 0; h < p.Hkv; ++h) {
+            const float4 v =
+                *reinterpret_cast<const float4 *>(p.dkr_part + ((((int64_t)s * p.B + b) * p.Hkv + h) * p.Tk + kj) * dr + e);
+            acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+        }
+    __nv_bfloat16 *dst = p.dk2 + (int64_t)b * p.dk2s[0] + (int64_t)kj * p.dk2s[1] + e;
+    *reinterpret_cast<uint2 *>(dst) =
+        make_uint2(pack_bf16(acc.x * p.scale, acc.y * p.scale), pack_bf16(acc.z * p.scale, acc.w * p.scale));
 }
 
 template <int D, int DV, int BR, int NH>
@@ -744,6 +804,11 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
     if (p.rsplit > 1 && p.Tk > 0) {
         const int64_t n = (int64_t)p.B * p.Hkv * p.Tk * ((D + DV) / 4);
         bwd_reduce_kernel<D, DV><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (p.mla && p.Tk > 0 && p.dk_cols < D) {
+        const int64_t n = (int64_t)p.B * p.Tk * ((D - p.dk_cols) / 4);
+        bwd_rope_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {

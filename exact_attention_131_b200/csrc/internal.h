@@ -148,12 +148,23 @@ struct BwdParams {
     CUtensorMap tm_q, tm_do;    // q / dO {D, H*Tq, B}, box {64, 128}      (dQ kernel)
     CUtensorMap tm_qr, tm_dor;  // the same, box {64, fold-tile rows}      (dK/dV kernel)
     CUtensorMap tm_k, tm_v;     // k / v {D, Tk, Hkv, B}, box {64, 128}
+    // MLA: q = q_nope || q_rope and k = k_nope || k_rope (shared by the heads) are
+    // concatenated on load; 64-column chunks from kc_first on come from the rope maps
+    CUtensorMap tm_q2, tm_qr2;  // q_rope {Dr, H*Tq, B}, boxes {64, 128} and {64, fold-tile rows}
+    CUtensorMap tm_k2;          // k_rope {Dr, Tk, B}, box {64, 128}
+    int mla, kc_first;
     int B, H, Hkv, G, Tq, Tk, D, Dv;
     int causal;
     const float *lse, *delta;   // [B,H,Tq]
     float scale, scale_log2;
     __nv_bfloat16 *dq, *dk, *dv;
     int64_t dqs[3], dks[3], dvs[3];
+    __nv_bfloat16 *dq2;         // MLA: dq_rope, strides dq2s; dq holds dq_nope
+    int64_t dq2s[3];
+    int dk_cols;                // columns of dK written to dk (D; MLA: Dn, the rope columns go to dkr_part)
+    float *dkr_part;            // MLA: fp32 [rsplit][B][H][Tk][Dr] per-head rope columns of dK (unscaled)
+    __nv_bfloat16 *dk2;         // MLA: dk_rope [B, Tk, Dr] (the sum over heads), strides dk2s
+    int64_t dk2s[2];
     int rsplit, tiles_per_split;// dK/dV CTAs per key tile along the fold rows, and fold tiles each
     float *dkv_part;            // rsplit > 1: fp32 [rsplit][B][Hkv][Tk][D + Dv] (dK unscaled, then dV)
     uint32_t *status;

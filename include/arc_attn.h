@@ -70,7 +70,7 @@ typedef enum { ARC_KV_Q4_0 = 2, ARC_KV_Q8_0 = 8 } arc_kv_type;
 
 typedef enum {
     ARC_OP_ATTN = 1, ARC_OP_MLA = 2, ARC_OP_SPARSE = 3, ARC_OP_DECODE = 4, ARC_OP_MERGE = 5,
-    ARC_OP_SPARSE_DECODE = 6, ARC_OP_ATTN_BWD = 7
+    ARC_OP_SPARSE_DECODE = 6, ARC_OP_ATTN_BWD = 7, ARC_OP_MLA_BWD = 8
 } arc_op;
 
 /* flags (all calls) */
@@ -442,6 +442,55 @@ typedef struct {
 size_t arc_attn_bwd_workspace_size(const arc_attn_bwd_args *args);
 
 arc_status arc_attn_bwd(const arc_attn_bwd_args *args, void *workspace, size_t ws_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * arc_mla_bwd: gradients of arc_mla_fwd.
+ *
+ * Source: "pith-train: FA4 b19 return arity and MLA q/k concat", MLA section:
+ * the model concatenates q = q_nope||q_rope and k = k_nope||k_rope and trains
+ * through the attention call, so the gradients reach each part through that
+ * concatenation.  They are those of arc_attn_bwd on the concatenated head dims
+ * (d_qk = Dn + Dr, one kv head per query head, no sinks), split back:
+ *     dq_nope, dq_rope   the first Dn and the last Dr columns of dQ
+ *     dk_nope            the first Dn columns of each head's dK
+ *     dk_rope            the sum over all H heads of the last Dr columns of dK
+ *                        (k_rope is one tensor shared by every head)
+ *     dv                 as arc_attn_bwd
+ *
+ *   q_nope ... v, o, lse   as arc_mla_fwd's arguments and outputs
+ *   dout [B,H,Tq,Dv] bf16; dlse [B,H,Tq] fp32 or NULL
+ *   dq_nope [B,H,Tq,Dn], dq_rope [B,H,Tq,Dr], dk_nope [B,H,Tk,Dn], dk_rope [B,Tk,Dr],
+ *   dv [B,H,Tk,Dv]        bf16, device, written
+ * (Dn + Dr, Dv) in {(128,128), (192,128)} with Dn, Dr multiples of 64; layout rules
+ * as arc_attn_bwd.  workspace: at least arc_mla_bwd_workspace_size(args) bytes,
+ * 256-byte aligned (delta, and each head's fp32 share of dk_rope before the
+ * sum over heads, which runs in a fixed order).  Errors as arc_attn_bwd.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int32_t B, H, Tq, Tk, Dn, Dr, Dv;
+    const void *q_nope; int64_t q_nope_strides[3];
+    const void *q_rope; int64_t q_rope_strides[3];
+    const void *k_nope; int64_t k_nope_strides[3];
+    const void *k_rope; int64_t k_rope_strides[2];
+    const void *v;      int64_t v_strides[3];
+    const void *o;      int64_t o_strides[3];
+    const void *dout;   int64_t do_strides[3];
+    const float *lse;
+    const float *dlse;
+    void *dq_nope;      int64_t dq_nope_strides[3];
+    void *dq_rope;      int64_t dq_rope_strides[3];
+    void *dk_nope;      int64_t dk_nope_strides[3];
+    void *dk_rope;      int64_t dk_rope_strides[2];
+    void *dv;           int64_t dv_strides[3];
+    float scale;
+    int32_t causal;
+    uint32_t flags;
+    uint32_t *status;
+} arc_mla_bwd_args;
+
+size_t arc_mla_bwd_workspace_size(const arc_mla_bwd_args *args);
+
+arc_status arc_mla_bwd(const arc_mla_bwd_args *args, void *workspace, size_t ws_bytes, void *stream);
 
 /* --------------------------------------------------------------------------
  * Engagement record and helpers.

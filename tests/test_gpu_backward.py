@@ -106,3 +106,29 @@ def test_backward_mla_shaped_head_dims():
     c, got, ref, _ = run_case(2, 4, 4, 1024, 1024, 192, 128, True, False, False, seed=453)
     for name, g, r in zip(("dq", "dk", "dv"), got[:3], ref[:3]):
         check(name, g, r)
+
+
+@pytest.mark.parametrize("B,H,T,Dn,Dr,Dv,causal,dlse", [
+    (1, 3, 300, 128, 64, 128, True, False),     # the MLA prefill's head dims, ragged tiles
+    (2, 2, 200, 64, 64, 128, False, True),      # d_qk 128, non-causal, upstream dLSE
+    (1, 4, 260, 128, 64, 128, True, False),     # four heads summed into dk_rope
+])
+def test_mla_backward_matches_oracle(B, H, T, Dn, Dr, Dv, causal, dlse):
+    """arc_mla_bwd: gradients through the q_nope||q_rope and k_nope||k_rope concatenation,
+    dk_rope summed over the heads that share it, against oracle/backward.py's mla_bwd."""
+    c = W.mla_case(B, H, T, T, Dn, Dr, Dv, causal=causal, seed=470 + T)
+    up = W.upstream(B, H, T, Dv, dlse=dlse, seed=471 + T)
+    t = [dev(x) for x in (c.q_nope, c.q_rope, c.k_nope, c.k_rope, c.v)]
+    o, lse = arc.mla_fwd(*t, scale=c.scale, causal=causal)
+    do = dev(up.do)
+    dl = dev(up.dlse) if dlse else None
+    st = status_word()
+    got = arc.mla_bwd(*t, o, lse, do, scale=c.scale, causal=causal, dlse=dl, status=st)
+    torch.cuda.synchronize()
+    assert arc.check_device_error(st) == arc.ARC_OK
+    info = arc.plan_mla_bwd(*t, o, lse, do, causal=causal)
+    assert info["kernel"] == "bwd_dkdv_kernel<mla>+bwd_dq_kernel" and info["tensor_cores"] == 1
+    ref = oracle.mla_bwd(c.q_nope, c.q_rope, c.k_nope, c.k_rope, c.v, up.do, scale=c.scale, causal=causal,
+                         dlse=up.dlse)
+    for name, g, r in zip(("dq_nope", "dq_rope", "dk_nope", "dk_rope", "dv"), got, ref):
+        check(name, g, r)

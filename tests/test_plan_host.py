@@ -462,3 +462,42 @@ def test_backward_validation_before_any_launch(arc):
     assert L.arc_attn_bwd(ctypes.byref(a), FAKE + 16, ws, None) == arc.ARC_ERR_WORKSPACE
     a.scale = float("nan")
     assert L.arc_attn_bwd(ctypes.byref(a), FAKE, ws, None) == arc.ARC_ERR_INVALID_ARG
+
+
+def mla_bwd_args(arc, B=2, H=16, T=4096, Dn=128, Dr=64, Dv=128):
+    a = arc.MlaBwdArgs()
+    a.B, a.H, a.Tq, a.Tk, a.Dn, a.Dr, a.Dv = B, H, T, T, Dn, Dr, Dv
+    for f in ("q_nope", "q_rope", "k_nope", "k_rope", "v", "o", "dout", "lse", "dq_nope", "dq_rope", "dk_nope",
+              "dk_rope", "dv"):
+        setattr(a, f, FAKE)
+    a.q_nope_strides = a.k_nope_strides = a.dq_nope_strides = a.dk_nope_strides = (arc._i64 * 3)(*contiguous(B, H, T, Dn))
+    a.q_rope_strides = a.dq_rope_strides = (arc._i64 * 3)(*contiguous(B, H, T, Dr))
+    a.k_rope_strides = a.dk_rope_strides = (arc._i64 * 2)(*contiguous(B, T, Dr))
+    a.v_strides = a.o_strides = a.do_strides = a.dv_strides = (arc._i64 * 3)(*contiguous(B, H, T, Dv))
+    a.scale, a.causal = (Dn + Dr) ** -0.5, 1
+    return a
+
+
+def test_mla_backward_plan_workspace_and_validation(arc):
+    """MLA prefill's shape: 2 x 16 heads x 32 key tiles = 1024 dK/dV CTAs (no split), 64-row
+    fold tiles at d_qk 192; the workspace holds delta and each head's fp32 share of dk_rope;
+    four launches: delta, dK / dV, the sum over heads, dQ."""
+    L = arc.lib()
+    a = mla_bwd_args(arc)
+    info = arc.plan(arc.ARC_OP_MLA_BWD, a)
+    assert info["kernel"] == "bwd_dkdv_kernel<mla>+bwd_dq_kernel" and info["splits"] == 1
+    assert info["n_ctas"] == 2 * 16 * 32 and info["tile_n"] == 64 and info["launches"] == 4
+    ws = L.arc_mla_bwd_workspace_size(ctypes.byref(a))
+    assert ws == 2 * 16 * 4096 * 4 + 2 * 16 * 4096 * 64 * 4
+    assert L.arc_mla_bwd(ctypes.byref(a), None, ws, None) == arc.ARC_ERR_WORKSPACE
+    for field, value, want in (("Dr", 0, arc.ARC_ERR_UNSUPPORTED), ("Dn", 96, arc.ARC_ERR_UNSUPPORTED),
+                               ("Dv", 256, arc.ARC_ERR_UNSUPPORTED)):
+        b = mla_bwd_args(arc)
+        setattr(b, field, value)
+        assert L.arc_mla_bwd(ctypes.byref(b), FAKE, 1 << 34, None) == want, field
+    b = mla_bwd_args(arc)
+    b.k_rope = FAKE + 8                                  # not 16-byte aligned
+    assert L.arc_mla_bwd(ctypes.byref(b), FAKE, 1 << 34, None) == arc.ARC_ERR_UNSUPPORTED
+    b = mla_bwd_args(arc)
+    b.dq_rope = None
+    assert L.arc_mla_bwd(ctypes.byref(b), FAKE, 1 << 34, None) == arc.ARC_ERR_INVALID_ARG
