@@ -541,8 +541,10 @@ struct WsLayout {
     static constexpr int SLICE = S::DT * RS;                                // one K (or V) slice box
     static constexpr int STAGE = S::NS * 2 * SLICE;                         // [slice][K, V] of one tile
     static constexpr int NST = STAGE >= 16384 ? 3 : 4;                      // stages in flight; three CTAs per SM fit
-    static constexpr int QS = D + 16;                                       // Q row stride (halfs)
-    static constexpr int QB = S::ROWS * QS * 2;                             // Q tile (f16, pre-scaled)
+    // Q tile (f16, pre-scaled), stored as the m16n8k16 A fragments themselves: one 16-byte
+    // record per (fragment, k-step, row group g, quad index t), so a lane's operand quad
+    // is one shared load (no register moves to assemble it)
+    static constexpr int QB = S::ROWS * D * 2;
     static constexpr int XB = S::NS > 1 ? 2 * S::NCG * S::NS * MF * 32 * 8 * 4 : 0;   // S partials, 2 buffers
     static constexpr int MAIN = NST * STAGE + QB + XB;
     // in-CTA merge: per cell group O [ROWS][OS] with OS = D + 8*NS (a skew of up to 6
@@ -832,16 +834,24 @@ __global__ void __launch_bounds__(WS_WARPS * 32, MF == 1 ? 3 : 2) decode_ws_kern
         const int vsh = (KVT == ARC_KV_Q4_0 && ve >= 16) ? 4 : 0;  // q4_0: high nibbles hold elements 16..31
 
         asm volatile("bar.sync 2, %0;" ::"n"(WS_WARPS * 32) : "memory");   // stage barriers initialised
-        // Q tile, shared by the four warps: ROWS fold rows x D, scaled into log2 units, f16.
+        // Q tile, shared by the four warps: ROWS fold rows x D, scaled into log2 units, f16,
+        // written as A fragments.  In k-step ks the lane with quad index t holds dims
+        // 16 ks + 4t .. +3 (the permuted k order below): record (f, ks, g, t) is
+        // {rows g, g+8} x {dims +0..1, +2..3}, as a0 = (g, +0..1), a1 = (g+8, +0..1),
+        // a2 = (g, +2..3), a3 = (g+8, +2..3).
+        uint32_t *qw = reinterpret_cast<uint32_t *>(qs);
 #pragma unroll
         for (int j = 0; j < QI; ++j) {
             const int x = threadIdx.x + j * 4 * 32;
             const int r = x / (D / 2), d = (x % (D / 2)) * 2;
             const float2 v = j < QP ? qv[j < QP ? j : 0] : q_load(j);
-            *reinterpret_cast<__half2 *>(qs + r * L::QS + d) = __floats2half2_rn(v.x * p.scale_log2, v.y * p.scale_log2);
+            const int f = r / 16, gg = r % 8, up = (r % 16) / 8;
+            const int ks = d / 16, t = (d % 16) / 4, hi = (d % 4) / 2;
+            qw[(((f * (D / 16) + ks) * 8 + gg) * 4 + t) * 4 + hi * 2 + up] =
+                h2_bits(__floats2half2_rn(v.x * p.scale_log2, v.y * p.scale_log2));
         }
         asm volatile("bar.sync 1, %0;" ::"n"(4 * 32) : "memory");   // consumer warps only
-        const __half *qrow = qs + g * L::QS + 4 * tq + s * KS;
+        const uint4 *qfrag = reinterpret_cast<const uint4 *>(qs) + ((s * (KS / 16)) * 8 + g) * 4 + tq;
 
         for (int i = 0; i < n_tiles; ++i) {
             const int st = i % L::NST;
@@ -875,9 +885,8 @@ __global__ void __launch_bounds__(WS_WARPS * 32, MF == 1 ? 3 : 2) decode_ws_kern
                 for (int f = 0; f < MF; ++f)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
-                        const __half *q0 = qrow + f * 16 * L::QS;
-                        const uint2 a0 = lds_u64(q0 + 32 * B + 16 * hh), a1 = lds_u64(q0 + 8 * L::QS + 32 * B + 16 * hh);
-                        const uint32_t a[4] = {a0.x, a1.x, a0.y, a1.y};
+                        const uint4 aq = qfrag[(f * (D / 16) + 2 * B + hh) * 32];
+                        const uint32_t a[4] = {aq.x, aq.y, aq.z, aq.w};
                         mma16816(sacc[f][0], a, kf0[hh][0], kf0[hh][1]);
                         mma16816(sacc[f][1], a, kf1[hh][0], kf1[hh][1]);
                     }
