@@ -7,25 +7,36 @@
 // the MMA is M = 64 rows (heads) tall.
 //
 // Data path per CTA
-//   warps 0-3   gather: Q rows once, then the top-k rows in tiles of 64 keys,
-//               16-byte cp.async per lane (a warp reads 512 contiguous bytes of
-//               one pool row), written straight into the 128-byte-swizzled
-//               K-major layout the tensor core reads; an index outside
-//               [0, Skv) writes zeros and clears its bit in the tile's validity
-//               mask.  A tile's 64 indices are read once per warp and the next
-//               tile's are fetched while this tile's rows are in flight.
-//               Two tile buffers alternate.
+//   warps 0-3   Q rows once, straight into tensor memory (each warp its own
+//               lane quadrant); then the top-k rows in tiles of 64 keys, 16-byte
+//               cp.async per lane (a warp reads 512 contiguous bytes of one pool
+//               row), written into the 128-byte-swizzled K-major layout the
+//               tensor core reads; an index outside [0, Skv) writes zeros and
+//               clears its bit in the tile's validity mask.  A tile's 64 indices
+//               are read once per warp and the next tile's are fetched while this
+//               tile's rows are in flight.  Three tile buffers rotate.
 //   warp 8      TMEM owner and MMA issuer:
-//                 S[buf] = Q K^T       M=64, N=64 keys,  A and B K-major
-//                 O     += P V         M=64, N<=256,     V read MN-major
+//                 S[buf] = Q K^T       M=64, N=64 keys,  A = Q from TMEM, B K-major
+//                 O     += P V         M=64, N<=256,     A = P, V MN-major (shared memory)
 //               When V is the latent (no separate V) the same gathered tile
 //               serves as K and V, so each row crosses L2 once.
 //   warps 4-7   softmax: two threads per head row, each holding 32 of the
 //               tile's 64 scores; P (bf16) goes to shared memory.
-// TMEM: an M=64 accumulator uses 16 of the 32 lanes of each quadrant.  O sits
-// in lanes 0-15 of each quadrant (columns 0..Dv), S in lanes 16-31 (columns
-// 0..63 and 64..127 for the two buffers), so O never moves.  All TMEM loads
-// and stores here use the 16-lane shape, which touches only its own half.
+// Holding Q in tensor memory (S reads it there as a TS-form A operand) frees the
+// 64 KB it would take in shared memory for a third tile buffer, so the gather of a
+// tile no longer waits for the P V of the tile two before it.  At d 512 the tensor
+// pipe is then busy for about 96% of a tile: S (32 K=16 steps at M=64, N=64) takes
+// about 2,000 cycles and P V (8 steps at N=256) about 1,300.  An M=64 step costs
+// about 32 cycles beyond its half-rate arithmetic whatever its operands' source
+// (two alternating accumulators did not change it), which bounds this shape.
+// TMEM: an M=64 operand or accumulator uses 16 of the 32 lanes of each quadrant
+// (rows 16q .. 16q+15 in lanes 32q .. 32q+15, or 32q+16 .. 32q+31 with the lane
+// field set to 16).  An A operand read from TMEM must sit in the same lanes as the
+// accumulator it feeds, so Q and S share the upper lanes: Q in columns 0..Dqk/2 (two
+// bf16 per column), S in columns 256..383 (two buffers).  The lower lanes hold O in
+// columns 0..Dv, which never moves; P V therefore takes P from shared memory (O
+// fills its half at d_v 512).  All TMEM loads and stores here use the 16-lane
+// shapes, which touch only their own half.
 // Every wait is bounded and reports through p.status.
 #include <math.h>
 
@@ -39,29 +50,33 @@ constexpr int SM_ROWS = 64;        // heads per CTA (MMA M)
 constexpr int SBN = 64;            // keys per tile
 constexpr int SCHUNK = 64 * 128;   // bytes of one [64 rows x 64 bf16] swizzled chunk
 constexpr int S_THREADS = 288;     // 9 warps
+constexpr int NSTG = 3;            // gathered tile buffers
 constexpr float S_LOG2E = 1.4426950408889634f;
 constexpr float S_LN2 = 0.6931471805599453f;
 constexpr float S_RESCALE = 8.0f;
+// TMEM addresses: O at column 0 of the lower 16 lanes of each quadrant; Q and S in
+// the upper 16 lanes (lane field 16)
+constexpr uint32_t TM_Q = (16u << 16) + 0;
+constexpr uint32_t TM_S = (16u << 16) + 256;
 
 struct SparseBars {
     uint64_t q_full;
-    uint64_t kv_full[2];
-    uint64_t kv_empty[2];
+    uint64_t kv_full[NSTG];
+    uint64_t kv_empty[NSTG];
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t o_done;
     uint64_t drain;
-    uint32_t mask[2][2];  // validity of the 64 slots of each tile buffer
+    uint32_t mask[NSTG][2];  // validity of the 64 slots of each tile buffer
     uint32_t tmem_base;
 };
 
 template <int KC, int VC, bool SEPV>
 struct SparseLayout {
     static constexpr int TILE_CHUNKS = KC + (SEPV ? VC : 0);
-    static constexpr int Q_BYTES = KC * SCHUNK;
     static constexpr int TILE_BYTES = TILE_CHUNKS * SCHUNK;
     static constexpr int P_BYTES = SCHUNK;  // [64 rows x 64 keys] bf16
-    static constexpr int BYTES = 1024 + Q_BYTES + 2 * TILE_BYTES + 2 * P_BYTES + (int)sizeof(SparseBars);
+    static constexpr int BYTES = 1024 + NSTG * TILE_BYTES + 2 * P_BYTES + (int)sizeof(SparseBars);
 };
 
 __device__ __forceinline__ bool warp_all_sparse(bool ok) { return __all_sync(0xffffffffu, ok); }
@@ -74,9 +89,8 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
     using L = SparseLayout<KC, VC, SEPV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = align_smem<1024>(smem_raw);
-    uint8_t *sQ = smem;
-    uint8_t *sKV = sQ + L::Q_BYTES;               // 2 tile buffers
-    uint8_t *sP = sKV + 2 * L::TILE_BYTES;        // 2 P buffers
+    uint8_t *sKV = smem;                              // NSTG tile buffers
+    uint8_t *sP = sKV + NSTG * L::TILE_BYTES;         // 2 P buffers
     SparseBars *bars = reinterpret_cast<SparseBars *>(sP + 2 * L::P_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,9 +104,11 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
 
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 128);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < NSTG; ++i) {
             mbar_init(&bars->kv_full[i], 128);
             mbar_init(&bars->kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&bars->s_full[i], 1);
             mbar_init(&bars->p_full[i], 128);
         }
@@ -111,18 +127,28 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
 
     if (warp < 4) {
         // =============================== gather
-        const int g = threadIdx.x;  // 0..127
-        // Q: 64 head rows x KC chunks of 8 units
-        for (int x = g; x < SM_ROWS * KC * 8; x += 128) {
-            const int r = x / (KC * 8), c = (x / 8) % KC, u = x % 8;
+        {
+            // Q row r = 16 * warp + (lane & 15) into this warp's lane quadrant: half
+            // (lane >> 4) of each 64-column group, i.e. 64 consecutive bf16 per store.
+            const int r = warp * 16 + (lane & 15), half = lane >> 4;
             const int h = h0 + r;
-            const __nv_bfloat16 *src = p.q + (int64_t)tok * p.qs[0] + (int64_t)(h < p.H ? h : 0) * p.qs[1] + c * 64 + u * 8;
-            cp_async16(sQ + c * SCHUNK + swz(r, u), src, h < p.H ? 16u : 0u);
+            const __nv_bfloat16 *qrow = p.q + (int64_t)tok * p.qs[0] + (int64_t)(h < p.H ? h : 0) * p.qs[1];
+            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + TM_Q;   // + upper-lane field
+#pragma unroll 1
+            for (int c = 0; c < KC / 2; ++c) {
+                uint32_t w[32];
+                const uint4 *src = reinterpret_cast<const uint4 *>(qrow + c * 128 + half * 64);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 v = h < p.H ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+                    w[4 * i] = v.x, w[4 * i + 1] = v.y, w[4 * i + 2] = v.z, w[4 * i + 3] = v.w;
+                }
+                tmem_st16x2_32(taddr + c * 64, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->q_full);
         }
-        cp_async_commit_group();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->q_full);
 
         const int32_t *idx_row = p.idx + (int64_t)tok * p.idx_stride + s_begin;
         // Lane i < 16 of warp w holds the index of tile row w + 4i; warp 0 also holds
@@ -140,9 +166,9 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
         if (nt > 0) fetch(0, mine, m0, m1);
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
-            const int b = j & 1;
-            if (j >= 2) {
-                ok = warp_all_sparse(mbar_wait(&bars->kv_empty[b], (uint32_t)(((j - 2) >> 1) & 1)));
+            const int b = j % NSTG;
+            if (j >= NSTG) {
+                ok = warp_all_sparse(mbar_wait(&bars->kv_empty[b], (uint32_t)((j / NSTG - 1) & 1)));
                 if (!ok) break;
             }
             uint8_t *tile = sKV + b * L::TILE_BYTES;
@@ -189,26 +215,25 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
             const uint32_t idesc_s = idesc_bf16(SM_ROWS, SBN, false, false);
             constexpr int NV = VC * 64;                 // O columns
             constexpr int NG = (NV + 255) / 256;        // N groups of <= 256
-            const uint64_t qd0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
             const uint64_t kvd0 = sdesc_sw128(smem_u32(sKV), 16, 1024);
             const uint64_t vd0 = sdesc_sw128(smem_u32(sKV), SCHUNK, 1024);
             const uint64_t pd0 = sdesc_sw128(smem_u32(sP), 16, 1024);
             bool ok = mbar_wait(&bars->q_full, 0);
             tc_fence_after();
             auto issue_s = [&](int j) {
-                const int b = j & 1;
+                const int b = j % NSTG;
                 tc_fence_after();
-                const uint32_t d = tmem + (16u << 16) + b * SBN;
+                const uint32_t d = tmem + TM_S + (j & 1) * SBN;
 #pragma unroll
                 for (int c = 0; c < KC; ++c)
-                    umma_ss_k64(d, qd0 + (uint64_t)(c * kChunkUnits),
-                                kvd0 + (uint64_t)((b * L::TILE_CHUNKS + c) * kChunkUnits), idesc_s, c > 0);
-                umma_commit(&bars->s_full[b]);
+                    umma_ts_k64(d, tmem + TM_Q + c * 32, kvd0 + (uint64_t)((b * L::TILE_CHUNKS + c) * kChunkUnits), 2,
+                                idesc_s, c > 0);
+                umma_commit(&bars->s_full[j & 1]);
             };
             auto issue_pv = [&](int j) {
-                const int b = j & 1;
+                const int b = j % NSTG;
                 tc_fence_after();
-                const uint64_t a = pd0 + (uint64_t)(b * kChunkUnits);
+                const uint64_t a = pd0 + (uint64_t)((j & 1) * kChunkUnits);
                 const int vfirst = b * L::TILE_CHUNKS + (SEPV ? KC : 0);
 #pragma unroll
                 for (int gi = 0; gi < NG; ++gi) {
@@ -229,7 +254,7 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
             int js = 0, jp = 0;
             uint64_t t_last = globaltimer_ns();
             while (ok && jp < nt) {
-                if (js < nt && js <= jp + 1 && mbar_test(&bars->kv_full[js & 1], (uint32_t)((js >> 1) & 1))) {
+                if (js < nt && js <= jp + 1 && mbar_test(&bars->kv_full[js % NSTG], (uint32_t)((js / NSTG) & 1))) {
                     issue_s(js++);
                     t_last = globaltimer_ns();
                 } else if (jp < js && mbar_test(&bars->p_full[jp & 1], (uint32_t)((jp >> 1) & 1))) {
@@ -251,21 +276,20 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
         const int h = h0 + r;
         const bool row_ok = h < p.H;
         const uint32_t o_lanes = (uint32_t)(q4 * 32) << 16;
-        const uint32_t s_lanes = (uint32_t)(q4 * 32 + 16) << 16;
         const float sl2 = p.scale_log2;
         float m_use = -INFINITY, l = 0.f;
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
-            const int b = j & 1;
-            ok = warp_all_sparse(mbar_wait(&bars->s_full[b], (uint32_t)((j >> 1) & 1)));
+            const int sb = j & 1, b = j % NSTG;
+            ok = warp_all_sparse(mbar_wait(&bars->s_full[sb], (uint32_t)((j >> 1) & 1)));
             if (!ok) break;
             tc_fence_after();
             uint32_t sv[32];
-            tmem_ld16x2_32(tmem + s_lanes + b * SBN, sv);
+            tmem_ld16x2_32(tmem + o_lanes + TM_S + sb * SBN, sv);
             tmem_wait_ld();
             // validity of this thread's 32 keys, published with the tile (kv_full is
             // already complete here; waiting on it orders the mask read after its write)
-            ok = warp_all_sparse(mbar_wait(&bars->kv_full[b], (uint32_t)((j >> 1) & 1)));
+            ok = warp_all_sparse(mbar_wait(&bars->kv_full[b], (uint32_t)((j / NSTG) & 1)));
             if (!ok) break;
             const uint32_t bits = bars->mask[b][half];
             float mx = -INFINITY;
@@ -292,8 +316,10 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                 pk[i] = pack_bf16(p0, p1);
             }
             l = l * alpha + rowsum;   // this thread's half of the row; halves are added at the end
-            // P row r, keys half*32 .. +31 = 16-byte units half*4 .. half*4+3
-            uint8_t *prow = sP + b * L::P_BYTES;
+            // P row r, keys half*32 .. +31 = 16-byte units half*4 .. half*4+3 of P buffer
+            // sb.  P V of tile j-2, the last reader of this buffer, completed before the
+            // o_done wait of tile j-1.
+            uint8_t *prow = sP + sb * L::P_BYTES;
 #pragma unroll
             for (int u = 0; u < 4; ++u)
                 *reinterpret_cast<uint4 *>(prow + swz(r, half * 4 + u)) =
@@ -313,11 +339,11 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                         for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
                         tmem_st16x2_32(tmem + o_lanes + c * 64, ov);
                     }
-                    tmem_wait_st();
                 }
             }
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars->p_full[b]);
+            mbar_arrive(&bars->p_full[sb]);
         }
         if (ok && nt > 0) {
             ok = warp_all_sparse(mbar_wait(&bars->o_done, (uint32_t)((nt - 1) & 1)));
@@ -400,7 +426,7 @@ int sparse_smem_bytes(int dqk, int dv, bool sepv)
 {
     const int kc = dqk / 64, vc = dv / 64;
     const int tile = (kc + (sepv ? vc : 0)) * SCHUNK;
-    return 1024 + kc * SCHUNK + 2 * tile + 2 * SCHUNK + (int)sizeof(SparseBars);
+    return 1024 + NSTG * tile + 2 * SCHUNK + (int)sizeof(SparseBars);
 }
 
 bool sparse_tc_supported(int dqk, int dv, bool sepv)

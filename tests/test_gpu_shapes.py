@@ -123,6 +123,49 @@ def test_sparse_every_listed_head_dim_pair(Dqk, Dv, sep_v):
     assert arc.check_device_error(st) == arc.ARC_OK
 
 
+@pytest.mark.parametrize("Dqk,Dv,sep_v", [(512, 512, False), (128, 64, True)])
+def test_sparse_invalid_slots_read_no_pool_row(Dqk, Dv, sep_v):
+    """The kernel gathers rows four slots at a time.  Invalid slots (-1, negative,
+    Skv and beyond) are placed as whole tiles, whole groups of four, one to three
+    slots of a group, every other slot, and a ragged last tile; every pool row that
+    no valid slot names holds NaN.  An invalid slot adds nothing, so the output must
+    be finite and equal the oracle's, which never reads such a row."""
+    c = W.sparse_case(8, 64, 3000, Dqk, Dv, 203, pad_frac=0.0, separate_v=sep_v, seed=262)
+    bad = np.array([-1, -5, c.Skv, c.Skv + 77, 2**31 - 1], dtype=np.int64)
+    rng = np.random.default_rng(263)
+    slots = np.arange(c.topk)
+    patterns = [
+        slots < 64,                                  # a whole tile
+        (slots // 4) % 3 == 1,                       # whole groups of four
+        slots % 4 == 1,                              # one slot of each group
+        slots % 4 != 0,                              # three slots of each group
+        slots % 2 == 0,                              # every other slot
+        slots >= 192,                                # the ragged last tile
+        rng.random(c.topk) < 0.5,
+        np.ones(c.topk, dtype=bool),                 # no valid slot at all
+    ]
+    for t, m in enumerate(patterns):
+        c.idx[t, m] = rng.choice(bad, size=int(m.sum())).astype(np.int32)
+    valid = c.idx[(c.idx >= 0) & (c.idx < c.Skv)]
+    unnamed = np.setdiff1d(np.arange(c.Skv), valid)
+    assert unnamed.size > 0
+    nan = np.uint16(0x7FC0)
+    c.kv[unnamed] = nan
+    if sep_v:
+        c.v[unnamed] = nan
+    q, kv, idx = dev(c.q), dev(c.kv), dev(c.idx)
+    v = dev(c.v) if sep_v else None
+    st = status_word()
+    o, lse = arc.sparse_mla_fwd(q, kv, idx, Dv=Dv, v=v, scale=c.scale, status=st)
+    torch.cuda.synchronize()
+    assert arc.plan_sparse(q, kv, idx, o, lse, Dv=Dv, v=v)["kernel"] == "sparse_tc_kernel"
+    assert bool(torch.isfinite(o).all())
+    ro, rl = oracle.run_case(c)
+    compare(o, lse, ro, rl, TOL_O_BF16)
+    assert float(o[7].abs().max()) == 0.0
+    assert arc.check_device_error(st) == arc.ARC_OK
+
+
 @pytest.mark.parametrize("Dqk,Dv", [(512, 512), (128, 64)])
 def test_sparse_sinks_and_a_row_with_no_valid_slot(Dqk, Dv):
     """Sinks in the sparse kernel's epilogue (sink max, rescale, the sink in the
