@@ -36,6 +36,7 @@
 // S and dP are computed in both main kernels (5 + 2 products per tile pair for
 // 5 algorithmic): the price of needing no atomics and no dS round trip
 // through memory.
+#include <limits.h>
 #include <math.h>
 
 #include "internal.h"
@@ -117,7 +118,8 @@ struct DkdvLayout {
     static constexpr int QCH = BR * 128;                      // one 64-column chunk of a fold tile
     static constexpr int STAGE = (KC + VC) * QCH;             // Q and dO of one fold tile
     static constexpr int FIXED = (KC + VC) * KCH;             // K and V of the CTA's key tile
-    static constexpr int BYTES = 1024 + FIXED + 2 * STAGE + 3 * 2 * 128 * 4 + (int)sizeof(BwdBars);
+    // + per fold tile (two buffers): (LSE, delta) pairs, last visible keys, per-warp minima
+    static constexpr int BYTES = 1024 + FIXED + 2 * STAGE + 2 * 128 * 12 + 2 * 4 * 4 + (int)sizeof(BwdBars);
     static constexpr int DV_COL = 0, DK_COL = DV;
     __host__ __device__ static constexpr int s_col(int h) { return DV + D + h * 2 * HR; }
     __host__ __device__ static constexpr int dp_col(int h) { return DV + D + h * 2 * HR + HR; }
@@ -135,10 +137,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
     uint8_t *smem = align_smem<1024>(smem_raw);
     uint8_t *sK = smem, *sV = sK + KC * KCH;
     uint8_t *sRing = sK + L::FIXED;                             // [2][Q chunks, dO chunks]
-    float *col_lse2 = reinterpret_cast<float *>(sRing + 2 * L::STAGE);   // [2][128]
-    float *col_delta = col_lse2 + 2 * 128;
-    int *col_lim = reinterpret_cast<int *>(col_delta + 2 * 128);
-    BwdBars *bars = reinterpret_cast<BwdBars *>(col_lim + 2 * 128);
+    float2 *col_ld = reinterpret_cast<float2 *>(sRing + 2 * L::STAGE);   // [2][128] (LSE in log2 units, delta)
+    int *col_lim = reinterpret_cast<int *>(col_ld + 2 * 128);             // [2][128] last key a row may see
+    int *col_wmin = col_lim + 2 * 128;                                    // [2][4] min of those per 32 rows
+    BwdBars *bars = reinterpret_cast<BwdBars *>(col_wmin + 2 * 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_kt = (p.Tk + BK - 1) / BK;
@@ -306,12 +308,15 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
         bool ok = true;
         for (int qt = next_live(qt_begin); qt < qt_end; qt = next_live(qt + 1)) {
             const int cb = (it & 1) * 128;
+            int lim_min = INT_MAX;    // a row past the group has P = 0 (LSE +inf) and bounds nothing
             if (tid < BR) {
                 const RowInfo ri = row_info(p, b, kvh, qt * BR + tid);
-                col_lse2[cb + tid] = ri.lse2;
-                col_delta[cb + tid] = ri.delta;
+                col_ld[cb + tid] = make_float2(ri.lse2, ri.delta);
                 col_lim[cb + tid] = ri.lim;
+                if (qt * BR + tid < p.G * p.Tq) lim_min = ri.lim;
             }
+            lim_min = __reduce_min_sync(0xffffffffu, lim_min);
+            if (lane == 0 && tid < BR) col_wmin[(it & 1) * 4 + (tid >> 5)] = lim_min;
             // every softmax thread has written its column (a bounded wait, unlike a named
             // barrier, so a thread that stopped early cannot hold the others forever)
             mbar_arrive(&bars->cols);
@@ -320,6 +325,13 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                 report(p.status, BW_AT_COLS);
                 break;
             }
+            // Every row of the tile sees every valid key of the CTA: no causal test per
+            // element.  (A key past Tk then gets a nonzero P, but it only feeds its own
+            // dK / dV rows, which are never stored.)
+            int tile_min = INT_MAX;
+#pragma unroll
+            for (int w = 0; w < BR / 32; ++w) tile_min = min(tile_min, col_wmin[(it & 1) * 4 + w]);
+            const bool whole = tile_min >= min(k0 + BK - 1, p.Tk - 1);
 #pragma unroll 1
             for (int h = 0; h < NH && ok; ++h) {
                 ok = bw_all(mbar_wait(&bars->s_full[h], (uint32_t)(it & 1)));
@@ -336,20 +348,35 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                     tmem_wait_ld();
                     const int c0 = cb + h * HR + 32 * ch;
                     uint32_t pk[16], dk[16];
+                    if (whole) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float pp[2], dd[2];
+                        for (int i = 0; i < 16; ++i) {
+                            float pp[2], dd[2];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int c = c0 + 2 * i + e;
-                            const float pe = kj <= col_lim[c]
-                                                 ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -col_lse2[c]))
-                                                 : 0.f;
-                            pp[e] = pe;
-                            dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - col_delta[c]);
+                            for (int e = 0; e < 2; ++e) {
+                                const float2 ld = col_ld[c0 + 2 * i + e];
+                                pp[e] = fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ld.x));
+                                dd[e] = pp[e] * (__uint_as_float(dv[2 * i + e]) - ld.y);
+                            }
+                            pk[i] = pack_bf16(pp[0], pp[1]);
+                            dk[i] = pack_bf16(dd[0], dd[1]);
                         }
-                        pk[i] = pack_bf16(pp[0], pp[1]);
-                        dk[i] = pack_bf16(dd[0], dd[1]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float pp[2], dd[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const int c = c0 + 2 * i + e;
+                                const float2 ld = col_ld[c];
+                                const float pe =
+                                    kj <= col_lim[c] ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ld.x)) : 0.f;
+                                pp[e] = pe;
+                                dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - ld.y);
+                            }
+                            pk[i] = pack_bf16(pp[0], pp[1]);
+                            dk[i] = pack_bf16(dd[0], dd[1]);
+                        }
                     }
                     // bf16 pairs over the first half of the columns just read
                     tmem_st16(tmem + lane_off + L::s_col(h) + 16 * ch, pk);
@@ -619,17 +646,32 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
                     tmem_wait_ld();
                     const int key0 = j * BK + h * HK + 32 * ch;
                     uint32_t dk[16];
+                    // all 32 keys visible to every row of the warp (a row past the group has
+                    // P = 0 from its +inf LSE): no causal test per element
+                    if (__all_sync(0xffffffffu, r >= rows || key0 + 31 <= ri.lim)) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float dd[2];
+                        for (int i = 0; i < 16; ++i) {
+                            float dd[2];
 #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const float pe = key0 + 2 * i + e <= ri.lim
-                                                 ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ri.lse2))
-                                                 : 0.f;
-                            dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - ri.delta);
+                            for (int e = 0; e < 2; ++e) {
+                                const float pe = fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ri.lse2));
+                                dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - ri.delta);
+                            }
+                            dk[i] = pack_bf16(dd[0], dd[1]);
                         }
-                        dk[i] = pack_bf16(dd[0], dd[1]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            float dd[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                const float pe = key0 + 2 * i + e <= ri.lim
+                                                     ? fast_exp2(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -ri.lse2))
+                                                     : 0.f;
+                                dd[e] = pe * (__uint_as_float(dv[2 * i + e]) - ri.delta);
+                            }
+                            dk[i] = pack_bf16(dd[0], dd[1]);
+                        }
                     }
                     tmem_st16(tmem + lane_off + L::s_col(h) + 16 * ch, dk);
                 }
