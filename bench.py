@@ -345,7 +345,9 @@ def kernel_source_hash(kernel):
              "tc_attn_pair_kernel<mla>": "attn_pair.cu",
              "tc_attn2_kernel": "attn_tc.cu", "tc_attn2_kernel<mla>": "attn_tc.cu",
              "sparse_tc_kernel": "sparse_tc.cu", "simple_attn_kernel<sparse>": "simple_kernels.cu",
-             "simple_attn_kernel": "simple_kernels.cu", "merge_kernel": "merge.cu"}
+             "simple_attn_kernel": "simple_kernels.cu", "merge_kernel": "merge.cu",
+             "sparse_tc_kernel<split>": "sparse_tc.cu", "bwd_dkdv_kernel+bwd_dq_kernel": "attn_bwd.cu",
+             "bwd_dkdv_kernel<mla>+bwd_dq_kernel": "attn_bwd.cu"}
     f = files.get(kernel)
     if kernel.startswith("decode_split_kernel") or kernel.startswith("decode_ws_kernel"):
         f = "decode.cu"
