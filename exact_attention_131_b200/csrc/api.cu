@@ -886,6 +886,22 @@ arc_status run_bwd(const arc_attn_bwd_args *a, const MlaBwdExtra *mla, void *wor
     p.dkv_part = pl.rsplit > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + pl.delta_bytes) : nullptr;
     p.status = a->status;
     if (a->Tk == 0) p.rsplit = 1;   // no key: every gradient is zero; the dQ kernel writes dQ
+    // dQ tiles by decreasing causal work (key tiles visible to the tile's last position),
+    // so the heaviest go out first; without a mask every tile is alike
+    const int n_rt = (G * a->Tq + 127) / 128;
+    if (a->causal && n_rt <= 1024) {
+        const int n_kt = (a->Tk + 127) / 128;
+        std::vector<std::pair<int, int>> w(n_rt);
+        for (int rt = 0; rt < n_rt; ++rt) {
+            const int r0 = rt * 128, rl = std::min(r0 + 128, G * a->Tq) - 1;
+            const int t_max = (r0 / a->Tq != rl / a->Tq) ? a->Tq - 1 : rl % a->Tq;
+            const int nk = std::max(0, std::min(a->Tk, t_max + a->Tk - a->Tq + 1));
+            w[rt] = {-std::min(n_kt, (nk + 127) / 128), rt};
+        }
+        std::stable_sort(w.begin(), w.end());
+        p.dq_order_n = n_rt;
+        for (int i = 0; i < n_rt; ++i) p.dq_order[i] = (uint16_t)w[i].second;
+    }
     note_dispatch(mla ? "bwd_dkdv_kernel<mla>" : "bwd_dkdv_kernel");
     note_dispatch("bwd_dq_kernel");
     return launch_bwd(p, s) == cudaSuccess ? ARC_OK : ARC_ERR_CUDA;

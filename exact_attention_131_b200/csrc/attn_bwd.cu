@@ -48,7 +48,12 @@ namespace {
 constexpr int BK = 128;                 // keys per tile (dK/dV: the CTA's keys; dQ: the streamed tile)
 constexpr int BQ = 128;                 // fold rows per dQ tile
 constexpr int KCH = 128 * 128;          // bytes of a [128 rows x 64 bf16] swizzled chunk
-constexpr int BW_THREADS = 256;         // producer, MMA issuer, 2 idle, 4 softmax / epilogue warps
+constexpr int BW_THREADS = 256;         // dQ: producer, MMA issuer, 2 idle, 4 softmax / epilogue warps
+// dK/dV: producer, MMA issuer, 2 idle, then two groups of 4 softmax / epilogue warps (two
+// warps per lane quadrant), each group taking every other 32-row chunk of a half, so the
+// TMEM load -> exp2 -> TMEM store chains of two chunks overlap
+constexpr int DKDV_GROUPS = 2;
+constexpr int DKDV_THREADS = 128 + DKDV_GROUPS * 128;
 constexpr int BW_SMEM_LIMIT = 232448;
 constexpr float BW_LOG2E = 1.4426950408889634f;
 
@@ -108,6 +113,8 @@ __device__ __forceinline__ RowInfo row_info(const BwdParams &p, int b, int kvh, 
 }
 
 
+static_assert(sizeof(BwdParams) <= 4096, "backward parameters fit the classic kernel-parameter space");
+
 // dK / dV.  A fold tile of BR rows is processed as NH halves of HR = BR/NH rows, each
 // with its own S^T / dP^T buffers in TMEM: while the softmax warps rebuild P and dS of
 // one half, the tensor core runs the other half's products.
@@ -129,7 +136,7 @@ struct DkdvLayout {
 };
 
 template <int D, int DV, int BR, int NH>
-__global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
+__global__ void __launch_bounds__(DKDV_THREADS, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams p)
 {
     using L = DkdvLayout<D, DV, BR, NH>;
     constexpr int KC = L::KC, VC = L::VC, HR = L::HR;
@@ -144,10 +151,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_kt = (p.Tk + BK - 1) / BK;
+    // key-tile-major: under a causal mask the first key tiles see the most fold rows, so
+    // the heaviest CTAs of every (batch, kv head) go out first and the light ones fill in
     const int rs = blockIdx.x % p.rsplit;
-    const int kt = (blockIdx.x / p.rsplit) % n_kt;
-    const int kvh = (blockIdx.x / (p.rsplit * n_kt)) % p.Hkv;
-    const int b = blockIdx.x / (p.rsplit * n_kt * p.Hkv);
+    const int kvh = (blockIdx.x / p.rsplit) % p.Hkv;
+    const int b = (blockIdx.x / (p.rsplit * p.Hkv)) % p.B;
+    const int kt = blockIdx.x / (p.rsplit * p.Hkv * p.B);
     const int k0 = kt * BK;
     const int n_qt = (p.G * p.Tq + BR - 1) / BR;
     const int qt_begin = rs * p.tiles_per_split, qt_end = min(n_qt, qt_begin + p.tiles_per_split);
@@ -164,10 +173,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
             mbar_init(&bars->full[i], 1);
             mbar_init(&bars->empty[i], 1);
             mbar_init(&bars->s_full[i], 1);
-            mbar_init(&bars->p_full[i], 128);
+            mbar_init(&bars->p_full[i], DKDV_GROUPS * 128);
         }
         mbar_init(&bars->done, 1);
-        mbar_init(&bars->cols, 128);
+        mbar_init(&bars->cols, DKDV_GROUPS * 128);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -270,16 +279,17 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                     }
                     tc_fence_after();
                     // dV += P^T_h dO_h, dK += dS^T_h Q_h: B read MN-major from the half's rows
-                    // (16 fold rows = 2048 B per K step)
+                    // (16 fold rows = 2048 B per K step).  The bf16 P^T / dS^T of 32-row chunk
+                    // c sit in the first 16 of that chunk's 32 columns.
                     const uint32_t acc = (it > 0 || h > 0) ? 1u : 0u;
 #pragma unroll
-                    for (int k4 = 0; k4 < HR / 64; ++k4)
-                        umma_ts_k64(tmem + L::DV_COL, tmem + L::s_col(h) + k4 * 32,
-                                    dob + (uint64_t)(h * kHalf + k4 * 512), 128, idesc_dv, acc | k4);
+                    for (int c2 = 0; c2 < HR / 32; ++c2)
+                        umma_ts_k32(tmem + L::DV_COL, tmem + L::s_col(h) + c2 * 32,
+                                    dob + (uint64_t)(h * kHalf + c2 * 256), 128, idesc_dv, acc | c2);
 #pragma unroll
-                    for (int k4 = 0; k4 < HR / 64; ++k4)
-                        umma_ts_k64(tmem + L::DK_COL, tmem + L::dp_col(h) + k4 * 32,
-                                    qb + (uint64_t)(h * kHalf + k4 * 512), 128, idesc_dk, acc | k4);
+                    for (int c2 = 0; c2 < HR / 32; ++c2)
+                        umma_ts_k32(tmem + L::DK_COL, tmem + L::dp_col(h) + c2 * 32,
+                                    qb + (uint64_t)(h * kHalf + c2 * 256), 128, idesc_dk, acc | c2);
                     if (h == NH - 1) umma_commit(&bars->empty[st]);   // the stage is free once these have read it
                     if (qn < qt_end) {
                         if (h == 0) {
@@ -299,8 +309,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
             mbar_wait(&bars->done, 0);
         }
     } else if (warp >= 4) {
-        // =============================== P^T, dS^T (one thread per key) and the epilogue
-        const int tid = threadIdx.x - 128;                      // key lane 0..127
+        // =============================== P^T, dS^T (one thread per key and chunk group) and the epilogue
+        const int tid = (threadIdx.x - 128) & 127;              // key lane 0..127 (the warp's TMEM quadrant)
+        const int grp = (threadIdx.x - 128) >> 7;               // chunk group
         const int kj = k0 + tid;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const float sl2 = p.scale_log2;
@@ -309,14 +320,14 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
         for (int qt = next_live(qt_begin); qt < qt_end; qt = next_live(qt + 1)) {
             const int cb = (it & 1) * 128;
             int lim_min = INT_MAX;    // a row past the group has P = 0 (LSE +inf) and bounds nothing
-            if (tid < BR) {
+            if (grp == 0 && tid < BR) {
                 const RowInfo ri = row_info(p, b, kvh, qt * BR + tid);
                 col_ld[cb + tid] = make_float2(ri.lse2, ri.delta);
                 col_lim[cb + tid] = ri.lim;
                 if (qt * BR + tid < p.G * p.Tq) lim_min = ri.lim;
             }
             lim_min = __reduce_min_sync(0xffffffffu, lim_min);
-            if (lane == 0 && tid < BR) col_wmin[(it & 1) * 4 + (tid >> 5)] = lim_min;
+            if (grp == 0 && lane == 0 && tid < BR) col_wmin[(it & 1) * 4 + (tid >> 5)] = lim_min;
             // every softmax thread has written its column (a bounded wait, unlike a named
             // barrier, so a thread that stopped early cannot hold the others forever)
             mbar_arrive(&bars->cols);
@@ -341,7 +352,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                 }
                 tc_fence_after();
 #pragma unroll 1
-                for (int ch = 0; ch < HR / 32; ++ch) {
+                for (int ch = grp; ch < HR / 32; ch += DKDV_GROUPS) {
                     uint32_t sv[32], dv[32];
                     tmem_ld32(tmem + lane_off + L::s_col(h) + 32 * ch, sv);
                     tmem_ld32(tmem + lane_off + L::dp_col(h) + 32 * ch, dv);
@@ -378,9 +389,10 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
                             dk[i] = pack_bf16(dd[0], dd[1]);
                         }
                     }
-                    // bf16 pairs over the first half of the columns just read
-                    tmem_st16(tmem + lane_off + L::s_col(h) + 16 * ch, pk);
-                    tmem_st16(tmem + lane_off + L::dp_col(h) + 16 * ch, dk);
+                    // bf16 pairs over the first half of the columns just read (no other
+                    // chunk group reads or writes these columns)
+                    tmem_st16(tmem + lane_off + L::s_col(h) + 32 * ch, pk);
+                    tmem_st16(tmem + lane_off + L::dp_col(h) + 32 * ch, dk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -402,7 +414,7 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dkdv_kernel(const __grid_co
         const int dr = D - p.dk_cols;                             // MLA: rope columns of dK (else 0)
         float *rrow = p.dkr_part + ((((int64_t)rs * p.B + b) * p.Hkv + kvh) * p.Tk + kj) * dr;
 #pragma unroll 1
-        for (int c = 0; c < (D + DV) / 32; ++c) {
+        for (int c = grp; c < (D + DV) / 32; c += DKDV_GROUPS) {
             uint32_t v[32];
             const bool is_k = c < D / 32;
             const int col = is_k ? L::DK_COL + 32 * c : L::DV_COL + 32 * (c - D / 32);
@@ -484,10 +496,12 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rows = p.G * p.Tq;
     const int n_rt = (rows + BQ - 1) / BQ;
-    // heavier tiles (later positions see more keys) first
-    const int rt = n_rt - 1 - blockIdx.x % n_rt;
-    const int kvh = (blockIdx.x / n_rt) % p.Hkv;
-    const int b = blockIdx.x / (n_rt * p.Hkv);
+    // heavier tiles (later positions see more keys) first, over all (batch, kv head) pairs
+    const int nbh = p.B * p.Hkv;
+    const int rank = blockIdx.x / nbh;
+    const int rt = p.dq_order_n ? (int)p.dq_order[rank] : n_rt - 1 - rank;
+    const int kvh = (blockIdx.x % nbh) % p.Hkv;
+    const int b = (blockIdx.x % nbh) / p.Hkv;
     const int r0 = rt * BQ;
     int nt;
     {
@@ -840,7 +854,7 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t s)
         const int bytes = L::BYTES > 118784 ? L::BYTES : 118784;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)) != cudaSuccess) return e;
         const int grid = p.B * p.Hkv * ((p.Tk + BK - 1) / BK) * p.rsplit;
-        if (grid > 0) kern<<<grid, BW_THREADS, bytes, s>>>(p);
+        if (grid > 0) kern<<<grid, DKDV_THREADS, bytes, s>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (p.rsplit > 1 && p.Tk > 0) {

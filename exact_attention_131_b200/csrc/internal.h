@@ -168,6 +168,10 @@ struct BwdParams {
     int rsplit, tiles_per_split;// dK/dV CTAs per key tile along the fold rows, and fold tiles each
     float *dkv_part;            // rsplit > 1: fp32 [rsplit][B][Hkv][Tk][D + Dv] (dK unscaled, then dV)
     uint32_t *status;
+    // dQ CTAs go out rank by rank over all (batch, kv head) pairs; rank i takes fold tile
+    // dq_order[i] (the tiles by decreasing causal work), or n_rt - 1 - i when dq_order_n is 0
+    int dq_order_n;
+    uint16_t dq_order[1024];
 };
 bool bwd_supported(int d, int dv);
 int bwd_tile_rows(int d, int dv);

@@ -255,6 +255,20 @@ ARC_DEV void umma_ts_k64(uint32_t d, uint32_t a_tm, uint64_t b, uint32_t b_step,
         : "memory");
 }
 
+// Two consecutive K=16 steps of a TS MMA: A in TMEM advances 8 columns per step,
+// B advances b_step descriptor units per step.
+ARC_DEV void umma_ts_k32(uint32_t d, uint32_t a_tm, uint64_t b, uint32_t b_step, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.eq.b32 q, %4, %4;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %3, q;\n\t}" ::"r"(d),
+        "r"(a_tm), "l"(b), "r"(idesc), "r"(acc), "r"(a_tm + 8), "l"(b + b_step)
+        : "memory");
+}
+
 // Four K=16 steps of an SS MMA with separate per-step descriptor advances for A and B
 // (e.g. B read MN-major, where one K step of 16 rows is 2048 bytes = 128 units).
 ARC_DEV void umma_ss_k64_step(uint32_t d, uint64_t a, uint32_t a_step, uint64_t b, uint32_t b_step, uint32_t idesc,
