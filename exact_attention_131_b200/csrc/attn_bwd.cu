@@ -734,36 +734,56 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
     }
 }
 
-// delta_i = sum_d dO_id O_id - dLSE_i.  A warp takes RPW = 256 / Dv rows (at least one):
-// each lane moves 8 elements (16 bytes) of one row per step, so a warp keeps 32 16-byte
-// loads of each tensor in flight; the lanes of a row reduce with shuffles.
+// delta_i = sum_d dO_id O_id - dLSE_i.  A warp takes PREP_U groups of RPW = 256 / Dv rows
+// (at least one row a group): each lane moves 8 elements (16 bytes) of one row per step,
+// and the loads of all PREP_U groups go out before any is used, so a lane keeps
+// 2 * PREP_U 16-byte loads in flight; the lanes of a row reduce with shuffles.
+constexpr int PREP_U = 4;
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __grid_constant__ BwdPrepParams p)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rpw = p.Dv >= 256 ? 1 : 256 / p.Dv;               // rows per warp (a power of two)
+    const int rpw = p.Dv >= 256 ? 1 : 256 / p.Dv;               // rows per group (a power of two)
     const int lpr = 32 / rpw;                                   // lanes per row
     const int64_t rows = (int64_t)p.B * p.H * p.Tq;
-    const int64_t row = ((int64_t)blockIdx.x * 8 + warp) * rpw + lane / lpr;
-    const bool live = row < rows;
-    float acc = 0.f;
-    if (live) {
-        const int t = (int)(row % p.Tq), h = (int)((row / p.Tq) % p.H), b = (int)(row / ((int64_t)p.Tq * p.H));
-        const __nv_bfloat16 *o = p.o + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)t * p.os[2];
-        const __nv_bfloat16 *g = p.dout + (int64_t)b * p.dos[0] + (int64_t)h * p.dos[1] + (int64_t)t * p.dos[2];
-        for (int d = (lane % lpr) * 8; d < p.Dv; d += lpr * 8) {
-            const uint4 x = *reinterpret_cast<const uint4 *>(o + d), y = *reinterpret_cast<const uint4 *>(g + d);
-            const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
+    const int64_t first = ((int64_t)blockIdx.x * 8 + warp) * PREP_U * rpw + lane / lpr;
+    const __nv_bfloat16 *o[PREP_U], *g[PREP_U];
+    bool live[PREP_U];
+    float acc[PREP_U];
+#pragma unroll
+    for (int u = 0; u < PREP_U; ++u) {
+        const int64_t row = first + (int64_t)u * rpw;
+        live[u] = row < rows;
+        acc[u] = 0.f;
+        const int64_t rr = live[u] ? row : 0;
+        const int t = (int)(rr % p.Tq), h = (int)((rr / p.Tq) % p.H), b = (int)(rr / ((int64_t)p.Tq * p.H));
+        o[u] = p.o + (int64_t)b * p.os[0] + (int64_t)h * p.os[1] + (int64_t)t * p.os[2];
+        g[u] = p.dout + (int64_t)b * p.dos[0] + (int64_t)h * p.dos[1] + (int64_t)t * p.dos[2];
+    }
+    for (int d = (lane % lpr) * 8; d < p.Dv; d += lpr * 8) {
+        uint4 x[PREP_U], y[PREP_U];
+#pragma unroll
+        for (int u = 0; u < PREP_U; ++u) {
+            x[u] = live[u] ? *reinterpret_cast<const uint4 *>(o[u] + d) : make_uint4(0u, 0u, 0u, 0u);
+            y[u] = live[u] ? *reinterpret_cast<const uint4 *>(g[u] + d) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < PREP_U; ++u) {
+            const uint32_t xw[4] = {x[u].x, x[u].y, x[u].z, x[u].w}, yw[4] = {y[u].x, y[u].y, y[u].z, y[u].w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&xw[k]));
                 const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&yw[k]));
-                acc = fmaf(a.x, c.x, acc);
-                acc = fmaf(a.y, c.y, acc);
+                acc[u] = fmaf(a.x, c.x, acc[u]);
+                acc[u] = fmaf(a.y, c.y, acc[u]);
             }
         }
     }
-    for (int s = lpr / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-    if (live && lane % lpr == 0) p.delta[row] = acc - (p.dlse ? p.dlse[row] : 0.f);
+#pragma unroll
+    for (int u = 0; u < PREP_U; ++u) {
+        for (int sh = lpr / 2; sh > 0; sh >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], sh);
+        const int64_t row = first + (int64_t)u * rpw;
+        if (live[u] && lane % lpr == 0) p.delta[row] = acc[u] - (p.dlse ? p.dlse[row] : 0.f);
+    }
 }
 
 // d sink_h = -sum_{b,t} exp(sink_h - LSE_bht) * delta_bht, one CTA per head, a fixed
@@ -889,8 +909,8 @@ cudaError_t launch_bwd_prep(const BwdPrepParams &p, cudaStream_t s)
 {
     const int64_t rows = (int64_t)p.B * p.H * p.Tq;
     if (rows == 0) return cudaSuccess;
-    const int rpw = p.Dv >= 256 ? 1 : 256 / p.Dv;             // rows per warp, as in the kernel
-    bwd_prep_kernel<<<(unsigned)((rows + 8 * rpw - 1) / (8 * rpw)), 256, 0, s>>>(p);
+    const int64_t per_cta = 8 * PREP_U * (p.Dv >= 256 ? 1 : 256 / p.Dv);   // rows per CTA, as in the kernel
+    bwd_prep_kernel<<<(unsigned)((rows + per_cta - 1) / per_cta), 256, 0, s>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || !p.sinks) return e;
     bwd_dsink_kernel<<<p.H, 256, 0, s>>>(p);
