@@ -10,6 +10,9 @@ kernel: the TMA split kernel, the cp.async split kernel (a cell stride that is
 not a multiple of 16 bytes) and the CUDA-core kernel (ARC_FLAG_FORCE_SIMPLE).  The file
 name sorts last so a stop-at-first-failure run has run everything else.
 """
+import ctypes
+
+import numpy as np
 import pytest
 import torch
 
@@ -95,3 +98,75 @@ def test_noalloc_decode_rejects_calls_beyond_its_buffer():
         arc.attn_decode_q8_noalloc(q, kc, vc, out=o, **_kw(c))
     assert e.value.status == arc.ARC_ERR_WORKSPACE
     assert torch.all(o == 3.0)
+
+
+class _DevBuf:
+    """A raw device allocation of the current driver context, shaped like the tensor it holds."""
+
+    def __init__(self, cu, host):
+        self.cu, self.host = cu, np.ascontiguousarray(host)
+        self.shape = self.host.shape
+        err, self.ptr = cu.cuMemAlloc(max(1, self.host.nbytes))
+        assert err == cu.CUresult.CUDA_SUCCESS, err
+        if self.host.nbytes:
+            (err,) = cu.cuMemcpyHtoD(self.ptr, self.host.ctypes.data, self.host.nbytes)
+            assert err == cu.CUresult.CUDA_SUCCESS, err
+
+    def data_ptr(self):
+        return int(self.ptr)
+
+    def read(self):
+        out = np.empty_like(self.host)
+        (err,) = self.cu.cuMemcpyDtoH(out.ctypes.data, self.ptr, out.nbytes)
+        assert err == self.cu.CUresult.CUDA_SUCCESS, err
+        return out
+
+    def free(self):
+        self.cu.cuMemFree(self.ptr)
+
+
+def test_noalloc_decode_in_a_second_context():
+    """The static scratch has a different device address in every CUDA context.  After a
+    call in the primary context (torch's), a call made with a second context current
+    (created through the driver API, its buffers allocated there) must use that context's
+    address; both results are checked against the oracle."""
+    from cuda.bindings import driver as cu
+
+    c = W.decode_case(2, 4, 700, 16, 4, 128, kv_type=W.KV_Q8_0, seed=47)
+    q, kc, vc = _inputs(c)
+    info = arc.plan_decode(c.kv_type, q, kc, vc, Hkv=c.Hkv, q_begin=c.q_begin, n_q=c.n_q, kv_begin=c.kv_begin,
+                           n_kv=c.n_kv)
+    assert info["splits"] > 1                       # the partials go through the scratch
+    ro, rl = oracle.run_case(c)
+    o, lse = arc.attn_decode_q8_noalloc(q, kc, vc, **_kw(c))
+    torch.cuda.synchronize()
+    compare(o, lse, ro, rl, TOL_O_BF16, TOL_LSE)
+
+    (err,) = cu.cuInit(0)
+    assert err == cu.CUresult.CUDA_SUCCESS, err
+    err, device = cu.cuDeviceGet(torch.cuda.current_device())
+    assert err == cu.CUresult.CUDA_SUCCESS, err
+    err, ctx = cu.cuCtxCreate(0, device)            # made current on this thread
+    assert err == cu.CUresult.CUDA_SUCCESS, err
+    bufs = []
+    try:
+        dq, dkc, dvc = (_DevBuf(cu, x) for x in (c.q.astype(np.float32), c.k_cache, c.v_cache))
+        do = _DevBuf(cu, np.full((c.n_tok, c.H, c.D), np.nan, dtype=np.float32))
+        dl = _DevBuf(cu, np.full((c.n_tok, c.H), np.nan, dtype=np.float32))
+        bufs = [dq, dkc, dvc, do, dl]
+        seqs = arc.make_seqs(c.q_begin, c.n_q, c.kv_begin, c.n_kv)
+        a = arc._decode_args(c.kv_type, dq, dkc, dvc, seqs, len(c.q_begin), c.Hkv, c.n_cells, do, dl, c.scale, 0,
+                             None)
+        for _ in range(2):
+            st = arc.lib().arc_attn_decode_q8_noalloc(ctypes.byref(a), None)
+            assert st == arc.ARC_OK, arc.status_string(st)
+            (err,) = cu.cuCtxSynchronize()
+            assert err == cu.CUresult.CUDA_SUCCESS, err
+            compare(torch.from_numpy(do.read()), torch.from_numpy(dl.read()), ro, rl, TOL_O_BF16, TOL_LSE)
+    finally:
+        for b in bufs:
+            b.free()
+        cu.cuCtxDestroy(ctx)                        # pops it: torch's context is current again
+    o2, lse2 = arc.attn_decode_q8_noalloc(q, kc, vc, **_kw(c))
+    torch.cuda.synchronize()
+    compare(o2, lse2, ro, rl, TOL_O_BF16, TOL_LSE)
