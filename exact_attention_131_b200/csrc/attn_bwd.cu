@@ -150,7 +150,6 @@ __global__ void __launch_bounds__(DKDV_THREADS, 1) bwd_dkdv_kernel(const __grid_
     BwdBars *bars = reinterpret_cast<BwdBars *>(col_wmin + 2 * 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_kt = (p.Tk + BK - 1) / BK;
     // key-tile-major: under a causal mask the first key tiles see the most fold rows, so
     // the heaviest CTAs of every (batch, kv head) go out first and the light ones fill in
     const int rs = blockIdx.x % p.rsplit;
