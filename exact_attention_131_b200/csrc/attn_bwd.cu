@@ -15,19 +15,22 @@
 // inside one accumulator, with no atomics.
 //
 // Kernels (every wait bounded; a wait that runs out reports through p.status):
-//   bwd_prep_kernel   one warp per row: delta_i = D_i - dLSE_i (HBM-bound)
+//   bwd_prep_kernel   delta_i = D_i - dLSE_i, a warp per few rows (HBM-bound)
 //   bwd_dsink_kernel  one CTA per head: the sink gradient, a fixed-order sum
-//   bwd_dkdv_kernel   one CTA per (batch, kv head, 128-key tile[, row split]):
+//   bwd_dkdv_kernel   one CTA per (128-key tile, batch, kv head[, row split]), key tiles
+//                     outermost so the causally heaviest CTAs start first:
 //                       S^T  = K Q^T       M=128 keys, N=64 fold rows (a half tile)
 //                       dP^T = V dO^T
-//                       P^T, dS^T from S^T, dP^T, LSE, delta (softmax warps),
-//                       written back over S^T / dP^T as bf16 (TMEM A operands)
+//                       P^T, dS^T from S^T, dP^T, LSE, delta (two groups of softmax
+//                       warps, a 32-row chunk each), written back over the chunk's
+//                       own S^T / dP^T columns as bf16 (TMEM A operands)
 //                       dV  += P^T dO      dK += dS^T Q   (dO, Q read MN-major)
 //                     TMEM: dV [0, DV), dK [DV, DV+D), then S^T / dP^T of each half;
 //                     the two halves of a 128-row fold tile alternate, so one half's
 //                     softmax overlaps the other half's products (one half of 64
 //                     rows per tile at d_qk 192, where TMEM has no room for two)
-//   bwd_dq_kernel     one CTA per (batch, kv head, 128-row fold tile):
+//   bwd_dq_kernel     one CTA per (batch, kv head, 128-row fold tile), the tiles in
+//                     order of decreasing causal work (a host-sorted table):
 //                       S = Q K^T, dP = dO V^T, dS (softmax warps, over S),
 //                       dQ += dS K         (K read MN-major)
 //                     TMEM: dQ [0, D), S / dP of two 64-key halves at 256 and 384,
