@@ -127,29 +127,6 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
 
     if (warp < 4) {
         // =============================== gather
-        {
-            // Q row r = 16 * warp + (lane & 15) into this warp's lane quadrant: half
-            // (lane >> 4) of each 64-column group, i.e. 64 consecutive bf16 per store.
-            const int r = warp * 16 + (lane & 15), half = lane >> 4;
-            const int h = h0 + r;
-            const __nv_bfloat16 *qrow = p.q + (int64_t)tok * p.qs[0] + (int64_t)(h < p.H ? h : 0) * p.qs[1];
-            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + TM_Q;   // + upper-lane field
-#pragma unroll 1
-            for (int c = 0; c < KC / 2; ++c) {
-                uint32_t w[32];
-                const uint4 *src = reinterpret_cast<const uint4 *>(qrow + c * 128 + half * 64);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint4 v = h < p.H ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-                    w[4 * i] = v.x, w[4 * i + 1] = v.y, w[4 * i + 2] = v.z, w[4 * i + 3] = v.w;
-                }
-                tmem_st16x2_32(taddr + c * 64, w);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bars->q_full);
-        }
-
         const int32_t *idx_row = p.idx + (int64_t)tok * p.idx_stride + s_begin;
         // Lane i < 16 of warp w holds the index of tile row w + 4i; warp 0 also holds
         // one index per lane for each half of the tile, for the validity mask.
@@ -162,8 +139,37 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
                 m1 = s1 < cnt ? idx_row[s1] : -1;
             }
         };
+        // The first tile's indices and every Q load go out together, before anything
+        // waits on either: the CTA's start-up is one memory round trip, not several.
         int32_t mine = -1, m0 = -1, m1 = -1;
         if (nt > 0) fetch(0, mine, m0, m1);
+        {
+            // Q row r = 16 * warp + (lane & 15) into this warp's lane quadrant: half
+            // (lane >> 4) of each 64-column group, i.e. 64 consecutive bf16 per store.
+            const int r = warp * 16 + (lane & 15), half = lane >> 4;
+            const int h = h0 + r;
+            const __nv_bfloat16 *qrow = p.q + (int64_t)tok * p.qs[0] + (int64_t)(h < p.H ? h : 0) * p.qs[1];
+            const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + TM_Q;   // + upper-lane field
+            uint4 qv[KC / 2][8];
+#pragma unroll
+            for (int c = 0; c < KC / 2; ++c) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(qrow + c * 128 + half * 64);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) qv[c][i] = h < p.H ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int c = 0; c < KC / 2; ++c) {
+                uint32_t w[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    w[4 * i] = qv[c][i].x, w[4 * i + 1] = qv[c][i].y, w[4 * i + 2] = qv[c][i].z, w[4 * i + 3] = qv[c][i].w;
+                tmem_st16x2_32(taddr + c * 64, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars->q_full);
+        }
+
         bool ok = true;
         for (int j = 0; j < nt; ++j) {
             const int b = j % NSTG;
