@@ -457,6 +457,9 @@ __global__ void __launch_bounds__(DKDV_THREADS, 1) bwd_dkdv_kernel(const __grid_
         }
     }
 
+    // Each warp arrives whole (a role branch may have left lanes behind, e.g. the MMA
+    // issuer's lane 0), so the barrier below holds until every warp is done with TMEM.
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -728,6 +731,9 @@ __global__ void __launch_bounds__(BW_THREADS, 1) bwd_dq_kernel(const __grid_cons
         }
     }
 
+    // Each warp arrives whole (a role branch may have left lanes behind, e.g. the MMA
+    // issuer's lane 0), so the barrier below holds until every warp is done with TMEM.
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -380,6 +380,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) tc_attn_kernel(const __grid_const
         if (row_ok && slice == 0) p.lse[((int64_t)b * p.H + h) * p.Tq + t] = lse;
     }
 
+    // Each warp arrives whole (a role branch may have left lanes behind, e.g. the MMA
+    // issuer's lane 0), so the barrier below holds until every warp is done with TMEM.
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -729,6 +732,9 @@ __global__ void __launch_bounds__(NTHREADS2, 1) tc_attn2_kernel(const __grid_con
         if (row_ok) p.lse[((int64_t)b * p.H + h) * p.Tq + tpos] = lse;
     }
 
+    // Each warp arrives whole (a role branch may have left lanes behind, e.g. the MMA
+    // issuer's lane 0), so the barrier below holds until every warp is done with TMEM.
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

@@ -405,6 +405,9 @@ __global__ void __launch_bounds__(S_THREADS, 1) sparse_tc_kernel(const __grid_co
         }
     }
 
+    // Each warp arrives whole (a role branch may have left lanes behind, e.g. the MMA
+    // issuer's lane 0), so the barrier below holds until every warp is done with TMEM.
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     if (warp == 8) {
