@@ -1018,7 +1018,10 @@ __global__ void __launch_bounds__(WS_WARPS * 32, MF == 1 ? 3 : 2) decode_ws_kern
             }
     }
 
-    // ---- merge the 4 consumer warps (the raw ring is idle now)
+    // ---- merge the 4 consumer warps (the raw ring is idle now).  The producer warp arrives
+    // whole (its lane 0 ran the load loop alone), so the merge's first barrier holds until
+    // every consumer warp is past its last read of the ring.
+    __syncwarp();
     write_ws_partial<KVT, D, MF>(o, m_r, l_r, cg, s, warp < 4, smem, p, part_index(p, s_idx, kvh, rg, sp));
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
