@@ -63,3 +63,22 @@ def test_merge_bytes():
     o_bytes = 1 * 4 * 10 * 8 * 2
     lse_bytes = 1 * 4 * 10 * 4
     assert bench.work(c) == (3 * (o_bytes + lse_bytes), "byte")
+
+
+def test_every_measured_kernel_maps_to_its_source_and_has_a_traffic_record():
+    """roofline.traffic is taken from profiles/traffic.json only while the recorded source
+    hash matches the kernel's source file: every kernel a measured workload names must map
+    to a file, and every measured workload must have a record naming that kernel."""
+    import json
+    import os
+    names = {"c2": "tc_attn_pair_kernel", "c3": "tc_attn_pair_kernel<mla>", "c4": "sparse_tc_kernel",
+             "c4d": "sparse_tc_kernel<split>", "c5q8": "decode_ws_kernel<q8_0>", "c5q4": "decode_ws_kernel<q4_0>",
+             "c5d256": "decode_ws_kernel<q8_0>", "c5g8": "decode_ws_kernel<q8_0>",
+             "bwd_gqa": "bwd_dkdv_kernel+bwd_dq_kernel", "bwd_mla": "bwd_dkdv_kernel<mla>+bwd_dq_kernel",
+             "merge": "merge_kernel"}
+    assert set(bench.GRADED) | {"merge"} == set(names)
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for cfg, kernel in names.items():
+        assert bench.kernel_source_hash(kernel) is not None, kernel
+        assert rec[cfg]["kernel"] == kernel, cfg
+        assert rec[cfg]["dram_bytes_per_launch"] > 0, cfg
